@@ -1,0 +1,421 @@
+"""Throughput of the gated delta rule on B200: chunked prefill (headline) and decode.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one chunked-prefill pass (gdn_chunk_fwd) over the prefill workload
+B=4, T=4096, H=16, d_k=d_v=128 (bf16 q/k/v, fp32 gates and states, chunk 64).
+`value` is prefill tokens/s over all ranks (every rank runs its own batch: weak
+scaling, no collective on the data path), timed with CUDA events around
+exactly K steps after W warm-up steps, max over ranks.  The inputs (~280 MB)
+are larger than L2, so no explicit flush is done between steps.
+
+The same line carries:
+  e2e          the same metric with host (pinned) inputs copied in and the
+               outputs copied back inside the timed region;
+  roofline     for the dominant kernel, from the library's own per-kernel event
+               timer in the timed region;
+  decode       decode tokens/s on 256 sequences x 32 heads (state updated in
+               place, 64 steps per pass) with its own roofline;
+  cpu_baseline the fp64 oracle on a bounded sample, on this host's cores;
+  clocks       SM clocks sampled with nvidia-smi during the timed region.
+
+--impl reference times the oracle (the CPU reference of the method) instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "gated-delta-rule prefill tokens/s & decode tokens/s, % of TC/HBM roofline"
+UNIT = "tokens/s"
+
+# Algorithmic traffic and work of the prefill workload, per head-token.
+# bytes: q, k, v in and o out (bf16, 128 each) + fp32 gate and beta;
+# states (initial read + final write, 2 x 64 KiB per (sequence, head)) are added per unit.
+PREFILL_BYTES_PER_HEAD_TOKEN = 4 * 128 * 2 + 4 + 4
+STATE_BYTES = 128 * 128 * 4
+# flops: 10*C*d + 6*d^2 + 2*C^2/3 per head-token for C = 64, d = 128
+PREFILL_FLOPS_PER_HEAD_TOKEN = 10 * 64 * 128 + 6 * 128 * 128 + 2 * 64 * 64 / 3
+# decode, per (sequence, head) and step: fp32 state read + written, q/k/v/o bf16, gate+beta fp32
+DECODE_BYTES_PER_UNIT = 2 * STATE_BYTES + 4 * 128 * 2 + 4 + 4
+
+
+def env_rank():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[5:10]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 1 <= r[0] <= (self.t1 or r[0]) + 1]
+        use = inside or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3][1:]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use)}
+
+
+# ---------------------------------------------------------------------------
+# Multi-rank plumbing (host logic; tested with gloo on CPU)
+# ---------------------------------------------------------------------------
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch of the workload (independent sequences)."""
+    return base + 1000 * rank
+
+
+# ---------------------------------------------------------------------------
+# Oracle (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(tokens_per_seq: int, seed: int = 1):
+    from gated_delta_rule_64_b200.inputs import PREFILL_BF16, make_inputs
+    w = PREFILL_BF16.replace(T=tokens_per_seq, seed=seed)
+    return w, make_inputs(w)
+
+
+def time_oracle(x, n_threads):
+    import oracle
+    t = time.perf_counter()
+    oracle.gated_delta_rule(x.q, x.k, x.v, x.g, x.beta, x.h0, n_threads=n_threads)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(target_s: float = 12.0):
+    import oracle
+    cores = oracle.host_threads()
+    w, x = oracle_sample(64)
+    dt = time_oracle(x, cores)
+    per_tok = dt / (w.B * 64)
+    T = int(max(64, min(4096, (target_s / per_tok) / w.B)) // 64 * 64)
+    w, x = oracle_sample(T)
+    dt = time_oracle(x, cores)
+    tokens = w.B * T
+    return {"value": tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"prefill workload B=4 H=16 d=128 bf16, first {T} of 4096 tokens per sequence "
+                      f"({tokens} tokens x 16 heads), fp64 token loop, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return 0
+    import oracle
+    cores = oracle.host_threads()
+    budget = 150.0
+    w, x = oracle_sample(64)
+    per_tok = time_oracle(x, cores) / (w.B * 64)
+    T = int(max(64, min(4096, budget / max(1, args.steps + args.warmup) / per_tok / w.B)) // 64 * 64)
+    w, x = oracle_sample(T)
+    for _ in range(args.warmup):
+        time_oracle(x, cores)
+    times = [time_oracle(x, cores) for _ in range(args.steps)]
+    dt = sum(times) / len(times)
+    value = w.B * T / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill B4 T4096 H16 d128 bf16 (bounded sample per step)", "global_batch": 4,
+                   "seq_len": 4096, "parallelism": "replicas only: oracle on rank 0", "sample_tokens_per_seq": T},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"first {T} tokens of each of the 4 sequences, all 16 heads, per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def traffic_for(kernel: str):
+    """ncu DRAM bytes per launch recorded for `kernel`, if its source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+        return None
+    return rec["bytes_per_launch"] * rec.get("scale_to_bench", 1.0)
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from gated_delta_rule_64_b200 import gdn
+    from gated_delta_rule_64_b200.inputs import DECODE, PREFILL_BF16, make_inputs
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    gdn.load_library()
+    pk = peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---------------- prefill ----------------
+    w = PREFILL_BF16.replace(seed=rank_seed(PREFILL_BF16.seed, rank))
+    x = make_inputs(w)
+    d = lambda t: t.to(dev).contiguous()
+    q, k, v, g, beta, h0 = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    fin = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.gdn_chunk_workspace_size(B, T, H, dk, dv, B, dtype=q.dtype), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdn.gdn_chunk_fwd(q, k, v, g, beta, h0, out=out, final_state=fin, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    gdn.profile_read()
+    gdn.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.mark_begin()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    barrier()
+    gdn.profile_enable(False)
+    kernels = gdn.profile_read()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_step = ms_total / args.steps
+    tokens_all = B * T * world
+    value = tokens_all / (ms_step * 1e-3)
+
+    # dominant kernel roofline (HBM-bound by arithmetic intensity)
+    top = max(kernels.items(), key=lambda kv: kv[1][1]) if kernels else ("none", (1, 0.0))
+    top_name, (top_launches, top_ms) = top
+    per_launch_s = top_ms / max(1, top_launches) * 1e-3
+    head_tokens = B * T * H
+    alg_bytes = head_tokens * PREFILL_BYTES_PER_HEAD_TOKEN + 2 * B * H * STATE_BYTES
+    alg_flops = head_tokens * PREFILL_FLOPS_PER_HEAD_TOKEN
+    achieved = alg_bytes / per_launch_s / 1e9 if per_launch_s > 0 else 0.0
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(top_name), "kernel": top_name,
+                "peak_source": f"{pk['source']} hbm_gbs",
+                "tensor": {"achieved_tflops": alg_flops / per_launch_s / 1e12 if per_launch_s > 0 else 0.0,
+                           "peak": pk["bf16_tflops"],
+                           "frac": (alg_flops / per_launch_s / 1e12) / pk["bf16_tflops"] if per_launch_s > 0 else 0},
+                "step": {"achieved_gbs": alg_bytes / (ms_step * 1e-3) / 1e9,
+                         "frac_hbm": alg_bytes / (ms_step * 1e-3) / 1e9 / pk["hbm_gbs"]},
+                "kernels_ms_per_step": {n: t / args.steps for n, (c, t) in kernels.items()}}
+    launches = sum(c for c, _ in kernels.values())
+
+    # ---------------- e2e through the public API with host buffers ----------------
+    pin = lambda t: t.pin_memory()
+    hq, hk, hv, hg, hb, hh0 = pin(x.q), pin(x.k), pin(x.v), pin(x.g), pin(x.beta), pin(x.h0)
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hfin = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hh0))
+    d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
+
+    def e2e_step():
+        for src, dst in ((hq, q), (hk, k), (hv, v), (hg, g), (hb, beta), (hh0, h0)):
+            dst.copy_(src, non_blocking=True)
+        gdn.gdn_chunk_fwd(q, k, v, g, beta, h0, out=out, final_state=fin, workspace=ws, stream=stream)
+        hout.copy_(out, non_blocking=True)
+        hfin.copy_(fin, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+    e2e = {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
+    del q, k, v, g, beta, h0, out, fin, ws, hq, hk, hv, hg, hb, hh0, hout, hfin
+    torch.cuda.empty_cache()
+
+    # ---------------- decode ----------------
+    wd = DECODE.replace(seed=rank_seed(DECODE.seed, rank))
+    xd = make_inputs(wd)
+    dq, dk_, dv_, dg, db = (d(t) for t in (xd.q, xd.k, xd.v, xd.g, xd.beta))
+    state = d(xd.h0)
+    steps_d = xd.q.shape[0]
+    dout = torch.empty((steps_d,) + tuple(xd.v.shape[1:]), dtype=dq.dtype, device=dev)
+
+    def decode_pass():
+        for s in range(steps_d):
+            gdn.gdn_decode_step(dq[s], dk_[s], dv_[s], dg[s], db[s], state, out=dout[s], stream=stream)
+
+    decode_pass()
+    torch.cuda.synchronize()
+    passes = max(2, min(10, args.steps // 10 + 1))
+    gdn.profile_read()
+    gdn.profile_enable(True)
+    barrier()
+    e0.record(stream)
+    for _ in range(passes):
+        decode_pass()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    gdn.profile_enable(False)
+    dk_times = gdn.profile_read()
+    dms = max_over_ranks(e0.elapsed_time(e1), world, dev) / (passes * steps_d)
+    nseq = xd.q.shape[1]
+    dec_units = nseq * xd.q.shape[3]
+    dname, (dl, dt_ms) = max(dk_times.items(), key=lambda kv: kv[1][1])
+    d_per_launch = dt_ms / dl * 1e-3
+    d_ach = dec_units * DECODE_BYTES_PER_UNIT / d_per_launch / 1e9
+    decode = {"metric": "decode tokens/s", "value": nseq * world / (dms * 1e-3), "unit": UNIT,
+              "ms_per_step": dms, "config": {"workload": wd.name, "sequences": nseq, "heads": xd.q.shape[3],
+                                             "state": "fp32 in HBM, updated in place"},
+              "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                           "frac": d_ach / pk["hbm_gbs"], "traffic": traffic_for(dname), "kernel": dname,
+                           "peak_source": f"{pk['source']} hbm_gbs"},
+              "gpu_launches": sum(c for c, _ in dk_times.values())}
+    del dq, dk_, dv_, dg, db, state, dout
+    clk = clocks.stop()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": B * world, "seq_len": T, "heads": H, "d_k": dk, "d_v": dv,
+                       "chunk": 64, "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": roofline, "decode": decode, "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
+            "gpu_launches": launches,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

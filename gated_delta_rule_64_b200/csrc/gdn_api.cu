@@ -1,0 +1,322 @@
+// C-ABI entry points: argument validation, workspace planning, launches and
+// the optional per-kernel event timer.  No device memory is allocated here.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+// ---------------------------------------------------------------------------
+// Error reporting
+// ---------------------------------------------------------------------------
+static thread_local char g_last_error[512] = "";
+
+gdn_status fail(gdn_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+gdn_status check_launch(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Event timer
+// ---------------------------------------------------------------------------
+namespace {
+struct ProfRecord {
+    const char *name;
+    cudaEvent_t start, stop;
+};
+struct ProfState {
+    std::mutex mu;
+    bool on = false;
+    std::vector<ProfRecord> open;     // recorded, not yet read
+    std::vector<cudaEvent_t> pool;    // free events
+    cudaEvent_t get() {
+        if (!pool.empty()) {
+            cudaEvent_t e = pool.back();
+            pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+        return e;
+    }
+};
+ProfState &prof() {
+    static ProfState *p = new ProfState();  // never destroyed: events may outlive static teardown
+    return *p;
+}
+}  // namespace
+
+LaunchScope::LaunchScope(const char *name, cudaStream_t s) : name_(name), stream_(s), slot_(-1) {
+    ProfState &P = prof();
+    std::lock_guard<std::mutex> lk(P.mu);
+    if (!P.on) return;
+    cudaEvent_t a = P.get(), b = P.get();
+    if (!a || !b) return;
+    cudaEventRecord(a, s);
+    P.open.push_back({name, a, b});
+    slot_ = (int)P.open.size() - 1;
+}
+
+LaunchScope::~LaunchScope() {
+    if (slot_ < 0) return;
+    ProfState &P = prof();
+    std::lock_guard<std::mutex> lk(P.mu);
+    if (slot_ < (int)P.open.size()) cudaEventRecord(P.open[slot_].stop, stream_);
+}
+
+// ---------------------------------------------------------------------------
+// Workspace plan of the chunked forward pass
+// ---------------------------------------------------------------------------
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed) {
+    ChunkPlan p{};
+    p.N = num_seqs;
+    p.rows = d.B * d.T;
+    p.H = d.H;
+    p.dk = d.dk;
+    p.dv = d.dv;
+    p.packed = packed;
+    p.per_channel = d.gate == GDN_GATE_CHANNEL;
+    // Every sequence of length L has ceil(L/64) chunks; over any packing of
+    // `rows` tokens into N sequences that is at most rows/64 + N.
+    p.max_chunks = packed ? (p.rows / kChunk + p.N) : (d.B * ((d.T + kChunk - 1) / kChunk));
+    const int64_t ch = p.max_chunks * p.H;
+    size_t off = 0;
+    p.off_chunk_offsets = off;
+    off = align_up(off + sizeof(int32_t) * (size_t)(p.N + 1), 256);
+    p.off_W = off;
+    off = align_up(off + sizeof(float) * (size_t)ch * kChunk * p.dk, 256);
+    p.off_U = off;
+    off = align_up(off + sizeof(float) * (size_t)ch * kChunk * p.dv, 256);
+    p.off_P = off;
+    off = align_up(off + sizeof(float) * (size_t)ch * kChunk * kChunk, 256);
+    p.off_b = off;
+    off = align_up(off + sizeof(float) * (size_t)ch * kChunk * (p.per_channel ? p.dk : 1), 256);
+    p.total = off;
+    return p;
+}
+
+// ---------------------------------------------------------------------------
+// Validation helpers
+// ---------------------------------------------------------------------------
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+static bool aligned4(const void *p) { return ((uintptr_t)p & 3u) == 0; }
+
+static gdn_status check_desc(const gdn_desc *d) {
+    if (!d) return fail(GDN_ERR_INVALID_ARG, "descriptor is NULL");
+    if (d->B < 0 || d->T < 0 || d->H <= 0)
+        return fail(GDN_ERR_INVALID_ARG, "need B >= 0, T >= 0, H > 0 (got B=%lld T=%lld H=%lld)",
+                    (long long)d->B, (long long)d->T, (long long)d->H);
+    if (d->dk <= 0 || d->dv <= 0)
+        return fail(GDN_ERR_INVALID_ARG, "head sizes must be positive");
+    if (!((d->dk == 64 || d->dk == 128) && (d->dv == 64 || d->dv == 128)))
+        return fail(GDN_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128 (got %lld, %lld)",
+                    (long long)d->dk, (long long)d->dv);
+    if (d->dtype != GDN_F32 && d->dtype != GDN_BF16)
+        return fail(GDN_ERR_INVALID_ARG, "unknown dtype %d", d->dtype);
+    if (d->gate != GDN_GATE_HEAD && d->gate != GDN_GATE_CHANNEL)
+        return fail(GDN_ERR_INVALID_ARG, "unknown gate kind %d", d->gate);
+    if (d->reserved != 0) return fail(GDN_ERR_INVALID_ARG, "reserved field must be 0");
+    if (!isfinite(d->scale)) return fail(GDN_ERR_INVALID_ARG, "scale must be finite");
+    // Keep every element index of every tensor well inside int64.
+    const double elems = (double)d->B * (double)d->T * (double)d->H * (double)(d->dk > d->dv ? d->dk : d->dv);
+    if (elems > 4.0e15) return fail(GDN_ERR_INVALID_ARG, "problem too large");
+    return GDN_OK;
+}
+
+struct Range {
+    uintptr_t lo, hi;
+};
+static bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+static Range range_of(const void *p, size_t bytes) { return {(uintptr_t)p, (uintptr_t)p + bytes}; }
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported";
+        case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_TIMEOUT: return "device wait timed out";
+        case GDN_ERR_INTERNAL: return "internal error";
+    }
+    return "unknown status";
+}
+
+const char *gdn_last_error(void) { return g_last_error; }
+
+gdn_status gdn_profile_enable(int on) {
+    ProfState &P = prof();
+    std::lock_guard<std::mutex> lk(P.mu);
+    P.on = on != 0;
+    return GDN_OK;
+}
+
+gdn_status gdn_profile_read(gdn_kernel_time *entries, int32_t cap, int32_t *count) {
+    if (!count || cap < 0 || (cap > 0 && !entries)) return fail(GDN_ERR_INVALID_ARG, "bad profile_read args");
+    ProfState &P = prof();
+    std::lock_guard<std::mutex> lk(P.mu);
+    std::vector<gdn_kernel_time> acc;
+    gdn_status st = GDN_OK;
+    for (auto &r : P.open) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess)
+            st = fail(GDN_ERR_CUDA, "profile: event query failed");
+        size_t i = 0;
+        for (; i < acc.size(); ++i)
+            if (strcmp(acc[i].name, r.name) == 0) break;
+        if (i == acc.size()) acc.push_back({r.name, 0, 0.0});
+        acc[i].launches += 1;
+        acc[i].total_ms += ms;
+        P.pool.push_back(r.start);
+        P.pool.push_back(r.stop);
+    }
+    P.open.clear();
+    *count = (int32_t)acc.size();
+    for (int32_t i = 0; i < cap && i < (int32_t)acc.size(); ++i) entries[i] = acc[i];
+    return st;
+}
+
+gdn_status gdn_chunk_workspace_size(const gdn_desc *d, int32_t num_seqs, size_t *bytes) {
+    gdn_status st = check_desc(d);
+    if (st != GDN_OK) return st;
+    if (!bytes) return fail(GDN_ERR_INVALID_ARG, "bytes is NULL");
+    if (num_seqs < 0) return fail(GDN_ERR_INVALID_ARG, "num_seqs < 0");
+    // The packed-sequence bound covers B fixed-length sequences too:
+    // B * ceil(T/64) <= B*T/64 + B.
+    ChunkPlan p = make_plan(*d, num_seqs, true);
+    *bytes = p.total;
+    return GDN_OK;
+}
+
+gdn_status gdn_chunk_fwd(const gdn_desc *d, const void *q, const void *k, const void *v,
+                         const float *log_gate, const float *beta, const float *initial_state,
+                         const int32_t *cu_seqlens, int32_t num_seqs, int64_t snapshot_stride,
+                         void *out, float *final_state, float *snapshots, void *workspace,
+                         size_t workspace_bytes, gdn_stream_t stream) {
+    g_last_error[0] = 0;
+    gdn_status st = check_desc(d);
+    if (st != GDN_OK) return st;
+    const bool packed = cu_seqlens != nullptr;
+    if (packed) {
+        if (d->B != 1) return fail(GDN_ERR_INVALID_ARG, "packed sequences need B == 1");
+        if (num_seqs < 0) return fail(GDN_ERR_INVALID_ARG, "num_seqs < 0");
+        if (((uintptr_t)cu_seqlens & 3u) != 0) return fail(GDN_ERR_INVALID_ARG, "cu_seqlens misaligned");
+        if (snapshot_stride != 0)
+            return fail(GDN_ERR_UNSUPPORTED, "snapshots are only supported without cu_seqlens");
+    }
+    const int64_t N = packed ? num_seqs : d->B;
+    if (snapshot_stride < 0 || snapshot_stride % kChunk != 0)
+        return fail(GDN_ERR_INVALID_ARG, "snapshot_stride must be 0 or a positive multiple of 64");
+    const int64_t n_snap = (snapshot_stride > 0 && !packed) ? d->T / snapshot_stride : 0;
+    const int64_t rows = d->B * d->T;
+    const size_t in_el = d->dtype == GDN_F32 ? 4 : 2;
+    const size_t qk_bytes = (size_t)rows * d->H * d->dk * in_el;
+    const size_t v_bytes = (size_t)rows * d->H * d->dv * in_el;
+    const size_t g_bytes = (size_t)rows * d->H * (d->gate == GDN_GATE_CHANNEL ? d->dk : 1) * 4;
+    const size_t b_bytes = (size_t)rows * d->H * 4;
+    const size_t st_bytes = (size_t)N * d->H * d->dv * d->dk * 4;
+    const size_t snap_bytes = (size_t)N * n_snap * d->H * d->dv * d->dk * 4;
+    if (rows > 0) {
+        if (!q || !k || !v || !log_gate || !beta || !out)
+            return fail(GDN_ERR_INVALID_ARG, "q, k, v, log_gate, beta and out are required");
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+            return fail(GDN_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+        if (!aligned4(log_gate) || !aligned4(beta))
+            return fail(GDN_ERR_INVALID_ARG, "log_gate and beta must be 4-byte aligned");
+        const Range ro = range_of(out, v_bytes);
+        const Range ins[] = {range_of(q, qk_bytes), range_of(k, qk_bytes), range_of(v, v_bytes),
+                             range_of(log_gate, g_bytes), range_of(beta, b_bytes)};
+        for (const Range &r : ins)
+            if (overlaps(ro, r)) return fail(GDN_ERR_INVALID_ARG, "out overlaps an input");
+        if (initial_state && overlaps(ro, range_of(initial_state, st_bytes)))
+            return fail(GDN_ERR_INVALID_ARG, "out overlaps initial_state");
+        if (final_state && overlaps(ro, range_of(final_state, st_bytes)))
+            return fail(GDN_ERR_INVALID_ARG, "out overlaps final_state");
+    }
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)) ||
+        (snapshots && !aligned16(snapshots)))
+        return fail(GDN_ERR_INVALID_ARG, "state pointers must be 16-byte aligned");
+    if (final_state && initial_state && final_state != initial_state &&
+        overlaps(range_of(final_state, st_bytes), range_of(initial_state, st_bytes)))
+        return fail(GDN_ERR_INVALID_ARG, "final_state partially overlaps initial_state");
+    if (n_snap > 0 && !snapshots) return fail(GDN_ERR_INVALID_ARG, "snapshots buffer is required");
+    if (n_snap > 0 && final_state && overlaps(range_of(snapshots, snap_bytes), range_of(final_state, st_bytes)))
+        return fail(GDN_ERR_INVALID_ARG, "snapshots overlap final_state");
+
+    ChunkPlan p = make_plan(*d, N, packed);
+    if (N == 0) return GDN_OK;
+    if (!workspace) return fail(GDN_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", p.total);
+    if (((uintptr_t)workspace & 255u) != 0) return fail(GDN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (workspace_bytes < p.total)
+        return fail(GDN_ERR_WORKSPACE, "workspace has %zu bytes, need %zu", workspace_bytes, p.total);
+
+    ChunkArgs a{};
+    a.q = q; a.k = k; a.v = v; a.g = log_gate; a.beta = beta; a.h0 = initial_state;
+    a.cu_seqlens = cu_seqlens;
+    a.T = d->T;
+    a.N = N;
+    a.H = d->H;
+    a.scale = d->scale;
+    a.snapshot_stride = snapshot_stride;
+    a.n_snap = n_snap;
+    a.out = out;
+    a.final_state = final_state;
+    a.snapshots = snapshots;
+    a.ws = (char *)workspace;
+    return launch_chunk_simt(p, a, d->dtype, (cudaStream_t)stream);
+}
+
+gdn_status gdn_decode_step(const gdn_desc *d, const void *q, const void *k, const void *v,
+                           const float *log_gate, const float *beta, float *state, void *out,
+                           gdn_stream_t stream) {
+    g_last_error[0] = 0;
+    gdn_status st = check_desc(d);
+    if (st != GDN_OK) return st;
+    if (d->T != 1) return fail(GDN_ERR_INVALID_ARG, "decode needs T == 1 (got %lld)", (long long)d->T);
+    if (d->B == 0) return GDN_OK;
+    if (!q || !k || !v || !log_gate || !beta || !state || !out)
+        return fail(GDN_ERR_INVALID_ARG, "all decode pointers are required");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out))
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v, state and out must be 16-byte aligned");
+    if (!aligned4(log_gate) || !aligned4(beta))
+        return fail(GDN_ERR_INVALID_ARG, "log_gate and beta must be 4-byte aligned");
+    const size_t in_el = d->dtype == GDN_F32 ? 4 : 2;
+    const Range ro = range_of(out, (size_t)d->B * d->H * d->dv * in_el);
+    const Range rs = range_of(state, (size_t)d->B * d->H * d->dv * d->dk * 4);
+    const Range ins[] = {range_of(q, (size_t)d->B * d->H * d->dk * in_el),
+                         range_of(k, (size_t)d->B * d->H * d->dk * in_el),
+                         range_of(v, (size_t)d->B * d->H * d->dv * in_el),
+                         range_of(log_gate, (size_t)d->B * d->H * (d->gate == GDN_GATE_CHANNEL ? d->dk : 1) * 4),
+                         range_of(beta, (size_t)d->B * d->H * 4)};
+    if (overlaps(ro, rs)) return fail(GDN_ERR_INVALID_ARG, "out overlaps state");
+    for (const Range &r : ins)
+        if (overlaps(ro, r) || overlaps(rs, r)) return fail(GDN_ERR_INVALID_ARG, "out or state overlaps an input");
+    return launch_decode(*d, q, k, v, log_gate, beta, state, out, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,80 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+constexpr int kChunk = 64;  // tokens per chunk of the chunkwise form
+
+// Where a kernel launch came from, for the optional event timer.
+struct LaunchScope {
+    LaunchScope(const char *name, cudaStream_t s);
+    ~LaunchScope();
+    const char *name_;
+    cudaStream_t stream_;
+    int slot_;
+};
+
+// Records a failure reason for gdn_last_error() and returns `st`.
+gdn_status fail(gdn_status st, const char *fmt, ...);
+
+// Map the result of a launch to a status.
+gdn_status check_launch(const char *what);
+
+// ---------------------------------------------------------------------------
+// Workspace of the chunked forward pass.
+// ---------------------------------------------------------------------------
+struct ChunkPlan {
+    int64_t N;           // sequences
+    int64_t rows;        // B*T packed token rows
+    int64_t H, dk, dv;
+    int64_t max_chunks;  // upper bound on sum_n ceil(len_n / 64)
+    bool packed;
+    bool per_channel;
+    // byte offsets into the workspace
+    size_t off_chunk_offsets;  // int32 (N+1): first global chunk index of each sequence
+    size_t off_W, off_U, off_P, off_b;
+    size_t total;
+};
+
+ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed);
+
+struct ChunkArgs {
+    const void *q, *k, *v;
+    const float *g, *beta, *h0;
+    const int32_t *cu_seqlens;  // nullptr: fixed-length sequences of length T
+    int64_t T;                  // per-sequence length when not packed
+    int64_t N, H;
+    float scale;
+    int64_t snapshot_stride;
+    int64_t n_snap;             // snapshots per sequence (fixed-length only)
+    void *out;
+    float *final_state, *snapshots;
+    char *ws;
+};
+
+gdn_status launch_chunk_simt(const ChunkPlan &p, const ChunkArgs &a, int dtype, cudaStream_t s);
+gdn_status launch_decode(const gdn_desc &d, const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, float *state, void *out,
+                         cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+}  // namespace gdn

@@ -1,0 +1,198 @@
+/*
+ * gdn.h -- C ABI of the gated delta rule for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  Per sequence and head, a d_v x d_k state S evolves token by
+ * token as
+ *
+ *     S_t = S_{t-1} D_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t (scale q_t)
+ *
+ * with D_t = alpha_t I (one gate per head: Gated DeltaNet) or
+ * D_t = Diag(alpha_t), alpha_t in (0,1]^{d_k} (one gate per key channel: the
+ * KDA variant).  Decay comes first, the delta correction is applied to the
+ * decayed state, and the output reads the state after the write.
+ *   - "Hybrid models: what Gated DeltaNet replaces in the KV cache", section
+ *     "Gated DeltaNet: add decay" (the update and the d_v x d_k state);
+ *   - "From Traditional Attention to hybrid ones", section 5 (decay, then the
+ *     delta update on the decayed state, then o_t = S_t q_t) and section 7
+ *     (the per-channel form S_{t-1} Diag(alpha_t)(I - beta_t k_t k_t^T) + ...);
+ *   - "Attention, Part 4: Linear Attention, Gated DeltaNet and Hybrid Models",
+ *     "Where alpha and beta come from" (the gate arrives as g = log alpha).
+ *
+ * Conventions shared by every entry point.
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates device memory; scratch memory comes only from
+ *     the caller's workspace.
+ *   - Layouts are dense row-major (C order), no strides:
+ *       q, k      (B, T, H, d_k)      dtype per gdn_desc.dtype
+ *       v, out    (B, T, H, d_v)      dtype per gdn_desc.dtype
+ *       log_gate  (B, T, H) fp32      one gate per head, or
+ *                 (B, T, H, d_k) fp32 one gate per key channel
+ *       beta      (B, T, H) fp32
+ *       states    (N, H, d_v, d_k) fp32, N = number of sequences
+ *     log_gate holds g = log(alpha): finite and <= 0 (alpha = 1 is allowed).
+ *     beta is used as given (the pages keep it in (0,1); 0 and 1 work).
+ *   - q, k, v, out and states must be 16-byte aligned, the workspace 256-byte;
+ *     log_gate, beta and cu_seqlens 4-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are detected on the host before
+ *     anything is launched and leave all outputs untouched.  A failed launch
+ *     returns GDN_ERR_CUDA.  gdn_last_error() gives a one-line reason for the
+ *     most recent failure on the calling thread.
+ *   - Supported sizes: d_k, d_v in {64, 128}.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *gdn_stream_t; /* same type as cudaStream_t */
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1, /* a size, pointer, alignment or flag is wrong      */
+    GDN_ERR_UNSUPPORTED = 2, /* valid request this build does not implement      */
+    GDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required       */
+    GDN_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed             */
+    GDN_ERR_TIMEOUT = 5,     /* reserved: a bounded device-side wait ran out     */
+    GDN_ERR_INTERNAL = 6     /* a device-side consistency check failed           */
+} gdn_status;
+
+typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+typedef enum gdn_gate_kind {
+    GDN_GATE_HEAD = 0,   /* alpha_t is one scalar per head and token (Gated DeltaNet) */
+    GDN_GATE_CHANNEL = 1 /* alpha_t is a d_k vector per head and token (KDA)          */
+} gdn_gate_kind;
+
+/* Problem description.  For packed sequences B = 1 and T is the total number
+ * of packed tokens.  For gdn_decode_step T = 1 and B is the number of live
+ * sequences. */
+typedef struct gdn_desc {
+    int64_t B, T, H, dk, dv;
+    int32_t dtype; /* gdn_dtype of q, k, v and out (gates, beta, states: fp32)  */
+    int32_t gate;  /* gdn_gate_kind                                              */
+    float scale;   /* multiplies q before the read; 1.0 gives o_t = S_t q_t      */
+    int32_t reserved; /* must be 0                                                */
+} gdn_desc;
+
+/* ---------------------------------------------------------------------------
+ * gdn_chunk_workspace_size -- bytes of device workspace gdn_chunk_fwd needs.
+ *
+ * num_seqs: number of sequences (B when cu_seqlens is NULL).  The bound
+ * covers any packing of d->T tokens into num_seqs sequences.
+ * Returns GDN_ERR_INVALID_ARG for a bad descriptor or a NULL `bytes`.
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_chunk_workspace_size(const gdn_desc *d, int32_t num_seqs, size_t *bytes);
+
+/* ---------------------------------------------------------------------------
+ * gdn_chunk_fwd -- chunkwise-parallel prefill.
+ *
+ * Computes the outputs o_t of every token and the state after each sequence,
+ * exactly as the token-by-token recurrence above (up to rounding), by the
+ * chunkwise form: within a chunk of 64 tokens the writes are coupled only
+ * through a small lower-triangular system, solved with matrix products; only
+ * the d_v x d_k state passes from one chunk to the next.
+ *   - "Hybrid attention: why new LLMs keep full attention in only a few
+ *     layers", section "Training a recurrence in parallel";
+ *   - "Hybrid Linear Attention Architecture Design Explained", section 4
+ *     (state update S[t+1] and output O[t] per chunk, cumulative decay in the
+ *     log domain);
+ *   - "Hybrid models ...", section "What a recurrent state changes for
+ *     serving", item 1 (snapshots of the state at chosen positions).
+ *
+ * Arguments
+ *   d              problem description (d->T >= 0; T = 0 is a no-op apart from
+ *                  copying initial states to final states)
+ *   q, k, v        inputs, layouts above
+ *   log_gate, beta gates, layouts above (log_gate per channel iff
+ *                  d->gate == GDN_GATE_CHANNEL)
+ *   initial_state  (N, H, d_v, d_k) fp32, or NULL for zero states
+ *   cu_seqlens     NULL: N = B sequences of T tokens each.  Otherwise a device
+ *                  array of num_seqs+1 non-decreasing int32 offsets into the
+ *                  B*T token rows with cu_seqlens[0] = 0 and
+ *                  cu_seqlens[num_seqs] = T (B must be 1).  Chunks restart at
+ *                  every sequence start.  The offsets are read on the device
+ *                  and are not validated there: wrong offsets give wrong
+ *                  results, but every access stays inside the B*T rows.
+ *   num_seqs       number of sequences when cu_seqlens != NULL (else ignored)
+ *   snapshot_stride 0 for none, else a positive multiple of 64: the state
+ *                  after the first n*stride tokens of each sequence,
+ *                  n = 1 .. floor(T/stride), is written to `snapshots`.
+ *                  Only without cu_seqlens (GDN_ERR_UNSUPPORTED otherwise).
+ *   out            (B, T, H, d_v), must not overlap any input
+ *   final_state    (N, H, d_v, d_k) fp32 or NULL; may be the same pointer as
+ *                  initial_state (read fully before it is written)
+ *   snapshots      (B, floor(T/stride), H, d_v, d_k) fp32, required iff
+ *                  snapshot_stride > 0
+ *   workspace      device scratch of at least gdn_chunk_workspace_size bytes,
+ *                  256-byte aligned; contents on entry do not matter and are
+ *                  clobbered.  Two calls in flight at once need two workspaces.
+ *   stream         CUDA stream
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_chunk_fwd(const gdn_desc *d,
+                         const void *q, const void *k, const void *v,
+                         const float *log_gate, const float *beta,
+                         const float *initial_state,
+                         const int32_t *cu_seqlens, int32_t num_seqs,
+                         int64_t snapshot_stride,
+                         void *out, float *final_state, float *snapshots,
+                         void *workspace, size_t workspace_bytes,
+                         gdn_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * gdn_decode_step -- one token of every live sequence, state updated in place.
+ *
+ * For each of the d->B sequences and d->H heads (d->T must be 1):
+ *     y = S D k,  z = S D (scale q)           (one read of S)
+ *     delta = beta (v - y)
+ *     S'  = S D + delta k^T                   (written over S)
+ *     o   = z + delta (k . scale q)  ( = S' scale q )
+ * with D = alpha I or Diag(alpha), alpha = exp(log_gate).
+ *   - "From Traditional Attention to hybrid ones", section 5 (the update on the
+ *     decayed state and the read o_t = S_t q_t) and "vLLM Storage" (the
+ *     recurrent state is fixed per live sequence and updated in place);
+ *   - "Attention, Part 4 ...", section 8 (one decode step updates the
+ *     32 x 128 x 128 memory once per token).
+ *
+ *   q, k (B, 1, H, d_k); v, out (B, 1, H, d_v); log_gate (B, 1, H) or
+ *   (B, 1, H, d_k); beta (B, 1, H); state (B, H, d_v, d_k) fp32, read and
+ *   overwritten.  `out` must not overlap the state or the inputs.
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_decode_step(const gdn_desc *d,
+                           const void *q, const void *k, const void *v,
+                           const float *log_gate, const float *beta,
+                           float *state, void *out, gdn_stream_t stream);
+
+/* Static description of a status code. */
+const char *gdn_status_string(gdn_status s);
+
+/* One-line reason for the most recent failed call on this thread ("" if none). */
+const char *gdn_last_error(void);
+
+/* ---------------------------------------------------------------------------
+ * Kernel timing.  While enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on the launch stream; gdn_profile_read
+ * waits for them and returns per kernel name the number of launches and the
+ * summed device time.  Events are created lazily (host resources only; no
+ * device memory is allocated).  Reading resets the counters.
+ * ------------------------------------------------------------------------- */
+typedef struct gdn_kernel_time {
+    const char *name;   /* static string, valid for the life of the library */
+    int64_t launches;
+    double total_ms;
+} gdn_kernel_time;
+
+gdn_status gdn_profile_enable(int on);
+/* Writes up to `cap` entries and stores the number of distinct kernels seen in
+ * *count (which may exceed cap). */
+gdn_status gdn_profile_read(gdn_kernel_time *entries, int32_t cap, int32_t *count);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_H_ */

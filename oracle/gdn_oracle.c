@@ -67,7 +67,7 @@ typedef struct {
     pthread_mutex_t lock;
 } oracle_job;
 
-static void run_unit(const oracle_job *J, int64_t unit, double *S, double *y)
+static void run_unit(const oracle_job *J, int64_t unit, double *S, double *y, double *al)
 {
     const int64_t H = J->H, dk = J->dk, dv = J->dv;
     const int64_t n = unit / H, h = unit % H;
@@ -88,9 +88,11 @@ static void run_unit(const oracle_job *J, int64_t unit, double *S, double *y)
         /* 1. forget */
         if (J->per_channel) {
             const double *gt = J->g + (row * H + h) * dk;
+            for (int64_t c = 0; c < dk; ++c)
+                al[c] = exp(gt[c]);
             for (int64_t i = 0; i < dv; ++i)
                 for (int64_t c = 0; c < dk; ++c)
-                    S[i * dk + c] *= exp(gt[c]);
+                    S[i * dk + c] *= al[c];
         } else {
             const double a = exp(J->g[row * H + h]);
             for (int64_t i = 0; i < dv * dk; ++i)
@@ -137,19 +139,21 @@ static void *worker(void *arg)
     oracle_job *J = (oracle_job *)arg;
     double *S = (double *)malloc(sizeof(double) * J->dv * J->dk);
     double *y = (double *)malloc(sizeof(double) * J->dv);
+    double *al = (double *)malloc(sizeof(double) * J->dk);
     const int64_t units = J->n_seqs * J->H;
-    if (S && y) {
+    if (S && y && al) {
         for (;;) {
             pthread_mutex_lock(&J->lock);
             const int64_t u = J->next_unit++;
             pthread_mutex_unlock(&J->lock);
             if (u >= units)
                 break;
-            run_unit(J, u, S, y);
+            run_unit(J, u, S, y, al);
         }
     }
     free(S);
     free(y);
+    free(al);
     return NULL;
 }
 

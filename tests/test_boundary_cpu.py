@@ -1,0 +1,186 @@
+"""The C-ABI library on the host: it loads, exports every declared entry point,
+and rejects bad arguments before launching anything (no GPU needed: every case
+here fails validation, so no CUDA call is reached)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_64_b200 import gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_64_b200 import build
+    build.build()
+    return gdn.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(gdn.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_struct_layout_matches_header():
+    assert ctypes.sizeof(gdn.GdnDesc) == 56
+
+
+def _desc(B=2, T=130, H=3, dk=128, dv=128, dtype=gdn.GDN_BF16, gate=gdn.GDN_GATE_HEAD, scale=1.0):
+    return gdn.GdnDesc(B, T, H, dk, dv, dtype, gate, scale, 0)
+
+
+A = 1 << 40  # fake, 256-byte aligned "device" addresses; never dereferenced
+
+
+def _addr(i, off=0):
+    return ctypes.c_void_p(A + i * (1 << 32) + off)
+
+
+def _fwd(lib, d, *, q=0, k=1, v=2, g=3, beta=4, h0=None, cu=None, n=0, snap=0, out=5, fin=None, snaps=None,
+         ws=7, ws_bytes=1 << 40, off=None):
+    off = off or {}
+    p = lambda i, name: None if i is None else _addr(i, off.get(name, 0))
+    return lib.gdn_chunk_fwd(ctypes.byref(d), p(q, "q"), p(k, "k"), p(v, "v"), p(g, "g"), p(beta, "beta"),
+                             p(h0, "h0"), p(cu, "cu"), n, snap, p(out, "out"), p(fin, "fin"), p(snaps, "snaps"),
+                             p(ws, "ws"), ws_bytes, None)
+
+
+def test_workspace_size(lib):
+    n = ctypes.c_size_t()
+    d = _desc()
+    assert lib.gdn_chunk_workspace_size(ctypes.byref(d), 2, ctypes.byref(n)) == gdn.GDN_OK
+    # 2 sequences of 130 tokens: at most 260/64 + 2 = 6 chunks x 3 heads
+    per_chunk_head = 4 * 64 * (128 + 128 + 64 + 1)
+    assert n.value >= 6 * 3 * per_chunk_head
+    assert n.value < 6 * 3 * per_chunk_head + 4096
+    d2 = _desc(gate=gdn.GDN_GATE_CHANNEL)
+    n2 = ctypes.c_size_t()
+    assert lib.gdn_chunk_workspace_size(ctypes.byref(d2), 2, ctypes.byref(n2)) == gdn.GDN_OK
+    assert n2.value > n.value
+    assert lib.gdn_chunk_workspace_size(ctypes.byref(d), 2, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("dk", 96, gdn.GDN_ERR_UNSUPPORTED),
+    ("dv", 32, gdn.GDN_ERR_UNSUPPORTED),
+    ("H", 0, gdn.GDN_ERR_INVALID_ARG),
+    ("T", -1, gdn.GDN_ERR_INVALID_ARG),
+    ("dtype", 7, gdn.GDN_ERR_INVALID_ARG),
+    ("gate", 3, gdn.GDN_ERR_INVALID_ARG),
+    ("reserved", 1, gdn.GDN_ERR_INVALID_ARG),
+    ("scale", float("nan"), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_bad_descriptor(lib, field, value, status):
+    d = _desc()
+    setattr(d, field, value)
+    assert _fwd(lib, d) == status
+    assert lib.gdn_last_error().decode()
+
+
+def test_null_descriptor(lib):
+    assert lib.gdn_chunk_fwd(None, *([None] * 7), 0, 0, None, None, None, None, 0, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,off", [("q", 8), ("k", 8), ("v", 8), ("out", 8), ("g", 2), ("beta", 1),
+                                      ("h0", 8)])
+def test_misaligned_pointer(lib, name, off):
+    kw = {"h0": 10} if name == "h0" else {}
+    assert _fwd(lib, _desc(), off={name: off}, **kw) == gdn.GDN_ERR_INVALID_ARG
+    assert "aligned" in lib.gdn_last_error().decode()
+
+
+def test_gates_need_only_4_byte_alignment(lib):
+    # passes validation (so it reaches the launch, which fails without a GPU)
+    st = _fwd(lib, _desc(), off={"g": 4, "beta": 8})
+    assert st in (gdn.GDN_OK, gdn.GDN_ERR_CUDA), st
+
+
+@pytest.mark.parametrize("name", ["q", "k", "v", "g", "beta", "out"])
+def test_null_required_pointer(lib, name):
+    kw = {name: None}
+    assert _fwd(lib, _desc(), **kw) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_out_overlapping_input(lib):
+    # out starts inside v
+    assert _fwd(lib, _desc(), out=2, off={"out": 256}) == gdn.GDN_ERR_INVALID_ARG
+    assert "overlap" in lib.gdn_last_error().decode()
+
+
+def test_workspace_checks(lib):
+    assert _fwd(lib, _desc(), ws=None) == gdn.GDN_ERR_WORKSPACE
+    assert _fwd(lib, _desc(), ws_bytes=1024) == gdn.GDN_ERR_WORKSPACE
+    assert _fwd(lib, _desc(), off={"ws": 16}) == gdn.GDN_ERR_WORKSPACE
+
+
+def test_snapshot_rules(lib):
+    d = _desc(T=512)
+    assert _fwd(lib, d, snap=100, snaps=8) == gdn.GDN_ERR_INVALID_ARG        # not a multiple of 64
+    assert _fwd(lib, d, snap=-64, snaps=8) == gdn.GDN_ERR_INVALID_ARG
+    assert _fwd(lib, d, snap=128, snaps=None) == gdn.GDN_ERR_INVALID_ARG     # buffer required
+    dp = _desc(B=1, T=512)
+    assert _fwd(lib, dp, cu=9, n=3, snap=128, snaps=8) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_packed_rules(lib):
+    assert _fwd(lib, _desc(B=2), cu=9, n=2) == gdn.GDN_ERR_INVALID_ARG       # packing needs B == 1
+    assert _fwd(lib, _desc(B=1), cu=9, n=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert _fwd(lib, _desc(B=1), cu=9, n=2, off={"cu": 2}) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_final_state_partial_overlap(lib):
+    assert _fwd(lib, _desc(), h0=10, fin=10, off={"fin": 256}) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_decode_validation(lib):
+    # argument order: q, k, v, log_gate, beta, state, out
+    d = _desc(B=4, T=2)
+    p = [_addr(i) for i in range(7)]
+    assert lib.gdn_decode_step(ctypes.byref(d), *p, None) == gdn.GDN_ERR_INVALID_ARG   # T must be 1
+    d = _desc(B=4, T=1)
+    q = list(p)
+    q[5] = None  # state
+    assert lib.gdn_decode_step(ctypes.byref(d), *q, None) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[6] = _addr(5, 64)  # out inside the state
+    assert lib.gdn_decode_step(ctypes.byref(d), *q, None) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[5] = _addr(0, 256)  # state overlapping q
+    assert lib.gdn_decode_step(ctypes.byref(d), *q, None) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[0] = _addr(0, 4)  # misaligned q
+    assert lib.gdn_decode_step(ctypes.byref(d), *q, None) == gdn.GDN_ERR_INVALID_ARG
+    d = _desc(B=4, T=1, dk=32)
+    assert lib.gdn_decode_step(ctypes.byref(d), *p, None) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.gdn_status_string(s)
+    assert lib.gdn_status_string(99) == b"unknown status"
+
+
+def test_profile_api_without_launches(lib):
+    assert lib.gdn_profile_enable(1) == gdn.GDN_OK
+    cnt = ctypes.c_int32(-1)
+    assert lib.gdn_profile_read(None, 0, ctypes.byref(cnt)) == gdn.GDN_OK
+    assert cnt.value == 0
+    assert lib.gdn_profile_enable(0) == gdn.GDN_OK
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 64, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        gdn.gdn_chunk_fwd(x, x, x, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1))

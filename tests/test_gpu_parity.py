@@ -1,0 +1,217 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, on the
+same seeded inputs, element by element (relative L2 over whole tensors).
+
+Tolerances: 1e-4 for fp32 inputs; 2e-2 on outputs and 1e-2 on states and
+snapshots for bf16 inputs with an fp32 state."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_64_b200 import gdn
+from gated_delta_rule_64_b200.inputs import (DECODE, KDA_PACKED, LONG_SNAPSHOTS, PREFILL_BF16, TINY_F32,
+                                             Workload, make_inputs)
+from tests.gpu_util import check, rel_l2, run_gpu, run_oracle, to_dev, tolerances
+
+pytestmark = pytest.mark.gpu
+
+def fresh(t):
+    """A freshly allocated contiguous copy (slices of packed tensors are views whose
+    start need not be 16-byte aligned, which the library requires)."""
+    return torch.empty_like(t, memory_format=torch.contiguous_format).copy_(t)
+
+
+SMALL = Workload("small", B=2, T=300, H=3, dk=128, dv=128, dtype="bf16", h0_std=0.1, seed=11)
+
+
+def test_tiny_f32_workload():
+    check(make_inputs(TINY_F32))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("per_channel", [False, True])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
+def test_shapes(dtype, per_channel, dk, dv):
+    check(make_inputs(SMALL.replace(dtype=dtype, per_channel=per_channel, dk=dk, dv=dv)))
+
+
+@pytest.mark.parametrize("T", [1, 5, 63, 64, 65, 128, 129])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_lengths_around_the_chunk(T, dtype):
+    check(make_inputs(SMALL.replace(T=T, dtype=dtype, seed=T)))
+
+
+def test_zero_length_copies_initial_state():
+    x = make_inputs(SMALL.replace(T=0, dtype="f32"))
+    dx = to_dev(x)
+    out, fin, _ = gdn.gdn_chunk_fwd(dx.q, dx.k, dx.v, dx.g, dx.beta, dx.h0)
+    torch.cuda.synchronize()
+    assert torch.equal(fin.cpu(), x.h0)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_packed_sequences(dtype, per_channel):
+    lengths = [1, 63, 64, 65, 130, 0, 7, 200]
+    w = SMALL.replace(dtype=dtype, per_channel=per_channel, seed=5)
+    check(make_inputs(w, lengths=lengths))
+
+
+def test_packed_equals_separate_runs():
+    lengths = [70, 129, 3]
+    x = make_inputs(SMALL.replace(seed=6), lengths=lengths)
+    out, fin, _ = run_gpu(x)
+    cu = x.cu_seqlens.tolist()
+    for n in range(len(lengths)):
+        a, b = cu[n], cu[n + 1]
+        dx = to_dev(x)
+        o1, f1, _ = gdn.gdn_chunk_fwd(fresh(dx.q[:, a:b]), fresh(dx.k[:, a:b]), fresh(dx.v[:, a:b]),
+                                      fresh(dx.g[:, a:b]), fresh(dx.beta[:, a:b]),
+                                      fresh(dx.h0[n:n + 1]))
+        assert rel_l2(o1, out[:, a:b].cpu().double().numpy()) < 1e-6
+        assert rel_l2(f1, fin[n:n + 1].cpu().double().numpy()) < 1e-6
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_snapshots(dtype):
+    x = make_inputs(SMALL.replace(T=640, dtype=dtype, seed=7))
+    check(x, snapshot_stride=128)
+
+
+def test_snapshot_resume_equals_full_run():
+    x = make_inputs(SMALL.replace(T=512, dtype="f32", seed=8))
+    dx = to_dev(x)
+    out, fin, snaps = gdn.gdn_chunk_fwd(dx.q, dx.k, dx.v, dx.g, dx.beta, dx.h0, snapshot_stride=192)
+    n = 192
+    o2, f2, _ = gdn.gdn_chunk_fwd(fresh(dx.q[:, n:]), fresh(dx.k[:, n:]), fresh(dx.v[:, n:]),
+                                  fresh(dx.g[:, n:]), fresh(dx.beta[:, n:]), fresh(snaps[:, 0]))
+    assert rel_l2(o2, out[:, n:].cpu().double().numpy()) < 1e-5
+    assert rel_l2(f2, fin.cpu().double().numpy()) < 1e-5
+
+
+def test_final_state_may_alias_initial_state():
+    x = make_inputs(SMALL.replace(dtype="f32", seed=9))
+    o_ref, f_ref, _ = run_oracle(x)
+    dx = to_dev(x)
+    st = dx.h0.clone()
+    out, fin, _ = gdn.gdn_chunk_fwd(dx.q, dx.k, dx.v, dx.g, dx.beta, st, final_state=st)
+    torch.cuda.synchronize()
+    assert fin.data_ptr() == st.data_ptr()
+    assert rel_l2(st, f_ref) <= 1e-4 and rel_l2(out, o_ref) <= 1e-4
+
+
+def test_query_scale():
+    check(make_inputs(SMALL.replace(seed=10)), scale=0.125)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_long_memory_gates(dtype, per_channel):
+    """alpha ~ 0.999 and weak writes: the state and the initial state carry
+    across many chunks."""
+    w = SMALL.replace(T=2048, H=2, dtype=dtype, per_channel=per_channel, gate_mu=-7.0, beta_mu=-4.0, h0_std=0.3,
+                      seed=12)
+    check(make_inputs(w))
+
+
+def _with_gates(x, g):
+    x.g = g
+    return x
+
+
+def test_extreme_gates_scalar():
+    """alpha = 1 (g = 0) with full-strength writes, and g = -80 on some tokens."""
+    x = make_inputs(SMALL.replace(dtype="f32", seed=13))
+    g = torch.zeros_like(x.g)
+    g[:, 100:110] = -80.0
+    x.beta = torch.ones_like(x.beta)
+    check(_with_gates(x, g))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_extreme_gates_per_channel(dtype):
+    """Per-channel gates mixing 0 and -80, with in-chunk gate sums far below the
+    fp32 exponent range: nothing may overflow."""
+    x = make_inputs(SMALL.replace(dtype=dtype, per_channel=True, seed=14))
+    g = torch.zeros_like(x.g)
+    g[..., ::3] = -80.0
+    g[:, 50:60, :, 1::3] = -5.0
+    check(_with_gates(x, g))
+
+
+# ---------------------------------------------------------------------------
+# Decode
+# ---------------------------------------------------------------------------
+
+def _decode_oracle(x):
+    """Steps as a sequence per (b, h): (steps, B, 1, H, .) -> (B, steps, H, .)."""
+    seq = lambda t: t[:, :, 0].transpose(0, 1)
+    return oracle.gated_delta_rule(seq(x.q), seq(x.k), seq(x.v), seq(x.g), seq(x.beta), x.h0)
+
+
+def _decode_gpu(x):
+    dx = to_dev(x)
+    state = dx.h0.clone()
+    outs = [gdn.gdn_decode_step(dx.q[s], dx.k[s], dx.v[s], dx.g[s], dx.beta[s], state) for s in range(x.q.shape[0])]
+    # (per-step slices of the gates start on 4-byte boundaries only, which the library accepts)
+    torch.cuda.synchronize()
+    return torch.stack([o[:, 0] for o in outs], 1), state
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("per_channel", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_steps(dtype, per_channel, d):
+    w = DECODE.replace(B=6, H=3, dk=d, dv=d, decode_steps=20, dtype=dtype, per_channel=per_channel, seed=20)
+    x = make_inputs(w)
+    o, s = _decode_gpu(x)
+    o_ref, s_ref, _ = _decode_oracle(x)
+    tol_o, tol_s = tolerances(x.q.dtype)
+    assert rel_l2(o, o_ref) <= tol_o and rel_l2(s, s_ref) <= tol_s
+
+
+def test_decode_continues_prefill():
+    """Prefill of T tokens then decode of more equals prefill of all of them."""
+    w = SMALL.replace(T=200, dtype="f32", seed=21)
+    x = make_inputs(w)
+    dx = to_dev(x)
+    P = 150
+    _, st, _ = gdn.gdn_chunk_fwd(fresh(dx.q[:, :P]), fresh(dx.k[:, :P]), fresh(dx.v[:, :P]),
+                                 fresh(dx.g[:, :P]), fresh(dx.beta[:, :P]), dx.h0)
+    outs = []
+    for t in range(P, 200):
+        outs.append(gdn.gdn_decode_step(fresh(dx.q[:, t:t + 1]), fresh(dx.k[:, t:t + 1]),
+                                        fresh(dx.v[:, t:t + 1]), fresh(dx.g[:, t:t + 1]),
+                                        fresh(dx.beta[:, t:t + 1]), st)[:, 0])
+    out_all, fin_all, _ = gdn.gdn_chunk_fwd(dx.q, dx.k, dx.v, dx.g, dx.beta, dx.h0)
+    torch.cuda.synchronize()
+    assert rel_l2(torch.stack(outs, 1), out_all[:, P:].cpu().double().numpy()) < 1e-4
+    assert rel_l2(st, fin_all.cpu().double().numpy()) < 1e-4
+
+
+# ---------------------------------------------------------------------------
+# The benchmark workloads at full size (oracle on sampled heads / sequences)
+# ---------------------------------------------------------------------------
+
+def test_prefill_workload_full_size():
+    check(make_inputs(PREFILL_BF16), heads=[0, 9])
+
+
+def test_long_snapshot_workload_full_size():
+    x = make_inputs(LONG_SNAPSHOTS)
+    check(x, snapshot_stride=LONG_SNAPSHOTS.snapshot_stride, heads=[5])
+
+
+def test_kda_packed_workload_full_size():
+    check(make_inputs(KDA_PACKED), heads=[17])
+
+
+def test_decode_workload_full_size():
+    x = make_inputs(DECODE)
+    o, s = _decode_gpu(x)
+    pick = [0, 77, 255]
+    sub = lambda t: t[:, pick]
+    from gated_delta_rule_64_b200.inputs import Inputs
+    xs = Inputs(q=sub(x.q), k=sub(x.k), v=sub(x.v), g=sub(x.g), beta=sub(x.beta), h0=x.h0[pick])
+    o_ref, s_ref, _ = _decode_oracle(xs)
+    assert rel_l2(o[pick], o_ref) <= 2e-2 and rel_l2(s[pick], s_ref) <= 1e-2

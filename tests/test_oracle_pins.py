@@ -33,7 +33,7 @@ MUTANTS = {
     "error sign": ("(vt[i] - y[i])", "(vt[i] + y[i])"),
     "no write strength": ("S[i * dk + c] += bt * e * kt[c];", "S[i * dk + c] += e * kt[c];"),
     "gate not exponentiated": ("const double a = exp(J->g[row * H + h]);", "const double a = 1.0 + J->g[row * H + h];"),
-    "channel gate on value rows": ("S[i * dk + c] *= exp(gt[c]);", "S[i * dk + c] *= exp(gt[i % dk]);"),
+    "channel gate on value rows": ("S[i * dk + c] *= al[c];", "S[i * dk + c] *= al[i % dk];"),
     "prediction uses the query": ("acc += S[i * dk + c] * kt[c];", "acc += S[i * dk + c] * qt[c];"),
     "read uses the key": ("acc += S[i * dk + c] * (J->scale * qt[c]);", "acc += S[i * dk + c] * (J->scale * kt[c]);"),
     "snapshot index off by one": ("(t + 1) / J->snapshot_stride - 1;", "(t + 1) / J->snapshot_stride;"),
