@@ -24,6 +24,7 @@
 // U) of every chunk in parallel and writes it to the workspace;
 // `gdn_scan_simt` walks the chunks of each sequence in order, carrying a
 // 32-row slice of the state in shared memory.
+#include "chunk_common.cuh"
 #include "gdn_internal.cuh"
 
 namespace gdn {
@@ -33,55 +34,6 @@ constexpr int C = kChunk;
 constexpr int kPrepThreads = 256;
 constexpr int kScanThreads = 128;
 constexpr int kScanRows = 32;  // rows of the state per scan block
-
-// Token range of the chunk `chunk` (global index), or false when the index is
-// past the last chunk.  Offsets from cu_seqlens are clamped into [0, rows].
-struct ChunkLoc {
-    int64_t n, c, start, len;  // sequence, chunk within it, first token row, tokens (<= 64)
-};
-
-__device__ __forceinline__ void seq_bounds(const int32_t *cu, int64_t n, int64_t T, int64_t rows,
-                                           int64_t &start, int64_t &len) {
-    if (cu) {
-        int64_t a = cu[n], b = cu[n + 1];
-        a = a < 0 ? 0 : (a > rows ? rows : a);
-        b = b < a ? a : (b > rows ? rows : b);
-        start = a;
-        len = b - a;
-    } else {
-        start = n * T;
-        len = T;
-    }
-}
-
-__device__ bool locate_chunk(int64_t chunk, const int32_t *cu, const int32_t *off, int64_t N, int64_t T,
-                             int64_t rows, ChunkLoc &loc) {
-    int64_t n, c;
-    if (cu) {
-        if (chunk >= off[N]) return false;
-        int64_t lo = 0, hi = N;  // find n with off[n] <= chunk < off[n+1]
-        while (hi - lo > 1) {
-            const int64_t mid = (lo + hi) / 2;
-            if (off[mid] <= chunk) lo = mid; else hi = mid;
-        }
-        n = lo;
-        c = chunk - off[n];
-    } else {
-        const int64_t cps = (T + C - 1) / C;
-        if (cps == 0) return false;
-        n = chunk / cps;
-        c = chunk % cps;
-        if (n >= N) return false;
-    }
-    int64_t start, len;
-    seq_bounds(cu, n, T, rows, start, len);
-    if (c * C >= len) return false;
-    loc.n = n;
-    loc.c = c;
-    loc.start = start + c * C;
-    loc.len = len - c * C < C ? len - c * C : C;
-    return true;
-}
 
 // Exclusive prefix sum of ceil(len_n / 64) over the packed sequences.
 __global__ void gdn_chunk_table(const int32_t *__restrict__ cu, int64_t N, int64_t rows, int32_t *__restrict__ off) {
@@ -379,12 +331,7 @@ gdn_status launch_typed(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s) 
     float *U = reinterpret_cast<float *>(a.ws + p.off_U);
     float *P = reinterpret_cast<float *>(a.ws + p.off_P);
     float *b = reinterpret_cast<float *>(a.ws + p.off_b);
-    if (a.cu_seqlens) {
-        LaunchScope ls("gdn_chunk_table", s);
-        gdn_chunk_table<<<1, 1024, 0, s>>>(a.cu_seqlens, a.N, p.rows,
-                                           reinterpret_cast<int32_t *>(a.ws + p.off_chunk_offsets));
-    }
-    gdn_status st = check_launch("gdn_chunk_table");
+    gdn_status st = launch_chunk_table(p, a, s);
     if (st != GDN_OK) return st;
     if (p.max_chunks > 0 && p.rows > 0) {
         const size_t smem = sizeof(PrepSmem<Tin, DK, DV, PC>);
@@ -428,6 +375,16 @@ gdn_status launch_dtype(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s) 
 }
 
 }  // namespace
+
+gdn_status launch_chunk_table(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s) {
+    if (!a.cu_seqlens) return GDN_OK;
+    {
+        LaunchScope ls("gdn_chunk_table", s);
+        gdn_chunk_table<<<1, 1024, 0, s>>>(a.cu_seqlens, a.N, p.rows,
+                                           reinterpret_cast<int32_t *>(a.ws + p.off_chunk_offsets));
+    }
+    return check_launch("gdn_chunk_table");
+}
 
 gdn_status launch_chunk_simt(const ChunkPlan &p, const ChunkArgs &a, int dtype, cudaStream_t s) {
     return dtype == GDN_BF16 ? launch_dtype<__nv_bfloat16>(p, a, s) : launch_dtype<float>(p, a, s);

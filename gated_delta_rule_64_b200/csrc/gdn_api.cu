@@ -98,18 +98,30 @@ ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed) {
     // Every sequence of length L has ceil(L/64) chunks; over any packing of
     // `rows` tokens into N sequences that is at most rows/64 + N.
     p.max_chunks = packed ? (p.rows / kChunk + p.N) : (d.B * ((d.T + kChunk - 1) / kChunk));
+    p.tc = tc_eligible(d) && p.rows < (1LL << 31);
     const int64_t ch = p.max_chunks * p.H;
     size_t off = 0;
     p.off_chunk_offsets = off;
     off = align_up(off + sizeof(int32_t) * (size_t)(p.N + 1), 256);
-    p.off_W = off;
-    off = align_up(off + sizeof(float) * (size_t)ch * kChunk * p.dk, 256);
-    p.off_U = off;
-    off = align_up(off + sizeof(float) * (size_t)ch * kChunk * p.dv, 256);
-    p.off_P = off;
-    off = align_up(off + sizeof(float) * (size_t)ch * kChunk * kChunk, 256);
-    p.off_b = off;
-    off = align_up(off + sizeof(float) * (size_t)ch * kChunk * (p.per_channel ? p.dk : 1), 256);
+    if (p.tc) {
+        p.off_W = off;
+        off = align_up(off + kTcWImg * (size_t)ch, 256);
+        p.off_P = off;
+        off = align_up(off + kTcPImg * (size_t)ch, 256);
+        p.off_U = off;
+        off = align_up(off + kTcUt * (size_t)ch, 256);
+        p.off_b = off;
+        off = align_up(off + kTcB * (size_t)ch, 256);
+    } else {
+        p.off_W = off;
+        off = align_up(off + sizeof(float) * (size_t)ch * kChunk * p.dk, 256);
+        p.off_U = off;
+        off = align_up(off + sizeof(float) * (size_t)ch * kChunk * p.dv, 256);
+        p.off_P = off;
+        off = align_up(off + sizeof(float) * (size_t)ch * kChunk * kChunk, 256);
+        p.off_b = off;
+        off = align_up(off + sizeof(float) * (size_t)ch * kChunk * (p.per_channel ? p.dk : 1), 256);
+    }
     p.total = off;
     return p;
 }
@@ -288,7 +300,7 @@ gdn_status gdn_chunk_fwd(const gdn_desc *d, const void *q, const void *k, const 
     a.final_state = final_state;
     a.snapshots = snapshots;
     a.ws = (char *)workspace;
-    return launch_chunk_simt(p, a, d->dtype, (cudaStream_t)stream);
+    return p.tc ? launch_chunk_tc(p, a, (cudaStream_t)stream) : launch_chunk_simt(p, a, d->dtype, (cudaStream_t)stream);
 }
 
 gdn_status gdn_decode_step(const gdn_desc *d, const void *q, const void *k, const void *v,

@@ -36,6 +36,7 @@ struct ChunkPlan {
     int64_t max_chunks;  // upper bound on sum_n ceil(len_n / 64)
     bool packed;
     bool per_channel;
+    bool tc;             // tensor-core path (bf16, d_k = d_v = 128, one gate per head)
     // byte offsets into the workspace
     size_t off_chunk_offsets;  // int32 (N+1): first global chunk index of each sequence
     size_t off_W, off_U, off_P, off_b;
@@ -43,6 +44,7 @@ struct ChunkPlan {
 };
 
 ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed);
+
 
 struct ChunkArgs {
     const void *q, *k, *v;
@@ -58,7 +60,14 @@ struct ChunkArgs {
     char *ws;
 };
 
+gdn_status launch_chunk_table(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s);
 gdn_status launch_chunk_simt(const ChunkPlan &p, const ChunkArgs &a, int dtype, cudaStream_t s);
+gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s);
+bool tc_eligible(const gdn_desc &d);
+
+// Per chunk-head workspace of the tensor-core path (bytes): the W^T operand
+// image, the P operand image, U^T (bf16) and the cumulative log gate.
+constexpr size_t kTcWImg = 128 * 128, kTcPImg = 64 * 128, kTcUt = 128 * 64 * 2, kTcB = 64 * 4;
 gdn_status launch_decode(const gdn_desc &d, const void *q, const void *k, const void *v,
                          const float *g, const float *beta, float *state, void *out,
                          cudaStream_t s);

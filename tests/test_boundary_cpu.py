@@ -57,17 +57,18 @@ def _fwd(lib, d, *, q=0, k=1, v=2, g=3, beta=4, h0=None, cu=None, n=0, snap=0, o
 
 
 def test_workspace_size(lib):
-    n = ctypes.c_size_t()
-    d = _desc()
-    assert lib.gdn_chunk_workspace_size(ctypes.byref(d), 2, ctypes.byref(n)) == gdn.GDN_OK
     # 2 sequences of 130 tokens: at most 260/64 + 2 = 6 chunks x 3 heads
-    per_chunk_head = 4 * 64 * (128 + 128 + 64 + 1)
-    assert n.value >= 6 * 3 * per_chunk_head
-    assert n.value < 6 * 3 * per_chunk_head + 4096
-    d2 = _desc(gate=gdn.GDN_GATE_CHANNEL)
-    n2 = ctypes.c_size_t()
-    assert lib.gdn_chunk_workspace_size(ctypes.byref(d2), 2, ctypes.byref(n2)) == gdn.GDN_OK
-    assert n2.value > n.value
+    def size(**kw):
+        n = ctypes.c_size_t()
+        d = _desc(**kw)
+        assert lib.gdn_chunk_workspace_size(ctypes.byref(d), 2, ctypes.byref(n)) == gdn.GDN_OK
+        return n.value
+    simt = 4 * 64 * (128 + 128 + 64 + 1)          # fp32 W, U, P and gate per chunk-head
+    assert 6 * 3 * simt <= size(dtype=gdn.GDN_F32) < 6 * 3 * simt + 4096
+    tc = 128 * 128 + 64 * 128 + 128 * 64 * 2 + 64 * 4  # bf16 operand images + U^T + gate
+    assert 6 * 3 * tc <= size() < 6 * 3 * tc + 4096
+    assert size(dtype=gdn.GDN_F32, gate=gdn.GDN_GATE_CHANNEL) > size(dtype=gdn.GDN_F32)
+    d = _desc()
     assert lib.gdn_chunk_workspace_size(ctypes.byref(d), 2, None) == gdn.GDN_ERR_INVALID_ARG
 
 
