@@ -24,8 +24,8 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUD
 GDN_F32, GDN_BF16 = 0, 1
 GDN_GATE_HEAD, GDN_GATE_CHANNEL = 0, 1
 
-EXPORTED = ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_decode_step", "gdn_status_string",
-            "gdn_last_error", "gdn_profile_enable", "gdn_profile_read")
+EXPORTED = ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
+            "gdn_status_string", "gdn_last_error", "gdn_profile_enable", "gdn_profile_read")
 
 
 class GdnDesc(ctypes.Structure):
@@ -62,6 +62,7 @@ def load_library(path: str = LIB_PATH):
         dp = ctypes.POINTER(GdnDesc)
         lib.gdn_chunk_workspace_size.argtypes = [dp, i32, ctypes.POINTER(sz)]
         lib.gdn_chunk_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp, sz, vp]
+        lib.gdn_chunk_fwd_static.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp]
         lib.gdn_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn_status_string.argtypes = [ctypes.c_int]
         lib.gdn_status_string.restype = ctypes.c_char_p
@@ -69,8 +70,8 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_last_error.restype = ctypes.c_char_p
         lib.gdn_profile_enable.argtypes = [ctypes.c_int]
         lib.gdn_profile_read.argtypes = [ctypes.POINTER(GdnKernelTime), i32, ctypes.POINTER(i32)]
-        for name in ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_decode_step", "gdn_profile_enable",
-                     "gdn_profile_read"):
+        for name in ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
+                     "gdn_profile_enable", "gdn_profile_read"):
             getattr(lib, name).restype = ctypes.c_int
         if path == LIB_PATH:
             _lib = lib
@@ -156,6 +157,36 @@ def gdn_chunk_fwd(q, k, v, log_gate, beta, initial_state=None, cu_seqlens=None, 
                            _ptr(initial_state), _ptr(cu_seqlens), int(N), int(snapshot_stride), _ptr(out),
                            _ptr(final_state), _ptr(snapshots), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(lib, st)
+    return out, final_state, snapshots
+
+
+def gdn_chunk_fwd_static(q, k, v, log_gate, beta, initial_state=None, cu_seqlens=None, *, scale=1.0,
+                         snapshot_stride=0, out=None, final_state=True, snapshots=None, stream=None):
+    """gdn_chunk_fwd for callers that cannot allocate device scratch: the library
+    uses its built-in 64 MiB scratch array instead of a workspace (requests
+    that need more are rejected).  This wrapper still allocates the outputs with
+    torch when they are not passed; a caller that cannot allocate passes them."""
+    lib = load_library()
+    _need_cuda(q, k, v, log_gate, beta, initial_state, cu_seqlens)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    per_channel = log_gate.dim() == 4
+    N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    if final_state is True:
+        final_state = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    elif final_state is False:
+        final_state = None
+    if snapshot_stride and snapshots is None:
+        snapshots = torch.empty((B, T // snapshot_stride, H, dv, dk), dtype=torch.float32, device=dev)
+    _need_cuda(out, final_state, snapshots)
+    d = make_desc(B, T, H, dk, dv, _dtype_code(q), per_channel, scale)
+    st = lib.gdn_chunk_fwd_static(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_gate), _ptr(beta),
+                                  _ptr(initial_state), _ptr(cu_seqlens), int(N), int(snapshot_stride), _ptr(out),
+                                  _ptr(final_state), _ptr(snapshots), _stream(stream))
     _check(lib, st)
     return out, final_state, snapshots
 

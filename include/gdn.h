@@ -145,6 +145,37 @@ gdn_status gdn_chunk_fwd(const gdn_desc *d,
                          gdn_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * gdn_chunk_fwd_static -- gdn_chunk_fwd without a caller-provided workspace.
+ *
+ * The source pages have no counterpart to this entry point; it exists for
+ * callers that cannot allocate device memory (a serving loop whose allocator
+ * owns a fixed, pre-partitioned budget, a real-time path that must not take
+ * the device synchronisation an allocation may cause, a plugin that is handed
+ * pointers but no allocator).  It computes exactly what gdn_chunk_fwd
+ * computes, with the same arguments minus `workspace`/`workspace_bytes`; its
+ * scratch is a 64 MiB array built into the library, which every GPU that
+ * loads the library holds until the process exits.
+ *
+ *   - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
+ *   - Requests whose scratch need (gdn_chunk_workspace_size) exceeds 64 MiB
+ *     return GDN_ERR_WORKSPACE before touching the device.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the array and it keeps the previous call's contents;
+ *     nothing needs to start at zero, but two calls that overlap on the GPU
+ *     (e.g. on unordered streams) race on it: serialise them.
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_chunk_fwd_static(const gdn_desc *d,
+                                const void *q, const void *k, const void *v,
+                                const float *log_gate, const float *beta,
+                                const float *initial_state,
+                                const int32_t *cu_seqlens, int32_t num_seqs,
+                                int64_t snapshot_stride,
+                                void *out, float *final_state, float *snapshots,
+                                gdn_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * gdn_decode_step -- one token of every live sequence, state updated in place.
  *
  * For each of the d->B sequences and d->H heads (d->T must be 1):
