@@ -20,24 +20,25 @@
 //
 // Two kernels:
 //   gdn_prep_tc  one CTA per (chunk, head), all chunks in parallel.  TMA loads
-//                K, Q, V; one MMA gives [K;Q] K^T (M = 128: the K rows give the
-//                Gram matrix, the Q rows give Q K^T); the unit-lower-triangular
-//                system is solved on CUDA cores in fp32; two MMAs give W^T and
-//                U^T.  W^T and P are written to the workspace as ready-made
-//                128-byte-swizzled shared-memory operand images, so the scan
-//                copies them with plain bulk copies.
+//                K, Q, V; one M = 128 MMA gives [K;Q] K^T (the K rows give the
+//                Gram matrix, the Q rows Q K^T); the unit-lower-triangular
+//                system is solved blockwise (16 x 16 diagonal blocks by forward
+//                substitution in fp32, off-diagonal blocks by tf32 warp MMAs);
+//                two MMAs give W^T and U^T.  The results are staged in shared
+//                memory as ready-made operand images and bulk-stored as one
+//                contiguous block per chunk-head.
 //   gdn_scan_tc  one CTA per (sequence, head).  The fp32 state lives in
-//                registers (thread v owns row v); per chunk it is rounded to a
-//                bf16 operand in shared memory and four MMAs (S0 W^T, S0 Q^T,
-//                U' P^T, U'_w K) with fp32 accumulators in TMEM produce U', O and
-//                the state increment.  The next chunk's operands are prefetched
-//                by TMA / bulk copies into a second stage while this one runs.
+//                registers (two threads per state row, 64 columns each); per
+//                chunk it is rounded to a bf16 operand in shared memory and four
+//                MMAs (S0 W^T, S0 Q^T, U' P^T, U'_w K) with fp32 accumulators in
+//                TMEM produce U', O and the state increment.  The next chunk's
+//                operands are prefetched (TMA + one bulk copy) into a second
+//                stage; full output tiles leave through a TMA store.
 //
-// All MMAs are M = 128 (the 128 rows of the state, or the 64 K rows stacked
-// on the 64 Q rows), so the accumulator rows map 1:1 onto TMEM lanes and
-// every thread reads exactly its own row.
+// All tcgen05 MMAs are M = 128 (the 128 rows of the state, or the 64 K rows
+// stacked on the 64 Q rows), so accumulator rows map 1:1 onto TMEM lanes and
+// every thread reads its own row.
 #include <cudaTypedefs.h>
-
 #include <string.h>
 
 #include <mutex>
@@ -53,11 +54,13 @@ using namespace sm100;
 
 constexpr int C = kChunk;  // 64
 constexpr int D = 128;     // d_k = d_v
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 
-// ---------------------------------------------------------------------------
-// Device error flag: set by a kernel whose bounded wait ran out.
-// ---------------------------------------------------------------------------
+// Offsets inside one workspace block (see kTcBlock).
+constexpr uint32_t kBlkW = 0, kBlkU = 16384, kBlkP = 32768, kBlkFac = 40960;
+// Gate factors: [0, 64) w_i = exp(b_L - b_i); [64, 128) scale * exp(b_i); [128] exp(b_L).
+constexpr int kFacW = 0, kFacSG = 64, kFacGL = 128;
+
 __device__ __forceinline__ void flag_error(int *err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
@@ -66,49 +69,102 @@ __device__ __forceinline__ uint8_t *align1024(unsigned char *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-__device__ __forceinline__ void st_global_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
+// fp32 64 x 64 matrix, rows of 256 bytes, 16-byte chunks rotated per row (conflict-free row/column access).
+__device__ __forceinline__ uint32_t f32_offset(int i, int j) {
+    return (uint32_t)i * 256u + (uint32_t)((((j >> 2) ^ (i & 15)) << 4) + (j & 3) * 4);
 }
 
 // ===========================================================================
-// Prep: chunk-local quantities
+// Prep
 // ===========================================================================
 // Shared memory (1024-aligned):
-//   KQ   [0, 32K)     K and Q tiles stacked as the M = 128 operand:
-//                     [c-block 0: K rows | Q rows][c-block 1: K rows | Q rows]
-//   V    [32K, 48K)   V tile [c-block 0][c-block 1]
-//   Tp   [48K, 56K)   T diag(beta gam)  (bf16, K-major rows i)
-//   Tpp  [56K, 64K)   T diag(beta)
-//   A (fp32 64 x 64) reuses the Q rows once the first MMA has consumed them:
-//     rows 0..31 in [8K, 16K), rows 32..63 in [24K, 32K).
-constexpr uint32_t kPrepSmem = 65536 + 1024;
+//   [0, 32K)    K and Q tiles stacked as the M = 128 operand of the first MMA:
+//               [c-block 0: K rows | Q rows][c-block 1: K rows | Q rows].
+//               After that MMA the Q rows hold A (fp32; rows 0-31 | 32-63),
+//               then T diag(beta gam) at [8K,16K) and T diag(beta) at [24K,32K)
+//               (bf16 operand images); after the last MMAs the whole range
+//               stages the W^T image [0,16K) and the U^T rows [16K,32K).
+//   [32K, 48K)  V tile
+//   [48K, 64K)  T (fp32)
+//   [64K, 68K)  per-warp 16 x 16 scratch of the blocked solve
+//   [68K, 76K)  P image (staged)
+//   [76K, +768) gate factors (staged)
+constexpr uint32_t kPrepTf = 49152, kPrepY = 65536, kPrepP = 69632, kPrepFac = 77824;
+constexpr uint32_t kPrepSmem = kPrepFac + 768 + 1024;
 
-__device__ __forceinline__ uint32_t a_offset(int i, int q4) {
-    // row i of A, 16-byte chunk q4 (floats 4*q4 .. 4*q4+3), chunks rotated per row
-    const uint32_t base = i < 32 ? 8192u : 24576u;
-    return base + (uint32_t)(i & 31) * 256u + (uint32_t)((q4 ^ (i & 15)) << 4);
+__device__ __forceinline__ uint32_t a_offset(int i, int j) {
+    // A (fp32) in the Q rows of the first operand: rows 0..31 at 8K, 32..63 at 24K
+    return (i < 32 ? 8192u : 24576u) + f32_offset(i & 31, j);
 }
 
-__global__ void __launch_bounds__(kThreads)
+// C (16x16) = sum over `nk` 16-wide K blocks of X_k (16x16) * Y_k (16x16); X and Y
+// are fp32 blocks in shared memory given by their (row, col) origins and an
+// offset function.  Warp-level m16n8k8 tf32 MMAs, fp32 accumulate.  The result
+// is returned in the MMA accumulator layout: c[nt][0..3] for the 8-column
+// tiles nt = 0, 1.
+template <typename OffX, typename OffY>
+__device__ __forceinline__ void warp_gemm16(const uint8_t *base, int nk, const int *xr, const int *xc, const int *yr,
+                                            const int *yc, OffX offx, OffY offy, float (&c)[2][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+    for (int kb = 0; kb < nk; ++kb) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const int k0 = ks * 8;
+            uint32_t a[4];
+            a[0] = to_tf32(*reinterpret_cast<const float *>(base + offx(xr[kb] + g, xc[kb] + k0 + t)));
+            a[1] = to_tf32(*reinterpret_cast<const float *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t)));
+            a[2] = to_tf32(*reinterpret_cast<const float *>(base + offx(xr[kb] + g, xc[kb] + k0 + t + 4)));
+            a[3] = to_tf32(*reinterpret_cast<const float *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t + 4)));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t b[2];
+                b[0] = to_tf32(*reinterpret_cast<const float *>(base + offy(yr[kb] + k0 + t, yc[kb] + nt * 8 + g)));
+                b[1] = to_tf32(*reinterpret_cast<const float *>(base + offy(yr[kb] + k0 + t + 4, yc[kb] + nt * 8 + g)));
+                mma_tf32_16x8x8(c[nt], a, b);
+            }
+        }
+    }
+}
+
+// Store a 16x16 accumulator (times `sign`) at (r0, c0) through the offset function.
+template <typename Off>
+__device__ __forceinline__ void warp_store16(uint8_t *base, int r0, int c0, const float (&c)[2][4], float sign, Off off) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int col = c0 + nt * 8 + 2 * t;
+        *reinterpret_cast<float *>(base + off(r0 + g, col)) = sign * c[nt][0];
+        *reinterpret_cast<float *>(base + off(r0 + g, col + 1)) = sign * c[nt][1];
+        *reinterpret_cast<float *>(base + off(r0 + g + 8, col)) = sign * c[nt][2];
+        *reinterpret_cast<float *>(base + off(r0 + g + 8, col + 1)) = sign * c[nt][3];
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
 gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
             const __grid_constant__ CUtensorMap mv, const float *__restrict__ g, const float *__restrict__ beta,
             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
-            int64_t H, float scale, uint8_t *__restrict__ Wimg, uint8_t *__restrict__ Pimg,
-            __nv_bfloat16 *__restrict__ Ut, float *__restrict__ bcum, int *err) {
+            int64_t H, float scale, uint8_t *__restrict__ blocks, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    uint8_t *KQ = sm, *Vt = sm + 32768, *Tp = sm + 49152, *Tpp = sm + 57344;
     __shared__ uint64_t bar_ld, bar_mma;
     __shared__ uint32_t tmem_base;
-    __shared__ float s_b[C], s_beta[C];
+    __shared__ float s_b[C], s_beta[C], s_bg[C];
 
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
     ChunkLoc loc;
     if (!locate_chunk(chunk, cu, off, N, T, rows, loc)) return;
     const int L = (int)loc.len;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qd = warp & 3, hf = warp >> 2;
     const int64_t ch = chunk * H + h;
     const int32_t tok0 = (int32_t)loc.start;
+    uint8_t *blk = blocks + (size_t)ch * kTcBlock;
+    float *fac = reinterpret_cast<float *>(sm + kPrepFac);
 
     if (tid == 0) {
         mbar_init(&bar_ld, 1);
@@ -116,7 +172,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(&tmem_base, 128);
+        tmem_alloc(&tmem_base, 256);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -126,14 +182,14 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
 
     if (tid == 0) {
         mbar_arrive_expect_tx(&bar_ld, 6 * 8192);
-        tma_load_3d(KQ + 0, &mk, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(KQ + 16384, &mk, 64, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(KQ + 8192, &mq, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(KQ + 24576, &mq, 64, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(Vt + 0, &mv, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(Vt + 8192, &mv, 64, (int32_t)h, tok0, &bar_ld);
+        tma_load_3d(sm + 0, &mk, 0, (int32_t)h, tok0, &bar_ld);
+        tma_load_3d(sm + 16384, &mk, 64, (int32_t)h, tok0, &bar_ld);
+        tma_load_3d(sm + 8192, &mq, 0, (int32_t)h, tok0, &bar_ld);
+        tma_load_3d(sm + 24576, &mq, 64, (int32_t)h, tok0, &bar_ld);
+        tma_load_3d(sm + 32768, &mv, 0, (int32_t)h, tok0, &bar_ld);
+        tma_load_3d(sm + 40960, &mv, 64, (int32_t)h, tok0, &bar_ld);
     }
-    // gates: beta and the in-chunk cumulative log gate (rows >= L: beta = 0, g = 0)
+    // Gates (rows >= L: beta = 0, g = 0): in-chunk inclusive cumsum of the log gate.
     if (tid < C) {
         const bool in = tid < L;
         s_beta[tid] = in ? beta[(int64_t)(tok0 + tid) * H + h] : 0.f;
@@ -148,11 +204,19 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     __syncthreads();
     if (tid >= 32 && tid < C) s_b[tid] += s_b[31];
     __syncthreads();
+    if (tid < C) {
+        const bool in = tid < L;
+        const float bl = s_b[L - 1], bi = s_b[tid];
+        s_bg[tid] = s_beta[tid] * __expf(bi);
+        fac[kFacW + tid] = in ? __expf(bl - bi) : 0.f;
+        fac[kFacSG + tid] = in ? scale * __expf(bi) : 0.f;
+        fac[kFacGL + tid] = tid == 0 ? __expf(bl) : 0.f;  // exp(b_L), then zero padding
+    }
 
     bool ok = mbar_wait(&bar_ld, 0);
     if (tid == 0 && ok) {
         tc_fence_after();
-        const uint32_t kq = smem_u32(KQ);
+        const uint32_t kq = smem_u32(sm);
         const uint32_t id = idesc_bf16(128, 64, 0, 0);
         for (int kk = 0; kk < 8; ++kk) {
             const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -163,71 +227,140 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     ok = ok && mbar_wait(&bar_mma, 0);
     tc_fence_after();
 
-    // Epilogue 1: rows 0..63 of the accumulator are K K^T -> A (fp32, smem);
-    // rows 64..127 are Q K^T -> P (bf16 operand image, workspace).
+    // Epilogue 1: accumulator row r = qd*32 + lane, columns [32 hf, 32 hf + 32).
+    // Rows 0..63 (K K^T) -> A in fp32; rows 64..127 (Q K^T) -> P image (bf16).
     if (ok) {
-        const uint32_t taddr = tm + ((uint32_t)(warp * 32) << 16);
-        const bool is_a = tid < C;
-        const int i = is_a ? tid : tid - C;
+        const int r = qd * 32 + lane;
+        const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
+        const bool is_a = r < C;
+        const int i = is_a ? r : r - C;
         const float bi = s_b[i];
         const float pre = is_a ? s_beta[i] : scale;
-        uint8_t *prow = Pimg + (size_t)ch * kTcPImg + (size_t)i * 128;
+        float v0[16], v1[16];
+        tmem_ld16(taddr, v0);
+        tmem_ld16(taddr + 16, v1);
+        tmem_wait_ld();
+        float rr[32];
 #pragma unroll
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float v[16];
-            tmem_ld16(taddr + c0, v);
-            tmem_wait_ld();
-            float r[16];
+        for (int t = 0; t < 32; ++t) {
+            const int j = 32 * hf + t;
+            const bool keep = i < L && (is_a ? j < i : j <= i);
+            rr[t] = keep ? pre * __expf(bi - s_b[j]) * (t < 16 ? v0[t] : v1[t - 16]) : 0.f;
+        }
+        if (is_a) {
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const int j = c0 + t;
-                const bool keep = i < L && (is_a ? j < i : j <= i);
-                r[t] = keep ? pre * __expf(bi - s_b[j]) * v[t] : 0.f;
-            }
-            if (is_a) {
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4 *>(sm + a_offset(i, 32 * hf + 4 * q)) =
+                    make_float4(rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
+        } else {
+            const uint32_t pimg = smem_u32(sm + kPrepP);
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<float4 *>(KQ + a_offset(i, c0 / 4 + q)) =
-                        make_float4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int chunk16 = c0 / 8 + q;  // 8 bf16 per 16-byte chunk
-                    st_global_v4(prow + ((chunk16 ^ (i & 7)) << 4), pack_bf16(r[8 * q], r[8 * q + 1]),
-                                 pack_bf16(r[8 * q + 2], r[8 * q + 3]), pack_bf16(r[8 * q + 4], r[8 * q + 5]),
-                                 pack_bf16(r[8 * q + 6], r[8 * q + 7]));
-                }
-            }
+            for (int q = 0; q < 4; ++q)
+                st_shared_v4(pimg + sw128_offset(i, 4 * hf + q), pack_bf16(rr[8 * q], rr[8 * q + 1]),
+                             pack_bf16(rr[8 * q + 2], rr[8 * q + 3]), pack_bf16(rr[8 * q + 4], rr[8 * q + 5]),
+                             pack_bf16(rr[8 * q + 6], rr[8 * q + 7]));
         }
     }
     tc_fence_before();
     __syncthreads();
 
-    // Solve T = (I + A)^-1, one column per thread (forward substitution in
-    // fp32); then T' = T diag(beta gam), T'' = T diag(beta) as bf16 operands.
-    if (ok && tid < C) {
-        const int col = tid;
-        float x[C];
+    // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks.
+    uint8_t *Tf = sm + kPrepTf;
+    auto offA = [](int i, int j) { return a_offset(i, j); };
+    auto offT = [](int i, int j) { return kPrepTf + f32_offset(i, j); };
+    auto offY = [](int i, int j) { return kPrepY + (uint32_t)i * 64u + (uint32_t)j * 4u; };  // 4 blocks, rows of 16
+    if (ok) {
+        if (warp < 4) {
+            // diagonal block p: column `col` of (I + A_pp)^-1 by forward substitution (fp32)
+            const int p = warp, col = lane & 15;
+            float x[16];
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+            for (int i = 0; i < 16; ++i) {
+                float acc = 0.f;
 #pragma unroll
-            for (int q = 0; q < (i + 3) / 4; ++q) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(KQ + a_offset(i, q));
-                if (4 * q + 0 < i) acc0 += a4.x * x[4 * q + 0];
-                if (4 * q + 1 < i) acc1 += a4.y * x[4 * q + 1];
-                if (4 * q + 2 < i) acc2 += a4.z * x[4 * q + 2];
-                if (4 * q + 3 < i) acc3 += a4.w * x[4 * q + 3];
+                for (int j = 0; j < i; ++j)
+                    acc += *reinterpret_cast<const float *>(sm + a_offset(16 * p + i, 16 * p + j)) * x[j];
+                x[i] = (i == col) ? 1.f : -acc;
             }
-            x[i] = (i == col) ? 1.f : -((acc0 + acc1) + (acc2 + acc3));
-        }
-        const float bc = s_beta[col];
-        const float bgc = bc * __expf(s_b[col]);
+            if (lane < 16)
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            const uint32_t o = sw128_offset(i, col >> 3) + (col & 7) * 2;
-            *reinterpret_cast<__nv_bfloat16 *>(Tp + o) = __float2bfloat16_rn(x[i] * bgc);
-            *reinterpret_cast<__nv_bfloat16 *>(Tpp + o) = __float2bfloat16_rn(x[i] * bc);
+                for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(Tf + f32_offset(16 * p + i, 16 * p + col)) = x[i];
+        } else {
+            // zero the strictly upper off-diagonal blocks
+            for (int e = tid - 128; e < 6 * 256; e += 128) {
+                const int b = e >> 8, w = e & 255;
+                const int pb = b < 3 ? 0 : (b < 5 ? 1 : 2);
+                const int qb = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
+                *reinterpret_cast<float *>(Tf + f32_offset(16 * pb + (w >> 4), 16 * qb + (w & 15))) = 0.f;
+            }
+        }
+    }
+    __syncthreads();
+    // level 1: T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
+    if (ok && warp < 2) {
+        const int p = 2 * warp + 1, q = 2 * warp;
+        float c[2][4];
+        const int xr[1] = {16 * p}, xc[1] = {16 * q}, yr[1] = {16 * q}, yc[1] = {16 * q};
+        warp_gemm16(sm, 1, xr, xc, yr, yc, offA, offT, c);
+        warp_store16(sm, 16 * warp, 0, c, 1.f, offY);
+        __syncwarp();
+        const int xr2[1] = {16 * p}, xc2[1] = {16 * p}, yr2[1] = {16 * warp}, yc2[1] = {0};
+        warp_gemm16(sm, 1, xr2, xc2, yr2, yc2, offT, offY, c);
+        warp_store16(sm, 16 * p, 16 * q, c, -1.f, offT);
+    }
+    __syncthreads();
+    // level 2, step 1: Y_pq = sum_{r in {0,1}} A_pr T_rq for p in {2,3}, q in {0,1}
+    if (ok && warp < 4) {
+        const int p = 2 + (warp >> 1), q = warp & 1;
+        float c[2][4];
+        if (q == 0) {
+            const int xr[2] = {16 * p, 16 * p}, xc[2] = {0, 16}, yr[2] = {0, 16}, yc[2] = {0, 0};
+            warp_gemm16(sm, 2, xr, xc, yr, yc, offA, offT, c);
+        } else {
+            const int xr[1] = {16 * p}, xc[1] = {16}, yr[1] = {16}, yc[1] = {16};
+            warp_gemm16(sm, 1, xr, xc, yr, yc, offA, offT, c);
+        }
+        warp_store16(sm, 16 * warp, 0, c, 1.f, offY);
+    }
+    __syncthreads();
+    // level 2, step 2: T_pq = -sum_{r in {2,3}, r <= p} T_pr Y_rq
+    if (ok && warp < 4) {
+        const int p = 2 + (warp >> 1), q = warp & 1;
+        float c[2][4];
+        // Y_rq lives in scratch block (r - 2) * 2 + q
+        if (p == 2) {
+            const int xr[1] = {32}, xc[1] = {32}, yr[1] = {16 * (0 * 2 + q)}, yc[1] = {0};
+            warp_gemm16(sm, 1, xr, xc, yr, yc, offT, offY, c);
+        } else {
+            const int xr[2] = {48, 48}, xc[2] = {32, 48}, yr[2] = {16 * (0 * 2 + q), 16 * (1 * 2 + q)}, yc[2] = {0, 0};
+            warp_gemm16(sm, 2, xr, xc, yr, yc, offT, offY, c);
+        }
+        warp_store16(sm, 16 * p, 16 * q, c, -1.f, offT);
+    }
+    __syncthreads();
+
+    // T' = T diag(beta gam), T'' = T diag(beta) as bf16 operand images (K-major rows i).
+    if (ok) {
+        const int i = tid >> 2, j0 = (tid & 3) * 16;
+        float tv[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 f = *reinterpret_cast<const float4 *>(Tf + f32_offset(i, j0 + 4 * q));
+            tv[4 * q] = f.x; tv[4 * q + 1] = f.y; tv[4 * q + 2] = f.z; tv[4 * q + 3] = f.w;
+        }
+        const uint32_t tp = smem_u32(sm + 8192), tpp = smem_u32(sm + 24576);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            float a[8], b[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int j = j0 + 8 * q + e;
+                a[e] = tv[8 * q + e] * s_bg[j];
+                b[e] = tv[8 * q + e] * s_beta[j];
+            }
+            const uint32_t o = sw128_offset(i, (j0 >> 3) + q);
+            st_shared_v4(tp + o, pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
+            st_shared_v4(tpp + o, pack_bf16(b[0], b[1]), pack_bf16(b[2], b[3]), pack_bf16(b[4], b[5]), pack_bf16(b[6], b[7]));
         }
     }
     fence_async_smem();
@@ -235,62 +368,72 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     __syncthreads();
     tc_fence_after();
 
-    // W^T = K^T T'^T (M = d_k rows), U^T = V^T T''^T (M = d_v rows); K = 64 tokens.
+    // W^T = K^T T'^T (M = d_k), U^T = V^T T''^T (M = d_v); K = 64 tokens.
     if (tid == 0 && ok) {
-        const uint32_t kq = smem_u32(KQ), vt = smem_u32(Vt), tp = smem_u32(Tp), tpp = smem_u32(Tpp);
+        const uint32_t kq = smem_u32(sm), vt = smem_u32(sm + 32768), tp = smem_u32(sm + 8192),
+                       tpp = smem_u32(sm + 24576);
         const uint32_t id = idesc_bf16(128, 64, 1, 0);
         for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tm, sdesc_sw128(kq + kk * 2048, 16384, 1024), sdesc_sw128(tp + kk * 32, 16, 1024), id, kk > 0);
+            mma_bf16(tm + 64, sdesc_sw128(kq + kk * 2048, 16384, 1024), sdesc_sw128(tp + kk * 32, 16, 1024), id, kk > 0);
         for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tm + 64, sdesc_sw128(vt + kk * 2048, 8192, 1024), sdesc_sw128(tpp + kk * 32, 16, 1024), id,
+            mma_bf16(tm + 128, sdesc_sw128(vt + kk * 2048, 8192, 1024), sdesc_sw128(tpp + kk * 32, 16, 1024), id,
                      kk > 0);
         mma_commit(&bar_mma);
+        // P image and gate factors are final: store them while the MMAs run
+        bulk_store(blk + kBlkP, sm + kPrepP, (uint32_t)kTcPImg);
+        bulk_store(blk + kBlkFac, sm + kPrepFac, (uint32_t)kTcFac);
+        bulk_commit();
     }
     ok = ok && mbar_wait(&bar_mma, 1);
     tc_fence_after();
 
-    // Epilogue 2: thread r owns row r (channel r) of W^T and U^T.
+    // Epilogue 2: row r (a channel) of W^T and U^T, tokens [32 hf, 32 hf + 32), as
+    // 128-byte-swizzled rows: the W^T image at [0, 16K), the U^T rows at [16K, 32K).
     if (ok) {
-        const uint32_t taddr = tm + ((uint32_t)(warp * 32) << 16);
-        const int r = tid;
-        uint8_t *wrow = Wimg + (size_t)ch * kTcWImg + (size_t)r * 128;
-        uint8_t *urow = reinterpret_cast<uint8_t *>(Ut) + (size_t)ch * kTcUt + (size_t)r * 128;
+        const int r = qd * 32 + lane;
+        const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
+        float w0[16], w1[16], u0[16], u1[16];
+        tmem_ld16(taddr + 64, w0);
+        tmem_ld16(taddr + 64 + 16, w1);
+        tmem_ld16(taddr + 128, u0);
+        tmem_ld16(taddr + 128 + 16, u1);
+        tmem_wait_ld();
+        const uint32_t wimg = smem_u32(sm), uimg = smem_u32(sm + 16384);
 #pragma unroll
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float w[16], u[16];
-            tmem_ld16(taddr + c0, w);
-            tmem_ld16(taddr + 64 + c0, u);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int chunk16 = c0 / 8 + q;
-                st_global_v4(wrow + ((chunk16 ^ (r & 7)) << 4), pack_bf16(w[8 * q], w[8 * q + 1]),
-                             pack_bf16(w[8 * q + 2], w[8 * q + 3]), pack_bf16(w[8 * q + 4], w[8 * q + 5]),
-                             pack_bf16(w[8 * q + 6], w[8 * q + 7]));
-                st_global_v4(urow + chunk16 * 16, pack_bf16(u[8 * q], u[8 * q + 1]), pack_bf16(u[8 * q + 2], u[8 * q + 3]),
-                             pack_bf16(u[8 * q + 4], u[8 * q + 5]), pack_bf16(u[8 * q + 6], u[8 * q + 7]));
-            }
+        for (int q = 0; q < 4; ++q) {
+            const float *w = q < 2 ? w0 + 8 * q : w1 + 8 * (q - 2);
+            const float *u = q < 2 ? u0 + 8 * q : u1 + 8 * (q - 2);
+            const uint32_t o = sw128_offset(r, 4 * hf + q);
+            st_shared_v4(wimg + o, pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+            st_shared_v4(uimg + o, pack_bf16(u[0], u[1]), pack_bf16(u[2], u[3]), pack_bf16(u[4], u[5]), pack_bf16(u[6], u[7]));
         }
-        if (tid < C) bcum[ch * C + tid] = s_b[tid];
-    } else if (tid == 0) {
-        flag_error(err, 1);
     }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, 128);
+    if (tid == 0) {
+        if (ok) {
+            bulk_store(blk + kBlkW, sm, 32768);  // W^T image then U^T rows, contiguous in both places
+            bulk_commit();
+        }
+        bulk_wait_all();
+        if (!ok) flag_error(err, 1);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, 256);
 }
 
 // ===========================================================================
-// Scan: the chunks of each sequence in order
+// Scan
 // ===========================================================================
-// Shared memory (1024-aligned): two stages of per-chunk operands, then the
-// per-chunk A operands written by the threads.
-constexpr uint32_t kStQ = 0, kStK = 16384, kStW = 32768, kStP = 49152, kStB = 57344, kStage = 58368;
-constexpr uint32_t kSImg = 2 * kStage;          // state, bf16, K-major rows v, 2 x 16K
-constexpr uint32_t kUpImg = kSImg + 32768;      // U' (rows v, K = tokens)
-constexpr uint32_t kUwImg = kUpImg + 16384;     // U' scaled by exp(b_L - b_i)
+// Shared memory (1024-aligned): two stages of per-chunk operands
+//   [Q tile 16K][K tile 16K][workspace block: W^T image 16K, U^T rows 16K, P image 8K, factors]
+// then the bf16 operands written by the threads: S0 (32K), U' and U'_w (16K each).
+// The U' region also stages full output tiles for the TMA store.
+constexpr uint32_t kStQ = 0, kStK = 16384, kStBlk = 32768, kStage = 75776;
+constexpr uint32_t kStageBytes = 32768 + (uint32_t)kTcBlock;
+constexpr uint32_t kSImg = 2 * kStage, kUpImg = kSImg + 32768, kUwImg = kUpImg + 16384;
 constexpr uint32_t kScanSmem = kUwImg + 16384 + 1024;
-constexpr uint32_t kStageBytes = 2 * 16384 + 16384 + 8192 + 256;
 
 struct ScanBars {
     uint64_t full[2];
@@ -299,18 +442,18 @@ struct ScanBars {
 
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_scan_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-            const float *h0, const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T,
-            int64_t rows, int64_t H, int64_t max_chunks, float scale, int64_t snap_stride, int64_t n_snap,
-            const uint8_t *__restrict__ Wimg, const uint8_t *__restrict__ Pimg, const __nv_bfloat16 *__restrict__ Ut,
-            const float *__restrict__ bcum, __nv_bfloat16 *__restrict__ out, float *final_state,
-            float *__restrict__ snaps, int *err) {
+            const __grid_constant__ CUtensorMap mo, const float *h0, const int32_t *__restrict__ cu,
+            const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t max_chunks,
+            int64_t snap_stride, int64_t n_snap, const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out,
+            float *final_state, float *__restrict__ snaps, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     __shared__ ScanBars bars;
     __shared__ uint32_t tmem_base;
     const int64_t n = blockIdx.x, h = blockIdx.y;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int v = tid;  // state row owned by this thread
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qd = warp & 3, hf = warp >> 2;
+    const int v = qd * 32 + lane;  // state row; this thread holds columns [64 hf, 64 hf + 64)
 
     int64_t start, len;
     seq_bounds(cu, n, T, rows, start, len);
@@ -332,8 +475,9 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tmem_base;
-    const uint32_t acc1 = tm, acc2 = tm + 64, acc3 = tm + 128, acc4 = tm + 256;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const uint32_t acc1 = tm + lane_off, acc2 = tm + 64 + lane_off, acc3 = tm + 128 + lane_off,
+                   acc4 = tm + 256 + lane_off;
 
     auto issue_loads = [&](int64_t c) {
         const int stage = (int)(c & 1);
@@ -346,189 +490,203 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         tma_load_3d(st + kStQ + 8192, &mq, 64, (int32_t)h, tok, bar);
         tma_load_3d(st + kStK, &mk, 0, (int32_t)h, tok, bar);
         tma_load_3d(st + kStK + 8192, &mk, 64, (int32_t)h, tok, bar);
-        bulk_load(st + kStW, Wimg + (size_t)chh * kTcWImg, (uint32_t)kTcWImg, bar);
-        bulk_load(st + kStP, Pimg + (size_t)chh * kTcPImg, (uint32_t)kTcPImg, bar);
-        bulk_load(st + kStB, bcum + (size_t)chh * C, (uint32_t)kTcB, bar);
+        bulk_load(st + kStBlk, blocks + (size_t)chh * kTcBlock, (uint32_t)kTcBlock, bar);
     };
     if (tid == 0) {
         if (nchunks > 0) issue_loads(0);
         if (nchunks > 1) issue_loads(1);
     }
 
-    // state row v in registers
-    float S[D];
-    const int64_t srow = ((n * H + h) * D + v) * (int64_t)D;
+    float S[64];
+    const int64_t srow = ((n * H + h) * D + v) * (int64_t)D + 64 * hf;
     if (h0) {
 #pragma unroll
-        for (int c = 0; c < D; c += 4) {
+        for (int c = 0; c < 64; c += 4) {
             const float4 t = *reinterpret_cast<const float4 *>(h0 + srow + c);
             S[c] = t.x; S[c + 1] = t.y; S[c + 2] = t.z; S[c + 3] = t.w;
         }
     } else {
 #pragma unroll
-        for (int c = 0; c < D; ++c) S[c] = 0.f;
+        for (int c = 0; c < 64; ++c) S[c] = 0.f;
     }
 
     const uint32_t s_img = smem_u32(sm + kSImg), up_img = smem_u32(sm + kUpImg), uw_img = smem_u32(sm + kUwImg);
+    const uint32_t id_w = idesc_bf16(128, 64, 0, 1), id_q = idesc_bf16(128, 64, 0, 0),
+                   id_k = idesc_bf16(128, 128, 0, 1), id_p = idesc_bf16(128, 64, 0, 0);
     bool ok = true;
-    for (int64_t c = 0; c < nchunks && ok; ++c) {
+    for (int64_t c = 0; c < nchunks; ++c) {
         const int stage = (int)(c & 1);
         uint8_t *st = sm + stage * kStage;
         const uint32_t st_u = smem_u32(st);
-        const int64_t chh = (chunk0 + c) * H + h;
         const int L = (int)(len - c * C < C ? len - c * C : C);
         const int64_t tok0 = start + c * C;
         const uint32_t par = (uint32_t)(c & 1);
+        const float *fac = reinterpret_cast<const float *>(st + kStBlk + kBlkFac);
 
-        // this chunk's U row (U[i, v], i = 0..63), bf16
-        uint4 ur[8];
-        const uint4 *usrc = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(Ut) +
-                                                            (size_t)chh * kTcUt + (size_t)v * 128);
+        // (a) S0 -> bf16 operand, K-major rows v; this thread writes its 64-column block
 #pragma unroll
-        for (int q = 0; q < 8; ++q) ur[q] = usrc[q];
-
-        // (a) S0 -> bf16 operand (K-major rows v, two 64-column blocks)
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk)
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float *s8 = S + blk * 64 + q * 8;
-                st_shared_v4(s_img + blk * 16384 + sw128_offset(v, q), pack_bf16(s8[0], s8[1]), pack_bf16(s8[2], s8[3]),
-                             pack_bf16(s8[4], s8[5]), pack_bf16(s8[6], s8[7]));
-            }
+        for (int q = 0; q < 8; ++q) {
+            const float *s8 = S + q * 8;
+            st_shared_v4(s_img + hf * 16384 + sw128_offset(v, q), pack_bf16(s8[0], s8[1]), pack_bf16(s8[2], s8[3]),
+                         pack_bf16(s8[4], s8[5]), pack_bf16(s8[6], s8[7]));
+        }
         fence_async_smem();
+        if (tid == 0) bulk_wait_read();  // the previous output tile has left the U' region
         ok = mbar_wait(&bars.full[stage], (uint32_t)((c >> 1) & 1));
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (!ok) break;
+        if (__syncthreads_or(!ok)) break;
 
         // (b) acc1 = S0 W^T, acc2 = S0 Q^T
         if (tid == 0) {
-            const uint32_t id_w = idesc_bf16(128, 64, 0, 1), id_q = idesc_bf16(128, 64, 0, 0);
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16(acc1, sdesc_sw128(s_img + o, 16, 1024), sdesc_sw128(st_u + kStW + kk * 2048, 16384, 1024),
-                         id_w, kk > 0);
+                mma_bf16(acc1 - lane_off, sdesc_sw128(s_img + o, 16, 1024),
+                         sdesc_sw128(st_u + kStBlk + kBlkW + kk * 2048, 16384, 1024), id_w, kk > 0);
             }
             mma_commit(&bars.mma[0]);
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16(acc2, sdesc_sw128(s_img + o, 16, 1024),
+                mma_bf16(acc2 - lane_off, sdesc_sw128(s_img + o, 16, 1024),
                          sdesc_sw128(st_u + kStQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_q, kk > 0);
             }
             mma_commit(&bars.mma[1]);
         }
 
-        // (c) U' = U - S0 W^T; write U' and U' * exp(b_L - b_i) as bf16 operands
-        const float *bs = reinterpret_cast<const float *>(st + kStB);
-        const float bl = bs[L - 1];
+        // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32); write U' and U' * w as bf16
         ok = mbar_wait(&bars.mma[0], par);
         tc_fence_after();
-        if (ok) {
+        {
+            float a0[16], a1[16];
+            tmem_ld16(acc1 + 32 * hf, a0);
+            tmem_ld16(acc1 + 32 * hf + 16, a1);
+            tmem_wait_ld();
+            const uint32_t urow = st_u + kStBlk + kBlkU;
 #pragma unroll
-            for (int c0 = 0; c0 < C; c0 += 16) {
-                float a[16];
-                tmem_ld16(acc1 + lane_off + c0, a);
-                tmem_wait_ld();
-                float up[16], uw[16];
+            for (int q = 0; q < 4; ++q) {
+                const int cq = 4 * hf + q;  // 16-byte chunk = tokens 8 cq .. 8 cq + 7
+                const uint4 u8 = ld_shared_v4(urow + sw128_offset(v, cq));
+                const float4 wlo = *reinterpret_cast<const float4 *>(fac + kFacW + 8 * cq);
+                const float4 whi = *reinterpret_cast<const float4 *>(fac + kFacW + 8 * cq + 4);
+                const float wv[8] = {wlo.x, wlo.y, wlo.z, wlo.w, whi.x, whi.y, whi.z, whi.w};
+                const uint32_t uw32[4] = {u8.x, u8.y, u8.z, u8.w};
+                float up[8], uw[8];
 #pragma unroll
-                for (int t = 0; t < 16; t += 2) {
-                    const uint32_t pr = (&ur[0].x)[(c0 + t) / 2];
-                    const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&pr);
-                    const int i = c0 + t;
-                    up[t] = i < L ? __low2float(u2) - a[t] : 0.f;
-                    up[t + 1] = i + 1 < L ? __high2float(u2) - a[t + 1] : 0.f;
-                    uw[t] = up[t] * __expf(bl - bs[i]);
-                    uw[t + 1] = up[t + 1] * __expf(bl - bs[i + 1]);
+                for (int e = 0; e < 8; e += 2) {
+                    const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
+                    const float acc_lo = (q < 2 ? a0[8 * q + e] : a1[8 * (q - 2) + e]);
+                    const float acc_hi = (q < 2 ? a0[8 * q + e + 1] : a1[8 * (q - 2) + e + 1]);
+                    up[e] = __low2float(u2) - acc_lo;
+                    up[e + 1] = __high2float(u2) - acc_hi;
+                    uw[e] = up[e] * wv[e];
+                    uw[e + 1] = up[e + 1] * wv[e + 1];
                 }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int chunk16 = c0 / 8 + q;
-                    st_shared_v4(up_img + sw128_offset(v, chunk16), pack_bf16(up[8 * q], up[8 * q + 1]),
-                                 pack_bf16(up[8 * q + 2], up[8 * q + 3]), pack_bf16(up[8 * q + 4], up[8 * q + 5]),
-                                 pack_bf16(up[8 * q + 6], up[8 * q + 7]));
-                    st_shared_v4(uw_img + sw128_offset(v, chunk16), pack_bf16(uw[8 * q], uw[8 * q + 1]),
-                                 pack_bf16(uw[8 * q + 2], uw[8 * q + 3]), pack_bf16(uw[8 * q + 4], uw[8 * q + 5]),
-                                 pack_bf16(uw[8 * q + 6], uw[8 * q + 7]));
-                }
+                const uint32_t o = sw128_offset(v, cq);
+                st_shared_v4(up_img + o, pack_bf16(up[0], up[1]), pack_bf16(up[2], up[3]), pack_bf16(up[4], up[5]),
+                             pack_bf16(up[6], up[7]));
+                st_shared_v4(uw_img + o, pack_bf16(uw[0], uw[1]), pack_bf16(uw[2], uw[3]), pack_bf16(uw[4], uw[5]),
+                             pack_bf16(uw[6], uw[7]));
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (!ok) break;
 
-        // (d) acc4 = U'_w K (state increment), acc3 = U' P^T (intra-chunk output)
+        // (d) acc4 = U'_w K (state increment), acc3 = U' P^T (in-chunk output)
         if (tid == 0) {
-            const uint32_t id_k = idesc_bf16(128, 128, 0, 1), id_p = idesc_bf16(128, 64, 0, 0);
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(acc4, sdesc_sw128(uw_img + kk * 32, 16, 1024), sdesc_sw128(st_u + kStK + kk * 2048, 8192, 1024),
-                         id_k, kk > 0);
+                mma_bf16(acc4 - lane_off, sdesc_sw128(uw_img + kk * 32, 16, 1024),
+                         sdesc_sw128(st_u + kStK + kk * 2048, 8192, 1024), id_k, kk > 0);
             mma_commit(&bars.mma[2]);
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(acc3, sdesc_sw128(up_img + kk * 32, 16, 1024), sdesc_sw128(st_u + kStP + kk * 32, 16, 1024),
-                         id_p, kk > 0);
+                mma_bf16(acc3 - lane_off, sdesc_sw128(up_img + kk * 32, 16, 1024),
+                         sdesc_sw128(st_u + kStBlk + kBlkP + kk * 32, 16, 1024), id_p, kk > 0);
             mma_commit(&bars.mma[3]);
         }
 
-        // (e) S = gam_L S0 + acc4
-        const float gl = __expf(bl);
-        ok = mbar_wait(&bars.mma[2], par);
+        // (e) S = gam_L S0 + acc4 (columns [64 hf, 64 hf + 64))
+        const float gl = fac[kFacGL];
+        ok = mbar_wait(&bars.mma[2], par) && ok;
         tc_fence_after();
-        if (ok) {
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float a[16];
-                tmem_ld16(acc4 + lane_off + c0, a);
-                tmem_wait_ld();
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+            float a[16];
+            tmem_ld16(acc4 + 64 * hf + c0, a);
+            tmem_wait_ld();
 #pragma unroll
-                for (int t = 0; t < 16; ++t) S[c0 + t] = gl * S[c0 + t] + a[t];
-            }
+            for (int t = 0; t < 16; ++t) S[c0 + t] = gl * S[c0 + t] + a[t];
         }
 
-        // (f) O = scale gam_i (S0 q_i) + (P U')_i
-        ok = ok && mbar_wait(&bars.mma[1], par) && mbar_wait(&bars.mma[3], par);
+        // (f) O = scale gam_i (S0 q_i) + (P U')_i for tokens [32 hf, 32 hf + 32)
+        ok = mbar_wait(&bars.mma[1], par) && mbar_wait(&bars.mma[3], par) && ok;
         tc_fence_after();
-        if (ok) {
-            __nv_bfloat16 *op = out + (tok0 * H + h) * D + v;
+        {
+            float a2[32], a3[32];
+            tmem_ld16(acc2 + 32 * hf, *reinterpret_cast<float(*)[16]>(a2));
+            tmem_ld16(acc2 + 32 * hf + 16, *reinterpret_cast<float(*)[16]>(a2 + 16));
+            tmem_ld16(acc3 + 32 * hf, *reinterpret_cast<float(*)[16]>(a3));
+            tmem_ld16(acc3 + 32 * hf + 16, *reinterpret_cast<float(*)[16]>(a3 + 16));
+            tmem_wait_ld();
+            float o[32];
 #pragma unroll
-            for (int c0 = 0; c0 < C; c0 += 16) {
-                float a2[16], a3[16];
-                tmem_ld16(acc2 + lane_off + c0, a2);
-                tmem_ld16(acc3 + lane_off + c0, a3);
-                tmem_wait_ld();
+            for (int t = 0; t < 32; t += 4) {
+                const float4 sg = *reinterpret_cast<const float4 *>(fac + kFacSG + 32 * hf + t);
+                o[t] = sg.x * a2[t] + a3[t];
+                o[t + 1] = sg.y * a2[t + 1] + a3[t + 1];
+                o[t + 2] = sg.z * a2[t + 2] + a3[t + 2];
+                o[t + 3] = sg.w * a2[t + 3] + a3[t + 3];
+            }
+            if (L == C) {
+                // stage [token][channel] tiles (two 64-channel boxes) in the U' region
+                uint8_t *ot = sm + kUpImg + (v >> 6) * 8192 + (v & 63) * 2;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const int i = c0 + t;
-                    if (i < L) op[(int64_t)i * H * D] = __float2bfloat16_rn(scale * __expf(bs[i]) * a2[t] + a3[t]);
+                for (int t = 0; t < 32; ++t)
+                    *reinterpret_cast<__nv_bfloat16 *>(ot + (32 * hf + t) * 128) = __float2bfloat16_rn(o[t]);
+            } else {
+                __nv_bfloat16 *op = out + (tok0 * H + h) * D + v;
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const int i = 32 * hf + t;
+                    if (i < L) op[(int64_t)i * H * D] = __float2bfloat16_rn(o[t]);
                 }
             }
         }
 
         // snapshot after n * stride tokens of the sequence
-        if (ok && snaps && snap_stride > 0 && ((c + 1) * C) % snap_stride == 0 && (c + 1) * C <= len) {
+        if (snaps && snap_stride > 0 && ((c + 1) * C) % snap_stride == 0 && (c + 1) * C <= len) {
             const int64_t s = (c + 1) * C / snap_stride - 1;
             if (s < n_snap) {
-                float *dst = snaps + (((n * n_snap + s) * H + h) * D + v) * (int64_t)D;
+                float *dst = snaps + (((n * n_snap + s) * H + h) * D + v) * (int64_t)D + 64 * hf;
 #pragma unroll
-                for (int cc = 0; cc < D; cc += 4)
+                for (int cc = 0; cc < 64; cc += 4)
                     *reinterpret_cast<float4 *>(dst + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
             }
         }
 
-        // release this stage: every MMA that read it has completed; refill with chunk c+2
+        // every MMA of this chunk has completed: release the stage, ship the output tile
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0 && ok && c + 2 < nchunks) issue_loads(c + 2);
+        if (tid == 0) {
+            if (L == C) {
+                tma_store_3d(&mo, sm + kUpImg, 0, (int32_t)h, (int32_t)tok0);
+                tma_store_3d(&mo, sm + kUpImg + 8192, 64, (int32_t)h, (int32_t)tok0);
+                bulk_commit();
+            }
+            if (c + 2 < nchunks) issue_loads(c + 2);
+        }
+        if (__syncthreads_or(!ok)) break;
     }
     if (!ok && tid == 0) flag_error(err, 2);
     if (ok && final_state) {
+        const int64_t frow = srow;
 #pragma unroll
-        for (int cc = 0; cc < D; cc += 4)
-            *reinterpret_cast<float4 *>(final_state + srow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
+        for (int cc = 0; cc < 64; cc += 4)
+            *reinterpret_cast<float4 *>(final_state + frow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
     }
+    if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
@@ -550,16 +708,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// (rows, H, 128) bf16 tensor, tiles of 64 tokens x 64 channels of one head, 128-byte swizzle.
-gdn_status make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t H) {
+// (rows, H, 128) bf16 tensor, tiles of 64 tokens x 64 channels of one head.
+gdn_status make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t H, bool swizzle) {
     auto enc = tensor_map_encoder();
     if (!enc) return fail(GDN_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
     cuuint32_t box[3] = {64, 1, 64}, es[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(GDN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return GDN_OK;
 }
@@ -574,21 +732,19 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     gdn_status st = launch_chunk_table(p, a, s);
     if (st != GDN_OK) return st;
     const int32_t *off = a.cu_seqlens ? reinterpret_cast<const int32_t *>(a.ws + p.off_chunk_offsets) : nullptr;
-    uint8_t *Wimg = reinterpret_cast<uint8_t *>(a.ws + p.off_W);
-    uint8_t *Pimg = reinterpret_cast<uint8_t *>(a.ws + p.off_P);
-    __nv_bfloat16 *Ut = reinterpret_cast<__nv_bfloat16 *>(a.ws + p.off_U);
-    float *bcum = reinterpret_cast<float *>(a.ws + p.off_b);
+    uint8_t *blocks = reinterpret_cast<uint8_t *>(a.ws + p.off_W);
     if (p.H > 65535 || p.max_chunks > 0x7fffffffLL || a.N > 0x7fffffffLL)
         return fail(GDN_ERR_UNSUPPORTED, "grid too large");
-    CUtensorMap mq, mk, mv;
-    const int64_t map_rows = p.rows > 0 ? p.rows : 1;
+    CUtensorMap mq, mk, mv, mo;
+    memset(&mq, 0, sizeof mq);
+    memset(&mk, 0, sizeof mk);
+    memset(&mv, 0, sizeof mv);
+    memset(&mo, 0, sizeof mo);
     if (p.rows > 0) {
-        if ((st = make_map(&mq, a.q, map_rows, p.H)) != GDN_OK) return st;
-        if ((st = make_map(&mk, a.k, map_rows, p.H)) != GDN_OK) return st;
-        if ((st = make_map(&mv, a.v, map_rows, p.H)) != GDN_OK) return st;
-    } else {
-        memset(&mq, 0, sizeof mq);
-        memset(&mk, 0, sizeof mk);
+        if ((st = make_map(&mq, a.q, p.rows, p.H, true)) != GDN_OK) return st;
+        if ((st = make_map(&mk, a.k, p.rows, p.H, true)) != GDN_OK) return st;
+        if ((st = make_map(&mv, a.v, p.rows, p.H, true)) != GDN_OK) return st;
+        if ((st = make_map(&mo, a.out, p.rows, p.H, false)) != GDN_OK) return st;
     }
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -601,14 +757,14 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     if (p.max_chunks > 0 && p.rows > 0) {
         LaunchScope ls("gdn_prep_tc", s);
         gdn_prep_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kPrepSmem, s>>>(
-            mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.scale, Wimg, Pimg, Ut, bcum, nullptr);
+            mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.scale, blocks, nullptr);
     }
     if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
     {
         LaunchScope ls("gdn_scan_tc", s);
         gdn_scan_tc<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
-            mq, mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.scale, a.snapshot_stride, a.n_snap,
-            Wimg, Pimg, Ut, bcum, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, nullptr);
+            mq, mk, mo, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap,
+            blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, nullptr);
     }
     return check_launch("gdn_scan_tc");
 }

@@ -65,9 +65,11 @@ gdn_status launch_chunk_simt(const ChunkPlan &p, const ChunkArgs &a, int dtype, 
 gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s);
 bool tc_eligible(const gdn_desc &d);
 
-// Per chunk-head workspace of the tensor-core path (bytes): the W^T operand
-// image, the P operand image, U^T (bf16) and the cumulative log gate.
-constexpr size_t kTcWImg = 128 * 128, kTcPImg = 64 * 128, kTcUt = 128 * 64 * 2, kTcB = 64 * 4;
+// Per chunk-head workspace block of the tensor-core path (bytes), in this
+// order: the W^T operand image, the U^T rows, the P operand image and the
+// per-token gate factors.  The scan copies each block with one bulk copy.
+constexpr size_t kTcWImg = 128 * 128, kTcUt = 128 * 128, kTcPImg = 64 * 128, kTcFac = 192 * 4;
+constexpr size_t kTcBlock = kTcWImg + kTcUt + kTcPImg + kTcFac;  // 41728
 gdn_status launch_decode(const gdn_desc &d, const void *q, const void *k, const void *v,
                          const float *g, const float *beta, float *state, void *out,
                          cudaStream_t s);
