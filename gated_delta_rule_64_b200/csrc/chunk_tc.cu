@@ -57,7 +57,7 @@ constexpr int D = 128;     // d_k = d_v
 constexpr int kThreads = 256;
 
 // Offsets inside one workspace block (see kTcBlock).
-constexpr uint32_t kBlkW = 0, kBlkU = 16384, kBlkP = 32768, kBlkFac = 40960;
+constexpr uint32_t kBlkWQ = 0, kBlkU = 32768, kBlkP = 49152, kBlkFac = 57344;
 // Gate factors: [0, 64) w_i = exp(b_L - b_i); [64, 128) scale * exp(b_i); [128] exp(b_L).
 constexpr int kFacW = 0, kFacSG = 64, kFacGL = 128;
 
@@ -82,15 +82,14 @@ __device__ __forceinline__ uint32_t f32_offset(int i, int j) {
 //               [c-block 0: K rows | Q rows][c-block 1: K rows | Q rows].
 //               After that MMA the Q rows hold A (fp32; rows 0-31 | 32-63),
 //               then T diag(beta gam) at [8K,16K) and T diag(beta) at [24K,32K)
-//               (bf16 operand images); after the last MMAs the whole range
-//               stages the W^T image [0,16K) and the U^T rows [16K,32K).
+//               (bf16 operand images).
 //   [32K, 48K)  V tile
 //   [48K, 64K)  T (fp32)
 //   [64K, 68K)  per-warp 16 x 16 scratch of the blocked solve
-//   [68K, 76K)  P image (staged)
-//   [76K, +768) gate factors (staged)
-constexpr uint32_t kPrepTf = 49152, kPrepY = 65536, kPrepP = 69632, kPrepFac = 77824;
-constexpr uint32_t kPrepSmem = kPrepFac + 768 + 1024;
+// The results (W image, U^T rows, P image, gate factors) are written straight
+// to the workspace block of the chunk-head.
+constexpr uint32_t kPrepTf = 49152, kPrepY = 65536;
+constexpr uint32_t kPrepSmem = kPrepY + 4096 + 1024;
 
 __device__ __forceinline__ uint32_t a_offset(int i, int j) {
     // A (fp32) in the Q rows of the first operand: rows 0..31 at 8K, 32..63 at 24K
@@ -99,9 +98,10 @@ __device__ __forceinline__ uint32_t a_offset(int i, int j) {
 
 // C (16x16) = sum over `nk` 16-wide K blocks of X_k (16x16) * Y_k (16x16); X and Y
 // are fp32 blocks in shared memory given by their (row, col) origins and an
-// offset function.  Warp-level m16n8k8 tf32 MMAs, fp32 accumulate.  The result
-// is returned in the MMA accumulator layout: c[nt][0..3] for the 8-column
-// tiles nt = 0, 1.
+// offset function.  Warp-level m16n8k8 tf32 MMAs, fp32 accumulate; the fp32
+// bit patterns are passed as they are (the tensor core reads them as tf32,
+// dropping the low mantissa bits).  The result is returned in the MMA
+// accumulator layout: c[nt][0..3] for the 8-column tiles nt = 0, 1.
 template <typename OffX, typename OffY>
 __device__ __forceinline__ void warp_gemm16(const uint8_t *base, int nk, const int *xr, const int *xc, const int *yr,
                                             const int *yc, OffX offx, OffY offy, float (&c)[2][4]) {
@@ -115,15 +115,15 @@ __device__ __forceinline__ void warp_gemm16(const uint8_t *base, int nk, const i
         for (int ks = 0; ks < 2; ++ks) {
             const int k0 = ks * 8;
             uint32_t a[4];
-            a[0] = to_tf32(*reinterpret_cast<const float *>(base + offx(xr[kb] + g, xc[kb] + k0 + t)));
-            a[1] = to_tf32(*reinterpret_cast<const float *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t)));
-            a[2] = to_tf32(*reinterpret_cast<const float *>(base + offx(xr[kb] + g, xc[kb] + k0 + t + 4)));
-            a[3] = to_tf32(*reinterpret_cast<const float *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t + 4)));
+            a[0] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g, xc[kb] + k0 + t));
+            a[1] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t));
+            a[2] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g, xc[kb] + k0 + t + 4));
+            a[3] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t + 4));
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 uint32_t b[2];
-                b[0] = to_tf32(*reinterpret_cast<const float *>(base + offy(yr[kb] + k0 + t, yc[kb] + nt * 8 + g)));
-                b[1] = to_tf32(*reinterpret_cast<const float *>(base + offy(yr[kb] + k0 + t + 4, yc[kb] + nt * 8 + g)));
+                b[0] = *reinterpret_cast<const uint32_t *>(base + offy(yr[kb] + k0 + t, yc[kb] + nt * 8 + g));
+                b[1] = *reinterpret_cast<const uint32_t *>(base + offy(yr[kb] + k0 + t + 4, yc[kb] + nt * 8 + g));
                 mma_tf32_16x8x8(c[nt], a, b);
             }
         }
@@ -144,7 +144,7 @@ __device__ __forceinline__ void warp_store16(uint8_t *base, int r0, int c0, cons
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
 gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
             const __grid_constant__ CUtensorMap mv, const float *__restrict__ g, const float *__restrict__ beta,
             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
@@ -153,7 +153,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     uint8_t *sm = align1024(smem_raw);
     __shared__ uint64_t bar_ld, bar_mma;
     __shared__ uint32_t tmem_base;
-    __shared__ float s_b[C], s_beta[C], s_bg[C];
+    __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C];
 
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
     ChunkLoc loc;
@@ -164,15 +164,20 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     const int64_t ch = chunk * H + h;
     const int32_t tok0 = (int32_t)loc.start;
     uint8_t *blk = blocks + (size_t)ch * kTcBlock;
-    float *fac = reinterpret_cast<float *>(sm + kPrepFac);
 
+    // gate loads first: their latency overlaps the set-up and the TMA loads
+    float g_in = 0.f, beta_in = 0.f;
+    if (tid < L) {
+        g_in = g[(int64_t)(tok0 + tid) * H + h];
+        beta_in = beta[(int64_t)(tok0 + tid) * H + h];
+    }
     if (tid == 0) {
         mbar_init(&bar_ld, 1);
         mbar_init(&bar_mma, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(&tmem_base, 256);
+        tmem_alloc(&tmem_base, 128);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -191,9 +196,8 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     }
     // Gates (rows >= L: beta = 0, g = 0): in-chunk inclusive cumsum of the log gate.
     if (tid < C) {
-        const bool in = tid < L;
-        s_beta[tid] = in ? beta[(int64_t)(tok0 + tid) * H + h] : 0.f;
-        float x = in ? g[(int64_t)(tok0 + tid) * H + h] : 0.f;
+        s_beta[tid] = beta_in;
+        float x = g_in;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -207,23 +211,54 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     if (tid < C) {
         const bool in = tid < L;
         const float bl = s_b[L - 1], bi = s_b[tid];
+        float *fac = reinterpret_cast<float *>(blk + kBlkFac);
         s_bg[tid] = s_beta[tid] * __expf(bi);
+        s_sg[tid] = in ? scale * __expf(bi) : 0.f;
         fac[kFacW + tid] = in ? __expf(bl - bi) : 0.f;
-        fac[kFacSG + tid] = in ? scale * __expf(bi) : 0.f;
+        fac[kFacSG + tid] = s_sg[tid];
         fac[kFacGL + tid] = tid == 0 ? __expf(bl) : 0.f;  // exp(b_L), then zero padding
     }
+    // In-chunk decay exp(b_i - b_j) for j <= i, computed once (both the Gram
+    // rows and the Q K^T rows use it); it lives in the T area until the solve.
+    for (int e = tid; e < C * C; e += kThreads) {
+        const int i = e >> 6, j = e & 63;
+        if (j <= i) *reinterpret_cast<float *>(sm + kPrepTf + f32_offset(i, j)) = __expf(s_b[i] - s_b[j]);
+    }
+    __syncthreads();
 
     bool ok = mbar_wait(&bar_ld, 0);
-    if (tid == 0 && ok) {
+    if (warp == 0 && __all_sync(0xffffffffu, ok)) {
         tc_fence_after();
-        const uint32_t kq = smem_u32(sm);
+        const uint64_t dkq = sdesc_sw128(smem_u32(sm), 16, 1024);
         const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16(tm, sdesc_sw128(kq + o, 16, 1024), sdesc_sw128(kq + o, 16, 1024), id, kk > 0);
+            const uint64_t o = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_bf16_ss(tm, dkq + o, dkq + o, id, kk > 0);
         }
-        mma_commit(&bar_mma);
+        mma_commit_warp(&bar_mma);
     }
+    // Qs = (scale * exp(b_i)) q_i, the rows of the Q tile rescaled (rows >= L: zero),
+    // written to the workspace with the tile's own byte layout.
+    if (ok) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int e = tid + kThreads * k;            // 16-byte chunk over both 8K blocks
+            const int qb = e >> 9, i = (e & 511) >> 3;   // block, token row
+            const uint32_t off = (uint32_t)((e & 511) << 4);
+            const uint4 src = *reinterpret_cast<const uint4 *>(sm + 8192 + qb * 16384 + off);
+            const float f = s_sg[i];
+            const uint32_t in[4] = {src.x, src.y, src.z, src.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&in[w]);
+                o4[w] = pack_bf16(f * __low2float(b2), f * __high2float(b2));
+            }
+            *reinterpret_cast<uint4 *>(blk + kBlkWQ + 8192 + qb * 16384 + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+    }
+    __syncthreads();  // every thread is done reading Q before A overwrites it
     ok = ok && mbar_wait(&bar_mma, 0);
     tc_fence_after();
 
@@ -234,18 +269,23 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
         const bool is_a = r < C;
         const int i = is_a ? r : r - C;
-        const float bi = s_b[i];
         const float pre = is_a ? s_beta[i] : scale;
         float v0[16], v1[16];
         tmem_ld16(taddr, v0);
         tmem_ld16(taddr + 16, v1);
         tmem_wait_ld();
+        float dec[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 d4 = *reinterpret_cast<const float4 *>(sm + kPrepTf + f32_offset(i, 32 * hf + 4 * q));
+            dec[4 * q] = d4.x; dec[4 * q + 1] = d4.y; dec[4 * q + 2] = d4.z; dec[4 * q + 3] = d4.w;
+        }
         float rr[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int j = 32 * hf + t;
             const bool keep = i < L && (is_a ? j < i : j <= i);
-            rr[t] = keep ? pre * __expf(bi - s_b[j]) * (t < 16 ? v0[t] : v1[t - 16]) : 0.f;
+            rr[t] = keep ? pre * dec[t] * (t < 16 ? v0[t] : v1[t - 16]) : 0.f;
         }
         if (is_a) {
 #pragma unroll
@@ -253,12 +293,12 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
                 *reinterpret_cast<float4 *>(sm + a_offset(i, 32 * hf + 4 * q)) =
                     make_float4(rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
         } else {
-            const uint32_t pimg = smem_u32(sm + kPrepP);
+            uint8_t *pimg = blk + kBlkP;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                st_shared_v4(pimg + sw128_offset(i, 4 * hf + q), pack_bf16(rr[8 * q], rr[8 * q + 1]),
-                             pack_bf16(rr[8 * q + 2], rr[8 * q + 3]), pack_bf16(rr[8 * q + 4], rr[8 * q + 5]),
-                             pack_bf16(rr[8 * q + 6], rr[8 * q + 7]));
+                *reinterpret_cast<uint4 *>(pimg + sw128_offset(i, 4 * hf + q)) =
+                    make_uint4(pack_bf16(rr[8 * q], rr[8 * q + 1]), pack_bf16(rr[8 * q + 2], rr[8 * q + 3]),
+                               pack_bf16(rr[8 * q + 4], rr[8 * q + 5]), pack_bf16(rr[8 * q + 6], rr[8 * q + 7]));
         }
     }
     tc_fence_before();
@@ -369,80 +409,81 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     tc_fence_after();
 
     // W^T = K^T T'^T (M = d_k), U^T = V^T T''^T (M = d_v); K = 64 tokens.
-    if (tid == 0 && ok) {
-        const uint32_t kq = smem_u32(sm), vt = smem_u32(sm + 32768), tp = smem_u32(sm + 8192),
-                       tpp = smem_u32(sm + 24576);
+    if (warp == 0 && __all_sync(0xffffffffu, ok)) {
+        const uint64_t dk = sdesc_sw128(smem_u32(sm), 16384, 1024), dv = sdesc_sw128(smem_u32(sm + 32768), 8192, 1024),
+                       dtp = sdesc_sw128(smem_u32(sm + 8192), 16, 1024), dtpp = sdesc_sw128(smem_u32(sm + 24576), 16, 1024);
         const uint32_t id = idesc_bf16(128, 64, 1, 0);
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tm + 64, sdesc_sw128(kq + kk * 2048, 16384, 1024), sdesc_sw128(tp + kk * 32, 16, 1024), id, kk > 0);
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tm + 128, sdesc_sw128(vt + kk * 2048, 8192, 1024), sdesc_sw128(tpp + kk * 32, 16, 1024), id,
-                     kk > 0);
-        mma_commit(&bar_mma);
-        // P image and gate factors are final: store them while the MMAs run
-        bulk_store(blk + kBlkP, sm + kPrepP, (uint32_t)kTcPImg);
-        bulk_store(blk + kBlkFac, sm + kPrepFac, (uint32_t)kTcFac);
-        bulk_commit();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm, dk + ((kk * 2048) >> 4), dtp + ((kk * 32) >> 4), id, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm + 64, dv + ((kk * 2048) >> 4), dtpp + ((kk * 32) >> 4), id, kk > 0);
+        mma_commit_warp(&bar_mma);
     }
     ok = ok && mbar_wait(&bar_mma, 1);
     tc_fence_after();
 
-    // Epilogue 2: row r (a channel) of W^T and U^T, tokens [32 hf, 32 hf + 32), as
-    // 128-byte-swizzled rows: the W^T image at [0, 16K), the U^T rows at [16K, 32K).
+    // Epilogue 2: thread row r is channel r of W^T and U^T, tokens [32 hf, 32 hf + 32).
+    // W goes out as a K-major operand image (rows = tokens, two 64-channel
+    // blocks), U^T as 128-byte-swizzled rows (row = channel).
     if (ok) {
         const int r = qd * 32 + lane;
         const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
         float w0[16], w1[16], u0[16], u1[16];
-        tmem_ld16(taddr + 64, w0);
-        tmem_ld16(taddr + 64 + 16, w1);
-        tmem_ld16(taddr + 128, u0);
-        tmem_ld16(taddr + 128 + 16, u1);
+        tmem_ld16(taddr, w0);
+        tmem_ld16(taddr + 16, w1);
+        tmem_ld16(taddr + 64, u0);
+        tmem_ld16(taddr + 64 + 16, u1);
         tmem_wait_ld();
-        const uint32_t wimg = smem_u32(sm), uimg = smem_u32(sm + 16384);
+        uint8_t *wimg = blk + kBlkWQ + (r >> 6) * 16384 + (r & 7) * 2;
+        const int wchunk = (r & 63) >> 3;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int i = 32 * hf + t;
+            *reinterpret_cast<__nv_bfloat16 *>(wimg + i * 128 + ((wchunk ^ (i & 7)) << 4)) =
+                __float2bfloat16_rn(t < 16 ? w0[t] : w1[t - 16]);
+        }
+        uint8_t *urow = blk + kBlkU;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float *w = q < 2 ? w0 + 8 * q : w1 + 8 * (q - 2);
             const float *u = q < 2 ? u0 + 8 * q : u1 + 8 * (q - 2);
-            const uint32_t o = sw128_offset(r, 4 * hf + q);
-            st_shared_v4(wimg + o, pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
-            st_shared_v4(uimg + o, pack_bf16(u[0], u[1]), pack_bf16(u[2], u[3]), pack_bf16(u[4], u[5]), pack_bf16(u[6], u[7]));
+            *reinterpret_cast<uint4 *>(urow + sw128_offset(r, 4 * hf + q)) =
+                make_uint4(pack_bf16(u[0], u[1]), pack_bf16(u[2], u[3]), pack_bf16(u[4], u[5]), pack_bf16(u[6], u[7]));
         }
+    } else if (tid == 0) {
+        flag_error(err, 1);
     }
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-        if (ok) {
-            bulk_store(blk + kBlkW, sm, 32768);  // W^T image then U^T rows, contiguous in both places
-            bulk_commit();
-        }
-        bulk_wait_all();
-        if (!ok) flag_error(err, 1);
-    }
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, 256);
+    if (warp == 0) tmem_dealloc(tm, 128);
 }
 
 // ===========================================================================
 // Scan
 // ===========================================================================
-// Shared memory (1024-aligned): two stages of per-chunk operands
-//   [Q tile 16K][K tile 16K][workspace block: W^T image 16K, U^T rows 16K, P image 8K, factors]
-// then the bf16 operands written by the threads: S0 (32K), U' and U'_w (16K each).
-// The U' region also stages full output tiles for the TMA store.
-constexpr uint32_t kStQ = 0, kStK = 16384, kStBlk = 32768, kStage = 75776;
-constexpr uint32_t kStageBytes = 32768 + (uint32_t)kTcBlock;
-constexpr uint32_t kSImg = 2 * kStage, kUpImg = kSImg + 32768, kUwImg = kUpImg + 16384;
-constexpr uint32_t kScanSmem = kUwImg + 16384 + 1024;
+// Shared memory (1024-aligned), three stages of per-chunk operands:
+//   [0, 32K)   [W rows | Qs rows] per 64-channel block: the N = 128 B operand
+//              of S0 [W ; Qs]^T (one bulk copy from the workspace block)
+//   [32K, 48K) K tile (TMA; the MN-major B operand of the state update)
+//   [48K, 72K) U^T rows, P image, gate factors (one bulk copy)
+// The operands the threads produce (S0 and U' in bf16) are written to TMEM
+// and used as A operands straight from there.
+// TMEM columns: [0,256) two buffers of [S0 W^T | S0 Qs^T + U' P^T] (the second
+// half is the chunk's output), [256,384) U'_w K, [384,448) S0, [448,480) U',
+// [480,512) U'_w.  The output of chunk c is read while chunk c+1's first MMAs run.
+constexpr uint32_t kStWQ = 0, kStK = 32768, kStRest = 49152, kStage = 75776;
+constexpr uint32_t kRestU = 0, kRestP = 16384, kRestFac = 24576;
+constexpr uint32_t kStageBytes = (uint32_t)kTcWQ + 16384 + (uint32_t)(kTcBlock - kTcWQ);
+constexpr int kStages = 3;
+constexpr uint32_t kScanSmem = kStages * kStage + 1024;
+constexpr uint32_t kTmD = 0, kTmAcc4 = 256, kTmAS = 384, kTmAUp = 448, kTmAUw = 480;
 
 struct ScanBars {
-    uint64_t full[2];
-    uint64_t mma[4];
+    uint64_t full[kStages];
+    uint64_t mma[3];
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-gdn_scan_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-            const __grid_constant__ CUtensorMap mo, const float *h0, const int32_t *__restrict__ cu,
+gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32_t *__restrict__ cu,
             const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t max_chunks,
             int64_t snap_stride, int64_t n_snap, const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out,
             float *final_state, float *__restrict__ snaps, int *err) {
@@ -462,9 +503,8 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     if (chunk0 + nchunks > max_chunks) nchunks = max_chunks > chunk0 ? max_chunks - chunk0 : 0;
 
     if (tid == 0) {
-        mbar_init(&bars.full[0], 1);
-        mbar_init(&bars.full[1], 1);
-        for (int i = 0; i < 4; ++i) mbar_init(&bars.mma[i], 1);
+        for (int i = 0; i < kStages; ++i) mbar_init(&bars.full[i], 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bars.mma[i], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -476,26 +516,22 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tm = tmem_base;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    const uint32_t acc1 = tm + lane_off, acc2 = tm + 64 + lane_off, acc3 = tm + 128 + lane_off,
-                   acc4 = tm + 256 + lane_off;
 
+    constexpr int kLoader = 128;  // warp 4 lane 0 issues the copies (warp 0 issues the MMAs)
     auto issue_loads = [&](int64_t c) {
-        const int stage = (int)(c & 1);
+        const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
-        const int64_t chh = (chunk0 + c) * H + h;
+        const uint8_t *blk = blocks + (size_t)((chunk0 + c) * H + h) * kTcBlock;
         const int32_t tok = (int32_t)(start + c * C);
         uint64_t *bar = &bars.full[stage];
         mbar_arrive_expect_tx(bar, kStageBytes);
-        tma_load_3d(st + kStQ, &mq, 0, (int32_t)h, tok, bar);
-        tma_load_3d(st + kStQ + 8192, &mq, 64, (int32_t)h, tok, bar);
+        bulk_load(st + kStWQ, blk + kBlkWQ, (uint32_t)kTcWQ, bar);
         tma_load_3d(st + kStK, &mk, 0, (int32_t)h, tok, bar);
         tma_load_3d(st + kStK + 8192, &mk, 64, (int32_t)h, tok, bar);
-        bulk_load(st + kStBlk, blocks + (size_t)chh * kTcBlock, (uint32_t)kTcBlock, bar);
+        bulk_load(st + kStRest, blk + kBlkU, (uint32_t)(kTcBlock - kTcWQ), bar);
     };
-    if (tid == 0) {
-        if (nchunks > 0) issue_loads(0);
-        if (nchunks > 1) issue_loads(1);
-    }
+    if (tid == kLoader)
+        for (int64_t c = 0; c < kStages && c < nchunks; ++c) issue_loads(c);
 
     float S[64];
     const int64_t srow = ((n * H + h) * D + v) * (int64_t)D + 64 * hf;
@@ -510,148 +546,128 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         for (int c = 0; c < 64; ++c) S[c] = 0.f;
     }
 
-    const uint32_t s_img = smem_u32(sm + kSImg), up_img = smem_u32(sm + kUpImg), uw_img = smem_u32(sm + kUwImg);
-    const uint32_t id_w = idesc_bf16(128, 64, 0, 1), id_q = idesc_bf16(128, 64, 0, 0),
-                   id_k = idesc_bf16(128, 128, 0, 1), id_p = idesc_bf16(128, 64, 0, 0);
+    // Output of chunk `c` (tokens [32 hf, 32 hf + 32) of column v): waits for its last MMA.
+    auto emit_output = [&](int64_t c) -> bool {
+        const bool ok_w = mbar_wait(&bars.mma[2], (uint32_t)(c & 1));
+        tc_fence_after();
+        const int L = (int)(len - c * C < C ? len - c * C : C);
+        float o[2][16];
+        const uint32_t dcol = kTmD + (uint32_t)(c & 1) * 128 + 64 + 32 * hf;
+        tmem_ld16(tm + lane_off + dcol, o[0]);
+        tmem_ld16(tm + lane_off + dcol + 16, o[1]);
+        tmem_wait_ld();
+        __nv_bfloat16 *op = out + ((start + c * C + 32 * hf) * H + h) * D + v;
+        const int64_t tstride = H * D;
+#pragma unroll
+        for (int tt = 0; tt < 32; ++tt)
+            if (32 * hf + tt < L) op[tt * tstride] = __float2bfloat16_rn(o[tt >> 4][tt & 15]);
+        return ok_w;
+    };
+
+    const uint32_t id_wq = idesc_bf16(128, 128, 0, 0), id_k = idesc_bf16(128, 128, 0, 1),
+                   id_p = idesc_bf16(128, 64, 0, 0);
     bool ok = true;
     for (int64_t c = 0; c < nchunks; ++c) {
-        const int stage = (int)(c & 1);
+        const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
         const uint32_t st_u = smem_u32(st);
-        const int L = (int)(len - c * C < C ? len - c * C : C);
-        const int64_t tok0 = start + c * C;
         const uint32_t par = (uint32_t)(c & 1);
-        const float *fac = reinterpret_cast<const float *>(st + kStBlk + kBlkFac);
+        const uint32_t dbuf = kTmD + par * 128;
+        const uint8_t *rest = st + kStRest;
+        const float *fac = reinterpret_cast<const float *>(rest + kRestFac);
 
-        // (a) S0 -> bf16 operand, K-major rows v; this thread writes its 64-column block
+        // (a) S0 -> bf16 pairs -> TMEM A operand (this thread: 32 columns of its row)
+        {
+            uint32_t w[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float *s8 = S + q * 8;
-            st_shared_v4(s_img + hf * 16384 + sw128_offset(v, q), pack_bf16(s8[0], s8[1]), pack_bf16(s8[2], s8[3]),
-                         pack_bf16(s8[4], s8[5]), pack_bf16(s8[6], s8[7]));
+            for (int q = 0; q < 2; ++q) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[e] = pack_bf16(S[32 * q + 2 * e], S[32 * q + 2 * e + 1]);
+                tmem_st16u(tm + lane_off + kTmAS + 32 * hf + 16 * q, w);
+            }
+            tmem_wait_st();
         }
-        fence_async_smem();
-        if (tid == 0) bulk_wait_read();  // the previous output tile has left the U' region
-        ok = mbar_wait(&bars.full[stage], (uint32_t)((c >> 1) & 1));
+        ok = mbar_wait(&bars.full[stage], (uint32_t)((c / kStages) & 1)) && ok;
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (__syncthreads_or(!ok)) break;
 
-        // (b) acc1 = S0 W^T, acc2 = S0 Q^T
-        if (tid == 0) {
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16(acc1 - lane_off, sdesc_sw128(s_img + o, 16, 1024),
-                         sdesc_sw128(st_u + kStBlk + kBlkW + kk * 2048, 16384, 1024), id_w, kk > 0);
-            }
-            mma_commit(&bars.mma[0]);
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16(acc2 - lane_off, sdesc_sw128(s_img + o, 16, 1024),
-                         sdesc_sw128(st_u + kStQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_q, kk > 0);
-            }
-            mma_commit(&bars.mma[1]);
+        // (b) D[buf] = S0 [W ; Qs]^T   (N = 128, K = 128): [U-correction | inter-chunk output]
+        if (warp == 0) {
+            const uint64_t bwq = sdesc_sw128(st_u + kStWQ, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_bf16_ts(tm + dbuf, tm + kTmAS + kk * 8, bwq + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                            id_wq, kk > 0);
+            mma_commit_warp(&bars.mma[0]);
         }
+        // the previous chunk's output, while this chunk's MMAs run; after it every MMA of
+        // chunk c-1 has completed, so its stage can take chunk c+2
+        if (c >= 1) ok = emit_output(c - 1) && ok;
+        if (tid == kLoader && c >= 1 && c + kStages - 1 < nchunks) issue_loads(c + kStages - 1);
 
-        // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32); write U' and U' * w as bf16
-        ok = mbar_wait(&bars.mma[0], par);
+        // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32) -> TMEM A operands U', U' * w
+        ok = mbar_wait(&bars.mma[0], par) && ok;
         tc_fence_after();
         {
             float a0[16], a1[16];
-            tmem_ld16(acc1 + 32 * hf, a0);
-            tmem_ld16(acc1 + 32 * hf + 16, a1);
+            tmem_ld16(tm + lane_off + dbuf + 32 * hf, a0);
+            tmem_ld16(tm + lane_off + dbuf + 32 * hf + 16, a1);
             tmem_wait_ld();
-            const uint32_t urow = st_u + kStBlk + kBlkU;
+            uint32_t wu[16], ww[16];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int cq = 4 * hf + q;  // 16-byte chunk = tokens 8 cq .. 8 cq + 7
-                const uint4 u8 = ld_shared_v4(urow + sw128_offset(v, cq));
+                const uint4 u8 = *reinterpret_cast<const uint4 *>(rest + kRestU + sw128_offset(v, cq));
                 const float4 wlo = *reinterpret_cast<const float4 *>(fac + kFacW + 8 * cq);
                 const float4 whi = *reinterpret_cast<const float4 *>(fac + kFacW + 8 * cq + 4);
                 const float wv[8] = {wlo.x, wlo.y, wlo.z, wlo.w, whi.x, whi.y, whi.z, whi.w};
                 const uint32_t uw32[4] = {u8.x, u8.y, u8.z, u8.w};
-                float up[8], uw[8];
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
                     const float acc_lo = (q < 2 ? a0[8 * q + e] : a1[8 * (q - 2) + e]);
                     const float acc_hi = (q < 2 ? a0[8 * q + e + 1] : a1[8 * (q - 2) + e + 1]);
-                    up[e] = __low2float(u2) - acc_lo;
-                    up[e + 1] = __high2float(u2) - acc_hi;
-                    uw[e] = up[e] * wv[e];
-                    uw[e + 1] = up[e + 1] * wv[e + 1];
+                    const float up0 = __low2float(u2) - acc_lo, up1 = __high2float(u2) - acc_hi;
+                    wu[4 * q + e / 2] = pack_bf16(up0, up1);
+                    ww[4 * q + e / 2] = pack_bf16(up0 * wv[e], up1 * wv[e + 1]);
                 }
-                const uint32_t o = sw128_offset(v, cq);
-                st_shared_v4(up_img + o, pack_bf16(up[0], up[1]), pack_bf16(up[2], up[3]), pack_bf16(up[4], up[5]),
-                             pack_bf16(up[6], up[7]));
-                st_shared_v4(uw_img + o, pack_bf16(uw[0], uw[1]), pack_bf16(uw[2], uw[3]), pack_bf16(uw[4], uw[5]),
-                             pack_bf16(uw[6], uw[7]));
             }
+            tmem_st16u(tm + lane_off + kTmAUp + 16 * hf, wu);
+            tmem_st16u(tm + lane_off + kTmAUw + 16 * hf, ww);
+            tmem_wait_st();
         }
-        fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        // (d) acc4 = U'_w K (state increment), acc3 = U' P^T (in-chunk output)
-        if (tid == 0) {
+        // (d) acc4 = U'_w K (state increment, first); D[buf] output half += U' P^T
+        if (warp == 0) {
+            const uint64_t bk = sdesc_sw128(st_u + kStK, 8192, 1024),
+                           bp = sdesc_sw128(st_u + kStRest + kRestP, 16, 1024);
+#pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(acc4 - lane_off, sdesc_sw128(uw_img + kk * 32, 16, 1024),
-                         sdesc_sw128(st_u + kStK + kk * 2048, 8192, 1024), id_k, kk > 0);
-            mma_commit(&bars.mma[2]);
+                mma_bf16_ts(tm + kTmAcc4, tm + kTmAUw + kk * 8, bk + (uint64_t)((kk * 2048) >> 4), id_k, kk > 0);
+            mma_commit_warp(&bars.mma[1]);
+#pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(acc3 - lane_off, sdesc_sw128(up_img + kk * 32, 16, 1024),
-                         sdesc_sw128(st_u + kStBlk + kBlkP + kk * 32, 16, 1024), id_p, kk > 0);
-            mma_commit(&bars.mma[3]);
+                mma_bf16_ts(tm + dbuf + 64, tm + kTmAUp + kk * 8, bp + (uint64_t)((kk * 32) >> 4), id_p, 1);
+            mma_commit_warp(&bars.mma[2]);
         }
 
         // (e) S = gam_L S0 + acc4 (columns [64 hf, 64 hf + 64))
         const float gl = fac[kFacGL];
-        ok = mbar_wait(&bars.mma[2], par) && ok;
-        tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 16) {
-            float a[16];
-            tmem_ld16(acc4 + 64 * hf + c0, a);
-            tmem_wait_ld();
-#pragma unroll
-            for (int t = 0; t < 16; ++t) S[c0 + t] = gl * S[c0 + t] + a[t];
-        }
-
-        // (f) O = scale gam_i (S0 q_i) + (P U')_i for tokens [32 hf, 32 hf + 32)
-        ok = mbar_wait(&bars.mma[1], par) && mbar_wait(&bars.mma[3], par) && ok;
+        ok = mbar_wait(&bars.mma[1], par) && ok;
         tc_fence_after();
         {
-            float a2[32], a3[32];
-            tmem_ld16(acc2 + 32 * hf, *reinterpret_cast<float(*)[16]>(a2));
-            tmem_ld16(acc2 + 32 * hf + 16, *reinterpret_cast<float(*)[16]>(a2 + 16));
-            tmem_ld16(acc3 + 32 * hf, *reinterpret_cast<float(*)[16]>(a3));
-            tmem_ld16(acc3 + 32 * hf + 16, *reinterpret_cast<float(*)[16]>(a3 + 16));
+            float a[4][16];
+#pragma unroll
+            for (int c0 = 0; c0 < 4; ++c0) tmem_ld16(tm + lane_off + kTmAcc4 + 64 * hf + 16 * c0, a[c0]);
             tmem_wait_ld();
-            float o[32];
 #pragma unroll
-            for (int t = 0; t < 32; t += 4) {
-                const float4 sg = *reinterpret_cast<const float4 *>(fac + kFacSG + 32 * hf + t);
-                o[t] = sg.x * a2[t] + a3[t];
-                o[t + 1] = sg.y * a2[t + 1] + a3[t + 1];
-                o[t + 2] = sg.z * a2[t + 2] + a3[t + 2];
-                o[t + 3] = sg.w * a2[t + 3] + a3[t + 3];
-            }
-            if (L == C) {
-                // stage [token][channel] tiles (two 64-channel boxes) in the U' region
-                uint8_t *ot = sm + kUpImg + (v >> 6) * 8192 + (v & 63) * 2;
+            for (int c0 = 0; c0 < 4; ++c0)
 #pragma unroll
-                for (int t = 0; t < 32; ++t)
-                    *reinterpret_cast<__nv_bfloat16 *>(ot + (32 * hf + t) * 128) = __float2bfloat16_rn(o[t]);
-            } else {
-                __nv_bfloat16 *op = out + (tok0 * H + h) * D + v;
-#pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const int i = 32 * hf + t;
-                    if (i < L) op[(int64_t)i * H * D] = __float2bfloat16_rn(o[t]);
-                }
-            }
+                for (int t = 0; t < 16; ++t) S[16 * c0 + t] = gl * S[16 * c0 + t] + a[c0][t];
         }
 
         // snapshot after n * stride tokens of the sequence
@@ -664,29 +680,15 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
                     *reinterpret_cast<float4 *>(dst + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
             }
         }
-
-        // every MMA of this chunk has completed: release the stage, ship the output tile
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            if (L == C) {
-                tma_store_3d(&mo, sm + kUpImg, 0, (int32_t)h, (int32_t)tok0);
-                tma_store_3d(&mo, sm + kUpImg + 8192, 64, (int32_t)h, (int32_t)tok0);
-                bulk_commit();
-            }
-            if (c + 2 < nchunks) issue_loads(c + 2);
-        }
         if (__syncthreads_or(!ok)) break;
     }
+    if (ok && nchunks > 0) ok = emit_output(nchunks - 1) && ok;
     if (!ok && tid == 0) flag_error(err, 2);
     if (ok && final_state) {
-        const int64_t frow = srow;
 #pragma unroll
         for (int cc = 0; cc < 64; cc += 4)
-            *reinterpret_cast<float4 *>(final_state + frow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
+            *reinterpret_cast<float4 *>(final_state + srow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
     }
-    if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
@@ -735,16 +737,14 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     uint8_t *blocks = reinterpret_cast<uint8_t *>(a.ws + p.off_W);
     if (p.H > 65535 || p.max_chunks > 0x7fffffffLL || a.N > 0x7fffffffLL)
         return fail(GDN_ERR_UNSUPPORTED, "grid too large");
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv;
     memset(&mq, 0, sizeof mq);
     memset(&mk, 0, sizeof mk);
     memset(&mv, 0, sizeof mv);
-    memset(&mo, 0, sizeof mo);
     if (p.rows > 0) {
         if ((st = make_map(&mq, a.q, p.rows, p.H, true)) != GDN_OK) return st;
         if ((st = make_map(&mk, a.k, p.rows, p.H, true)) != GDN_OK) return st;
         if ((st = make_map(&mv, a.v, p.rows, p.H, true)) != GDN_OK) return st;
-        if ((st = make_map(&mo, a.out, p.rows, p.H, false)) != GDN_OK) return st;
     }
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -763,7 +763,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         LaunchScope ls("gdn_scan_tc", s);
         gdn_scan_tc<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
-            mq, mk, mo, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap,
+            mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap,
             blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, nullptr);
     }
     return check_launch("gdn_scan_tc");

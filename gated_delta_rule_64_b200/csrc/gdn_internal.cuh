@@ -65,11 +65,14 @@ gdn_status launch_chunk_simt(const ChunkPlan &p, const ChunkArgs &a, int dtype, 
 gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s);
 bool tc_eligible(const gdn_desc &d);
 
-// Per chunk-head workspace block of the tensor-core path (bytes), in this
-// order: the W^T operand image, the U^T rows, the P operand image and the
-// per-token gate factors.  The scan copies each block with one bulk copy.
-constexpr size_t kTcWImg = 128 * 128, kTcUt = 128 * 128, kTcPImg = 64 * 128, kTcFac = 192 * 4;
-constexpr size_t kTcBlock = kTcWImg + kTcUt + kTcPImg + kTcFac;  // 41728
+// Per chunk-head workspace block of the tensor-core path (bytes):
+//   [W (channels 0-63) 8K][Qs (0-63) 8K][W (64-127) 8K][Qs (64-127) 8K]
+//   [U^T rows 16K][P image 8K][gate factors 768]
+// W and Qs = (scale * exp(b_i)) q_i are K-major operand images (rows = tokens)
+// laid out so that [W ; Qs] is one N = 128 operand; the scan copies the block
+// with two bulk copies.
+constexpr size_t kTcWQ = 32768, kTcUt = 128 * 128, kTcPImg = 64 * 128, kTcFac = 192 * 4;
+constexpr size_t kTcBlock = kTcWQ + kTcUt + kTcPImg + kTcFac;  // 58112
 gdn_status launch_decode(const gdn_desc &d, const void *q, const void *k, const void *v,
                          const float *g, const float *beta, float *state, void *out,
                          cudaStream_t s);

@@ -65,7 +65,7 @@ def test_workspace_size(lib):
         return n.value
     simt = 4 * 64 * (128 + 128 + 64 + 1)          # fp32 W, U, P and gate per chunk-head
     assert 6 * 3 * simt <= size(dtype=gdn.GDN_F32) < 6 * 3 * simt + 4096
-    tc = 128 * 128 + 128 * 128 + 64 * 128 + 192 * 4  # bf16 operand images, U^T rows, gate factors
+    tc = 32768 + 128 * 128 + 64 * 128 + 192 * 4  # [W;Qs] image, U^T rows, P image, gate factors
     assert 6 * 3 * tc <= size() < 6 * 3 * tc + 4096
     assert size(dtype=gdn.GDN_F32, gate=gdn.GDN_GATE_CHANNEL) > size(dtype=gdn.GDN_F32)
     d = _desc()
