@@ -556,11 +556,30 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         tmem_ld16(tm + lane_off + dcol, o[0]);
         tmem_ld16(tm + lane_off + dcol + 16, o[1]);
         tmem_wait_ld();
-        __nv_bfloat16 *op = out + ((start + c * C + 32 * hf) * H + h) * D + v;
+        // 4 x 4 transposes among groups of 4 lanes (4 adjacent channels): afterwards
+        // lane j of a group holds those 4 channels of token 4 b + j -> one 8-byte store.
+        const int j4 = lane & 3;
         const int64_t tstride = H * D;
+        __nv_bfloat16 *op = out + ((start + c * C + 32 * hf + j4) * H + h) * D + (v - j4);
 #pragma unroll
-        for (int tt = 0; tt < 32; ++tt)
-            if (32 * hf + tt < L) op[tt * tstride] = __float2bfloat16_rn(o[tt >> 4][tt & 15]);
+        for (int b = 0; b < 8; ++b) {
+            float x0 = o[b >> 2][4 * (b & 3)], x1 = o[b >> 2][4 * (b & 3) + 1], x2 = o[b >> 2][4 * (b & 3) + 2],
+                  x3 = o[b >> 2][4 * (b & 3) + 3];
+            {
+                const bool hi = lane & 1;
+                const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x1, 1);
+                const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x2 : x3, 1);
+                if (hi) { x0 = r0; x2 = r1; } else { x1 = r0; x3 = r1; }
+            }
+            {
+                const bool hi = lane & 2;
+                const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x2, 2);
+                const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x1 : x3, 2);
+                if (hi) { x0 = r0; x1 = r1; } else { x2 = r0; x3 = r1; }
+            }
+            if (32 * hf + 4 * b + j4 < L)
+                *reinterpret_cast<uint2 *>(op + (int64_t)(4 * b) * tstride) = make_uint2(pack_bf16(x0, x1), pack_bf16(x2, x3));
+        }
         return ok_w;
     };
 
@@ -641,14 +660,16 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         __syncthreads();
         tc_fence_after();
 
-        // (d) acc4 = U'_w K (state increment, first); D[buf] output half += U' P^T
+        // (d) acc4 = U'_w K (state increment; warp 0) and, from warp 1 at the same time,
+        // D[buf] output half += U' P^T
         if (warp == 0) {
-            const uint64_t bk = sdesc_sw128(st_u + kStK, 8192, 1024),
-                           bp = sdesc_sw128(st_u + kStRest + kRestP, 16, 1024);
+            const uint64_t bk = sdesc_sw128(st_u + kStK, 8192, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ts(tm + kTmAcc4, tm + kTmAUw + kk * 8, bk + (uint64_t)((kk * 2048) >> 4), id_k, kk > 0);
             mma_commit_warp(&bars.mma[1]);
+        } else if (warp == 1) {
+            const uint64_t bp = sdesc_sw128(st_u + kStRest + kRestP, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ts(tm + dbuf + 64, tm + kTmAUp + kk * 8, bp + (uint64_t)((kk * 32) >> 4), id_p, 1);
