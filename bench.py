@@ -215,18 +215,35 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def kernel_source_hash(path: str, name: str):
+    """sha256 of the source text of the __global__ function `name` in `path`."""
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    i = text.find(f"\n{name}(")
+    if i < 0:
+        i = text.find(f" {name}(")
+    if i < 0:
+        return None
+    start = text.rfind("__global__", 0, i)
+    end = text.find("\n}\n", i)
+    if start < 0 or end < 0:
+        return None
+    return hashlib.sha256(text[start:end].encode()).hexdigest()
+
+
 def traffic_for(kernel: str):
-    """ncu DRAM bytes per launch recorded for `kernel`, if its source is unchanged."""
+    """ncu DRAM bytes (read + write) per launch recorded in profiles/traffic.json for
+    `kernel` on the benchmark workload, or None when the kernel's source changed."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     rec = json.load(open(p)).get(kernel)
     if not rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+    if kernel_source_hash(os.path.join(ROOT, rec["source"]), kernel) != rec["sha256"]:
         return None
-    return rec["bytes_per_launch"] * rec.get("scale_to_bench", 1.0)
+    return float(rec["bytes_per_launch"])
 
 
 def run_gpu(args):
@@ -290,23 +307,27 @@ def run_gpu(args):
     tokens_all = B * T * world
     value = tokens_all / (ms_step * 1e-3)
 
-    # dominant kernel roofline (HBM-bound by arithmetic intensity)
-    top = max(kernels.items(), key=lambda kv: kv[1][1]) if kernels else ("none", (1, 0.0))
-    top_name, (top_launches, top_ms) = top
-    per_launch_s = top_ms / max(1, top_launches) * 1e-3
+    # Roofline of the prefill step.  The step is two kernels (chunk-local prep of
+    # every chunk in parallel, then the in-order scan); neither moves the path's
+    # algorithmic bytes on its own, so the HBM roofline is taken over both.
     head_tokens = B * T * H
     alg_bytes = head_tokens * PREFILL_BYTES_PER_HEAD_TOKEN + 2 * B * H * STATE_BYTES
     alg_flops = head_tokens * PREFILL_FLOPS_PER_HEAD_TOKEN
-    achieved = alg_bytes / per_launch_s / 1e9 if per_launch_s > 0 else 0.0
+    per_launch = {n: t / max(1, c) * 1e-3 for n, (c, t) in kernels.items()}
+    step_kernel_s = sum(per_launch.values()) or ms_step * 1e-3
+    achieved = alg_bytes / step_kernel_s / 1e9
+    traffics = [traffic_for(n) for n in per_launch]
+    traffic = sum(traffics) if traffics and all(t is not None for t in traffics) else None
+    top_name = max(per_launch, key=per_launch.get) if per_launch else "none"
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(top_name), "kernel": top_name,
-                "peak_source": f"{pk['source']} hbm_gbs",
-                "tensor": {"achieved_tflops": alg_flops / per_launch_s / 1e12 if per_launch_s > 0 else 0.0,
-                           "peak": pk["bf16_tflops"],
-                           "frac": (alg_flops / per_launch_s / 1e12) / pk["bf16_tflops"] if per_launch_s > 0 else 0},
-                "step": {"achieved_gbs": alg_bytes / (ms_step * 1e-3) / 1e9,
-                         "frac_hbm": alg_bytes / (ms_step * 1e-3) / 1e9 / pk["hbm_gbs"]},
-                "kernels_ms_per_step": {n: t / args.steps for n, (c, t) in kernels.items()}}
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                "kernel": " + ".join(sorted(per_launch)) + " (one prefill step)",
+                "algorithmic_bytes": alg_bytes, "peak_source": f"{pk['source']} hbm_gbs (burst copy)",
+                "tensor": {"achieved_tflops": alg_flops / step_kernel_s / 1e12, "peak": pk["bf16_tflops"],
+                           "frac": alg_flops / step_kernel_s / 1e12 / pk["bf16_tflops"]},
+                "kernels": {n: {"us_per_launch": per_launch[n] * 1e6, "share": per_launch[n] / step_kernel_s,
+                                "traffic": traffic_for(n)} for n in per_launch},
+                "dominant_kernel": top_name}
     launches = sum(c for c, _ in kernels.values())
 
     # ---------------- e2e through the public API with host buffers ----------------
@@ -402,6 +423,26 @@ def run_gpu(args):
     return 0
 
 
+def run_profile(which: str) -> int:
+    import torch
+
+    from gated_delta_rule_64_b200 import gdn
+    from gated_delta_rule_64_b200.inputs import DECODE, PREFILL_BF16, make_inputs
+    d = lambda t: t.cuda()
+    if which == "prefill":
+        x = make_inputs(PREFILL_BF16)
+        q, k, v, g, b, h0 = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0)
+        for _ in range(3):
+            gdn.gdn_chunk_fwd(q, k, v, g, b, h0)
+    else:
+        x = make_inputs(DECODE.replace(decode_steps=3))
+        st = d(x.h0)
+        for s in range(3):
+            gdn.gdn_decode_step(d(x.q[s]), d(x.k[s]), d(x.v[s]), d(x.g[s]), d(x.beta[s]), st)
+    torch.cuda.synchronize()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -409,7 +450,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["prefill", "decode"],
+                    help="run three calls of one workload and exit (for ncu captures; prints nothing to time)")
     args = ap.parse_args(argv)
+    if args.profile:
+        return run_profile(args.profile)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
