@@ -43,36 +43,13 @@
 
 #include <mutex>
 
-#include "chunk_common.cuh"
-#include "gdn_internal.cuh"
-#include "sm100.cuh"
+#include "tc_common.cuh"
 
 namespace gdn {
 namespace {
 
 using namespace sm100;
-
-constexpr int C = kChunk;  // 64
-constexpr int D = 128;     // d_k = d_v
-constexpr int kThreads = 256;
-
-// Offsets inside one workspace block (see kTcBlock).
-constexpr uint32_t kBlkWQ = 0, kBlkU = 32768, kBlkP = 49152, kBlkFac = 57344;
-// Gate factors: [0, 64) w_i = exp(b_L - b_i); [64, 128) scale * exp(b_i); [128] exp(b_L).
-constexpr int kFacW = 0, kFacSG = 64, kFacGL = 128;
-
-__device__ __forceinline__ void flag_error(int *err, int code) {
-    if (err) atomicCAS(err, 0, code);
-}
-
-__device__ __forceinline__ uint8_t *align1024(unsigned char *p) {
-    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// fp32 64 x 64 matrix, rows of 256 bytes, 16-byte chunks rotated per row (conflict-free row/column access).
-__device__ __forceinline__ uint32_t f32_offset(int i, int j) {
-    return (uint32_t)i * 256u + (uint32_t)((((j >> 2) ^ (i & 15)) << 4) + (j & 3) * 4);
-}
+using namespace tc;
 
 // ===========================================================================
 // Prep
@@ -94,54 +71,6 @@ constexpr uint32_t kPrepSmem = kPrepY + 4096 + 1024;
 __device__ __forceinline__ uint32_t a_offset(int i, int j) {
     // A (fp32) in the Q rows of the first operand: rows 0..31 at 8K, 32..63 at 24K
     return (i < 32 ? 8192u : 24576u) + f32_offset(i & 31, j);
-}
-
-// C (16x16) = sum over `nk` 16-wide K blocks of X_k (16x16) * Y_k (16x16); X and Y
-// are fp32 blocks in shared memory given by their (row, col) origins and an
-// offset function.  Warp-level m16n8k8 tf32 MMAs, fp32 accumulate; the fp32
-// bit patterns are passed as they are (the tensor core reads them as tf32,
-// dropping the low mantissa bits).  The result is returned in the MMA
-// accumulator layout: c[nt][0..3] for the 8-column tiles nt = 0, 1.
-template <typename OffX, typename OffY>
-__device__ __forceinline__ void warp_gemm16(const uint8_t *base, int nk, const int *xr, const int *xc, const int *yr,
-                                            const int *yc, OffX offx, OffY offy, float (&c)[2][4]) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
-    for (int kb = 0; kb < nk; ++kb) {
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            const int k0 = ks * 8;
-            uint32_t a[4];
-            a[0] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g, xc[kb] + k0 + t));
-            a[1] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t));
-            a[2] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g, xc[kb] + k0 + t + 4));
-            a[3] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t + 4));
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                uint32_t b[2];
-                b[0] = *reinterpret_cast<const uint32_t *>(base + offy(yr[kb] + k0 + t, yc[kb] + nt * 8 + g));
-                b[1] = *reinterpret_cast<const uint32_t *>(base + offy(yr[kb] + k0 + t + 4, yc[kb] + nt * 8 + g));
-                mma_tf32_16x8x8(c[nt], a, b);
-            }
-        }
-    }
-}
-
-// Store a 16x16 accumulator (times `sign`) at (r0, c0) through the offset function.
-template <typename Off>
-__device__ __forceinline__ void warp_store16(uint8_t *base, int r0, int c0, const float (&c)[2][4], float sign, Off off) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int col = c0 + nt * 8 + 2 * t;
-        *reinterpret_cast<float *>(base + off(r0 + g, col)) = sign * c[nt][0];
-        *reinterpret_cast<float *>(base + off(r0 + g, col + 1)) = sign * c[nt][1];
-        *reinterpret_cast<float *>(base + off(r0 + g + 8, col)) = sign * c[nt][2];
-        *reinterpret_cast<float *>(base + off(r0 + g + 8, col + 1)) = sign * c[nt][3];
-    }
 }
 
 __global__ void __launch_bounds__(kThreads, 3)
@@ -306,78 +235,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
 
     // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks.
     uint8_t *Tf = sm + kPrepTf;
-    auto offA = [](int i, int j) { return a_offset(i, j); };
-    auto offT = [](int i, int j) { return kPrepTf + f32_offset(i, j); };
-    auto offY = [](int i, int j) { return kPrepY + (uint32_t)i * 64u + (uint32_t)j * 4u; };  // 4 blocks, rows of 16
-    if (ok) {
-        if (warp < 4) {
-            // diagonal block p: column `col` of (I + A_pp)^-1 by forward substitution (fp32)
-            const int p = warp, col = lane & 15;
-            float x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float acc = 0.f;
-#pragma unroll
-                for (int j = 0; j < i; ++j)
-                    acc += *reinterpret_cast<const float *>(sm + a_offset(16 * p + i, 16 * p + j)) * x[j];
-                x[i] = (i == col) ? 1.f : -acc;
-            }
-            if (lane < 16)
-#pragma unroll
-                for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(Tf + f32_offset(16 * p + i, 16 * p + col)) = x[i];
-        } else {
-            // zero the strictly upper off-diagonal blocks
-            for (int e = tid - 128; e < 6 * 256; e += 128) {
-                const int b = e >> 8, w = e & 255;
-                const int pb = b < 3 ? 0 : (b < 5 ? 1 : 2);
-                const int qb = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
-                *reinterpret_cast<float *>(Tf + f32_offset(16 * pb + (w >> 4), 16 * qb + (w & 15))) = 0.f;
-            }
-        }
-    }
-    __syncthreads();
-    // level 1: T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
-    if (ok && warp < 2) {
-        const int p = 2 * warp + 1, q = 2 * warp;
-        float c[2][4];
-        const int xr[1] = {16 * p}, xc[1] = {16 * q}, yr[1] = {16 * q}, yc[1] = {16 * q};
-        warp_gemm16(sm, 1, xr, xc, yr, yc, offA, offT, c);
-        warp_store16(sm, 16 * warp, 0, c, 1.f, offY);
-        __syncwarp();
-        const int xr2[1] = {16 * p}, xc2[1] = {16 * p}, yr2[1] = {16 * warp}, yc2[1] = {0};
-        warp_gemm16(sm, 1, xr2, xc2, yr2, yc2, offT, offY, c);
-        warp_store16(sm, 16 * p, 16 * q, c, -1.f, offT);
-    }
-    __syncthreads();
-    // level 2, step 1: Y_pq = sum_{r in {0,1}} A_pr T_rq for p in {2,3}, q in {0,1}
-    if (ok && warp < 4) {
-        const int p = 2 + (warp >> 1), q = warp & 1;
-        float c[2][4];
-        if (q == 0) {
-            const int xr[2] = {16 * p, 16 * p}, xc[2] = {0, 16}, yr[2] = {0, 16}, yc[2] = {0, 0};
-            warp_gemm16(sm, 2, xr, xc, yr, yc, offA, offT, c);
-        } else {
-            const int xr[1] = {16 * p}, xc[1] = {16}, yr[1] = {16}, yc[1] = {16};
-            warp_gemm16(sm, 1, xr, xc, yr, yc, offA, offT, c);
-        }
-        warp_store16(sm, 16 * warp, 0, c, 1.f, offY);
-    }
-    __syncthreads();
-    // level 2, step 2: T_pq = -sum_{r in {2,3}, r <= p} T_pr Y_rq
-    if (ok && warp < 4) {
-        const int p = 2 + (warp >> 1), q = warp & 1;
-        float c[2][4];
-        // Y_rq lives in scratch block (r - 2) * 2 + q
-        if (p == 2) {
-            const int xr[1] = {32}, xc[1] = {32}, yr[1] = {16 * (0 * 2 + q)}, yc[1] = {0};
-            warp_gemm16(sm, 1, xr, xc, yr, yc, offT, offY, c);
-        } else {
-            const int xr[2] = {48, 48}, xc[2] = {32, 48}, yr[2] = {16 * (0 * 2 + q), 16 * (1 * 2 + q)}, yc[2] = {0, 0};
-            warp_gemm16(sm, 2, xr, xc, yr, yc, offT, offY, c);
-        }
-        warp_store16(sm, 16 * p, 16 * q, c, -1.f, offT);
-    }
-    __syncthreads();
+    blocked_solve<kPrepTf, kPrepY>(sm, [](int i, int j) { return a_offset(i, j); }, ok);
 
     // T' = T diag(beta gam), T'' = T diag(beta) as bf16 operand images (K-major rows i).
     if (ok) {
@@ -426,29 +284,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     // W goes out as a K-major operand image (rows = tokens, two 64-channel
     // blocks), U^T as 128-byte-swizzled rows (row = channel).
     if (ok) {
-        const int r = qd * 32 + lane;
-        const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
-        float w0[16], w1[16], u0[16], u1[16];
-        tmem_ld16(taddr, w0);
-        tmem_ld16(taddr + 16, w1);
-        tmem_ld16(taddr + 64, u0);
-        tmem_ld16(taddr + 64 + 16, u1);
-        tmem_wait_ld();
-        uint8_t *wimg = blk + kBlkWQ + (r >> 6) * 16384 + (r & 7) * 2;
-        const int wchunk = (r & 63) >> 3;
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int i = 32 * hf + t;
-            *reinterpret_cast<__nv_bfloat16 *>(wimg + i * 128 + ((wchunk ^ (i & 7)) << 4)) =
-                __float2bfloat16_rn(t < 16 ? w0[t] : w1[t - 16]);
-        }
-        uint8_t *urow = blk + kBlkU;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float *u = q < 2 ? u0 + 8 * q : u1 + 8 * (q - 2);
-            *reinterpret_cast<uint4 *>(urow + sw128_offset(r, 4 * hf + q)) =
-                make_uint4(pack_bf16(u[0], u[1]), pack_bf16(u[2], u[3]), pack_bf16(u[4], u[5]), pack_bf16(u[6], u[7]));
-        }
+        store_wu(tm, blk, qd, hf, lane);
     } else if (tid == 0) {
         flag_error(err, 1);
     }
@@ -472,7 +308,12 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
 // [480,512) U'_w.  The output of chunk c is read while chunk c+1's first MMAs run.
 constexpr uint32_t kStWQ = 0, kStK = 32768, kStRest = 49152, kStage = 75776;
 constexpr uint32_t kRestU = 0, kRestP = 16384, kRestFac = 24576;
-constexpr uint32_t kStageBytes = (uint32_t)kTcWQ + 16384 + (uint32_t)(kTcBlock - kTcWQ);
+// bytes of the [U, P, factors] part of a block, and of one stage's copies
+template <bool KDA> constexpr uint32_t rest_bytes() {
+    return KDA ? (uint32_t)(kTcUt + kTcPImg + kTcFacKda) : (uint32_t)(kTcBlock - kTcWQ);
+}
+template <bool KDA> constexpr uint32_t stage_bytes() { return (uint32_t)kTcWQ + 16384 + rest_bytes<KDA>(); }
+static_assert(kStRest + rest_bytes<true>() <= kStage && kStRest + rest_bytes<false>() <= kStage, "stage layout");
 constexpr int kStages = 3;
 constexpr uint32_t kScanSmem = kStages * kStage + 1024;
 constexpr uint32_t kTmD = 0, kTmAcc4 = 256, kTmAS = 384, kTmAUp = 448, kTmAUw = 480;
@@ -482,6 +323,10 @@ struct ScanBars {
     uint64_t mma[3];
 };
 
+// KDA: per-channel gate.  The state-update operand is then K~ from the block
+// (instead of the K tile), U'_w = U', and the carried state is scaled per key
+// channel by exp(b_L).
+template <bool KDA>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32_t *__restrict__ cu,
             const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t max_chunks,
@@ -521,14 +366,18 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
     auto issue_loads = [&](int64_t c) {
         const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
-        const uint8_t *blk = blocks + (size_t)((chunk0 + c) * H + h) * kTcBlock;
+        const uint8_t *blk = blocks + (size_t)((chunk0 + c) * H + h) * (KDA ? kTcBlockKda : kTcBlock);
         const int32_t tok = (int32_t)(start + c * C);
         uint64_t *bar = &bars.full[stage];
-        mbar_arrive_expect_tx(bar, kStageBytes);
+        mbar_arrive_expect_tx(bar, stage_bytes<KDA>());
         bulk_load(st + kStWQ, blk + kBlkWQ, (uint32_t)kTcWQ, bar);
-        tma_load_3d(st + kStK, &mk, 0, (int32_t)h, tok, bar);
-        tma_load_3d(st + kStK + 8192, &mk, 64, (int32_t)h, tok, bar);
-        bulk_load(st + kStRest, blk + kBlkU, (uint32_t)(kTcBlock - kTcWQ), bar);
+        if (KDA) {
+            bulk_load(st + kStK, blk + kBlkKt, (uint32_t)kTcKt, bar);
+        } else {
+            tma_load_3d(st + kStK, &mk, 0, (int32_t)h, tok, bar);
+            tma_load_3d(st + kStK + 8192, &mk, 64, (int32_t)h, tok, bar);
+        }
+        bulk_load(st + kStRest, blk + kBlkU, rest_bytes<KDA>(), bar);
     };
     if (tid == kLoader)
         for (int64_t c = 0; c < kStages && c < nchunks; ++c) issue_loads(c);
@@ -676,7 +525,7 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
             mma_commit_warp(&bars.mma[2]);
         }
 
-        // (e) S = gam_L S0 + acc4 (columns [64 hf, 64 hf + 64))
+        // (e) S = gam_L S0 + acc4 (columns [64 hf, 64 hf + 64)); per key channel for KDA
         const float gl = fac[kFacGL];
         ok = mbar_wait(&bars.mma[1], par) && ok;
         tc_fence_after();
@@ -685,10 +534,22 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
 #pragma unroll
             for (int c0 = 0; c0 < 4; ++c0) tmem_ld16(tm + lane_off + kTmAcc4 + 64 * hf + 16 * c0, a[c0]);
             tmem_wait_ld();
+            if (KDA) {
+                const float4 *gl4 = reinterpret_cast<const float4 *>(fac + kFacGL + 64 * hf);
 #pragma unroll
-            for (int c0 = 0; c0 < 4; ++c0)
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const float4 f = gl4[c4];
+                    S[4 * c4] = f.x * S[4 * c4] + a[c4 >> 2][(4 * c4) & 15];
+                    S[4 * c4 + 1] = f.y * S[4 * c4 + 1] + a[c4 >> 2][(4 * c4 + 1) & 15];
+                    S[4 * c4 + 2] = f.z * S[4 * c4 + 2] + a[c4 >> 2][(4 * c4 + 2) & 15];
+                    S[4 * c4 + 3] = f.w * S[4 * c4 + 3] + a[c4 >> 2][(4 * c4 + 3) & 15];
+                }
+            } else {
 #pragma unroll
-                for (int t = 0; t < 16; ++t) S[16 * c0 + t] = gl * S[16 * c0 + t] + a[c0][t];
+                for (int c0 = 0; c0 < 4; ++c0)
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) S[16 * c0 + t] = gl * S[16 * c0 + t] + a[c0][t];
+            }
         }
 
         // snapshot after n * stride tokens of the sequence
@@ -748,7 +609,7 @@ gdn_status make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t H, b
 }  // namespace
 
 bool tc_eligible(const gdn_desc &d) {
-    return d.dtype == GDN_BF16 && d.dk == 128 && d.dv == 128 && d.gate == GDN_GATE_HEAD;
+    return d.dtype == GDN_BF16 && d.dk == 128 && d.dv == 128 && (d.gate == GDN_GATE_HEAD || d.gate == GDN_GATE_CHANNEL);
 }
 
 gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s) {
@@ -772,18 +633,27 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     std::call_once(attr_once, [] {
         attr_err = cudaFuncSetAttribute(gdn_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrepSmem);
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(gdn_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
+            attr_err = cudaFuncSetAttribute(gdn_scan_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)kScanSmem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(gdn_scan_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)kScanSmem);
     });
     if (attr_err != cudaSuccess) return fail(GDN_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(attr_err));
     if (p.max_chunks > 0 && p.rows > 0) {
-        LaunchScope ls("gdn_prep_tc", s);
-        gdn_prep_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kPrepSmem, s>>>(
-            mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.scale, blocks, nullptr);
+        if (p.per_channel) {
+            if ((st = tc::launch_prep_kda(mq, mk, mv, p, a, off, blocks, s)) != GDN_OK) return st;
+        } else {
+            LaunchScope ls("gdn_prep_tc", s);
+            gdn_prep_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kPrepSmem, s>>>(
+                mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.scale, blocks, nullptr);
+            if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
+        }
     }
-    if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
     {
         LaunchScope ls("gdn_scan_tc", s);
-        gdn_scan_tc<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
+        auto kern = p.per_channel ? gdn_scan_tc<true> : gdn_scan_tc<false>;
+        kern<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
             mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap,
             blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, nullptr);
     }

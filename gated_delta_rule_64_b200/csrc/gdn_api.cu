@@ -104,8 +104,9 @@ ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed) {
     p.off_chunk_offsets = off;
     off = align_up(off + sizeof(int32_t) * (size_t)(p.N + 1), 256);
     if (p.tc) {
-        p.off_W = p.off_U = p.off_P = p.off_b = off;  // one block of kTcBlock bytes per chunk-head
-        off = align_up(off + kTcBlock * (size_t)ch, 256);
+        p.tc_block = p.per_channel ? kTcBlockKda : kTcBlock;
+        p.off_W = p.off_U = p.off_P = p.off_b = off;  // one block of tc_block bytes per chunk-head
+        off = align_up(off + p.tc_block * (size_t)ch, 256);
     } else {
         p.off_W = off;
         off = align_up(off + sizeof(float) * (size_t)ch * kChunk * p.dk, 256);

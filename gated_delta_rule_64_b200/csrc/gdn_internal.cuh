@@ -36,7 +36,8 @@ struct ChunkPlan {
     int64_t max_chunks;  // upper bound on sum_n ceil(len_n / 64)
     bool packed;
     bool per_channel;
-    bool tc;             // tensor-core path (bf16, d_k = d_v = 128, one gate per head)
+    bool tc;             // tensor-core path (bf16, d_k = d_v = 128)
+    size_t tc_block;     // bytes per chunk-head of the tensor-core workspace
     // byte offsets into the workspace
     size_t off_chunk_offsets;  // int32 (N+1): first global chunk index of each sequence
     size_t off_W, off_U, off_P, off_b;
@@ -70,9 +71,14 @@ bool tc_eligible(const gdn_desc &d);
 //   [U^T rows 16K][P image 8K][gate factors 768]
 // W and Qs = (scale * exp(b_i)) q_i are K-major operand images (rows = tokens)
 // laid out so that [W ; Qs] is one N = 128 operand; the scan copies the block
-// with two bulk copies.
+// with two bulk copies.  The per-channel gate's block has 1 KB of gate
+// factors and adds K~ = K * exp(b_L - b) (16K, the layout of a K tile), the
+// operand of its state update:
+//   [W|Qs 32K][U^T rows 16K][P image 8K][gate factors 1K][K~ 16K]
 constexpr size_t kTcWQ = 32768, kTcUt = 128 * 128, kTcPImg = 64 * 128, kTcFac = 192 * 4;
 constexpr size_t kTcBlock = kTcWQ + kTcUt + kTcPImg + kTcFac;  // 58112
+constexpr size_t kTcFacKda = 256 * 4, kTcKt = 64 * 128 * 2;
+constexpr size_t kTcBlockKda = kTcWQ + kTcUt + kTcPImg + kTcFacKda + kTcKt;  // 74752
 gdn_status launch_decode(const gdn_desc &d, const void *q, const void *k, const void *v,
                          const float *g, const float *beta, float *state, void *out,
                          cudaStream_t s);

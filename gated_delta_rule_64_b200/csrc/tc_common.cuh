@@ -1,0 +1,210 @@
+// Pieces shared by the tensor-core prefill kernels (one gate per head, and the
+// per-channel gate): workspace block layout, the blocked solve of the
+// unit-lower-triangular chunk system and the W/U epilogue.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include "chunk_common.cuh"
+#include "gdn_internal.cuh"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace tc {
+
+using namespace sm100;
+
+constexpr int C = kChunk;  // 64 tokens per chunk
+constexpr int D = 128;     // d_k = d_v
+constexpr int kThreads = 256;
+
+// Offsets inside one workspace block (kTcBlock bytes for the per-head gate,
+// kTcBlockKda for the per-channel gate, whose block adds K~ at the end).
+constexpr uint32_t kBlkWQ = 0, kBlkU = 32768, kBlkP = 49152, kBlkFac = 57344;
+constexpr uint32_t kBlkKt = kBlkFac + (uint32_t)kTcFacKda;  // per-channel gate only
+// Gate factors (floats):
+//   per-head gate:    [0, 64) w_i = exp(b_L - b_i); [64, 128) scale exp(b_i); [128] exp(b_L)
+//   per-channel gate: [0, 64) w_i = 1 (0 past the chunk end); [128, 256) exp(b_L) per key channel
+constexpr int kFacW = 0, kFacSG = 64, kFacGL = 128;
+
+__device__ __forceinline__ void flag_error(int *err, int code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+__device__ __forceinline__ uint8_t *align1024(unsigned char *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// fp32 64 x 64 matrix, rows of 256 bytes, 16-byte chunks rotated per row (conflict-free row/column access).
+__device__ __forceinline__ uint32_t f32_offset(int i, int j) {
+    return (uint32_t)i * 256u + (uint32_t)((((j >> 2) ^ (i & 15)) << 4) + (j & 3) * 4);
+}
+
+// C (16x16) = sum over `nk` 16-wide K blocks of X_k (16x16) * Y_k (16x16); X and Y
+// are fp32 blocks in shared memory given by their (row, col) origins and an
+// offset function.  Warp-level m16n8k8 tf32 MMAs, fp32 accumulate; the fp32
+// bit patterns are passed as they are (the tensor core reads them as tf32,
+// dropping the low mantissa bits).  The result is returned in the MMA
+// accumulator layout: c[nt][0..3] for the 8-column tiles nt = 0, 1.
+template <typename OffX, typename OffY>
+__device__ __forceinline__ void warp_gemm16(const uint8_t *base, int nk, const int *xr, const int *xc, const int *yr,
+                                            const int *yc, OffX offx, OffY offy, float (&c)[2][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+    for (int kb = 0; kb < nk; ++kb) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const int k0 = ks * 8;
+            uint32_t a[4];
+            a[0] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g, xc[kb] + k0 + t));
+            a[1] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t));
+            a[2] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g, xc[kb] + k0 + t + 4));
+            a[3] = *reinterpret_cast<const uint32_t *>(base + offx(xr[kb] + g + 8, xc[kb] + k0 + t + 4));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t b[2];
+                b[0] = *reinterpret_cast<const uint32_t *>(base + offy(yr[kb] + k0 + t, yc[kb] + nt * 8 + g));
+                b[1] = *reinterpret_cast<const uint32_t *>(base + offy(yr[kb] + k0 + t + 4, yc[kb] + nt * 8 + g));
+                mma_tf32_16x8x8(c[nt], a, b);
+            }
+        }
+    }
+}
+
+// Store a 16x16 accumulator (times `sign`) at (r0, c0) through the offset function.
+template <typename Off>
+__device__ __forceinline__ void warp_store16(uint8_t *base, int r0, int c0, const float (&c)[2][4], float sign, Off off) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int col = c0 + nt * 8 + 2 * t;
+        *reinterpret_cast<float *>(base + off(r0 + g, col)) = sign * c[nt][0];
+        *reinterpret_cast<float *>(base + off(r0 + g, col + 1)) = sign * c[nt][1];
+        *reinterpret_cast<float *>(base + off(r0 + g + 8, col)) = sign * c[nt][2];
+        *reinterpret_cast<float *>(base + off(r0 + g + 8, col + 1)) = sign * c[nt][3];
+    }
+}
+
+// T = (I + A)^-1 for the 64 x 64 strictly lower A of a chunk, in 16 x 16 blocks.
+// A is read through `offA` (only its strictly lower part: the diagonal blocks
+// below their diagonal and the blocks below the block diagonal); T is written
+// in fp32 at byte offset TF of `sm` (f32_offset layout, upper blocks zeroed);
+// TY is 4 KB of scratch.  Diagonal blocks: forward substitution in fp32 (one
+// column per lane); off-diagonal blocks by the block recurrence
+// T_pq = -T_pp sum_{q <= r < p} A_pr T_rq with tf32 warp MMAs.  Every thread
+// of the block calls it (it synchronises internally).
+template <uint32_t TF, uint32_t TY, typename OffA>
+__device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto offT = [](int i, int j) { return TF + f32_offset(i, j); };
+    auto offY = [](int i, int j) { return TY + (uint32_t)i * 64u + (uint32_t)j * 4u; };  // 4 blocks, rows of 16
+    if (ok) {
+        if (warp < 4) {
+            // diagonal block p: column `col` of (I + A_pp)^-1 by forward substitution (fp32)
+            const int p = warp, col = lane & 15;
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < i; ++j) acc += *reinterpret_cast<const float *>(sm + offA(16 * p + i, 16 * p + j)) * x[j];
+                x[i] = (i == col) ? 1.f : -acc;
+            }
+            if (lane < 16)
+#pragma unroll
+                for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + offT(16 * p + i, 16 * p + col)) = x[i];
+        } else {
+            // zero the strictly upper off-diagonal blocks
+            for (int e = tid - 128; e < 6 * 256; e += 128) {
+                const int b = e >> 8, w = e & 255;
+                const int pb = b < 3 ? 0 : (b < 5 ? 1 : 2);
+                const int qb = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
+                *reinterpret_cast<float *>(sm + offT(16 * pb + (w >> 4), 16 * qb + (w & 15))) = 0.f;
+            }
+        }
+    }
+    __syncthreads();
+    // level 1: T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
+    if (ok && warp < 2) {
+        const int p = 2 * warp + 1, q = 2 * warp;
+        float c[2][4];
+        const int xr[1] = {16 * p}, xc[1] = {16 * q}, yr[1] = {16 * q}, yc[1] = {16 * q};
+        warp_gemm16(sm, 1, xr, xc, yr, yc, offA, offT, c);
+        warp_store16(sm, 16 * warp, 0, c, 1.f, offY);
+        __syncwarp();
+        const int xr2[1] = {16 * p}, xc2[1] = {16 * p}, yr2[1] = {16 * warp}, yc2[1] = {0};
+        warp_gemm16(sm, 1, xr2, xc2, yr2, yc2, offT, offY, c);
+        warp_store16(sm, 16 * p, 16 * q, c, -1.f, offT);
+    }
+    __syncthreads();
+    // level 2, step 1: Y_pq = sum_{r in {0,1}} A_pr T_rq for p in {2,3}, q in {0,1}
+    if (ok && warp < 4) {
+        const int p = 2 + (warp >> 1), q = warp & 1;
+        float c[2][4];
+        if (q == 0) {
+            const int xr[2] = {16 * p, 16 * p}, xc[2] = {0, 16}, yr[2] = {0, 16}, yc[2] = {0, 0};
+            warp_gemm16(sm, 2, xr, xc, yr, yc, offA, offT, c);
+        } else {
+            const int xr[1] = {16 * p}, xc[1] = {16}, yr[1] = {16}, yc[1] = {16};
+            warp_gemm16(sm, 1, xr, xc, yr, yc, offA, offT, c);
+        }
+        warp_store16(sm, 16 * warp, 0, c, 1.f, offY);
+    }
+    __syncthreads();
+    // level 2, step 2: T_pq = -sum_{r in {2,3}, r <= p} T_pr Y_rq
+    if (ok && warp < 4) {
+        const int p = 2 + (warp >> 1), q = warp & 1;
+        float c[2][4];
+        // Y_rq lives in scratch block (r - 2) * 2 + q
+        if (p == 2) {
+            const int xr[1] = {32}, xc[1] = {32}, yr[1] = {16 * (0 * 2 + q)}, yc[1] = {0};
+            warp_gemm16(sm, 1, xr, xc, yr, yc, offT, offY, c);
+        } else {
+            const int xr[2] = {48, 48}, xc[2] = {32, 48}, yr[2] = {16 * (0 * 2 + q), 16 * (1 * 2 + q)}, yc[2] = {0, 0};
+            warp_gemm16(sm, 2, xr, xc, yr, yc, offT, offY, c);
+        }
+        warp_store16(sm, 16 * p, 16 * q, c, -1.f, offT);
+    }
+    __syncthreads();
+}
+
+// Epilogue of the W / U MMAs: TMEM columns [0, 64) hold W^T and [64, 128) U^T
+// (lane = channel, column = token).  Thread row r = qd*32 + lane writes
+// tokens [32 hf, 32 hf + 32): W as a K-major operand image (rows = tokens, two
+// 64-channel blocks), U^T as 128-byte-swizzled rows (row = channel).
+// (Kept out of line: inlined, it pushes the per-head prep kernel past its register budget.)
+static __device__ __noinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
+    const int r = qd * 32 + lane;
+    const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
+    float w0[16], w1[16], u0[16], u1[16];
+    tmem_ld16(taddr, w0);
+    tmem_ld16(taddr + 16, w1);
+    tmem_ld16(taddr + 64, u0);
+    tmem_ld16(taddr + 64 + 16, u1);
+    tmem_wait_ld();
+    uint8_t *wimg = blk + kBlkWQ + (r >> 6) * 16384 + (r & 7) * 2;
+    const int wchunk = (r & 63) >> 3;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+        const int i = 32 * hf + t;
+        *reinterpret_cast<__nv_bfloat16 *>(wimg + i * 128 + ((wchunk ^ (i & 7)) << 4)) =
+            __float2bfloat16_rn(t < 16 ? w0[t] : w1[t - 16]);
+    }
+    uint8_t *urow = blk + kBlkU;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float *u = q < 2 ? u0 + 8 * q : u1 + 8 * (q - 2);
+        *reinterpret_cast<uint4 *>(urow + sw128_offset(r, 4 * hf + q)) =
+            make_uint4(pack_bf16(u[0], u[1]), pack_bf16(u[2], u[3]), pack_bf16(u[4], u[5]), pack_bf16(u[6], u[7]));
+    }
+}
+
+// Prep kernel of the per-channel gate (its own translation unit).
+gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const ChunkPlan &p,
+                           const ChunkArgs &a, const int32_t *off, uint8_t *blocks, cudaStream_t s);
+
+}  // namespace tc
+}  // namespace gdn

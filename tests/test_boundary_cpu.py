@@ -67,6 +67,8 @@ def test_workspace_size(lib):
     assert 6 * 3 * simt <= size(dtype=gdn.GDN_F32) < 6 * 3 * simt + 4096
     tc = 32768 + 128 * 128 + 64 * 128 + 192 * 4  # [W;Qs] image, U^T rows, P image, gate factors
     assert 6 * 3 * tc <= size() < 6 * 3 * tc + 4096
+    kda = tc + (1024 - 192 * 4) + 64 * 128 * 2  # per-channel gate: 1 KB of factors and K~
+    assert 6 * 3 * kda <= size(gate=gdn.GDN_GATE_CHANNEL) < 6 * 3 * kda + 4096
     assert size(dtype=gdn.GDN_F32, gate=gdn.GDN_GATE_CHANNEL) > size(dtype=gdn.GDN_F32)
     d = _desc()
     assert lib.gdn_chunk_workspace_size(ctypes.byref(d), 2, None) == gdn.GDN_ERR_INVALID_ARG

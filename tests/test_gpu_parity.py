@@ -37,8 +37,9 @@ def test_shapes(dtype, per_channel, dk, dv):
 
 @pytest.mark.parametrize("T", [1, 5, 63, 64, 65, 128, 129])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_lengths_around_the_chunk(T, dtype):
-    check(make_inputs(SMALL.replace(T=T, dtype=dtype, seed=T)))
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_lengths_around_the_chunk(T, dtype, per_channel):
+    check(make_inputs(SMALL.replace(T=T, dtype=dtype, per_channel=per_channel, seed=T)))
 
 
 def test_zero_length_copies_initial_state():
@@ -73,8 +74,9 @@ def test_packed_equals_separate_runs():
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_snapshots(dtype):
-    x = make_inputs(SMALL.replace(T=640, dtype=dtype, seed=7))
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_snapshots(dtype, per_channel):
+    x = make_inputs(SMALL.replace(T=640, dtype=dtype, per_channel=per_channel, seed=7))
     check(x, snapshot_stride=128)
 
 
@@ -137,6 +139,13 @@ def test_extreme_gates_per_channel(dtype):
     g[..., ::3] = -80.0
     g[:, 50:60, :, 1::3] = -5.0
     check(_with_gates(x, g))
+
+
+@pytest.mark.parametrize("gate_mu", [2.0, 6.0])
+def test_strong_per_channel_gates(gate_mu):
+    """Strong decays on every channel (alpha ~ e^-2 .. e^-6 per token): in-chunk
+    cumulative gates of several hundred, far outside the fp32 range of exp."""
+    check(make_inputs(SMALL.replace(per_channel=True, gate_mu=gate_mu, seed=15)))
 
 
 # ---------------------------------------------------------------------------
