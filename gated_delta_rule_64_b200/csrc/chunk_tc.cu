@@ -592,16 +592,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// (rows, H, 128) bf16 tensor, tiles of 64 tokens x 64 channels of one head.
-gdn_status make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t H, bool swizzle) {
+// (rows, H, 128) tensor of bf16 (tiles of 64 tokens x 64 channels of one head) or
+// fp32 (tiles of 64 tokens x 32 channels), 128-byte swizzle.
+gdn_status make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t H, bool f32 = false) {
     auto enc = tensor_map_encoder();
     if (!enc) return fail(GDN_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t es_bytes = f32 ? 4 : 2;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    cuuint32_t box[3] = {64, 1, 64}, es[3] = {1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    cuuint64_t strides[2] = {(cuuint64_t)D * es_bytes, (cuuint64_t)H * D * es_bytes};
+    cuuint32_t box[3] = {f32 ? 32u : 64u, 1, 64}, es[3] = {1, 1, 1};
+    CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                     const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(GDN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return GDN_OK;
 }
@@ -619,14 +621,16 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     uint8_t *blocks = reinterpret_cast<uint8_t *>(a.ws + p.off_W);
     if (p.H > 65535 || p.max_chunks > 0x7fffffffLL || a.N > 0x7fffffffLL)
         return fail(GDN_ERR_UNSUPPORTED, "grid too large");
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mg;
     memset(&mq, 0, sizeof mq);
     memset(&mk, 0, sizeof mk);
     memset(&mv, 0, sizeof mv);
+    memset(&mg, 0, sizeof mg);
     if (p.rows > 0) {
-        if ((st = make_map(&mq, a.q, p.rows, p.H, true)) != GDN_OK) return st;
-        if ((st = make_map(&mk, a.k, p.rows, p.H, true)) != GDN_OK) return st;
-        if ((st = make_map(&mv, a.v, p.rows, p.H, true)) != GDN_OK) return st;
+        if ((st = make_map(&mq, a.q, p.rows, p.H)) != GDN_OK) return st;
+        if ((st = make_map(&mk, a.k, p.rows, p.H)) != GDN_OK) return st;
+        if ((st = make_map(&mv, a.v, p.rows, p.H)) != GDN_OK) return st;
+        if (p.per_channel && (st = make_map(&mg, a.g, p.rows, p.H, true)) != GDN_OK) return st;
     }
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -642,7 +646,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     if (attr_err != cudaSuccess) return fail(GDN_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(attr_err));
     if (p.max_chunks > 0 && p.rows > 0) {
         if (p.per_channel) {
-            if ((st = tc::launch_prep_kda(mq, mk, mv, p, a, off, blocks, s)) != GDN_OK) return st;
+            if ((st = tc::launch_prep_kda(mq, mk, mv, mg, p, a, off, blocks, s)) != GDN_OK) return st;
         } else {
             LaunchScope ls("gdn_prep_tc", s);
             gdn_prep_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kPrepSmem, s>>>(

@@ -255,6 +255,8 @@ gdn_status gdn_chunk_fwd(const gdn_desc *d, const void *q, const void *k, const 
             return fail(GDN_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
         if (!aligned4(log_gate) || !aligned4(beta))
             return fail(GDN_ERR_INVALID_ARG, "log_gate and beta must be 4-byte aligned");
+        if (d->gate == GDN_GATE_CHANNEL && !aligned16(log_gate))
+            return fail(GDN_ERR_INVALID_ARG, "a per-channel log_gate must be 16-byte aligned");
         const Range ro = range_of(out, v_bytes);
         const Range ins[] = {range_of(q, qk_bytes), range_of(k, qk_bytes), range_of(v, v_bytes),
                              range_of(log_gate, g_bytes), range_of(beta, b_bytes)};

@@ -203,8 +203,10 @@ static __device__ __noinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, 
 }
 
 // Prep kernel of the per-channel gate (its own translation unit).
-gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const ChunkPlan &p,
-                           const ChunkArgs &a, const int32_t *off, uint8_t *blocks, cudaStream_t s);
+// (mg: the per-channel log gate as a (rows, H, 128) fp32 tensor, 32 x 1 x 64 boxes, 128-byte swizzle.)
+gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                           const CUtensorMap &mg, const ChunkPlan &p, const ChunkArgs &a, const int32_t *off,
+                           uint8_t *blocks, cudaStream_t s);
 
 }  // namespace tc
 }  // namespace gdn

@@ -32,7 +32,9 @@
  *     log_gate holds g = log(alpha): finite and <= 0 (alpha = 1 is allowed).
  *     beta is used as given (the pages keep it in (0,1); 0 and 1 work).
  *   - q, k, v, out and states must be 16-byte aligned, the workspace 256-byte;
- *     log_gate, beta and cu_seqlens 4-byte aligned.
+ *     log_gate, beta and cu_seqlens 4-byte aligned, except that the chunked
+ *     calls take a per-channel log_gate 16-byte aligned (its rows are d_k
+ *     floats, so any row of an aligned tensor qualifies).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream).  Argument errors are detected on the host before
  *     anything is launched and leave all outputs untouched.  A failed launch

@@ -109,6 +109,14 @@ def test_gates_need_only_4_byte_alignment(lib):
     assert st in (gdn.GDN_OK, gdn.GDN_ERR_CUDA), st
 
 
+def test_per_channel_gate_alignment(lib):
+    d = _desc(gate=gdn.GDN_GATE_CHANNEL)
+    assert _fwd(lib, d, off={"g": 4}) == gdn.GDN_ERR_INVALID_ARG
+    assert "16-byte" in lib.gdn_last_error().decode()
+    st = _fwd(lib, _desc(gate=gdn.GDN_GATE_CHANNEL), off={"g": 16, "beta": 4})
+    assert st in (gdn.GDN_OK, gdn.GDN_ERR_CUDA), st
+
+
 @pytest.mark.parametrize("name", ["q", "k", "v", "g", "beta", "out"])
 def test_null_required_pointer(lib, name):
     kw = {name: None}
