@@ -13,15 +13,18 @@
 //   Qs   = scale Q * Gam,            K~ = K * exp(b_L - b)
 //
 // (Gam_i = exp(b_i)); the scan then carries S0 Diag(Gam_L) + U'^T K~.
-// Writing the decay as a product of per-token factors (K * Gam)(K / Gam)^T
-// overflows for strong gates, so A and P are formed in 16 x 16 blocks:
-//   * a block (p, q) below the diagonal (rows 16p.., columns 16q.., q < p) is
-//     a tensor-core product of K_p * exp(b - r) and K_q * exp(r - b) with the
-//     reference r = b at row 16p - 1; both factors are <= 1 because the
-//     cumulative log gate does not increase;
-//   * a diagonal block is formed on the CUDA cores from running products of
-//     alpha = exp(g): walking j down from i, exp(b_i - b_j) gains one factor
-//     alpha_{j+1} per step, so no exponential of a large argument appears.
+// Writing the decay as one product (K * Gam)(K / Gam)^T overflows for strong
+// gates, so A and P are formed in 16 x 16 blocks.  With r_p = b at the row
+// before block p (r_0 = 0) and e_p = b at its last row, every row i of block p
+// gets the two factors L_i = exp(b_i - r_p) <= 1 and R_i = exp(e_p - b_i) <= 1,
+// and for i in block p, j in block q:
+//   * q < p:  exp(b_i - b_j) = L_i * exp(r_p - e_q) * R_j, all three <= 1, so the
+//             block is the tensor-core product of K * L (or Q * L) with K * R
+//             scaled per channel by exp(r_p - e_q) (= 1 for q = p - 1);
+//   * q = p:  exp(b_i - b_j) = L_i * exp(r_p - e_p) * R_j where the middle
+//             factor is >= 1: fine as long as the block's decay is moderate
+//             (2^64 at most); otherwise the block is formed term by term from
+//             exp(b_i - b_j) on the CUDA cores.
 // The triangular solve and the W / U tensor-core products are those of the
 // per-head kernel.
 #include <string.h>
@@ -36,22 +39,22 @@ namespace {
 
 // Shared memory (1024-aligned):
 //   [0, 32K)    K and Q tiles: [K ch 0-63 | Q ch 0-63 | K ch 64-127 | Q ch 64-127],
-//               64 token rows of 128 bytes each, 128-byte swizzle (TMA).  K is
-//               replaced by K * Gam (the A operand of the W product) before the solve.
-//   [32K, 48K)  V tile
-//   [48K, 80K)  gate tile (TMA: four [64 tokens][32 channels] fp32 quarters, 128-byte
-//               swizzle), turned in place into b in log2 units; after the gate passes
-//               it holds T (fp32, 16K), the solve's scratch (4K) and the T diag(beta)
-//               operand image (8K, at +24K)
-//   [80K, 96K)  A (fp32, f32_offset layout)
+//               64 token rows of 128 bytes each, 128-byte swizzle (TMA).  They become
+//               K * L and Q * L, and then K * L becomes K * Gam (the A operand of W).
+//   [32K, 64K)  gate tile (TMA: four [64 tokens][32 channels] fp32 quarters, 128-byte
+//               swizzle), turned in place into b in log2 units; once the factors are
+//               formed: A (fp32, f32_offset layout) at 32K and the V tile at 48K
+//   [64K, 80K)  K * R (layout of a K tile, channel halves 8K apart); after the blocks:
+//               T (fp32)
+//   [80K, 96K)  after the blocks: the solve's scratch (4K) and T diag(beta) (8K at 88K)
 //   [96K, 104K) P image (bf16, K-major rows of 64 tokens)
-constexpr uint32_t kSmKQ = 0, kSmV = 32768, kSmB = 49152, kSmA = 81920, kSmP = 98304;
-constexpr uint32_t kSmT = kSmB, kSmY = kSmB + 16384, kSmTp = kSmB + 24576;
+constexpr uint32_t kSmKQ = 0, kSmB = 32768, kSmA = 32768, kSmV = 49152, kSmZ = 65536, kSmP = 98304;
+constexpr uint32_t kSmT = 65536, kSmY = 81920, kSmTp = 90112;
 constexpr uint32_t kSmem = kSmP + 8192 + 1024;
 constexpr float kLog2e = 1.4426950408889634f;
-// Largest in-block decay (log2 units) for which a diagonal block is formed as a
-// product of scaled operands: its right factors reach 2^kSpanMax (far inside the
-// bf16 / fp32 range); beyond it the block is formed term by term.
+// Largest decay inside a diagonal block (log2 units) for which the block is a
+// product of scaled operands: its middle factor reaches 2^kSpanMax (far inside
+// the bf16 / fp32 range).
 constexpr float kSpanMax = 64.f;
 
 // Element (token i, channel c) of the gate / b tile.
@@ -62,8 +65,10 @@ __device__ __forceinline__ uint32_t b_off(int i, int c) {
 __device__ __forceinline__ uint32_t kq_chunk(int qk, int i, int cc) {
     return (uint32_t)((cc >> 3) * 16384 + qk * 8192 + i * 128 + (((cc & 7) ^ (i & 7)) << 4));
 }
-// bf16 pair (c, c+1), c even, of row i of the K / Q tile.
-__device__ __forceinline__ uint32_t kq_pair(int qk, int i, int c) { return kq_chunk(qk, i, c >> 3) + (c & 7) * 2; }
+// 8-channel chunk `cc` of row i of the K * R image.
+__device__ __forceinline__ uint32_t z_chunk(int i, int cc) {
+    return (uint32_t)(kSmZ + (cc >> 3) * 8192 + i * 128 + (((cc & 7) ^ (i & 7)) << 4));
+}
 // bf16 pair (j, j+1), j even, of row i of the P image.
 __device__ __forceinline__ uint32_t p_pair(int i, int j) {
     return (uint32_t)(i * 128 + (((j >> 3) ^ (i & 7)) << 4) + (j & 7) * 2);
@@ -71,28 +76,37 @@ __device__ __forceinline__ uint32_t p_pair(int i, int j) {
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ uint32_t scale_pair(uint32_t w, float2 f) { return pack_bf16(bf_lo(w) * f.x, bf_hi(w) * f.y); }
 
 __device__ __forceinline__ void unpack8(const uint4 &w, float *f) {
     f[0] = bf_lo(w.x); f[1] = bf_hi(w.x); f[2] = bf_lo(w.y); f[3] = bf_hi(w.y);
     f[4] = bf_lo(w.z); f[5] = bf_hi(w.z); f[6] = bf_lo(w.w); f[7] = bf_hi(w.w);
 }
+__device__ __forceinline__ void ld_f8(const uint8_t *sm, int i, int c8, float *f) {
+    *reinterpret_cast<float4 *>(f) = *reinterpret_cast<const float4 *>(sm + kSmB + b_off(i, c8));
+    *reinterpret_cast<float4 *>(f + 4) = *reinterpret_cast<const float4 *>(sm + kSmB + b_off(i, c8 + 4));
+}
+
+// Per-channel factors of one chunk (fp32): exp(r_p) per block, exp(r_p - e_p) per
+// diagonal block, exp(r_p - e_q) for the blocks (2,0), (3,0), (3,1).
+struct Factors {
+    float rp[4][D];
+    float sp[4][D];
+    float d[3][D];
+};
 
 // One warp's share of A and P by bf16 m16n8k16 MMAs: row block p against
-// column blocks q0 .. q0 + nq - 1 (q <= p), with the reference r = b at row
-// 16p - 1 (r = 0 for p = 0).  Left operand rows K_i, Q_i times exp(b_i - r) <= 1;
-// right operand rows K_j times exp(r - b_j), <= 1 below the diagonal block and
-// <= 2^kSpanMax inside it.
-__device__ __forceinline__ void ap_blocks(uint8_t *sm, int p, int q0, int nq, int L, float scale, const float *s_beta) {
+// column blocks q0 .. q0 + nq - 1 (q <= p).  Operands from the K * L, Q * L and
+// K * R images; the right operand is scaled per channel by exp(r_p - e_q).
+__device__ __forceinline__ void ap_blocks(uint8_t *sm, const Factors &f, int p, int q0, int nq, int L, float scale,
+                                          const float *s_beta) {
     const int lane = threadIdx.x & 31, g8 = lane >> 2, t = lane & 3;
-    const int R = 16 * p - 1, i0 = 16 * p + g8, i1 = i0 + 8;
-    auto bpair = [&](int i, int c) { return *reinterpret_cast<const float2 *>(sm + kSmB + b_off(i, c)); };
-    auto scaled = [&](int qk, int i, int c, float2 r2, bool left) {
-        const float2 bi = bpair(i, c);
-        const float e0 = left ? ex2(bi.x - r2.x) : ex2(r2.x - bi.x);
-        const float e1 = left ? ex2(bi.y - r2.y) : ex2(r2.y - bi.y);
-        const uint32_t w = *reinterpret_cast<const uint32_t *>(sm + kSmKQ + kq_pair(qk, i, c));
-        return pack_bf16(bf_lo(w) * e0, bf_hi(w) * e1);
-    };
+    const int i0 = 16 * p + g8, i1 = i0 + 8;
+    const uint32_t sb = smem_u32(sm);
+    // ldmatrix row of this lane: left operand (matrix m = lane / 8: rows +8 (m & 1), columns +8 (m >> 1));
+    // right operand (rows +8 (m >> 1) = second n-tile, columns +8 (m & 1))
+    const int m = lane >> 3, lr = lane & 7;
+    const int arow = 16 * p + lr + 8 * (m & 1), acol = m >> 1;
     float cA[2][2][4], cP[2][2][4];
 #pragma unroll
     for (int b = 0; b < 2; ++b)
@@ -100,26 +114,31 @@ __device__ __forceinline__ void ap_blocks(uint8_t *sm, int p, int q0, int nq, in
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) cA[b][nt][e] = cP[b][nt][e] = 0.f;
-#pragma unroll 1
+#pragma unroll 2
     for (int kk = 0; kk < 8; ++kk) {
-        const int ca = 16 * kk + 2 * t, cb = ca + 8;
-        const float2 ra = p > 0 ? bpair(R, ca) : make_float2(0.f, 0.f);
-        const float2 rb = p > 0 ? bpair(R, cb) : make_float2(0.f, 0.f);
-        const uint32_t ak[4] = {scaled(0, i0, ca, ra, true), scaled(0, i1, ca, ra, true),
-                                scaled(0, i0, cb, rb, true), scaled(0, i1, cb, rb, true)};
-        const uint32_t aq[4] = {scaled(1, i0, ca, ra, true), scaled(1, i1, ca, ra, true),
-                                scaled(1, i0, cb, rb, true), scaled(1, i1, cb, rb, true)};
+        uint32_t ak[4], aq[4];
+        ldsm_x4(sb + kq_chunk(0, arow, 2 * kk + acol), ak);
+        ldsm_x4(sb + kq_chunk(1, arow, 2 * kk + acol), aq);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-            if (b < nq) {
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int j = 16 * (q0 + b) + 8 * nt + g8;
-                    const uint32_t bz[2] = {scaled(0, j, ca, ra, false), scaled(0, j, cb, rb, false)};
-                    mma_bf16_16x8x16(cA[b][nt], ak, bz);
-                    mma_bf16_16x8x16(cP[b][nt], aq, bz);
-                }
+            if (b >= nq) continue;
+            const int q = q0 + b;
+            uint32_t bz[4];
+            ldsm_x4(sb + z_chunk(16 * q + lr + 8 * (m >> 1), 2 * kk + (m & 1)), bz);
+            const float *sc = q == p ? f.sp[p] : (q == p - 1 ? nullptr : f.d[p == 2 ? 0 : (q == 0 ? 1 : 2)]);
+            if (sc) {
+                const int c = 16 * kk + 2 * t;
+                const float2 lo = *reinterpret_cast<const float2 *>(sc + c), hi = *reinterpret_cast<const float2 *>(sc + c + 8);
+                bz[0] = scale_pair(bz[0], lo);
+                bz[1] = scale_pair(bz[1], hi);
+                bz[2] = scale_pair(bz[2], lo);
+                bz[3] = scale_pair(bz[3], hi);
             }
+            const uint32_t b0[2] = {bz[0], bz[1]}, b1[2] = {bz[2], bz[3]};
+            mma_bf16_16x8x16(cA[b][0], ak, b0);
+            mma_bf16_16x8x16(cP[b][0], aq, b0);
+            mma_bf16_16x8x16(cA[b][1], ak, b1);
+            mma_bf16_16x8x16(cP[b][1], aq, b1);
         }
     }
     const float be0 = s_beta[i0], be1 = s_beta[i1];
@@ -146,10 +165,15 @@ __device__ __forceinline__ void ap_blocks(uint8_t *sm, int p, int q0, int nq, in
     }
 }
 
-// Diagonal blocks term by term (for chunks whose gates decay too fast for
-// ap_blocks): warp pair (2p, 2p+1) takes block p; lane = (row pair, 16-channel
-// group); rows r and 15 - r of a block together need 17 (i, j) steps.
-__device__ __forceinline__ void diag_exact(uint8_t *sm, int L, float scale, const float *s_beta) {
+// Diagonal blocks term by term, for chunks whose gates decay too fast for the
+// factored form: warp pair (2p, 2p+1) takes block p; lane = (row pair, 16-channel
+// group); rows r and 15 - r of a block together need 17 (i, j) steps.  It reads
+// the raw K and Q tiles and b; the butterfly leaves every sum in all 8 lanes of a
+// group, and lane s keeps the steps it = s (mod 8) for diag_exact_store.
+struct DiagKeep {
+    float a[3], p[3];
+};
+__device__ __forceinline__ void diag_exact(const uint8_t *sm, DiagKeep &keep) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int p = warp >> 1, rl = lane >> 3, s = lane & 7;
     const int r = 4 * (warp & 1) + rl, base = 16 * p;
@@ -191,12 +215,28 @@ __device__ __forceinline__ void diag_exact(uint8_t *sm, int L, float scale, cons
             a += __shfl_xor_sync(0xffffffffu, a, o);
             pp += __shfl_xor_sync(0xffffffffu, pp, o);
         }
-        if (s == 0) {
-            const int i = base + il, j = base + jl;
-            *reinterpret_cast<float *>(sm + kSmA + f32_offset(i, j)) = s_beta[i] * a;
-            *reinterpret_cast<__nv_bfloat16 *>(sm + kSmP + p_pair(i, j & ~1) + (j & 1) * 2) =
-                __float2bfloat16_rn(i < L ? scale * pp : 0.f);
+        if ((it & 7) == s) {
+            const int k = it >> 3;
+            if (k == 0) { keep.a[0] = a; keep.p[0] = pp; }
+            else if (k == 1) { keep.a[1] = a; keep.p[1] = pp; }
+            else { keep.a[2] = a; keep.p[2] = pp; }
         }
+    }
+}
+__device__ __forceinline__ void diag_exact_store(uint8_t *sm, const DiagKeep &keep, int L, float scale,
+                                                 const float *s_beta) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int p = warp >> 1, rl = lane >> 3, s = lane & 7;
+    const int r = 4 * (warp & 1) + rl, base = 16 * p;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const int it = 8 * k + s;
+        if (it >= 17) continue;
+        const bool first = it <= r;
+        const int i = base + (first ? r : 15 - r), j = base + (first ? r - it : 16 - it);
+        *reinterpret_cast<float *>(sm + kSmA + f32_offset(i, j)) = s_beta[i] * keep.a[k];
+        *reinterpret_cast<__nv_bfloat16 *>(sm + kSmP + p_pair(i, j & ~1) + (j & 1) * 2) =
+            __float2bfloat16_rn(i < L ? scale * keep.p[k] : 0.f);
     }
 }
 
@@ -207,9 +247,10 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                 int64_t N, int64_t T, int64_t rows, int64_t H, float scale, uint8_t *__restrict__ blocks, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    __shared__ uint64_t bar_g, bar_ld, bar_mma;
+    __shared__ uint64_t bar_g, bar_ld, bar_v, bar_mma;
     __shared__ uint32_t tmem_base;
     __shared__ float s_beta[C], s_tot[D];
+    __shared__ __align__(16) Factors fct;
 
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
     ChunkLoc loc;
@@ -224,18 +265,17 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     if (tid == 0) {
         mbar_init(&bar_g, 1);
         mbar_init(&bar_ld, 1);
+        mbar_init(&bar_v, 1);
         mbar_init(&bar_mma, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(&bar_g, 4 * 8192);
 #pragma unroll
         for (int qt = 0; qt < 4; ++qt) tma_load_3d(sm + kSmB + qt * 8192, &mg, 32 * qt, (int32_t)h, tok0, &bar_g);
-        mbar_arrive_expect_tx(&bar_ld, 6 * 8192);
+        mbar_arrive_expect_tx(&bar_ld, 4 * 8192);
         tma_load_3d(sm + kSmKQ, &mk, 0, (int32_t)h, tok0, &bar_ld);
         tma_load_3d(sm + kSmKQ + 16384, &mk, 64, (int32_t)h, tok0, &bar_ld);
         tma_load_3d(sm + kSmKQ + 8192, &mq, 0, (int32_t)h, tok0, &bar_ld);
         tma_load_3d(sm + kSmKQ + 24576, &mq, 64, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + kSmV, &mv, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + kSmV + 8192, &mv, 64, (int32_t)h, tok0, &bar_ld);
     }
     if (warp == 0) {
         tmem_alloc(&tmem_base, 128);
@@ -253,91 +293,149 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     // largest decay inside any 16-token block decides how the diagonal blocks
     // are formed.
     bool ok = mbar_wait(&bar_g, 0);
-    float vals[32];
     const int c_own = tid & 127, half = tid >> 7;
-    if (ok) {
+    {
+        float vals[32];
+        if (ok) {
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
-            const int i = 32 * half + r;
-            vals[r] = i < L ? *reinterpret_cast<const float *>(sm + kSmB + b_off(i, c_own)) : 0.f;
+            for (int r = 0; r < 32; ++r) {
+                const int i = 32 * half + r;
+                vals[r] = i < L ? *reinterpret_cast<const float *>(sm + kSmB + b_off(i, c_own)) : 0.f;
+            }
+#pragma unroll
+            for (int r = 1; r < 32; ++r) vals[r] += vals[r - 1];
+            if (half == 0) s_tot[c_own] = vals[31];
         }
+        __syncthreads();
+        bool wide = false;
+        if (ok) {
+            const float base = half ? s_tot[c_own] : 0.f;
 #pragma unroll
-        for (int r = 1; r < 32; ++r) vals[r] += vals[r - 1];
-        if (half == 0) s_tot[c_own] = vals[31];
+            for (int r = 0; r < 32; ++r) {
+                vals[r] = (vals[r] + base) * kLog2e;
+                *reinterpret_cast<float *>(sm + kSmB + b_off(32 * half + r, c_own)) = vals[r];
+            }
+            // block p = 2 half (+1): r_p = b before it, e_p = b at its last row
+            const float r0 = base * kLog2e, e0 = vals[15], e1 = vals[31];
+            fct.rp[2 * half][c_own] = ex2(r0);
+            fct.rp[2 * half + 1][c_own] = ex2(e0);
+            fct.sp[2 * half][c_own] = ex2(r0 - e0);
+            fct.sp[2 * half + 1][c_own] = ex2(e0 - e1);
+            wide = (r0 - e0 > kSpanMax) || (e0 - e1 > kSpanMax);
+        }
+        const bool any_wide = __syncthreads_or(wide);  // uniform over the block
+        // exp(r_p - e_q) for (p, q) = (2, 0), (3, 0), (3, 1)
+        if (ok && tid < D) {
+            const float e0 = *reinterpret_cast<const float *>(sm + kSmB + b_off(15, tid));
+            const float e1 = *reinterpret_cast<const float *>(sm + kSmB + b_off(31, tid));
+            const float r3 = *reinterpret_cast<const float *>(sm + kSmB + b_off(47, tid));
+            fct.d[0][tid] = ex2(e1 - e0);
+            fct.d[1][tid] = ex2(r3 - e0);
+            fct.d[2][tid] = ex2(r3 - e1);
+        }
+        ok = mbar_wait(&bar_ld, 0) && ok;
+        // exact diagonal blocks need the raw tiles and b: before the factor pass
+        DiagKeep keep = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+        if (any_wide) {
+            if (ok) diag_exact(sm, keep);
+            __syncthreads();
+        }
+
+        // Factor pass over (token, 8-channel) chunks: K * L and Q * L in place,
+        // K * R to its image; Qs = scale Q * Gam and K~ = K * exp(b_L - b) to the block.
+        if (ok) {
+            const int Lm1 = L - 1;
+#pragma unroll 1
+            for (int k = 0; k < 4; ++k) {
+                const int e = tid + kThreads * k;
+                const int hc = e >> 9, i = (e & 511) >> 3, pc = e & 7, p = i >> 4;
+                const int c8 = hc * 64 + ((pc ^ (i & 7)) << 3);
+                const uint32_t so = (uint32_t)(hc * 16384 + i * 128 + pc * 16);
+                float kf[8], qf[8], bi[8], rr[8], ee[8], bl[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + kSmKQ + so), kf);
+                unpack8(*reinterpret_cast<const uint4 *>(sm + kSmKQ + so + 8192), qf);
+                ld_f8(sm, i, c8, bi);
+                ld_f8(sm, 16 * p + 15, c8, ee);
+                ld_f8(sm, Lm1, c8, bl);
+                if (p > 0) ld_f8(sm, 16 * p - 1, c8, rr);
+                else
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) rr[u] = 0.f;
+                float er[8];  // exp(r_p): Gam_i = L_i exp(r_p), both factors <= 1
+                *reinterpret_cast<float4 *>(er) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8);
+                *reinterpret_cast<float4 *>(er + 4) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8 + 4);
+                uint32_t xk[4], xq[4], zr[4], kt[4], qs[4];
+                const bool in = i < L;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int a = 2 * u, b = 2 * u + 1;
+                    const float la = ex2(bi[a] - rr[a]), lb = ex2(bi[b] - rr[b]);
+                    const float ra = ex2(ee[a] - bi[a]), rb = ex2(ee[b] - bi[b]);
+                    const float ga = la * er[a], gb = lb * er[b];
+                    const float ta = ex2(bl[a] - bi[a]), tb = ex2(bl[b] - bi[b]);
+                    xk[u] = pack_bf16(kf[a] * la, kf[b] * lb);
+                    xq[u] = pack_bf16(qf[a] * la, qf[b] * lb);
+                    zr[u] = pack_bf16(kf[a] * ra, kf[b] * rb);
+                    kt[u] = in ? pack_bf16(kf[a] * ta, kf[b] * tb) : 0u;
+                    qs[u] = in ? pack_bf16(scale * qf[a] * ga, scale * qf[b] * gb) : 0u;
+                }
+                *reinterpret_cast<uint4 *>(blk + kBlkKt + hc * 8192 + i * 128 + pc * 16) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+                *reinterpret_cast<uint4 *>(blk + kBlkWQ + 8192 + hc * 16384 + i * 128 + pc * 16) =
+                    make_uint4(qs[0], qs[1], qs[2], qs[3]);
+                // (no other thread reads this chunk of the tiles)
+                *reinterpret_cast<uint4 *>(sm + kSmKQ + so) = make_uint4(xk[0], xk[1], xk[2], xk[3]);
+                *reinterpret_cast<uint4 *>(sm + kSmKQ + so + 8192) = make_uint4(xq[0], xq[1], xq[2], xq[3]);
+                *reinterpret_cast<uint4 *>(sm + kSmZ + hc * 8192 + i * 128 + pc * 16) = make_uint4(zr[0], zr[1], zr[2], zr[3]);
+            }
+            float *fac = reinterpret_cast<float *>(blk + kBlkFac);
+            if (tid < D) fac[kFacGL + tid] = ex2(*reinterpret_cast<const float *>(sm + kSmB + b_off(Lm1, tid)));
+            else if (tid < D + C) fac[kFacW + tid - D] = tid - D < L ? 1.f : 0.f;
+            else if (tid < D + 2 * C) fac[kFacSG + tid - D - C] = 0.f;
+        }
+        fence_async_smem();  // the b region is taken over by the V tile (TMA) below
+        __syncthreads();
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&bar_v, 2 * 8192);
+            tma_load_3d(sm + kSmV, &mv, 0, (int32_t)h, tok0, &bar_v);
+            tma_load_3d(sm + kSmV + 8192, &mv, 64, (int32_t)h, tok0, &bar_v);
+        }
+
+        // A and P.  Warp w takes row block p against column blocks [q0, q0 + nq);
+        // (p, q0, nq) per warp, one hex digit each, with the diagonal blocks (10
+        // blocks) or without them (6), spread so that warps w and w + 4 (which
+        // share a scheduler) hold at most 3 blocks between them.
+        if (ok) {
+            if (any_wide) diag_exact_store(sm, keep, L, scale, s_beta);
+            const uint32_t P = any_wide ? 0x00100233u : 0x01102233u, Q0 = any_wide ? 0x00000020u : 0x01002020u,
+                           NQ = any_wide ? 0x00100212u : 0x01111222u;
+            const int p = (P >> (4 * warp)) & 15, q0 = (Q0 >> (4 * warp)) & 15, nq = (NQ >> (4 * warp)) & 15;
+            if (nq > 0) ap_blocks(sm, fct, p, q0, nq, L, scale, s_beta);
+        }
     }
     __syncthreads();
-    bool wide = false;
-    if (ok) {
-        const float base = half ? s_tot[c_own] : 0.f;
-#pragma unroll
-        for (int r = 0; r < 32; ++r) {
-            vals[r] = (vals[r] + base) * kLog2e;
-            *reinterpret_cast<float *>(sm + kSmB + b_off(32 * half + r, c_own)) = vals[r];
-        }
-        const float b_before = base * kLog2e;  // b at the row before this half
-        wide = (b_before - vals[15] > kSpanMax) || (vals[15] - vals[31] > kSpanMax);
-    }
-    const bool exact_diag = __syncthreads_or(wide);
-    ok = mbar_wait(&bar_ld, 0) && ok;
 
-    // A and P.  Warp w < 6 takes row block p against column blocks [q0, q0 + nq).
+    // P image to the block; K * L -> K * Gam = K * L * exp(r_p) in place.
     if (ok) {
-        if (exact_diag) diag_exact(sm, L, scale, s_beta);
-        // (p, q0, nq) per warp, one hex digit each: with the diagonal blocks (10
-        // blocks on warps 0-5) or without them (6 blocks on warps 0-3)
-        const uint32_t P = exact_diag ? 0x3321u : 0x332210u, Q0 = exact_diag ? 0x2000u : 0x202000u,
-                       NQ = exact_diag ? 0x1221u : 0x221221u;
-        const int p = (P >> (4 * warp)) & 15, q0 = (Q0 >> (4 * warp)) & 15, nq = (NQ >> (4 * warp)) & 15;
-        if (nq > 0) ap_blocks(sm, p, q0, nq, L, scale, s_beta);
-    }
-    __syncthreads();
-
-    // Gate passes over the K and Q tiles (16-byte chunks, 8 channels each):
-    // K * Gam in place, K~ = K * exp(b_L - b) and Qs = scale Q * Gam to the block.
-    if (ok) {
-        const int Lm1 = L - 1;
+        for (int e = tid; e < 512; e += kThreads)
+            *reinterpret_cast<uint4 *>(blk + kBlkP + e * 16) = *reinterpret_cast<const uint4 *>(sm + kSmP + e * 16);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int e = tid + kThreads * k;
             const int hc = e >> 9, i = (e & 511) >> 3, pc = e & 7;
             const int c8 = hc * 64 + ((pc ^ (i & 7)) << 3);
             const uint32_t so = (uint32_t)(hc * 16384 + i * 128 + pc * 16);
-            const uint4 kw = *reinterpret_cast<const uint4 *>(sm + kSmKQ + so);
-            const uint4 qw = *reinterpret_cast<const uint4 *>(sm + kSmKQ + so + 8192);
-            float kf[8], qf[8], bi[8], bl[8];
-            unpack8(kw, kf);
-            unpack8(qw, qf);
-            *reinterpret_cast<float4 *>(bi) = *reinterpret_cast<const float4 *>(sm + kSmB + b_off(i, c8));
-            *reinterpret_cast<float4 *>(bi + 4) = *reinterpret_cast<const float4 *>(sm + kSmB + b_off(i, c8 + 4));
-            *reinterpret_cast<float4 *>(bl) = *reinterpret_cast<const float4 *>(sm + kSmB + b_off(Lm1, c8));
-            *reinterpret_cast<float4 *>(bl + 4) = *reinterpret_cast<const float4 *>(sm + kSmB + b_off(Lm1, c8 + 4));
-            uint32_t kg[4], kt[4], qs[4];
-            const bool in = i < L;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float g0 = ex2(bi[2 * m]), g1 = ex2(bi[2 * m + 1]);
-                const float t0 = ex2(bl[2 * m] - bi[2 * m]), t1 = ex2(bl[2 * m + 1] - bi[2 * m + 1]);
-                kg[m] = in ? pack_bf16(kf[2 * m] * g0, kf[2 * m + 1] * g1) : 0u;
-                kt[m] = in ? pack_bf16(kf[2 * m] * t0, kf[2 * m + 1] * t1) : 0u;
-                qs[m] = in ? pack_bf16(scale * qf[2 * m] * g0, scale * qf[2 * m + 1] * g1) : 0u;
-            }
-            *reinterpret_cast<uint4 *>(sm + kSmKQ + so) = make_uint4(kg[0], kg[1], kg[2], kg[3]);
-            *reinterpret_cast<uint4 *>(blk + kBlkKt + hc * 8192 + i * 128 + pc * 16) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
-            *reinterpret_cast<uint4 *>(blk + kBlkWQ + 8192 + hc * 16384 + i * 128 + pc * 16) =
-                make_uint4(qs[0], qs[1], qs[2], qs[3]);
+            const uint4 w = *reinterpret_cast<const uint4 *>(sm + kSmKQ + so);
+            const float *rp = fct.rp[i >> 4] + c8;
+            const float4 f0 = *reinterpret_cast<const float4 *>(rp), f1 = *reinterpret_cast<const float4 *>(rp + 4);
+            *reinterpret_cast<uint4 *>(sm + kSmKQ + so) =
+                make_uint4(scale_pair(w.x, make_float2(f0.x, f0.y)), scale_pair(w.y, make_float2(f0.z, f0.w)),
+                           scale_pair(w.z, make_float2(f1.x, f1.y)), scale_pair(w.w, make_float2(f1.z, f1.w)));
         }
-        // the P image, and the gate factors
-        for (int e = tid; e < 512; e += kThreads)
-            *reinterpret_cast<uint4 *>(blk + kBlkP + e * 16) = *reinterpret_cast<const uint4 *>(sm + kSmP + e * 16);
-        float *fac = reinterpret_cast<float *>(blk + kBlkFac);
-        if (tid < D) fac[kFacGL + tid] = ex2(*reinterpret_cast<const float *>(sm + kSmB + b_off(Lm1, tid)));
-        else if (tid < D + C) fac[kFacW + tid - D] = tid - D < L ? 1.f : 0.f;
-        else if (tid < D + 2 * C) fac[kFacSG + tid - D - C] = 0.f;
     }
     fence_async_smem();  // K * Gam is read by the tensor core
     __syncthreads();
 
-    // T = (I + A)^-1 into the (now free) b region.
+    // T = (I + A)^-1 into the (now free) K * R region.
     blocked_solve<kSmT, kSmY>(sm, [](int i, int j) { return kSmA + f32_offset(i, j); }, ok);
 
     // T'' = T diag(beta) as a bf16 operand image (K-major rows i).
@@ -365,6 +463,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     tc_fence_after();
 
     // W^T = (K * Gam)^T T''^T (M = d_k), U^T = V^T T''^T (M = d_v); K = 64 tokens.
+    ok = mbar_wait(&bar_v, 0) && ok;
     if (warp == 0 && __all_sync(0xffffffffu, ok)) {
         const uint64_t dk = sdesc_sw128(smem_u32(sm + kSmKQ), 16384, 1024), dv = sdesc_sw128(smem_u32(sm + kSmV), 8192, 1024),
                        dt = sdesc_sw128(smem_u32(sm + kSmTp), 16, 1024);

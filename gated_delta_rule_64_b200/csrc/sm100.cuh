@@ -267,6 +267,15 @@ __device__ __forceinline__ void mma_bf16_16x8x16(float (&d)[4], const uint32_t (
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// Four 8 x 8 b16 matrices from shared memory: lanes 8m .. 8m+7 give the row
+// addresses (16 bytes each) of matrix m; register m receives matrix m in the
+// MMA fragment layout (lane l: row l / 4, columns 2 (l % 4), +1).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
 // 2^x by the hardware approximation (subnormal results flush to zero).
 __device__ __forceinline__ float ex2(float x) {
     float y;

@@ -1,5 +1,7 @@
 """Helpers for the GPU parity tests: run the library and the oracle on the same
 seeded inputs and compare."""
+import os
+
 import numpy as np
 import torch
 
@@ -57,5 +59,9 @@ def check(x: Inputs, *, scale=1.0, snapshot_stride=0, heads=None):
     tol_o, tol_s = tolerances(x.q.dtype)
     eo, ef = rel_l2(out, o_ref), rel_l2(fin, f_ref)
     es = rel_l2(snaps, s_ref) if snapshot_stride else 0.0
+    report = os.environ.get("GDN_PARITY_REPORT")
+    if report:  # optional record of the measured errors, one line per check
+        with open(report, "a") as f:
+            f.write(f"{os.environ.get('PYTEST_CURRENT_TEST', '?').split(' ')[0]}\t{eo:.3e}\t{ef:.3e}\t{es:.3e}\n")
     assert eo <= tol_o and ef <= tol_s and es <= tol_s, f"rel-L2 out {eo:.2e} state {ef:.2e} snaps {es:.2e}"
     return eo, ef, es
