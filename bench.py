@@ -423,17 +423,91 @@ def run_gpu(args):
     return 0
 
 
+SECONDARY = {"kda": "KDA_PACKED", "long": "LONG_SNAPSHOTS", "tiny": "TINY_F32"}
+
+
+def run_secondary(args) -> int:
+    """Time one of the other chunked workloads (the parity configurations) the way the
+    headline line times the prefill workload; prints one JSON line of its own."""
+    import torch
+
+    from gated_delta_rule_64_b200 import gdn, inputs
+
+    w = getattr(inputs, SECONDARY[args.workload])
+    torch.cuda.set_device(0)
+    pk = peaks()
+    x = inputs.make_inputs(w)
+    d = lambda t: None if t is None else t.cuda().contiguous()
+    q, k, v, g, beta, h0, cu = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0), d(x.cu_seqlens)
+    N = x.n_seqs
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    rows = B * T
+    out = torch.empty_like(v)
+    fin = torch.empty((N, H, dv, dk), dtype=torch.float32, device="cuda")
+    n_snap = T // w.snapshot_stride if w.snapshot_stride else 0
+    snaps = torch.empty((N, n_snap, H, dv, dk), dtype=torch.float32, device="cuda") if n_snap else None
+    ws = torch.empty(gdn.gdn_chunk_workspace_size(B, T, H, dk, dv, N, dtype=q.dtype, per_channel=w.per_channel),
+                     dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdn.gdn_chunk_fwd(q, k, v, g, beta, h0, cu, snapshot_stride=w.snapshot_stride, out=out, final_state=fin,
+                          snapshots=snaps, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    gdn.profile_read()
+    gdn.profile_enable(True)
+    clocks.mark_begin()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    gdn.profile_enable(False)
+    kernels = gdn.profile_read()
+    clk = clocks.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    tokens = x.tokens()
+    el = q.element_size()
+    gate_per_tok = 4 * (dk if w.per_channel else 1)
+    alg_bytes = (tokens * H * ((2 * dk + 2 * dv) * el + gate_per_tok + 4)
+                 + (2 if h0 is not None else 1) * N * H * STATE_BYTES + n_snap * N * H * STATE_BYTES)
+    per_launch = {n: t / max(1, c) * 1e-3 for n, (c, t) in kernels.items()}
+    step_s = sum(per_launch.values()) or ms_step * 1e-3
+    achieved = alg_bytes / step_s / 1e9
+    line = {"metric": "chunked prefill tokens/s (secondary workload)", "value": tokens / (ms_step * 1e-3),
+            "unit": UNIT, "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "tokens": tokens, "sequences": N, "heads": H, "d_k": dk, "d_v": dv,
+                       "per_channel_gate": w.per_channel, "snapshot_stride": w.snapshot_stride},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": alg_bytes,
+                         "kernels": {n: {"us_per_launch": per_launch[n] * 1e6, "share": per_launch[n] / step_s}
+                                     for n in per_launch}},
+            "gpu_launches": sum(c for c, _ in kernels.values()), "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_profile(which: str) -> int:
     import torch
 
     from gated_delta_rule_64_b200 import gdn
-    from gated_delta_rule_64_b200.inputs import DECODE, PREFILL_BF16, make_inputs
-    d = lambda t: t.cuda()
-    if which == "prefill":
-        x = make_inputs(PREFILL_BF16)
-        q, k, v, g, b, h0 = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0)
+    from gated_delta_rule_64_b200.inputs import DECODE, KDA_PACKED, PREFILL_BF16, make_inputs
+    d = lambda t: None if t is None else t.cuda()
+    if which in ("prefill", "kda-small"):
+        # kda-small: the per-channel packed workload on 8 of its 32 heads (about 1.5 GB on the device)
+        x = make_inputs(PREFILL_BF16) if which == "prefill" else make_inputs(KDA_PACKED, heads=8)
+        q, k, v, g, b, h0, cu = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0), d(x.cu_seqlens)
         for _ in range(3):
-            gdn.gdn_chunk_fwd(q, k, v, g, b, h0)
+            gdn.gdn_chunk_fwd(q, k, v, g, b, h0, cu)
     else:
         x = make_inputs(DECODE.replace(decode_steps=3))
         st = d(x.h0)
@@ -450,8 +524,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "decode"],
+    ap.add_argument("--profile", choices=["prefill", "decode", "kda-small"],
                     help="run three calls of one workload and exit (for ncu captures; prints nothing to time)")
+    ap.add_argument("--workload", choices=["prefill"] + sorted(SECONDARY), default="prefill",
+                    help="prefill (default): the headline line; kda / long / tiny: time that chunked "
+                         "workload instead (one GPU, its own JSON line)")
     args = ap.parse_args(argv)
     if args.profile:
         return run_profile(args.profile)
@@ -459,6 +536,8 @@ def main(argv=None):
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload != "prefill":
+        return run_secondary(args)
     return run_gpu(args)
 
 

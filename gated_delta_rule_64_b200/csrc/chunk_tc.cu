@@ -326,26 +326,82 @@ struct ScanBars {
 // KDA: per-channel gate.  The state-update operand is then K~ from the block
 // (instead of the K tile), U'_w = U', and the carried state is scaled per key
 // channel by exp(b_L).
+// Sequence split of long fixed-length sequences (G >= 3 segments of `seg` chunks).
+// A segment's end state is an affine function of its start state,
+// S_end = S_start M_g + B_g.  Pass 1 runs, in parallel, segment 0 from the true
+// initial state (outputs included) and every middle segment twice: from zero
+// (giving B_g) and from the identity with the writes U dropped (giving M_g; the
+// state has d_k rows then, which needs d_v = d_k).  gdn_seg_combine chains the
+// maps into the start state of every segment; pass 2 runs segments 1 .. G-1 from
+// those, with outputs, snapshots and the final state.
+struct ScanSplit {
+    int32_t G;      // segments per sequence; 1: no split
+    int32_t seg;    // chunks per segment
+    int32_t pass;   // 1 or 2 (with G >= 3)
+    float *states;  // [N][G][3][H][D][D] fp32: B_g, M_g and the start state of segment g
+};
+__device__ __forceinline__ float *split_state(const ScanSplit &sp, int64_t n, int64_t g, int slot, int64_t H,
+                                              int64_t h) {
+    return sp.states + ((((n * sp.G + g) * 3 + slot) * H + h) * (int64_t)D) * D;
+}
+
 template <bool KDA>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32_t *__restrict__ cu,
             const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t max_chunks,
             int64_t snap_stride, int64_t n_snap, const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out,
-            float *final_state, float *__restrict__ snaps, int *err) {
+            float *final_state, float *__restrict__ snaps, const ScanSplit sp, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     __shared__ ScanBars bars;
     __shared__ uint32_t tmem_base;
-    const int64_t n = blockIdx.x, h = blockIdx.y;
+    const int64_t h = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, hf = warp >> 2;
     const int v = qd * 32 + lane;  // state row; this thread holds columns [64 hf, 64 hf + 64)
 
+    // This block's work: sequence n, chunks [cb, ce) of it, its start state and
+    // where its end state goes (both D x D fp32 states of this (sequence, head)).
+    enum { kStartGiven, kStartZero, kStartIdentity };
+    int64_t n = blockIdx.x, g = 0;
+    int start_kind = kStartGiven;
+    bool emit = true;
+    if (sp.G > 1) {
+        if (sp.pass == 1) {
+            const int64_t per = 1 + 2 * (sp.G - 2), i = n % per;
+            n /= per;
+            if (i > 0) {
+                g = 1 + (i - 1) / 2;
+                start_kind = ((i - 1) & 1) ? kStartIdentity : kStartZero;
+                emit = false;
+            }
+        } else {
+            const int64_t per = sp.G - 1;
+            g = 1 + n % per;
+            n /= per;
+        }
+    }
+    const int64_t sh = (n * H + h) * (int64_t)D * D;  // this (sequence, head)'s state in h0 / final_state
+    const float *s_init = h0 ? h0 + sh : nullptr;     // kStartGiven: this state (nullptr: zero)
+    float *s_end = final_state ? final_state + sh : nullptr;
+    if (sp.G > 1) {
+        if (sp.pass == 1)
+            s_end = g == 0 ? split_state(sp, n, 1, 2, H, h) : split_state(sp, n, g, start_kind == kStartZero ? 0 : 1, H, h);
+        else {
+            s_init = split_state(sp, n, g, 2, H, h);
+            if (g != sp.G - 1) s_end = nullptr;
+        }
+    }
+
     int64_t start, len;
     seq_bounds(cu, n, T, rows, start, len);
-    int64_t nchunks = (len + C - 1) / C;
+    int64_t ntot = (len + C - 1) / C;
     const int64_t chunk0 = cu ? (int64_t)off[n] : n * ((T + C - 1) / C);
-    if (chunk0 + nchunks > max_chunks) nchunks = max_chunks > chunk0 ? max_chunks - chunk0 : 0;
+    if (chunk0 + ntot > max_chunks) ntot = max_chunks > chunk0 ? max_chunks - chunk0 : 0;
+    const int64_t cb = sp.G > 1 ? g * sp.seg : 0;
+    const int64_t ce = sp.G > 1 && g < sp.G - 1 ? (cb + sp.seg < ntot ? cb + sp.seg : ntot) : ntot;
+    const int64_t nchunks = ce > cb ? ce - cb : 0;  // chunks of this block; chunk i is cb + i of the sequence
+    const float umul = start_kind == kStartIdentity ? 0.f : 1.f;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(&bars.full[i], 1);
@@ -366,8 +422,8 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
     auto issue_loads = [&](int64_t c) {
         const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
-        const uint8_t *blk = blocks + (size_t)((chunk0 + c) * H + h) * (KDA ? kTcBlockKda : kTcBlock);
-        const int32_t tok = (int32_t)(start + c * C);
+        const uint8_t *blk = blocks + (size_t)((chunk0 + cb + c) * H + h) * (KDA ? kTcBlockKda : kTcBlock);
+        const int32_t tok = (int32_t)(start + (cb + c) * C);
         uint64_t *bar = &bars.full[stage];
         mbar_arrive_expect_tx(bar, stage_bytes<KDA>());
         bulk_load(st + kStWQ, blk + kBlkWQ, (uint32_t)kTcWQ, bar);
@@ -383,23 +439,24 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         for (int64_t c = 0; c < kStages && c < nchunks; ++c) issue_loads(c);
 
     float S[64];
-    const int64_t srow = ((n * H + h) * D + v) * (int64_t)D + 64 * hf;
-    if (h0) {
+    const int64_t srow = (int64_t)v * D + 64 * hf;  // this thread's part of a state
+    if (start_kind == kStartGiven && s_init) {
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-            const float4 t = *reinterpret_cast<const float4 *>(h0 + srow + c);
+            const float4 t = *reinterpret_cast<const float4 *>(s_init + srow + c);
             S[c] = t.x; S[c + 1] = t.y; S[c + 2] = t.z; S[c + 3] = t.w;
         }
     } else {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) S[c] = 0.f;
+        for (int c = 0; c < 64; ++c) S[c] = (start_kind == kStartIdentity && 64 * hf + c == v) ? 1.f : 0.f;
     }
 
     // Output of chunk `c` (tokens [32 hf, 32 hf + 32) of column v): waits for its last MMA.
     auto emit_output = [&](int64_t c) -> bool {
         const bool ok_w = mbar_wait(&bars.mma[2], (uint32_t)(c & 1));
         tc_fence_after();
-        const int L = (int)(len - c * C < C ? len - c * C : C);
+        const int64_t ca = cb + c;
+        const int L = (int)(len - ca * C < C ? len - ca * C : C);
         float o[2][16];
         const uint32_t dcol = kTmD + (uint32_t)(c & 1) * 128 + 64 + 32 * hf;
         tmem_ld16(tm + lane_off + dcol, o[0]);
@@ -409,7 +466,7 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         // lane j of a group holds those 4 channels of token 4 b + j -> one 8-byte store.
         const int j4 = lane & 3;
         const int64_t tstride = H * D;
-        __nv_bfloat16 *op = out + ((start + c * C + 32 * hf + j4) * H + h) * D + (v - j4);
+        __nv_bfloat16 *op = out + ((start + ca * C + 32 * hf + j4) * H + h) * D + (v - j4);
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
             float x0 = o[b >> 2][4 * (b & 3)], x1 = o[b >> 2][4 * (b & 3) + 1], x2 = o[b >> 2][4 * (b & 3) + 2],
@@ -471,7 +528,8 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         }
         // the previous chunk's output, while this chunk's MMAs run; after it every MMA of
         // chunk c-1 has completed, so its stage can take chunk c+2
-        if (c >= 1) ok = emit_output(c - 1) && ok;
+        // (without outputs every MMA of chunk c-1 was waited for in its steps (c) and (e))
+        if (c >= 1 && emit) ok = emit_output(c - 1) && ok;
         if (tid == kLoader && c >= 1 && c + kStages - 1 < nchunks) issue_loads(c + kStages - 1);
 
         // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32) -> TMEM A operands U', U' * w
@@ -496,7 +554,7 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
                     const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
                     const float acc_lo = (q < 2 ? a0[8 * q + e] : a1[8 * (q - 2) + e]);
                     const float acc_hi = (q < 2 ? a0[8 * q + e + 1] : a1[8 * (q - 2) + e + 1]);
-                    const float up0 = __low2float(u2) - acc_lo, up1 = __high2float(u2) - acc_hi;
+                    const float up0 = umul * __low2float(u2) - acc_lo, up1 = umul * __high2float(u2) - acc_hi;
                     wu[4 * q + e / 2] = pack_bf16(up0, up1);
                     ww[4 * q + e / 2] = pack_bf16(up0 * wv[e], up1 * wv[e + 1]);
                 }
@@ -517,7 +575,7 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ts(tm + kTmAcc4, tm + kTmAUw + kk * 8, bk + (uint64_t)((kk * 2048) >> 4), id_k, kk > 0);
             mma_commit_warp(&bars.mma[1]);
-        } else if (warp == 1) {
+        } else if (warp == 1 && emit) {
             const uint64_t bp = sdesc_sw128(st_u + kStRest + kRestP, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -553,8 +611,8 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         }
 
         // snapshot after n * stride tokens of the sequence
-        if (snaps && snap_stride > 0 && ((c + 1) * C) % snap_stride == 0 && (c + 1) * C <= len) {
-            const int64_t s = (c + 1) * C / snap_stride - 1;
+        if (emit && snaps && snap_stride > 0 && ((cb + c + 1) * C) % snap_stride == 0 && (cb + c + 1) * C <= len) {
+            const int64_t s = (cb + c + 1) * C / snap_stride - 1;
             if (s < n_snap) {
                 float *dst = snaps + (((n * n_snap + s) * H + h) * D + v) * (int64_t)D + 64 * hf;
 #pragma unroll
@@ -564,16 +622,74 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         }
         if (__syncthreads_or(!ok)) break;
     }
-    if (ok && nchunks > 0) ok = emit_output(nchunks - 1) && ok;
+    if (ok && nchunks > 0 && emit) ok = emit_output(nchunks - 1) && ok;
     if (!ok && tid == 0) flag_error(err, 2);
-    if (ok && final_state) {
+    if (ok && s_end) {
 #pragma unroll
         for (int cc = 0; cc < 64; cc += 4)
-            *reinterpret_cast<float4 *>(final_state + srow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
+            *reinterpret_cast<float4 *>(s_end + srow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+// Start states of the segments: S_{g+1} = S_g M_g + B_g for g = 1 .. G-2 (S_1
+// comes from pass 1), one block per (sequence, head), fp32 on the CUDA cores.
+// Thread (v, half) computes 64 entries of row v; S_g rows are padded to 132
+// floats in shared memory so that a warp's 16-byte row reads hit distinct banks.
+constexpr int kCombPad = D + 4;
+constexpr uint32_t kCombSmem = (uint32_t)(D * kCombPad + D * D) * 4;
+
+__global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit sp, int64_t H) {
+    extern __shared__ float4 comb_raw[];
+    float *Ss = reinterpret_cast<float *>(comb_raw);  // S_g, rows of kCombPad
+    float *Ms = Ss + D * kCombPad;                      // M_g, rows of D
+    const int64_t n = blockIdx.x, h = blockIdx.y;
+    const int tid = threadIdx.x, v = tid & 127, c0 = 64 * (tid >> 7);
+    {
+        const float *s1 = split_state(sp, n, 1, 2, H, h);
+        for (int e = tid; e < D * D / 4; e += kThreads) {
+            const int r = e >> 5, c4 = e & 31;
+            *reinterpret_cast<float4 *>(Ss + r * kCombPad + 4 * c4) = reinterpret_cast<const float4 *>(s1)[e];
+        }
+    }
+    for (int g = 1; g <= sp.G - 2; ++g) {
+        const float *M = split_state(sp, n, g, 1, H, h), *B = split_state(sp, n, g, 0, H, h);
+        for (int e = tid; e < D * D / 4; e += kThreads) reinterpret_cast<float4 *>(Ms)[e] = reinterpret_cast<const float4 *>(M)[e];
+        float acc[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+            const float4 b4 = *reinterpret_cast<const float4 *>(B + v * D + c0 + c);
+            acc[c] = b4.x; acc[c + 1] = b4.y; acc[c + 2] = b4.z; acc[c + 3] = b4.w;
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int k4 = 0; k4 < D / 4; ++k4) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(Ss + v * kCombPad + 4 * k4);
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float *mrow = Ms + (4 * k4 + j) * D + c0;
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4 *>(mrow + c);
+                    acc[c] = fmaf(sv[j], m4.x, acc[c]);
+                    acc[c + 1] = fmaf(sv[j], m4.y, acc[c + 1]);
+                    acc[c + 2] = fmaf(sv[j], m4.z, acc[c + 2]);
+                    acc[c + 3] = fmaf(sv[j], m4.w, acc[c + 3]);
+                }
+            }
+        }
+        __syncthreads();  // every read of S_g and M_g is done
+        float *dst = split_state(sp, n, g + 1, 2, H, h) + v * D + c0;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+            const float4 a4 = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+            *reinterpret_cast<float4 *>(dst + c) = a4;
+            *reinterpret_cast<float4 *>(Ss + v * kCombPad + c0 + c) = a4;
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -642,6 +758,9 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         if (attr_err == cudaSuccess)
             attr_err = cudaFuncSetAttribute(gdn_scan_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)kScanSmem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(gdn_seg_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)kCombSmem);
     });
     if (attr_err != cudaSuccess) return fail(GDN_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(attr_err));
     if (p.max_chunks > 0 && p.rows > 0) {
@@ -654,14 +773,59 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
             if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
         }
     }
-    {
+    auto kern = p.per_channel ? gdn_scan_tc<true> : gdn_scan_tc<false>;
+    ScanSplit sp{1, 0, 0, nullptr};
+    if (p.split_G < 3) {
         LaunchScope ls("gdn_scan_tc", s);
-        auto kern = p.per_channel ? gdn_scan_tc<true> : gdn_scan_tc<false>;
         kern<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
             mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap,
-            blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, nullptr);
+            blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
+        return check_launch("gdn_scan_tc");
+    }
+    // sequence split: pass 1, the chained start states, pass 2
+    sp = ScanSplit{p.split_G, p.split_seg, 1, reinterpret_cast<float *>(a.ws + p.off_split)};
+    const int64_t per1 = 1 + 2 * (int64_t)(p.split_G - 2), per2 = p.split_G - 1;
+    if (a.N * per1 > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
+    {
+        LaunchScope ls("gdn_scan_tc", s);
+        kern<<<dim3((unsigned)(a.N * per1), (unsigned)p.H), kThreads, kScanSmem, s>>>(
+            mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+            (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
+    }
+    if ((st = check_launch("gdn_scan_tc")) != GDN_OK) return st;
+    {
+        LaunchScope ls("gdn_seg_combine", s);
+        gdn_seg_combine<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kCombSmem, s>>>(sp, p.H);
+    }
+    if ((st = check_launch("gdn_seg_combine")) != GDN_OK) return st;
+    sp.pass = 2;
+    {
+        LaunchScope ls("gdn_scan_tc", s);
+        kern<<<dim3((unsigned)(a.N * per2), (unsigned)p.H), kThreads, kScanSmem, s>>>(
+            mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+            (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
     }
     return check_launch("gdn_scan_tc");
+}
+
+SplitChoice choose_split(int64_t N, int64_t H, int64_t nch, int sms) {
+    SplitChoice best{1, (int32_t)nch};
+    if (sms <= 0 || nch < 96) return best;
+    auto waves = [sms](int64_t ctas) { return (ctas + sms - 1) / sms; };
+    // cost in chunk steps of one block; a combine step costs about 4
+    double best_cost = (double)waves(N * H) * nch;
+    for (int64_t G = 3; G <= 128; ++G) {
+        const int64_t seg = (nch + G - 1) / G;
+        if (seg < 32) break;
+        const int64_t Gr = (nch + seg - 1) / seg;  // no empty segments
+        if (Gr < 3) continue;
+        const double cost = (double)(waves(N * H * (1 + 2 * (Gr - 2))) + waves(N * H * (Gr - 1))) * seg + 4.0 * (Gr - 2);
+        if (cost < 0.98 * best_cost) {
+            best_cost = cost;
+            best = SplitChoice{(int32_t)Gr, (int32_t)seg};
+        }
+    }
+    return best;
 }
 
 }  // namespace gdn

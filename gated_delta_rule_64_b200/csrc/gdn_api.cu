@@ -103,10 +103,28 @@ ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed) {
     size_t off = 0;
     p.off_chunk_offsets = off;
     off = align_up(off + sizeof(int32_t) * (size_t)(p.N + 1), 256);
+    p.split_G = 1;
+    p.split_seg = 0;
+    p.off_split = 0;
     if (p.tc) {
         p.tc_block = p.per_channel ? kTcBlockKda : kTcBlock;
         p.off_W = p.off_U = p.off_P = p.off_b = off;  // one block of tc_block bytes per chunk-head
         off = align_up(off + p.tc_block * (size_t)ch, 256);
+        if (!packed && d.T > 0) {
+            int dev = 0, sms = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+                cudaGetLastError();
+                sms = 148;
+            }
+            const SplitChoice sc = choose_split(p.N, p.H, (d.T + kChunk - 1) / kChunk, sms);
+            if (sc.G >= 3) {
+                p.split_G = sc.G;
+                p.split_seg = sc.seg;
+                p.off_split = off;
+                off = align_up(off + sizeof(float) * (size_t)p.N * sc.G * 3 * p.H * p.dv * p.dk, 256);
+            }
+        }
     } else {
         p.off_W = off;
         off = align_up(off + sizeof(float) * (size_t)ch * kChunk * p.dk, 256);
@@ -213,10 +231,15 @@ gdn_status gdn_chunk_workspace_size(const gdn_desc *d, int32_t num_seqs, size_t 
     if (st != GDN_OK) return st;
     if (!bytes) return fail(GDN_ERR_INVALID_ARG, "bytes is NULL");
     if (num_seqs < 0) return fail(GDN_ERR_INVALID_ARG, "num_seqs < 0");
-    // The packed-sequence bound covers B fixed-length sequences too:
-    // B * ceil(T/64) <= B*T/64 + B.
-    ChunkPlan p = make_plan(*d, num_seqs, true);
-    *bytes = p.total;
+    // The packed-sequence bound covers B fixed-length sequences too
+    // (B * ceil(T/64) <= B*T/64 + B); fixed-length sequences may add the state
+    // maps of the split scan.
+    size_t total = make_plan(*d, num_seqs, true).total;
+    if (num_seqs == d->B) {
+        const size_t fixed = make_plan(*d, num_seqs, false).total;
+        total = fixed > total ? fixed : total;
+    }
+    *bytes = total;
     return GDN_OK;
 }
 

@@ -38,11 +38,21 @@ struct ChunkPlan {
     bool per_channel;
     bool tc;             // tensor-core path (bf16, d_k = d_v = 128)
     size_t tc_block;     // bytes per chunk-head of the tensor-core workspace
+    int32_t split_G;     // tensor-core path, fixed-length sequences: segments per sequence (1: none)
+    int32_t split_seg;   // chunks per segment
     // byte offsets into the workspace
     size_t off_chunk_offsets;  // int32 (N+1): first global chunk index of each sequence
     size_t off_W, off_U, off_P, off_b;
+    size_t off_split;    // [N][G][3][H][d_v][d_k] fp32 segment maps and start states
     size_t total;
 };
+
+// Segments per sequence for the split scan of N fixed-length sequences of
+// `nch` chunks on `sms` multiprocessors (G = 1: no split).
+struct SplitChoice {
+    int32_t G, seg;
+};
+SplitChoice choose_split(int64_t N, int64_t H, int64_t nch, int sms);
 
 ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed);
 

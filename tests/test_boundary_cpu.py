@@ -195,3 +195,45 @@ def test_python_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 64, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         gdn.gdn_chunk_fwd(x, x, x, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1))
+
+
+def _split_policy(N, H, nch, sms=148):
+    """Segments per sequence the split scan picks (restated from the host code's
+    cost model: blocks waves x chunks per segment, plus 4 chunk steps per combine)."""
+    waves = lambda ctas: -(-ctas // sms)
+    best, best_cost = (1, nch), waves(N * H) * nch
+    if nch < 96:
+        return best
+    for G in range(3, 129):
+        seg = -(-nch // G)
+        if seg < 32:
+            break
+        Gr = -(-nch // seg)
+        if Gr < 3:
+            continue
+        cost = (waves(N * H * (1 + 2 * (Gr - 2))) + waves(N * H * (Gr - 1))) * seg + 4.0 * (Gr - 2)
+        if cost < 0.98 * best_cost:
+            best, best_cost = (Gr, seg), cost
+    return best
+
+
+def test_split_scan_workspace(lib):
+    """Long fixed-length sequences on few (sequence, head) pairs get the split scan and
+    its per-segment state maps in the workspace; short or many sequences do not.
+    (Without a GPU the library plans for 148 multiprocessors.)"""
+    def size(**kw):
+        n = ctypes.c_size_t()
+        d = _desc(**kw)
+        assert lib.gdn_chunk_workspace_size(ctypes.byref(d), kw.get("B", 2), ctypes.byref(n)) == gdn.GDN_OK
+        return n.value
+    blk = 32768 + 128 * 128 + 64 * 128 + 192 * 4
+    # one sequence of 262144 tokens, 16 heads: 4096 chunks
+    G, seg = _split_policy(1, 16, 4096)
+    assert G >= 3 and (G - 1) * seg < 4096 <= G * seg
+    fixed = 256 + 4096 * 16 * blk + 1 * G * 3 * 16 * 128 * 128 * 4
+    packed = 256 + (262144 // 64 + 1) * 16 * blk
+    got = size(B=1, T=262144, H=16)
+    assert max(fixed, packed) <= got < max(fixed, packed) + 1024
+    # the prefill workload (64 (sequence, head) pairs of 64 chunks) runs unsplit
+    assert _split_policy(4, 16, 64) == (1, 64)
+    assert size(B=4, T=4096, H=16) < 256 + (4 * 4096 // 64 + 4) * 16 * blk + 1024

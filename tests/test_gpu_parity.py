@@ -148,6 +148,29 @@ def test_strong_per_channel_gates(gate_mu):
     check(make_inputs(SMALL.replace(per_channel=True, gate_mu=gate_mu, seed=15)))
 
 
+@pytest.mark.parametrize("per_channel", [False, True])
+@pytest.mark.parametrize("gate_mu", [-2.0, -7.0])
+def test_split_scan(per_channel, gate_mu):
+    """One long sequence on two heads (128 chunks): the scan splits it into segments
+    (state maps per segment, chained start states); gate_mu = -7 keeps the state
+    alive across every segment boundary."""
+    w = SMALL.replace(B=1, T=8192, H=2, per_channel=per_channel, gate_mu=gate_mu, h0_std=0.1, seed=16)
+    check(make_inputs(w), snapshot_stride=1024)
+
+
+def test_split_scan_final_state_aliases_initial():
+    w = SMALL.replace(B=1, T=8192, H=2, h0_std=0.1, seed=17)
+    x = make_inputs(w)
+    dx = to_dev(x)
+    st = dx.h0.clone()
+    out, fin, _ = gdn.gdn_chunk_fwd(dx.q, dx.k, dx.v, dx.g, dx.beta, st, final_state=st)
+    torch.cuda.synchronize()
+    o_ref, f_ref, _ = run_oracle(x)
+    tol_o, tol_s = tolerances(x.q.dtype)
+    assert fin.data_ptr() == st.data_ptr()
+    assert rel_l2(out, o_ref) <= tol_o and rel_l2(st, f_ref) <= tol_s
+
+
 # ---------------------------------------------------------------------------
 # Decode
 # ---------------------------------------------------------------------------
