@@ -83,6 +83,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     __shared__ uint64_t bar_ld, bar_mma;
     __shared__ uint32_t tmem_base;
     __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C];
+    __shared__ __align__(16) float s_b2[C];  // b in log2 units
 
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
     ChunkLoc loc;
@@ -141,17 +142,12 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         const bool in = tid < L;
         const float bl = s_b[L - 1], bi = s_b[tid];
         float *fac = reinterpret_cast<float *>(blk + kBlkFac);
+        s_b2[tid] = bi * 1.4426950408889634f;
         s_bg[tid] = s_beta[tid] * __expf(bi);
         s_sg[tid] = in ? scale * __expf(bi) : 0.f;
         fac[kFacW + tid] = in ? __expf(bl - bi) : 0.f;
         fac[kFacSG + tid] = s_sg[tid];
         fac[kFacGL + tid] = tid == 0 ? __expf(bl) : 0.f;  // exp(b_L), then zero padding
-    }
-    // In-chunk decay exp(b_i - b_j) for j <= i, computed once (both the Gram
-    // rows and the Q K^T rows use it); it lives in the T area until the solve.
-    for (int e = tid; e < C * C; e += kThreads) {
-        const int i = e >> 6, j = e & 63;
-        if (j <= i) *reinterpret_cast<float *>(sm + kPrepTf + f32_offset(i, j)) = __expf(s_b[i] - s_b[j]);
     }
     __syncthreads();
 
@@ -203,11 +199,14 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         tmem_ld16(taddr, v0);
         tmem_ld16(taddr + 16, v1);
         tmem_wait_ld();
+        // in-chunk decay exp(b_i - b_j) = 2^(b2_i - b2_j) (used only for j <= i, where it is <= 1)
         float dec[32];
+        const float bi2 = s_b2[i];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const float4 d4 = *reinterpret_cast<const float4 *>(sm + kPrepTf + f32_offset(i, 32 * hf + 4 * q));
-            dec[4 * q] = d4.x; dec[4 * q + 1] = d4.y; dec[4 * q + 2] = d4.z; dec[4 * q + 3] = d4.w;
+            const float4 b4 = *reinterpret_cast<const float4 *>(s_b2 + 32 * hf + 4 * q);
+            dec[4 * q] = ex2(bi2 - b4.x); dec[4 * q + 1] = ex2(bi2 - b4.y);
+            dec[4 * q + 2] = ex2(bi2 - b4.z); dec[4 * q + 3] = ex2(bi2 - b4.w);
         }
         float rr[32];
 #pragma unroll
@@ -345,7 +344,8 @@ __device__ __forceinline__ float *split_state(const ScanSplit &sp, int64_t n, in
     return sp.states + ((((n * sp.G + g) * 3 + slot) * H + h) * (int64_t)D) * D;
 }
 
-template <bool KDA>
+// SPLIT: launched as a pass of the split scan (the block's work then comes from `sp`).
+template <bool KDA, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32_t *__restrict__ cu,
             const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t max_chunks,
@@ -365,15 +365,15 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
     enum { kStartGiven, kStartZero, kStartIdentity };
     int64_t n = blockIdx.x, g = 0;
     int start_kind = kStartGiven;
-    bool emit = true;
-    if (sp.G > 1) {
+    bool emit_rt = true;
+    if (SPLIT) {
         if (sp.pass == 1) {
             const int64_t per = 1 + 2 * (sp.G - 2), i = n % per;
             n /= per;
             if (i > 0) {
                 g = 1 + (i - 1) / 2;
                 start_kind = ((i - 1) & 1) ? kStartIdentity : kStartZero;
-                emit = false;
+                emit_rt = false;
             }
         } else {
             const int64_t per = sp.G - 1;
@@ -384,7 +384,7 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
     const int64_t sh = (n * H + h) * (int64_t)D * D;  // this (sequence, head)'s state in h0 / final_state
     const float *s_init = h0 ? h0 + sh : nullptr;     // kStartGiven: this state (nullptr: zero)
     float *s_end = final_state ? final_state + sh : nullptr;
-    if (sp.G > 1) {
+    if (SPLIT) {
         if (sp.pass == 1)
             s_end = g == 0 ? split_state(sp, n, 1, 2, H, h) : split_state(sp, n, g, start_kind == kStartZero ? 0 : 1, H, h);
         else {
@@ -398,10 +398,11 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
     int64_t ntot = (len + C - 1) / C;
     const int64_t chunk0 = cu ? (int64_t)off[n] : n * ((T + C - 1) / C);
     if (chunk0 + ntot > max_chunks) ntot = max_chunks > chunk0 ? max_chunks - chunk0 : 0;
-    const int64_t cb = sp.G > 1 ? g * sp.seg : 0;
-    const int64_t ce = sp.G > 1 && g < sp.G - 1 ? (cb + sp.seg < ntot ? cb + sp.seg : ntot) : ntot;
+    const int64_t cb = SPLIT ? g * sp.seg : 0;
+    const int64_t ce = SPLIT && g < sp.G - 1 ? (cb + sp.seg < ntot ? cb + sp.seg : ntot) : ntot;
     const int64_t nchunks = ce > cb ? ce - cb : 0;  // chunks of this block; chunk i is cb + i of the sequence
-    const float umul = start_kind == kStartIdentity ? 0.f : 1.f;
+    const bool emit = !SPLIT || emit_rt;
+    const float umul = SPLIT && start_kind == kStartIdentity ? 0.f : 1.f;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(&bars.full[i], 1);
@@ -554,7 +555,13 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
                     const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
                     const float acc_lo = (q < 2 ? a0[8 * q + e] : a1[8 * (q - 2) + e]);
                     const float acc_hi = (q < 2 ? a0[8 * q + e + 1] : a1[8 * (q - 2) + e + 1]);
-                    const float up0 = umul * __low2float(u2) - acc_lo, up1 = umul * __high2float(u2) - acc_hi;
+                    float up0 = __low2float(u2), up1 = __high2float(u2);
+                    if (SPLIT) {
+                        up0 *= umul;
+                        up1 *= umul;
+                    }
+                    up0 -= acc_lo;
+                    up1 -= acc_hi;
                     wu[4 * q + e / 2] = pack_bf16(up0, up1);
                     ww[4 * q + e / 2] = pack_bf16(up0 * wv[e], up1 * wv[e + 1]);
                 }
@@ -752,12 +759,11 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
         attr_err = cudaFuncSetAttribute(gdn_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrepSmem);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(gdn_scan_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)kScanSmem);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(gdn_scan_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)kScanSmem);
+        const void *scans[4] = {(const void *)gdn_scan_tc<false, false>, (const void *)gdn_scan_tc<false, true>,
+                                (const void *)gdn_scan_tc<true, false>, (const void *)gdn_scan_tc<true, true>};
+        for (const void *k : scans)
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
         if (attr_err == cudaSuccess)
             attr_err = cudaFuncSetAttribute(gdn_seg_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)kCombSmem);
@@ -773,9 +779,9 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
             if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
         }
     }
-    auto kern = p.per_channel ? gdn_scan_tc<true> : gdn_scan_tc<false>;
     ScanSplit sp{1, 0, 0, nullptr};
     if (p.split_G < 3) {
+        auto kern = p.per_channel ? gdn_scan_tc<true, false> : gdn_scan_tc<false, false>;
         LaunchScope ls("gdn_scan_tc", s);
         kern<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
             mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap,
@@ -783,6 +789,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         return check_launch("gdn_scan_tc");
     }
     // sequence split: pass 1, the chained start states, pass 2
+    auto kern = p.per_channel ? gdn_scan_tc<true, true> : gdn_scan_tc<false, true>;
     sp = ScanSplit{p.split_G, p.split_seg, 1, reinterpret_cast<float *>(a.ws + p.off_split)};
     const int64_t per1 = 1 + 2 * (int64_t)(p.split_G - 2), per2 = p.split_G - 1;
     if (a.N * per1 > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
