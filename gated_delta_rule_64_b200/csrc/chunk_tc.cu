@@ -643,58 +643,63 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
 
 // Start states of the segments: S_{g+1} = S_g M_g + B_g for g = 1 .. G-2 (S_1
 // comes from pass 1), one block per (sequence, head), fp32 on the CUDA cores.
-// Thread (v, half) computes 64 entries of row v; S_g rows are padded to 132
-// floats in shared memory so that a warp's 16-byte row reads hit distinct banks.
-constexpr int kCombPad = D + 4;
-constexpr uint32_t kCombSmem = (uint32_t)(D * kCombPad + D * D) * 4;
+// Thread t computes a 4-row x 16-column tile (rows 4 (t % 32) .., columns
+// 16 (t / 32) ..), so every value loaded from shared memory feeds 4 or 16 FMAs.
+// S_g is kept transposed (column k = row of St) so the 4 row values of a k are
+// one 16-byte load.
+constexpr uint32_t kCombSmem = (uint32_t)(2 * D * D) * 4;
 
 __global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit sp, int64_t H) {
     extern __shared__ float4 comb_raw[];
-    float *Ss = reinterpret_cast<float *>(comb_raw);  // S_g, rows of kCombPad
-    float *Ms = Ss + D * kCombPad;                      // M_g, rows of D
+    float *St = reinterpret_cast<float *>(comb_raw);  // S_g transposed: St[k][v]
+    float *Ms = St + D * D;                             // M_g: Ms[k][c]
     const int64_t n = blockIdx.x, h = blockIdx.y;
-    const int tid = threadIdx.x, v = tid & 127, c0 = 64 * (tid >> 7);
+    const int tid = threadIdx.x, r0 = 4 * (tid & 31), c0 = 16 * (tid >> 5);
     {
         const float *s1 = split_state(sp, n, 1, 2, H, h);
-        for (int e = tid; e < D * D / 4; e += kThreads) {
-            const int r = e >> 5, c4 = e & 31;
-            *reinterpret_cast<float4 *>(Ss + r * kCombPad + 4 * c4) = reinterpret_cast<const float4 *>(s1)[e];
+        for (int e = tid; e < D * D / 4; e += kThreads) {  // lanes take consecutive rows v
+            const int v = e & 127, c4 = e >> 7;
+            const float4 x = *reinterpret_cast<const float4 *>(s1 + v * D + 4 * c4);
+            St[(4 * c4) * D + v] = x.x;
+            St[(4 * c4 + 1) * D + v] = x.y;
+            St[(4 * c4 + 2) * D + v] = x.z;
+            St[(4 * c4 + 3) * D + v] = x.w;
         }
     }
     for (int g = 1; g <= sp.G - 2; ++g) {
         const float *M = split_state(sp, n, g, 1, H, h), *B = split_state(sp, n, g, 0, H, h);
         for (int e = tid; e < D * D / 4; e += kThreads) reinterpret_cast<float4 *>(Ms)[e] = reinterpret_cast<const float4 *>(M)[e];
-        float acc[64];
+        float acc[4][16];
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-            const float4 b4 = *reinterpret_cast<const float4 *>(B + v * D + c0 + c);
-            acc[c] = b4.x; acc[c + 1] = b4.y; acc[c + 2] = b4.z; acc[c + 3] = b4.w;
-        }
-        __syncthreads();
-#pragma unroll 1
-        for (int k4 = 0; k4 < D / 4; ++k4) {
-            const float4 s4 = *reinterpret_cast<const float4 *>(Ss + v * kCombPad + 4 * k4);
-            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float *mrow = Ms + (4 * k4 + j) * D + c0;
-#pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    const float4 m4 = *reinterpret_cast<const float4 *>(mrow + c);
-                    acc[c] = fmaf(sv[j], m4.x, acc[c]);
-                    acc[c + 1] = fmaf(sv[j], m4.y, acc[c + 1]);
-                    acc[c + 2] = fmaf(sv[j], m4.z, acc[c + 2]);
-                    acc[c + 3] = fmaf(sv[j], m4.w, acc[c + 3]);
-                }
+            for (int c = 0; c < 16; c += 4) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(B + (r0 + i) * D + c0 + c);
+                acc[i][c] = b4.x; acc[i][c + 1] = b4.y; acc[i][c + 2] = b4.z; acc[i][c + 3] = b4.w;
             }
+        __syncthreads();
+#pragma unroll 2
+        for (int k = 0; k < D; ++k) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(St + k * D + r0);
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+            float mv[16];
+#pragma unroll
+            for (int c = 0; c < 16; c += 4) *reinterpret_cast<float4 *>(mv + c) = *reinterpret_cast<const float4 *>(Ms + k * D + c0 + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int c = 0; c < 16; ++c) acc[i][c] = fmaf(sv[i], mv[c], acc[i][c]);
         }
         __syncthreads();  // every read of S_g and M_g is done
-        float *dst = split_state(sp, n, g + 1, 2, H, h) + v * D + c0;
+        float *dst = split_state(sp, n, g + 1, 2, H, h);
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-            const float4 a4 = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-            *reinterpret_cast<float4 *>(dst + c) = a4;
-            *reinterpret_cast<float4 *>(Ss + v * kCombPad + c0 + c) = a4;
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int c = 0; c < 16; c += 4)
+                *reinterpret_cast<float4 *>(dst + (r0 + i) * D + c0 + c) =
+                    make_float4(acc[i][c], acc[i][c + 1], acc[i][c + 2], acc[i][c + 3]);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) St[(c0 + c) * D + r0 + i] = acc[i][c];
         }
     }
 }
