@@ -423,7 +423,77 @@ def run_gpu(args):
     return 0
 
 
-SECONDARY = {"kda": "KDA_PACKED", "long": "LONG_SNAPSHOTS", "tiny": "TINY_F32"}
+SECONDARY = {"kda": "KDA_PACKED", "long": "LONG_SNAPSHOTS", "tiny": "TINY_F32", "spec": "DECODE"}
+SPEC_K = 4  # draft tokens per sequence in the speculative-decoding measurement
+
+
+def run_spec(args) -> int:
+    """Speculative decoding on the decode workload's shape (256 sequences x 32 heads,
+    d = 128): one gdn_decode_multi call per SPEC_K draft tokens, (a) committing all
+    of them, (b) verifying without commit while writing every step's state, then
+    adopting the accepted step (gdn_state_select, all drafts accepted)."""
+    import torch
+
+    from gated_delta_rule_64_b200 import gdn
+    from gated_delta_rule_64_b200.inputs import DECODE, make_inputs
+
+    torch.cuda.set_device(0)
+    pk = peaks()
+    w = DECODE.replace(decode_steps=0, T=SPEC_K)
+    x = make_inputs(w)
+    d = lambda t: t.cuda().contiguous()
+    q, k, v, g, beta, h0 = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    state = h0.clone()
+    out = torch.empty_like(v)
+    steps = torch.empty((B, T, H, dv, dk), dtype=torch.float32, device="cuda")
+    accept = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    modes = {
+        "commit": lambda: gdn.gdn_decode_multi(q, k, v, g, beta, state, commit=True, out=out, stream=stream),
+        "verify_select": lambda: (gdn.gdn_decode_multi(q, k, v, g, beta, state, commit=False, step_states=steps,
+                                                       out=out, stream=stream),
+                                  gdn.gdn_state_select(steps, accept, state, stream=stream)),
+    }
+    tok_bytes = T * (2 * dk + 2 * dv) * q.element_size() + T * 8
+    bytes_per_unit = {"commit": 2 * STATE_BYTES + tok_bytes,
+                      "verify_select": STATE_BYTES + T * STATE_BYTES + tok_bytes + 2 * STATE_BYTES}
+    res = {}
+    clocks = ClockSampler(0)
+    clocks.start()
+    for name, f in modes.items():
+        for _ in range(args.warmup):
+            f()
+        torch.cuda.synchronize()
+        gdn.profile_read()
+        gdn.profile_enable(True)
+        clocks.mark_begin()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks.mark_end()
+        gdn.profile_enable(False)
+        kern = gdn.profile_read()
+        ms = e0.elapsed_time(e1) / args.steps
+        achieved = B * H * bytes_per_unit[name] / (ms * 1e-3) / 1e9
+        res[name] = {"ms_per_call": ms, "tokens_per_s": B * T / (ms * 1e-3), "hbm_gbs": achieved,
+                     "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": B * H * bytes_per_unit[name],
+                     "kernels": {n: t / max(1, c) * 1e3 for n, (c, t) in kern.items()}}
+    clk = clocks.stop()
+    line = {"metric": "speculative decode tokens/s (secondary workload)", "value": res["commit"]["tokens_per_s"],
+            "unit": UNIT, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": {"workload": f"{w.name}: {T} tokens per sequence per call", "sequences": B, "heads": H,
+                       "d_k": dk, "d_v": dv},
+            "modes": res, "roofline": {"bound": "hbm", "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                       "achieved": res["commit"]["hbm_gbs"], "frac": res["commit"]["frac"]},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_secondary(args) -> int:
@@ -528,7 +598,8 @@ def main(argv=None):
                     help="run three calls of one workload and exit (for ncu captures; prints nothing to time)")
     ap.add_argument("--workload", choices=["prefill"] + sorted(SECONDARY), default="prefill",
                     help="prefill (default): the headline line; kda / long / tiny: time that chunked "
-                         "workload instead (one GPU, its own JSON line)")
+                         "workload instead; spec: multi-token decode / speculative verify (one GPU, its own "
+                         "JSON line)")
     args = ap.parse_args(argv)
     if args.profile:
         return run_profile(args.profile)
@@ -536,6 +607,8 @@ def main(argv=None):
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "spec":
+        return run_spec(args)
     if args.workload != "prefill":
         return run_secondary(args)
     return run_gpu(args)

@@ -351,4 +351,62 @@ gdn_status gdn_decode_step(const gdn_desc *d, const void *q, const void *k, cons
     return launch_decode(*d, q, k, v, log_gate, beta, state, out, (cudaStream_t)stream);
 }
 
+gdn_status gdn_decode_multi(const gdn_desc *d, const void *q, const void *k, const void *v,
+                            const float *log_gate, const float *beta, const int32_t *n_tokens, float *state,
+                            int32_t commit, void *out, float *step_states, gdn_stream_t stream) {
+    g_last_error[0] = 0;
+    gdn_status st = check_desc(d);
+    if (st != GDN_OK) return st;
+    if (d->T < 1 || d->T > kMaxMultiTokens)
+        return fail(GDN_ERR_INVALID_ARG, "multi-token decode needs 1 <= T <= %lld (got %lld)",
+                    (long long)kMaxMultiTokens, (long long)d->T);
+    if (commit != 0 && commit != 1) return fail(GDN_ERR_INVALID_ARG, "commit must be 0 or 1");
+    if (d->B == 0) return GDN_OK;
+    if (!q || !k || !v || !log_gate || !beta || !state || !out)
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v, log_gate, beta, state and out are required");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out) ||
+        (step_states && !aligned16(step_states)))
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v, state, out and step_states must be 16-byte aligned");
+    if (!aligned4(log_gate) || !aligned4(beta) || (n_tokens && !aligned4(n_tokens)))
+        return fail(GDN_ERR_INVALID_ARG, "log_gate, beta and n_tokens must be 4-byte aligned");
+    const size_t in_el = d->dtype == GDN_F32 ? 4 : 2;
+    const size_t bth = (size_t)d->B * d->T * d->H;
+    const size_t sbytes = (size_t)d->dv * d->dk * 4;
+    const Range ro = range_of(out, bth * d->dv * in_el);
+    const Range rs = range_of(state, (size_t)d->B * d->H * sbytes);
+    const Range rss = range_of(step_states, step_states ? bth * sbytes : 0);
+    const Range ins[] = {range_of(q, bth * d->dk * in_el), range_of(k, bth * d->dk * in_el),
+                         range_of(v, bth * d->dv * in_el),
+                         range_of(log_gate, bth * (d->gate == GDN_GATE_CHANNEL ? d->dk : 1) * 4),
+                         range_of(beta, bth * 4), range_of(n_tokens, n_tokens ? (size_t)d->B * 4 : 0)};
+    if (overlaps(ro, rs) || overlaps(ro, rss) || overlaps(rs, rss))
+        return fail(GDN_ERR_INVALID_ARG, "out, state and step_states must not overlap");
+    for (const Range &r : ins)
+        if (overlaps(ro, r) || overlaps(rs, r) || overlaps(rss, r))
+            return fail(GDN_ERR_INVALID_ARG, "out, state or step_states overlaps an input");
+    return launch_decode_multi(*d, q, k, v, log_gate, beta, n_tokens, state, commit, out, step_states,
+                               (cudaStream_t)stream);
+}
+
+gdn_status gdn_state_select(const gdn_desc *d, const float *step_states, const int32_t *accept, float *state,
+                            gdn_stream_t stream) {
+    g_last_error[0] = 0;
+    gdn_status st = check_desc(d);
+    if (st != GDN_OK) return st;
+    if (d->T < 1 || d->T > kMaxMultiTokens)
+        return fail(GDN_ERR_INVALID_ARG, "state select needs 1 <= T <= %lld (got %lld)",
+                    (long long)kMaxMultiTokens, (long long)d->T);
+    if (d->B == 0) return GDN_OK;
+    if (!step_states || !accept || !state)
+        return fail(GDN_ERR_INVALID_ARG, "step_states, accept and state are required");
+    if (!aligned16(step_states) || !aligned16(state) || !aligned4(accept))
+        return fail(GDN_ERR_INVALID_ARG, "step_states and state must be 16-byte aligned, accept 4-byte");
+    const size_t sbytes = (size_t)d->dv * d->dk * 4;
+    const Range rs = range_of(state, (size_t)d->B * d->H * sbytes);
+    if (overlaps(rs, range_of(step_states, (size_t)d->B * d->T * d->H * sbytes)) ||
+        overlaps(rs, range_of(accept, (size_t)d->B * 4)))
+        return fail(GDN_ERR_INVALID_ARG, "state overlaps step_states or accept");
+    return launch_state_select(*d, step_states, accept, state, (cudaStream_t)stream);
+}
+
 }  // extern "C"

@@ -92,6 +92,12 @@ constexpr size_t kTcBlockKda = kTcWQ + kTcUt + kTcPImg + kTcFacKda + kTcKt;  // 
 gdn_status launch_decode(const gdn_desc &d, const void *q, const void *k, const void *v,
                          const float *g, const float *beta, float *state, void *out,
                          cudaStream_t s);
+constexpr int64_t kMaxMultiTokens = 64;  // tokens per sequence of one gdn_decode_multi call
+gdn_status launch_decode_multi(const gdn_desc &d, const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const int32_t *n_tokens, float *state, int commit, void *out,
+                               float *step_states, cudaStream_t s);
+gdn_status launch_state_select(const gdn_desc &d, const float *step_states, const int32_t *accept, float *state,
+                               cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Device helpers

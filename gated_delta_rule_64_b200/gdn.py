@@ -25,7 +25,8 @@ GDN_F32, GDN_BF16 = 0, 1
 GDN_GATE_HEAD, GDN_GATE_CHANNEL = 0, 1
 
 EXPORTED = ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
-            "gdn_status_string", "gdn_last_error", "gdn_profile_enable", "gdn_profile_read")
+            "gdn_decode_multi", "gdn_state_select", "gdn_status_string", "gdn_last_error", "gdn_profile_enable",
+            "gdn_profile_read")
 
 
 class GdnDesc(ctypes.Structure):
@@ -64,6 +65,8 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_chunk_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp, sz, vp]
         lib.gdn_chunk_fwd_static.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp]
         lib.gdn_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.gdn_decode_multi.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
+        lib.gdn_state_select.argtypes = [dp, vp, vp, vp, vp]
         lib.gdn_status_string.argtypes = [ctypes.c_int]
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_last_error.argtypes = []
@@ -71,7 +74,7 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_profile_enable.argtypes = [ctypes.c_int]
         lib.gdn_profile_read.argtypes = [ctypes.POINTER(GdnKernelTime), i32, ctypes.POINTER(i32)]
         for name in ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
-                     "gdn_profile_enable", "gdn_profile_read"):
+                     "gdn_decode_multi", "gdn_state_select", "gdn_profile_enable", "gdn_profile_read"):
             getattr(lib, name).restype = ctypes.c_int
         if path == LIB_PATH:
             _lib = lib
@@ -206,6 +209,41 @@ def gdn_decode_step(q, k, v, log_gate, beta, state, *, scale=1.0, out=None, stre
                              _ptr(out), _stream(stream))
     _check(lib, st)
     return out
+
+
+def gdn_decode_multi(q, k, v, log_gate, beta, state, *, n_tokens=None, commit=True, step_states=None, scale=1.0,
+                     out=None, stream=None):
+    """Up to T tokens per sequence in one pass over the state (speculative verify / multi-token decode).
+    q, k (B,T,H,dk); v (B,T,H,dv); log_gate (B,T,H) or (B,T,H,dk); beta (B,T,H); state (B,H,dv,dk) fp32;
+    n_tokens: int32 (B) on the device or None (all T); commit: write the state after n_tokens back;
+    step_states: True to allocate, a (B,T,H,dv,dk) fp32 tensor, or None.  Returns (out, step_states)."""
+    lib = load_library()
+    _need_cuda(q, k, v, log_gate, beta, state)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    per_channel = log_gate.dim() == 4
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if step_states is True:
+        step_states = torch.empty((B, T, H, dv, dk), dtype=torch.float32, device=q.device)
+    _need_cuda(out)
+    d = make_desc(B, T, H, dk, dv, _dtype_code(q), per_channel, scale)
+    st = lib.gdn_decode_multi(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_gate), _ptr(beta),
+                              _ptr(n_tokens), _ptr(state), 1 if commit else 0, _ptr(out), _ptr(step_states),
+                              _stream(stream))
+    _check(lib, st)
+    return out, step_states
+
+
+def gdn_state_select(step_states, accept, state, *, stream=None):
+    """state[b] = step_states[b, accept[b] - 1] where accept[b] > 0 (int32 device tensor)."""
+    lib = load_library()
+    _need_cuda(step_states, accept, state)
+    B, T, H, dv, dk = step_states.shape
+    d = make_desc(B, T, H, dk, dv, GDN_F32, False, 1.0)
+    _check(lib, lib.gdn_state_select(ctypes.byref(d), _ptr(step_states), _ptr(accept), _ptr(state),
+                                     _stream(stream)))
+    return state
 
 
 def profile_enable(on: bool = True):

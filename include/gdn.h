@@ -201,6 +201,62 @@ gdn_status gdn_decode_step(const gdn_desc *d,
                            const float *log_gate, const float *beta,
                            float *state, void *out, gdn_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * gdn_decode_multi -- up to d->T tokens of every live sequence in one pass over
+ * its state: the verify step of speculative decoding and multi-token decode.
+ *
+ * A recurrent state has absorbed every token it saw, so rejecting draft tokens
+ * needs the state from before them ("Hybrid models: what Gated DeltaNet
+ * replaces in the KV cache", section "What a recurrent state changes for
+ * serving", item 2; "Hybrid attention: why new LLMs keep full attention in
+ * only a few layers", closing section: rolling back a rejected speculative
+ * token needs the state from a step earlier).
+ *
+ * For sequence b (d->B of them) and head h, with n_b = n_tokens[b] clamped to
+ * [0, d->T] (d->T when n_tokens is NULL), tokens t = 0 .. n_b - 1 are applied in
+ * order exactly as gdn_decode_step would apply them, starting from state[b, h]:
+ *   out[b, t, h]          = the token's output (rows t >= n_b are not written);
+ *   step_states[b, t, h]  = the state after token t, if step_states != NULL
+ *                           (entries t >= n_b are not written);
+ *   state[b, h]           = the state after n_b tokens if commit == 1; left
+ *                           unchanged (the pre-draft state) if commit == 0.
+ * The state is read from HBM once for all tokens.
+ *
+ *   d        B = live sequences, T = token slots per sequence (1 .. 64), H, d_k, d_v,
+ *            dtype, gate, scale as for gdn_decode_step
+ *   q, k     (B, T, H, d_k); v, out (B, T, H, d_v); log_gate (B, T, H) or
+ *            (B, T, H, d_k); beta (B, T, H)  -- token t of sequence b at [b, t]
+ *   n_tokens device int32 (B), or NULL for all T tokens
+ *   state    (B, H, d_v, d_k) fp32
+ *   commit   0 or 1
+ *   step_states (B, T, H, d_v, d_k) fp32 or NULL
+ * Alignment as for gdn_decode_step (step_states 16-byte, n_tokens 4-byte);
+ * out, state and step_states must not overlap each other or the inputs.
+ * Returns GDN_ERR_INVALID_ARG for T outside 1 .. 64, a bad commit value, NULL
+ * required pointers, misalignment or overlap (nothing launched).
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_decode_multi(const gdn_desc *d,
+                            const void *q, const void *k, const void *v,
+                            const float *log_gate, const float *beta,
+                            const int32_t *n_tokens, float *state, int32_t commit,
+                            void *out, float *step_states, gdn_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * gdn_state_select -- adopt the state after an accepted prefix of the drafts.
+ *
+ * For every sequence b with m = accept[b] > 0 (clamped to d->T) and every head
+ * h: state[b, h] = step_states[b, m - 1, h], the state gdn_decode_multi wrote
+ * after token m - 1; sequences with accept[b] <= 0 keep their state (the
+ * pre-draft state when the verify call did not commit).
+ *   d            B, T (token slots of step_states), H, d_k, d_v as in the
+ *                gdn_decode_multi call that wrote step_states
+ *   step_states  (B, T, H, d_v, d_k) fp32, 16-byte aligned
+ *   accept       device int32 (B), 4-byte aligned
+ *   state        (B, H, d_v, d_k) fp32, 16-byte aligned, not overlapping the others
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_state_select(const gdn_desc *d, const float *step_states, const int32_t *accept,
+                            float *state, gdn_stream_t stream);
+
 /* Static description of a status code. */
 const char *gdn_status_string(gdn_status s);
 

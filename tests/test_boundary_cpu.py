@@ -176,6 +176,53 @@ def test_decode_validation(lib):
     assert lib.gdn_decode_step(ctypes.byref(d), *p, None) == gdn.GDN_ERR_UNSUPPORTED
 
 
+def _multi(lib, d, p, commit=1):
+    # argument order: q, k, v, log_gate, beta, n_tokens, state, commit, out, step_states
+    return lib.gdn_decode_multi(ctypes.byref(d), p[0], p[1], p[2], p[3], p[4], p[5], p[6], commit, p[7], p[8], None)
+
+
+def test_decode_multi_validation(lib):
+    p = [_addr(i) for i in range(9)]
+    for T in (0, 65):  # 1 .. 64 token slots
+        assert _multi(lib, _desc(B=4, T=T), p) == gdn.GDN_ERR_INVALID_ARG
+    d = _desc(B=4, T=8)
+    assert _multi(lib, d, p, commit=2) == gdn.GDN_ERR_INVALID_ARG
+    for i, bad in ((6, None), (0, None), (7, None)):  # state, q, out are required
+        q = list(p)
+        q[i] = bad
+        assert _multi(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[8] = _addr(6, 4096)  # step_states inside the state
+    assert _multi(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    assert "overlap" in lib.gdn_last_error().decode()
+    q = list(p)
+    q[7] = _addr(8, 16)  # out inside step_states
+    assert _multi(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[5] = _addr(5, 2)  # misaligned n_tokens
+    assert _multi(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[8] = _addr(8, 8)  # misaligned step_states
+    assert _multi(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    # optional pointers may be NULL: validation passes (the launch then needs a GPU)
+    q = list(p)
+    q[5] = None
+    q[8] = None
+    assert _multi(lib, d, q) in (gdn.GDN_OK, gdn.GDN_ERR_CUDA)
+    assert _multi(lib, _desc(B=0, T=8), p) == gdn.GDN_OK
+
+
+def test_state_select_validation(lib):
+    d = _desc(B=4, T=8)
+    ss, acc, st = _addr(0), _addr(1), _addr(2)
+    sel = lambda d, a, b, c: lib.gdn_state_select(ctypes.byref(d), a, b, c, None)
+    assert sel(_desc(B=4, T=0), ss, acc, st) == gdn.GDN_ERR_INVALID_ARG
+    assert sel(d, None, acc, st) == gdn.GDN_ERR_INVALID_ARG
+    assert sel(d, ss, _addr(1, 2), st) == gdn.GDN_ERR_INVALID_ARG
+    assert sel(d, ss, acc, _addr(0, 1024)) == gdn.GDN_ERR_INVALID_ARG  # state inside step_states
+    assert sel(d, ss, acc, st) in (gdn.GDN_OK, gdn.GDN_ERR_CUDA)
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.gdn_status_string(s)

@@ -222,6 +222,92 @@ def test_decode_continues_prefill():
 
 
 # ---------------------------------------------------------------------------
+# Multi-token decode (speculative verify) and rollback
+# ---------------------------------------------------------------------------
+
+def _multi_inputs(dtype, per_channel, d, B=5, T=6, H=3, seed=30):
+    w = DECODE.replace(B=B, H=H, dk=d, dv=d, decode_steps=0, T=T, dtype=dtype, per_channel=per_channel,
+                       h0_std=0.1, seed=seed)
+    return make_inputs(w)
+
+
+def _multi_oracle(x, n):
+    """Per sequence b: its first n[b] tokens from its own initial state, with the
+    state after every token (snapshot stride 1)."""
+    B = x.q.shape[0]
+    outs, finals, steps = [], [], []
+    for b in range(B):
+        nb = int(n[b])
+        sl = lambda t: t[b:b + 1, :nb]
+        if nb == 0:
+            outs.append(None); finals.append(x.h0[b].double().numpy()); steps.append(None)
+            continue
+        o, f, sn = oracle.gated_delta_rule(sl(x.q), sl(x.k), sl(x.v), sl(x.g), sl(x.beta), x.h0[b:b + 1],
+                                           snapshot_stride=1)
+        outs.append(o[0]); finals.append(f[0]); steps.append(sn[0])
+    return outs, finals, steps
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("per_channel", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_multi_commit(dtype, per_channel, d):
+    x = _multi_inputs(dtype, per_channel, d)
+    dx = to_dev(x)
+    st = dx.h0.clone()
+    out, steps = gdn.gdn_decode_multi(dx.q, dx.k, dx.v, dx.g, dx.beta, st, commit=True, step_states=True)
+    torch.cuda.synchronize()
+    B, T = x.q.shape[:2]
+    o_ref, f_ref, s_ref = _multi_oracle(x, [T] * B)
+    tol_o, tol_s = tolerances(x.q.dtype)
+    assert rel_l2(out, np.stack(o_ref)) <= tol_o
+    assert rel_l2(st, np.stack(f_ref)) <= tol_s
+    assert rel_l2(steps, np.stack(s_ref)) <= tol_s
+
+
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_decode_multi_rollback(per_channel):
+    """Verify drafts without committing (the pre-draft state stays bit for bit),
+    then adopt the state after each sequence's accepted prefix."""
+    x = _multi_inputs("bf16", per_channel, 128, B=6, T=8, seed=31)
+    dx = to_dev(x)
+    n = torch.tensor([0, 3, 8, 1, 5, 8], dtype=torch.int32)
+    st = dx.h0.clone()
+    out, steps = gdn.gdn_decode_multi(dx.q, dx.k, dx.v, dx.g, dx.beta, st, n_tokens=n.cuda(), commit=False,
+                                      step_states=True)
+    torch.cuda.synchronize()
+    assert torch.equal(st, dx.h0)
+    o_ref, f_ref, s_ref = _multi_oracle(x, n.tolist())
+    tol_o, tol_s = tolerances(x.q.dtype)
+    for b, nb in enumerate(n.tolist()):
+        if nb:
+            assert rel_l2(out[b, :nb], o_ref[b]) <= tol_o
+            assert rel_l2(steps[b, :nb], s_ref[b]) <= tol_s
+    accept = torch.tensor([0, 2, 8, 1, 0, 4], dtype=torch.int32)
+    gdn.gdn_state_select(steps, accept.cuda(), st)
+    # the same states by committing only the accepted tokens from the pre-draft state
+    st2 = dx.h0.clone()
+    gdn.gdn_decode_multi(dx.q, dx.k, dx.v, dx.g, dx.beta, st2, n_tokens=accept.cuda(), commit=True)
+    torch.cuda.synchronize()
+    assert torch.equal(st, st2)
+    _, f_acc, _ = _multi_oracle(x, accept.tolist())
+    assert rel_l2(st, np.stack(f_acc)) <= tol_s
+
+
+def test_decode_multi_equals_single_steps():
+    x = _multi_inputs("f32", False, 128, B=4, T=5, seed=32)
+    dx = to_dev(x)
+    st = dx.h0.clone()
+    out, _ = gdn.gdn_decode_multi(dx.q, dx.k, dx.v, dx.g, dx.beta, st)
+    st1 = dx.h0.clone()
+    outs = [gdn.gdn_decode_step(fresh(dx.q[:, t:t + 1]), fresh(dx.k[:, t:t + 1]), fresh(dx.v[:, t:t + 1]),
+                                fresh(dx.g[:, t:t + 1]), fresh(dx.beta[:, t:t + 1]), st1)[:, 0] for t in range(5)]
+    torch.cuda.synchronize()
+    assert rel_l2(out, torch.stack(outs, 1).cpu().double().numpy()) < 1e-6
+    assert rel_l2(st, st1.cpu().double().numpy()) < 1e-6
+
+
+# ---------------------------------------------------------------------------
 # The benchmark workloads at full size (oracle on sampled heads / sequences)
 # ---------------------------------------------------------------------------
 
