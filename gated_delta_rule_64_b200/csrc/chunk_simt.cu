@@ -92,8 +92,9 @@ template <typename Tin, int DK, int DV, bool PC>
 __global__ void __launch_bounds__(kPrepThreads)
 gdn_prep_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const float *__restrict__ beta, const int32_t *__restrict__ cu,
-              const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, float scale,
-              float *__restrict__ Wg, float *__restrict__ Ug, float *__restrict__ Pg, float *__restrict__ bg) {
+              const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk,
+              float scale, float *__restrict__ Wg, float *__restrict__ Ug, float *__restrict__ Pg,
+              float *__restrict__ bg) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto &sm = *reinterpret_cast<PrepSmem<Tin, DK, DV, PC> *>(smem_raw);
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
@@ -102,13 +103,14 @@ gdn_prep_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     const int L = (int)loc.len;
     const int tid = threadIdx.x;
     const int64_t ch = chunk * H + h;  // chunk-head index into the workspace
+    const int64_t hk = h / (H / Hk);   // query/key head of value head h
 
     // 1. inputs of the chunk (rows >= L are zero)
     for (int idx = tid; idx < C * DK; idx += kPrepThreads) {
         const int i = idx / DK, c = idx % DK;
         float kv = 0.f, qv = 0.f;
         if (i < L) {
-            const int64_t e = ((loc.start + i) * H + h) * DK + c;
+            const int64_t e = ((loc.start + i) * Hk + hk) * DK + c;
             kv = to_f32<Tin>(k[e]);
             qv = to_f32<Tin>(q[e]) * scale;
         }
@@ -227,7 +229,8 @@ template <typename Tin, int DK, int DV, bool PC>
 __global__ void __launch_bounds__(kScanThreads)
 gdn_scan_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const float *__restrict__ h0,
               const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T,
-              int64_t rows, int64_t H, int64_t max_chunks, float scale, int64_t snap_stride, int64_t n_snap,
+              int64_t rows, int64_t H, int64_t Hk, int64_t max_chunks, float scale, int64_t snap_stride,
+              int64_t n_snap,
               const float *__restrict__ Wg, const float *__restrict__ Ug, const float *__restrict__ Pg,
               const float *__restrict__ bg, Tin *__restrict__ out, float *final_state, float *__restrict__ snaps) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -259,7 +262,7 @@ gdn_scan_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const float 
             const int i = idx / DK, cc = idx % DK;
             float wq = 0.f, kq = 0.f, kg = 0.f;
             if (i < L) {
-                const int64_t e = ((tok0 + i) * H + h) * DK + cc;
+                const int64_t e = ((tok0 + i) * Hk + h / (H / Hk)) * DK + cc;
                 const float bi = PC ? bch[i * DK + cc] : bch[i];
                 const float bl = PC ? bch[(L - 1) * DK + cc] : bch[L - 1];
                 wq = Wg[ch * C * DK + idx];
@@ -342,7 +345,7 @@ gdn_status launch_typed(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s) 
         LaunchScope ls("gdn_prep_simt", s);
         kern<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kPrepThreads, smem, s>>>(
             (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows,
-            p.H, a.scale, W, U, P, b);
+            p.H, a.Hk, a.scale, W, U, P, b);
     }
     st = check_launch("gdn_prep_simt");
     if (st != GDN_OK) return st;
@@ -354,7 +357,7 @@ gdn_status launch_typed(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s) 
         if (a.N > 0x7fffffffLL || p.H > 65535) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
         LaunchScope ls("gdn_scan_simt", s);
         kern<<<dim3((unsigned)a.N, (unsigned)p.H, DV / kScanRows), kScanThreads, smem, s>>>(
-            (const Tin *)a.q, (const Tin *)a.k, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks,
+            (const Tin *)a.q, (const Tin *)a.k, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, p.max_chunks,
             a.scale, a.snapshot_stride, a.n_snap, W, U, P, b, (Tin *)a.out, a.final_state, a.snapshots);
     }
     return check_launch("gdn_scan_simt");

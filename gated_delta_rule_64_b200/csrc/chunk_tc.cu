@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kThreads, 3)
 gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
             const __grid_constant__ CUtensorMap mv, const float *__restrict__ g, const float *__restrict__ beta,
             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
-            int64_t H, float scale, uint8_t *__restrict__ blocks, int *err) {
+            int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     __shared__ uint64_t bar_ld, bar_mma;
@@ -117,10 +117,11 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
 
     if (tid == 0) {
         mbar_arrive_expect_tx(&bar_ld, 6 * 8192);
-        tma_load_3d(sm + 0, &mk, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + 16384, &mk, 64, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + 8192, &mq, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + 24576, &mq, 64, (int32_t)h, tok0, &bar_ld);
+        const int32_t hq = (int32_t)(h / (H / Hk));  // query/key head of value head h
+        tma_load_3d(sm + 0, &mk, 0, hq, tok0, &bar_ld);
+        tma_load_3d(sm + 16384, &mk, 64, hq, tok0, &bar_ld);
+        tma_load_3d(sm + 8192, &mq, 0, hq, tok0, &bar_ld);
+        tma_load_3d(sm + 24576, &mq, 64, hq, tok0, &bar_ld);
         tma_load_3d(sm + 32768, &mv, 0, (int32_t)h, tok0, &bar_ld);
         tma_load_3d(sm + 40960, &mv, 64, (int32_t)h, tok0, &bar_ld);
     }
@@ -348,7 +349,8 @@ __device__ __forceinline__ float *split_state(const ScanSplit &sp, int64_t n, in
 template <bool KDA, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32_t *__restrict__ cu,
-            const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t max_chunks,
+            const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk,
+            int64_t max_chunks,
             int64_t snap_stride, int64_t n_snap, const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out,
             float *final_state, float *__restrict__ snaps, const ScanSplit sp, int *err) {
     extern __shared__ unsigned char smem_raw[];
@@ -431,8 +433,8 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         if (KDA) {
             bulk_load(st + kStK, blk + kBlkKt, (uint32_t)kTcKt, bar);
         } else {
-            tma_load_3d(st + kStK, &mk, 0, (int32_t)h, tok, bar);
-            tma_load_3d(st + kStK + 8192, &mk, 64, (int32_t)h, tok, bar);
+            tma_load_3d(st + kStK, &mk, 0, (int32_t)(h / (H / Hk)), tok, bar);
+            tma_load_3d(st + kStK + 8192, &mk, 64, (int32_t)(h / (H / Hk)), tok, bar);
         }
         bulk_load(st + kStRest, blk + kBlkU, rest_bytes<KDA>(), bar);
     };
@@ -755,8 +757,8 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     memset(&mv, 0, sizeof mv);
     memset(&mg, 0, sizeof mg);
     if (p.rows > 0) {
-        if ((st = make_map(&mq, a.q, p.rows, p.H)) != GDN_OK) return st;
-        if ((st = make_map(&mk, a.k, p.rows, p.H)) != GDN_OK) return st;
+        if ((st = make_map(&mq, a.q, p.rows, a.Hk)) != GDN_OK) return st;
+        if ((st = make_map(&mk, a.k, p.rows, a.Hk)) != GDN_OK) return st;
         if ((st = make_map(&mv, a.v, p.rows, p.H)) != GDN_OK) return st;
         if (p.per_channel && (st = make_map(&mg, a.g, p.rows, p.H, true)) != GDN_OK) return st;
     }
@@ -780,7 +782,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         } else {
             LaunchScope ls("gdn_prep_tc", s);
             gdn_prep_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kPrepSmem, s>>>(
-                mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.scale, blocks, nullptr);
+                mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, nullptr);
             if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
         }
     }
@@ -789,7 +791,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         auto kern = p.per_channel ? gdn_scan_tc<true, false> : gdn_scan_tc<false, false>;
         LaunchScope ls("gdn_scan_tc", s);
         kern<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
-            mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap,
+            mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap,
             blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
         return check_launch("gdn_scan_tc");
     }
@@ -801,7 +803,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         LaunchScope ls("gdn_scan_tc", s);
         kern<<<dim3((unsigned)(a.N * per1), (unsigned)p.H), kThreads, kScanSmem, s>>>(
-            mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+            mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
             (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
     }
     if ((st = check_launch("gdn_scan_tc")) != GDN_OK) return st;
@@ -814,7 +816,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         LaunchScope ls("gdn_scan_tc", s);
         kern<<<dim3((unsigned)(a.N * per2), (unsigned)p.H), kThreads, kScanSmem, s>>>(
-            mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+            mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
             (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
     }
     return check_launch("gdn_scan_tc");

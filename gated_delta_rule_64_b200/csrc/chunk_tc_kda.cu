@@ -244,7 +244,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                 const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
                 const float *__restrict__ beta, const int32_t *__restrict__ cu, const int32_t *__restrict__ off,
-                int64_t N, int64_t T, int64_t rows, int64_t H, float scale, uint8_t *__restrict__ blocks, int *err) {
+                int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks,
+                int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     __shared__ uint64_t bar_g, bar_ld, bar_v, bar_mma;
@@ -272,10 +273,11 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
 #pragma unroll
         for (int qt = 0; qt < 4; ++qt) tma_load_3d(sm + kSmB + qt * 8192, &mg, 32 * qt, (int32_t)h, tok0, &bar_g);
         mbar_arrive_expect_tx(&bar_ld, 4 * 8192);
-        tma_load_3d(sm + kSmKQ, &mk, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + kSmKQ + 16384, &mk, 64, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + kSmKQ + 8192, &mq, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + kSmKQ + 24576, &mq, 64, (int32_t)h, tok0, &bar_ld);
+        const int32_t hq = (int32_t)(h / (H / Hk));  // query/key head of value head h
+        tma_load_3d(sm + kSmKQ, &mk, 0, hq, tok0, &bar_ld);
+        tma_load_3d(sm + kSmKQ + 16384, &mk, 64, hq, tok0, &bar_ld);
+        tma_load_3d(sm + kSmKQ + 8192, &mq, 0, hq, tok0, &bar_ld);
+        tma_load_3d(sm + kSmKQ + 24576, &mq, 64, hq, tok0, &bar_ld);
     }
     if (warp == 0) {
         tmem_alloc(&tmem_base, 128);
@@ -499,7 +501,7 @@ gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const C
     if (attr != cudaSuccess) return fail(GDN_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(attr));
     LaunchScope ls("gdn_prep_kda_tc", s);
     gdn_prep_kda_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kSmem, s>>>(
-        mq, mk, mv, mg, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.scale, blocks, nullptr);
+        mq, mk, mv, mg, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, nullptr);
     return check_launch("gdn_prep_kda_tc");
 }
 

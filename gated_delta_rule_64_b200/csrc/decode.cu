@@ -62,15 +62,16 @@ template <int DK, typename Tin, bool PER_CHANNEL>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
 gdn_decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                   const float *__restrict__ g, const float *__restrict__ beta, float *__restrict__ state,
-                  Tin *__restrict__ out, int dv, float scale) {
+                  Tin *__restrict__ out, int dv, int64_t H, int64_t Hk, float scale) {
     constexpr int VEC = DK / 32;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int64_t unit = blockIdx.x;  // b * H + h
+    const int64_t qu = (unit / H) * Hk + (unit % H) / (H / Hk);  // its query/key head
 
     float kr[VEC], qr[VEC], a[VEC];
-    load_in<VEC>(k + unit * DK + lane * VEC, kr);
-    load_in<VEC>(q + unit * DK + lane * VEC, qr);
+    load_in<VEC>(k + qu * DK + lane * VEC, kr);
+    load_in<VEC>(q + qu * DK + lane * VEC, qr);
     if (PER_CHANNEL) {
 #pragma unroll
         for (int c = 0; c < VEC; ++c) a[c] = expf(g[unit * DK + lane * VEC + c]);
@@ -133,11 +134,13 @@ gdn_status launch_dk(const gdn_desc &d, const void *q, const void *k, const void
     if (d.gate == GDN_GATE_CHANNEL) {
         LaunchScope ls("gdn_decode_kernel", s);
         gdn_decode_kernel<DK, Tin, true><<<grid, block, 0, s>>>(
-            (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, (Tin *)out, (int)d.dv, d.scale);
+            (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, (Tin *)out, (int)d.dv, d.H, qk_heads(d),
+            d.scale);
     } else {
         LaunchScope ls("gdn_decode_kernel", s);
         gdn_decode_kernel<DK, Tin, false><<<grid, block, 0, s>>>(
-            (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, (Tin *)out, (int)d.dv, d.scale);
+            (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, (Tin *)out, (int)d.dv, d.H, qk_heads(d),
+            d.scale);
     }
     return check_launch("gdn_decode_kernel");
 }

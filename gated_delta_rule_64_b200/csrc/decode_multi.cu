@@ -40,7 +40,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
 gdn_decode_multi_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                         const float *__restrict__ g, const float *__restrict__ beta,
                         const int32_t *__restrict__ n_tokens, float *__restrict__ state, int commit,
-                        Tin *__restrict__ out, float *__restrict__ step_states, int T, int64_t H, float scale) {
+                        Tin *__restrict__ out, float *__restrict__ step_states, int T, int64_t H, int64_t Hk,
+                        float scale) {
     constexpr int TPR = kWarps * 32 / DV, NCH = DK / 4 / TPR, VEC = DK / 32;  // NCH chunks per thread
     extern __shared__ float4 dm_raw[];
     float *sm = reinterpret_cast<float *>(dm_raw);
@@ -57,14 +58,15 @@ gdn_decode_multi_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, co
 
     // stage the tokens' vectors (warp w takes tokens w, w + 8, ...)
     for (int t = warp; t < n; t += kWarps) {
-        const int64_t tk = (b * T + t) * H + h;  // (b, t, h)
+        const int64_t tk = (b * T + t) * H + h;             // (b, t, h)
+        const int64_t tq = (b * T + t) * Hk + h / (H / Hk);  // its query/key head
         float *st = sm + (size_t)t * per_tok;
         float kq = 0.f;
 #pragma unroll
         for (int c = 0; c < VEC; ++c) {
             const int col = lane * VEC + c;
-            const float kc = to_f32<Tin>(k[tk * DK + col]);
-            const float qc = scale * to_f32<Tin>(q[tk * DK + col]);
+            const float kc = to_f32<Tin>(k[tq * DK + col]);
+            const float qc = scale * to_f32<Tin>(q[tq * DK + col]);
             const float a = expf(PER_CHANNEL ? g[tk * DK + col] : g[tk]);
             st[col] = a * kc;
             st[DK + col] = a * qc;
@@ -158,7 +160,7 @@ gdn_status launch_multi(const gdn_desc &d, const void *q, const void *k, const v
         LaunchScope ls("gdn_decode_multi_kernel", s);
         kern<<<(unsigned)units, kWarps * 32, smem, s>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta,
                                                         n_tokens, state, commit, (Tin *)out, step_states,
-                                                        (int)d.T, d.H, d.scale);
+                                                        (int)d.T, d.H, qk_heads(d), d.scale);
     }
     return check_launch("gdn_decode_multi_kernel");
 }

@@ -159,7 +159,9 @@ static gdn_status check_desc(const gdn_desc *d) {
         return fail(GDN_ERR_INVALID_ARG, "unknown dtype %d", d->dtype);
     if (d->gate != GDN_GATE_HEAD && d->gate != GDN_GATE_CHANNEL)
         return fail(GDN_ERR_INVALID_ARG, "unknown gate kind %d", d->gate);
-    if (d->reserved != 0) return fail(GDN_ERR_INVALID_ARG, "reserved field must be 0");
+    if (d->hk < 0 || d->hk > d->H || (d->hk > 0 && d->H % d->hk != 0))
+        return fail(GDN_ERR_INVALID_ARG, "hk must be 0 or a divisor of H (got %d for H = %lld)", d->hk,
+                    (long long)d->H);
     if (!isfinite(d->scale)) return fail(GDN_ERR_INVALID_ARG, "scale must be finite");
     // Keep every element index of every tensor well inside int64.
     const double elems = (double)d->B * (double)d->T * (double)d->H * (double)(d->dk > d->dv ? d->dk : d->dv);
@@ -265,7 +267,7 @@ gdn_status gdn_chunk_fwd(const gdn_desc *d, const void *q, const void *k, const 
     const int64_t n_snap = (snapshot_stride > 0 && !packed) ? d->T / snapshot_stride : 0;
     const int64_t rows = d->B * d->T;
     const size_t in_el = d->dtype == GDN_F32 ? 4 : 2;
-    const size_t qk_bytes = (size_t)rows * d->H * d->dk * in_el;
+    const size_t qk_bytes = (size_t)rows * qk_heads(*d) * d->dk * in_el;
     const size_t v_bytes = (size_t)rows * d->H * d->dv * in_el;
     const size_t g_bytes = (size_t)rows * d->H * (d->gate == GDN_GATE_CHANNEL ? d->dk : 1) * 4;
     const size_t b_bytes = (size_t)rows * d->H * 4;
@@ -313,6 +315,7 @@ gdn_status gdn_chunk_fwd(const gdn_desc *d, const void *q, const void *k, const 
     a.T = d->T;
     a.N = N;
     a.H = d->H;
+    a.Hk = qk_heads(*d);
     a.scale = d->scale;
     a.snapshot_stride = snapshot_stride;
     a.n_snap = n_snap;
@@ -340,8 +343,8 @@ gdn_status gdn_decode_step(const gdn_desc *d, const void *q, const void *k, cons
     const size_t in_el = d->dtype == GDN_F32 ? 4 : 2;
     const Range ro = range_of(out, (size_t)d->B * d->H * d->dv * in_el);
     const Range rs = range_of(state, (size_t)d->B * d->H * d->dv * d->dk * 4);
-    const Range ins[] = {range_of(q, (size_t)d->B * d->H * d->dk * in_el),
-                         range_of(k, (size_t)d->B * d->H * d->dk * in_el),
+    const Range ins[] = {range_of(q, (size_t)d->B * qk_heads(*d) * d->dk * in_el),
+                         range_of(k, (size_t)d->B * qk_heads(*d) * d->dk * in_el),
                          range_of(v, (size_t)d->B * d->H * d->dv * in_el),
                          range_of(log_gate, (size_t)d->B * d->H * (d->gate == GDN_GATE_CHANNEL ? d->dk : 1) * 4),
                          range_of(beta, (size_t)d->B * d->H * 4)};
@@ -375,7 +378,8 @@ gdn_status gdn_decode_multi(const gdn_desc *d, const void *q, const void *k, con
     const Range ro = range_of(out, bth * d->dv * in_el);
     const Range rs = range_of(state, (size_t)d->B * d->H * sbytes);
     const Range rss = range_of(step_states, step_states ? bth * sbytes : 0);
-    const Range ins[] = {range_of(q, bth * d->dk * in_el), range_of(k, bth * d->dk * in_el),
+    const size_t btk = (size_t)d->B * d->T * qk_heads(*d);
+    const Range ins[] = {range_of(q, btk * d->dk * in_el), range_of(k, btk * d->dk * in_el),
                          range_of(v, bth * d->dv * in_el),
                          range_of(log_gate, bth * (d->gate == GDN_GATE_CHANNEL ? d->dk : 1) * 4),
                          range_of(beta, bth * 4), range_of(n_tokens, n_tokens ? (size_t)d->B * 4 : 0)};

@@ -20,6 +20,9 @@ struct LaunchScope {
     int slot_;
 };
 
+// Query/key heads of a description (hk = 0 means H).
+inline int64_t qk_heads(const gdn_desc &d) { return d.hk > 0 ? d.hk : d.H; }
+
 // Records a failure reason for gdn_last_error() and returns `st`.
 gdn_status fail(gdn_status st, const char *fmt, ...);
 
@@ -63,6 +66,7 @@ struct ChunkArgs {
     const int32_t *cu_seqlens;  // nullptr: fixed-length sequences of length T
     int64_t T;                  // per-sequence length when not packed
     int64_t N, H;
+    int64_t Hk;                 // query/key heads (divides H)
     float scale;
     int64_t snapshot_stride;
     int64_t n_snap;             // snapshots per sequence (fixed-length only)

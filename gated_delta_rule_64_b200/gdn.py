@@ -32,7 +32,7 @@ EXPORTED = ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static",
 class GdnDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("H", ctypes.c_int64),
                 ("dk", ctypes.c_int64), ("dv", ctypes.c_int64), ("dtype", ctypes.c_int32),
-                ("gate", ctypes.c_int32), ("scale", ctypes.c_float), ("reserved", ctypes.c_int32)]
+                ("gate", ctypes.c_int32), ("scale", ctypes.c_float), ("hk", ctypes.c_int32)]
 
 
 class GdnKernelTime(ctypes.Structure):
@@ -114,14 +114,16 @@ def _need_cuda(*ts):
                 raise ValueError("tensors must be contiguous")
 
 
-def make_desc(B, T, H, dk, dv, dtype_code, per_channel, scale) -> GdnDesc:
+def make_desc(B, T, H, dk, dv, dtype_code, per_channel, scale, hk=0) -> GdnDesc:
+    """hk: query/key heads when fewer than the H value heads (0: H)."""
     return GdnDesc(B, T, H, dk, dv, dtype_code, GDN_GATE_CHANNEL if per_channel else GDN_GATE_HEAD,
-                   float(scale), 0)
+                   float(scale), int(hk) if hk != H else 0)
 
 
-def gdn_chunk_workspace_size(B, T, H, dk, dv, num_seqs, *, dtype=torch.bfloat16, per_channel=False) -> int:
+def gdn_chunk_workspace_size(B, T, H, dk, dv, num_seqs, *, dtype=torch.bfloat16, per_channel=False,
+                             hk=0) -> int:
     lib = load_library()
-    d = make_desc(B, T, H, dk, dv, GDN_F32 if dtype == torch.float32 else GDN_BF16, per_channel, 1.0)
+    d = make_desc(B, T, H, dk, dv, GDN_F32 if dtype == torch.float32 else GDN_BF16, per_channel, 1.0, hk)
     n = ctypes.c_size_t(0)
     _check(lib, lib.gdn_chunk_workspace_size(ctypes.byref(d), int(num_seqs), ctypes.byref(n)))
     return int(n.value)
@@ -131,14 +133,14 @@ def gdn_chunk_fwd(q, k, v, log_gate, beta, initial_state=None, cu_seqlens=None, 
                   snapshot_stride=0, out=None, final_state=True, snapshots=None, workspace=None,
                   stream=None):
     """Chunkwise prefill.  Shapes as in include/gdn.h:
-    q, k (B,T,H,dk); v (B,T,H,dv); log_gate (B,T,H) or (B,T,H,dk); beta (B,T,H);
+    q, k (B,T,Hk,dk) with Hk dividing H (value head h reads query/key head h // (H // Hk)); v (B,T,H,dv); log_gate (B,T,H) or (B,T,H,dk); beta (B,T,H);
     initial_state (N,H,dv,dk) fp32 or None; cu_seqlens int32 (N+1) on the device or None.
     final_state: True to allocate, a tensor to fill (may be initial_state), or None.
     Returns (out, final_state, snapshots)."""
     lib = load_library()
     _need_cuda(q, k, v, log_gate, beta, initial_state, cu_seqlens)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, Hq, dk = q.shape
+    H, dv = v.shape[-2], v.shape[-1]  # value heads; q and k may have fewer (Hq divides H)
     per_channel = log_gate.dim() == 4
     N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
     dev = q.device
@@ -151,9 +153,9 @@ def gdn_chunk_fwd(q, k, v, log_gate, beta, initial_state=None, cu_seqlens=None, 
     if snapshot_stride and snapshots is None:
         n_snap = T // snapshot_stride
         snapshots = torch.empty((B, n_snap, H, dv, dk), dtype=torch.float32, device=dev)
-    d = make_desc(B, T, H, dk, dv, _dtype_code(q), per_channel, scale)
+    d = make_desc(B, T, H, dk, dv, _dtype_code(q), per_channel, scale, Hq)
     if workspace is None:
-        ws_bytes = gdn_chunk_workspace_size(B, T, H, dk, dv, N, dtype=q.dtype, per_channel=per_channel)
+        ws_bytes = gdn_chunk_workspace_size(B, T, H, dk, dv, N, dtype=q.dtype, per_channel=per_channel, hk=Hq)
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     _need_cuda(out, final_state, snapshots, workspace)
     st = lib.gdn_chunk_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_gate), _ptr(beta),
@@ -172,8 +174,8 @@ def gdn_chunk_fwd_static(q, k, v, log_gate, beta, initial_state=None, cu_seqlens
     torch when they are not passed; a caller that cannot allocate passes them."""
     lib = load_library()
     _need_cuda(q, k, v, log_gate, beta, initial_state, cu_seqlens)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, Hq, dk = q.shape
+    H, dv = v.shape[-2], v.shape[-1]  # value heads; q and k may have fewer (Hq divides H)
     per_channel = log_gate.dim() == 4
     N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
     dev = q.device
@@ -186,7 +188,7 @@ def gdn_chunk_fwd_static(q, k, v, log_gate, beta, initial_state=None, cu_seqlens
     if snapshot_stride and snapshots is None:
         snapshots = torch.empty((B, T // snapshot_stride, H, dv, dk), dtype=torch.float32, device=dev)
     _need_cuda(out, final_state, snapshots)
-    d = make_desc(B, T, H, dk, dv, _dtype_code(q), per_channel, scale)
+    d = make_desc(B, T, H, dk, dv, _dtype_code(q), per_channel, scale, Hq)
     st = lib.gdn_chunk_fwd_static(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_gate), _ptr(beta),
                                   _ptr(initial_state), _ptr(cu_seqlens), int(N), int(snapshot_stride), _ptr(out),
                                   _ptr(final_state), _ptr(snapshots), _stream(stream))
@@ -204,7 +206,7 @@ def gdn_decode_step(q, k, v, log_gate, beta, state, *, scale=1.0, out=None, stre
     if out is None:
         out = torch.empty((B, 1, H, dv), dtype=q.dtype, device=q.device)
     _need_cuda(out)
-    d = make_desc(B, 1, H, dk, dv, _dtype_code(q), per_channel, scale)
+    d = make_desc(B, 1, H, dk, dv, _dtype_code(q), per_channel, scale, q.shape[-2])
     st = lib.gdn_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_gate), _ptr(beta), _ptr(state),
                              _ptr(out), _stream(stream))
     _check(lib, st)
@@ -219,15 +221,15 @@ def gdn_decode_multi(q, k, v, log_gate, beta, state, *, n_tokens=None, commit=Tr
     step_states: True to allocate, a (B,T,H,dv,dk) fp32 tensor, or None.  Returns (out, step_states)."""
     lib = load_library()
     _need_cuda(q, k, v, log_gate, beta, state)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, Hq, dk = q.shape
+    H, dv = v.shape[-2], v.shape[-1]
     per_channel = log_gate.dim() == 4
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     if step_states is True:
         step_states = torch.empty((B, T, H, dv, dk), dtype=torch.float32, device=q.device)
     _need_cuda(out)
-    d = make_desc(B, T, H, dk, dv, _dtype_code(q), per_channel, scale)
+    d = make_desc(B, T, H, dk, dv, _dtype_code(q), per_channel, scale, Hq)
     st = lib.gdn_decode_multi(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_gate), _ptr(beta),
                               _ptr(n_tokens), _ptr(state), 1 if commit else 0, _ptr(out), _ptr(step_states),
                               _stream(stream))

@@ -79,7 +79,8 @@ typedef struct gdn_desc {
     int32_t dtype; /* gdn_dtype of q, k, v and out (gates, beta, states: fp32)  */
     int32_t gate;  /* gdn_gate_kind                                              */
     float scale;   /* multiplies q before the read; 1.0 gives o_t = S_t q_t      */
-    int32_t reserved; /* must be 0                                                */
+    int32_t hk;    /* query/key heads: 0 (= H) or a divisor of H; value head h
+                      reads query/key head h / (H / hk)                         */
 } gdn_desc;
 
 /* ---------------------------------------------------------------------------

@@ -81,7 +81,9 @@ def test_workspace_size(lib):
     ("T", -1, gdn.GDN_ERR_INVALID_ARG),
     ("dtype", 7, gdn.GDN_ERR_INVALID_ARG),
     ("gate", 3, gdn.GDN_ERR_INVALID_ARG),
-    ("reserved", 1, gdn.GDN_ERR_INVALID_ARG),
+    ("hk", 2, gdn.GDN_ERR_INVALID_ARG),   # H = 3: not a divisor
+    ("hk", -1, gdn.GDN_ERR_INVALID_ARG),
+    ("hk", 6, gdn.GDN_ERR_INVALID_ARG),
     ("scale", float("nan"), gdn.GDN_ERR_INVALID_ARG),
 ])
 def test_bad_descriptor(lib, field, value, status):

@@ -11,6 +11,7 @@ import oracle
 from gated_delta_rule_64_b200 import gdn
 from gated_delta_rule_64_b200.inputs import (DECODE, KDA_PACKED, LONG_SNAPSHOTS, PREFILL_BF16, TINY_F32,
                                              Workload, make_inputs)
+from gated_delta_rule_64_b200.inputs import Inputs
 from tests.gpu_util import check, rel_l2, run_gpu, run_oracle, to_dev, tolerances
 
 pytestmark = pytest.mark.gpu
@@ -305,6 +306,66 @@ def test_decode_multi_equals_single_steps():
     torch.cuda.synchronize()
     assert rel_l2(out, torch.stack(outs, 1).cpu().double().numpy()) < 1e-6
     assert rel_l2(st, st1.cpu().double().numpy()) < 1e-6
+
+
+# ---------------------------------------------------------------------------
+# Shared query/key heads (fewer q/k heads than value heads)
+# ---------------------------------------------------------------------------
+
+def _share_qk(x, hk):
+    """Keep the first hk query/key heads; the oracle sees them repeated so that
+    value head h reads query/key head h // (H // hk)."""
+    H = x.q.shape[-2]
+    rep = lambda t: t.repeat_interleave(H // hk, dim=-2)
+    q_small, k_small = x.q[..., :hk, :].contiguous(), x.k[..., :hk, :].contiguous()
+    ref = Inputs(q=rep(q_small), k=rep(k_small), v=x.v, g=x.g, beta=x.beta, h0=x.h0, cu_seqlens=x.cu_seqlens,
+                 workload=x.workload)
+    gpu = Inputs(q=q_small, k=k_small, v=x.v, g=x.g, beta=x.beta, h0=x.h0, cu_seqlens=x.cu_seqlens,
+                 workload=x.workload)
+    return gpu, ref
+
+
+@pytest.mark.parametrize("dtype,per_channel", [("bf16", False), ("bf16", True), ("f32", False), ("f32", True)])
+@pytest.mark.parametrize("hk", [1, 2])
+def test_shared_qk_heads_prefill(dtype, per_channel, hk):
+    x = make_inputs(SMALL.replace(H=4, T=200, dtype=dtype, per_channel=per_channel, seed=40), lengths=None)
+    gx, rx = _share_qk(x, hk)
+    out, fin, _ = run_gpu(gx)
+    o_ref, f_ref, _ = run_oracle(rx)
+    tol_o, tol_s = tolerances(x.q.dtype)
+    assert rel_l2(out, o_ref) <= tol_o and rel_l2(fin, f_ref) <= tol_s
+
+
+def test_shared_qk_heads_packed_and_split():
+    # packed sequences, then one long fixed-length sequence (split scan), 4 value heads on 2 q/k heads
+    x = make_inputs(SMALL.replace(H=4, seed=41), lengths=[70, 1, 300, 64])
+    gx, rx = _share_qk(x, 2)
+    out, fin, _ = run_gpu(gx)
+    o_ref, f_ref, _ = run_oracle(rx)
+    assert rel_l2(out, o_ref) <= 2e-2 and rel_l2(fin, f_ref) <= 1e-2
+    x = make_inputs(SMALL.replace(B=1, T=8192, H=2, h0_std=0.1, seed=42))
+    gx, rx = _share_qk(x, 1)
+    out, fin, snaps = run_gpu(gx, snapshot_stride=2048)
+    o_ref, f_ref, s_ref = run_oracle(rx, snapshot_stride=2048)
+    assert rel_l2(out, o_ref) <= 2e-2 and rel_l2(fin, f_ref) <= 1e-2 and rel_l2(snaps, s_ref) <= 1e-2
+
+
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_shared_qk_heads_decode(per_channel):
+    x = _multi_inputs("bf16", per_channel, 128, B=4, T=5, H=4, seed=43)
+    gx, rx = _share_qk(x, 2)
+    dx = to_dev(gx)
+    st = dx.h0.clone()
+    out, steps = gdn.gdn_decode_multi(dx.q, dx.k, dx.v, dx.g, dx.beta, st, step_states=True)
+    st1 = dx.h0.clone()
+    out1 = gdn.gdn_decode_step(fresh(dx.q[:, :1]), fresh(dx.k[:, :1]), fresh(dx.v[:, :1]), fresh(dx.g[:, :1]),
+                               fresh(dx.beta[:, :1]), st1)
+    torch.cuda.synchronize()
+    o_ref, f_ref, s_ref = _multi_oracle(rx, [5] * 4)
+    tol_o, tol_s = tolerances(x.q.dtype)
+    assert rel_l2(out, np.stack(o_ref)) <= tol_o and rel_l2(st, np.stack(f_ref)) <= tol_s
+    assert rel_l2(out1[:, 0], np.stack(o_ref)[:, 0]) <= tol_o
+    assert rel_l2(st1, np.stack(s_ref)[:, 0]) <= tol_s
 
 
 # ---------------------------------------------------------------------------
