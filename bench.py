@@ -423,8 +423,77 @@ def run_gpu(args):
     return 0
 
 
-SECONDARY = {"kda": "KDA_PACKED", "long": "LONG_SNAPSHOTS", "tiny": "TINY_F32", "spec": "DECODE"}
+SECONDARY = {"kda": "KDA_PACKED", "long": "LONG_SNAPSHOTS", "tiny": "TINY_F32", "spec": "DECODE",
+             "prerule": "PREFILL_BF16"}
 SPEC_K = 4  # draft tokens per sequence in the speculative-decoding measurement
+
+
+def run_prerule(args) -> int:
+    """The work before the recurrence (gdn_prerule: short convolution + SiLU, q/k length,
+    gates) on the prefill workload's shape, with the convolution history read and
+    written, then the same followed by the chunked prefill (the layer core)."""
+    import torch
+
+    from gated_delta_rule_64_b200 import gdn
+    from gated_delta_rule_64_b200.inputs import PREFILL_BF16, make_prerule_inputs
+
+    torch.cuda.set_device(0)
+    pk = peaks()
+    w = PREFILL_BF16
+    pi = make_prerule_inputs(B=w.B, T=w.T, H=w.H, hk=w.H, dk=w.dk, dv=w.dv, dtype=w.dtype, seed=w.seed)
+    d = lambda t: t.cuda().contiguous()
+    x, a, b, cw, al, dtb, hist = (d(t) for t in (pi.x, pi.a, pi.b, pi.conv_w, pi.A_log, pi.dt_bias, pi.hist))
+    h0 = torch.zeros((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    B, T, C = x.shape
+    K = cw.shape[1]
+    ws = torch.empty(gdn.gdn_chunk_workspace_size(B, T, w.H, w.dk, w.dv, B), dtype=torch.uint8, device="cuda")
+    res = {}
+    modes = {
+        "prerule": lambda: gdn.gdn_prerule(x, a, b, cw, al, dtb, hk=w.H, dk=w.dk, H=w.H, dv=w.dv,
+                                           conv_state_in=hist, conv_state_out=hist, stream=stream),
+        "prerule+prefill": lambda: gdn.gdn_chunk_fwd(*gdn.gdn_prerule(x, a, b, cw, al, dtb, hk=w.H, dk=w.dk, H=w.H,
+                                                                      dv=w.dv, conv_state_in=hist,
+                                                                      conv_state_out=hist, stream=stream),
+                                                     h0, final_state=h0, workspace=ws, stream=stream),
+    }
+    el = x.element_size()
+    pre_bytes = B * T * (C * el + 2 * w.H * el) + 2 * B * C * (K - 1) * 4 + B * T * C * el + B * T * w.H * 8
+    clocks = ClockSampler(0)
+    clocks.start()
+    for name, f in modes.items():
+        for _ in range(args.warmup):
+            f()
+        torch.cuda.synchronize()
+        gdn.profile_read()
+        gdn.profile_enable(True)
+        clocks.mark_begin()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks.mark_end()
+        gdn.profile_enable(False)
+        kern = gdn.profile_read()
+        ms = e0.elapsed_time(e1) / args.steps
+        res[name] = {"ms_per_step": ms, "tokens_per_s": B * T / (ms * 1e-3),
+                     "kernels_us": {n: t / max(1, c) * 1e3 for n, (c, t) in kern.items()}}
+    pre_us = res["prerule"]["kernels_us"].get("gdn_prerule_kernel", 0.0) + \
+        res["prerule"]["kernels_us"].get("gdn_prerule_history", 0.0)
+    achieved = pre_bytes / (pre_us * 1e-6) / 1e9 if pre_us else None
+    clk = clocks.stop()
+    line = {"metric": "pre-rule tokens/s (secondary workload)", "value": res["prerule"]["tokens_per_s"], "unit": UNIT,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": {"workload": f"raw projections of {w.name}, convolution width {K}", "channels": C},
+            "modes": res,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"] if achieved else None, "algorithmic_bytes": pre_bytes},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_spec(args) -> int:
@@ -598,8 +667,8 @@ def main(argv=None):
                     help="run three calls of one workload and exit (for ncu captures; prints nothing to time)")
     ap.add_argument("--workload", choices=["prefill"] + sorted(SECONDARY), default="prefill",
                     help="prefill (default): the headline line; kda / long / tiny: time that chunked "
-                         "workload instead; spec: multi-token decode / speculative verify (one GPU, its own "
-                         "JSON line)")
+                         "workload instead; spec: multi-token decode / speculative verify; prerule: the work before "
+                         "the recurrence (one GPU, its own JSON line)")
     args = ap.parse_args(argv)
     if args.profile:
         return run_profile(args.profile)
@@ -609,6 +678,8 @@ def main(argv=None):
         return run_reference(args)
     if args.workload == "spec":
         return run_spec(args)
+    if args.workload == "prerule":
+        return run_prerule(args)
     if args.workload != "prefill":
         return run_secondary(args)
     return run_gpu(args)

@@ -392,6 +392,70 @@ gdn_status gdn_decode_multi(const gdn_desc *d, const void *q, const void *k, con
                                (cudaStream_t)stream);
 }
 
+gdn_status gdn_prerule(const gdn_desc *d, const void *x, const void *a, const void *b, const float *conv_w,
+                       int32_t K, const float *A_log, const float *dt_bias, const int32_t *cu_seqlens,
+                       int32_t num_seqs, const float *conv_state_in, float *conv_state_out, void *q, void *k,
+                       void *v, float *log_gate, float *beta, gdn_stream_t stream) {
+    g_last_error[0] = 0;
+    gdn_status st = check_desc(d);
+    if (st != GDN_OK) return st;
+    if (d->gate != GDN_GATE_HEAD)
+        return fail(GDN_ERR_UNSUPPORTED, "the pre-rule gate formula is the per-head one");
+    if (K < 1 || K > 4) return fail(GDN_ERR_UNSUPPORTED, "convolution width %d (1 .. 4 supported)", K);
+    const bool packed = cu_seqlens != nullptr;
+    if (packed && d->B != 1) return fail(GDN_ERR_INVALID_ARG, "packed sequences need B == 1");
+    if (packed && num_seqs < 0) return fail(GDN_ERR_INVALID_ARG, "num_seqs < 0");
+    const int64_t N = packed ? num_seqs : d->B;
+    const int64_t rows = d->B * d->T, Hk = qk_heads(*d);
+    const int64_t C = 2 * Hk * d->dk + d->H * d->dv;
+    if (rows == 0 && N == 0) return GDN_OK;
+    if (!x || !a || !b || !conv_w || !A_log || !dt_bias || !q || !k || !v || !log_gate || !beta)
+        return fail(GDN_ERR_INVALID_ARG, "x, a, b, conv_w, A_log, dt_bias and the five outputs are required");
+    const size_t el = d->dtype == GDN_F32 ? 4 : 2;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(k) || !aligned16(v))
+        return fail(GDN_ERR_INVALID_ARG, "x, q, k and v must be 16-byte aligned");
+    if (((uintptr_t)a % el) || ((uintptr_t)b % el) || !aligned4(conv_w) || !aligned4(A_log) || !aligned4(dt_bias) ||
+        !aligned4(log_gate) || !aligned4(beta) || (conv_state_in && !aligned4(conv_state_in)) ||
+        (conv_state_out && !aligned4(conv_state_out)) || (cu_seqlens && !aligned4(cu_seqlens)))
+        return fail(GDN_ERR_INVALID_ARG, "a, b: element-aligned; conv_w, A_log, dt_bias, gates, states, "
+                                         "cu_seqlens: 4-byte aligned");
+    const size_t hist_bytes = (size_t)N * C * (K - 1) * 4;
+    const Range outs[] = {range_of(q, (size_t)rows * Hk * d->dk * el), range_of(k, (size_t)rows * Hk * d->dk * el),
+                          range_of(v, (size_t)rows * d->H * d->dv * el), range_of(log_gate, (size_t)rows * d->H * 4),
+                          range_of(beta, (size_t)rows * d->H * 4),
+                          range_of(conv_state_out, conv_state_out ? hist_bytes : 0)};
+    const Range ins[] = {range_of(x, (size_t)rows * C * el), range_of(a, (size_t)rows * d->H * el),
+                         range_of(b, (size_t)rows * d->H * el), range_of(conv_w, (size_t)C * K * 4),
+                         range_of(A_log, (size_t)d->H * 4), range_of(dt_bias, (size_t)d->H * 4),
+                         range_of(cu_seqlens, cu_seqlens ? (size_t)(N + 1) * 4 : 0)};
+    for (int i = 0; i < 6; ++i) {
+        for (const Range &r : ins)
+            if (overlaps(outs[i], r)) return fail(GDN_ERR_INVALID_ARG, "an output overlaps an input");
+        for (int j = i + 1; j < 6; ++j)
+            if (overlaps(outs[i], outs[j])) return fail(GDN_ERR_INVALID_ARG, "outputs overlap");
+    }
+    // the new history may replace the old one in place, but not overlap it partly
+    if (conv_state_in && conv_state_out && conv_state_in != conv_state_out &&
+        overlaps(range_of(conv_state_in, hist_bytes), range_of(conv_state_out, hist_bytes)))
+        return fail(GDN_ERR_INVALID_ARG, "conv_state_out partially overlaps conv_state_in");
+    PreruleArgs pa{};
+    pa.dtype = d->dtype;
+    pa.K = K;
+    pa.T = d->T;
+    pa.N = N;
+    pa.rows = rows;
+    pa.H = d->H;
+    pa.Hk = Hk;
+    pa.dk = d->dk;
+    pa.dv = d->dv;
+    pa.x = x; pa.a = a; pa.b = b;
+    pa.conv_w = conv_w; pa.A_log = A_log; pa.dt_bias = dt_bias;
+    pa.cu_seqlens = cu_seqlens;
+    pa.hist_in = conv_state_in; pa.hist_out = conv_state_out;
+    pa.q = q; pa.k = k; pa.v = v; pa.g = log_gate; pa.beta = beta;
+    return launch_prerule(pa, (cudaStream_t)stream);
+}
+
 gdn_status gdn_state_select(const gdn_desc *d, const float *step_states, const int32_t *accept, float *state,
                             gdn_stream_t stream) {
     g_last_error[0] = 0;

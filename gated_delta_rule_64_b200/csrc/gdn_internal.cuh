@@ -103,6 +103,20 @@ gdn_status launch_decode_multi(const gdn_desc &d, const void *q, const void *k, 
 gdn_status launch_state_select(const gdn_desc &d, const float *step_states, const int32_t *accept, float *state,
                                cudaStream_t s);
 
+// The work before the recurrence (short convolution, SiLU, q/k length, gates).
+struct PreruleArgs {
+    int dtype, K;
+    int64_t T, N, rows, H, Hk, dk, dv;
+    const void *x, *a, *b;
+    const float *conv_w, *A_log, *dt_bias;
+    const int32_t *cu_seqlens;  // nullptr: N sequences of T tokens
+    const float *hist_in;
+    float *hist_out;
+    void *q, *k, *v;
+    float *g, *beta;
+};
+gdn_status launch_prerule(const PreruleArgs &a, cudaStream_t s);
+
 // ---------------------------------------------------------------------------
 // Device helpers
 // ---------------------------------------------------------------------------

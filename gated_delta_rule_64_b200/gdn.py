@@ -25,8 +25,8 @@ GDN_F32, GDN_BF16 = 0, 1
 GDN_GATE_HEAD, GDN_GATE_CHANNEL = 0, 1
 
 EXPORTED = ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
-            "gdn_decode_multi", "gdn_state_select", "gdn_status_string", "gdn_last_error", "gdn_profile_enable",
-            "gdn_profile_read")
+            "gdn_decode_multi", "gdn_state_select", "gdn_prerule", "gdn_status_string", "gdn_last_error",
+            "gdn_profile_enable", "gdn_profile_read")
 
 
 class GdnDesc(ctypes.Structure):
@@ -67,6 +67,7 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn_decode_multi.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
         lib.gdn_state_select.argtypes = [dp, vp, vp, vp, vp]
+        lib.gdn_prerule.argtypes = [dp, vp, vp, vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn_status_string.argtypes = [ctypes.c_int]
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_last_error.argtypes = []
@@ -74,7 +75,8 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_profile_enable.argtypes = [ctypes.c_int]
         lib.gdn_profile_read.argtypes = [ctypes.POINTER(GdnKernelTime), i32, ctypes.POINTER(i32)]
         for name in ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
-                     "gdn_decode_multi", "gdn_state_select", "gdn_profile_enable", "gdn_profile_read"):
+                     "gdn_decode_multi", "gdn_state_select", "gdn_prerule", "gdn_profile_enable",
+                     "gdn_profile_read"):
             getattr(lib, name).restype = ctypes.c_int
         if path == LIB_PATH:
             _lib = lib
@@ -235,6 +237,31 @@ def gdn_decode_multi(q, k, v, log_gate, beta, state, *, n_tokens=None, commit=Tr
                               _stream(stream))
     _check(lib, st)
     return out, step_states
+
+
+def gdn_prerule(x, a, b, conv_w, A_log, dt_bias, *, hk, dk, H, dv, cu_seqlens=None, conv_state_in=None,
+                conv_state_out=None, stream=None):
+    """Short convolution + SiLU, length-1 q/k and the gates from the raw projections.
+    x (B,T,2*hk*dk+H*dv); a, b (B,T,H) in x's dtype; conv_w (C,K) fp32; A_log, dt_bias (H,) fp32;
+    conv states (N,C,K-1) fp32 or None (conv_state_out may be conv_state_in).
+    Returns (q (B,T,hk,dk), k, v (B,T,H,dv), log_gate (B,T,H), beta (B,T,H))."""
+    lib = load_library()
+    _need_cuda(x, a, b, conv_w, A_log, dt_bias, cu_seqlens, conv_state_in, conv_state_out)
+    B, T, C = x.shape
+    K = conv_w.shape[1]
+    N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+    dev = x.device
+    q = torch.empty((B, T, hk, dk), dtype=x.dtype, device=dev)
+    k = torch.empty((B, T, hk, dk), dtype=x.dtype, device=dev)
+    v = torch.empty((B, T, H, dv), dtype=x.dtype, device=dev)
+    g = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    beta = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    d = make_desc(B, T, H, dk, dv, _dtype_code(x), False, 1.0, hk)
+    st = lib.gdn_prerule(ctypes.byref(d), _ptr(x), _ptr(a), _ptr(b), _ptr(conv_w), int(K), _ptr(A_log),
+                         _ptr(dt_bias), _ptr(cu_seqlens), int(N), _ptr(conv_state_in), _ptr(conv_state_out),
+                         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _stream(stream))
+    _check(lib, st)
+    return q, k, v, g, beta
 
 
 def gdn_state_select(step_states, accept, state, *, stream=None):

@@ -161,3 +161,49 @@ def make_inputs(w: Workload, *, lengths=None, heads: int | None = None) -> Input
         h0=None if h0 is None else torch.from_numpy(h0),
         cu_seqlens=None if cu is None else torch.from_numpy(cu),
         workload=w.replace(H=H))
+
+
+@dataclass
+class PreruleInputs:
+    """Raw projections of a Gated DeltaNet layer (CPU tensors): x (B, T, C) with
+    C = 2 hk dk + H dv, a and b (B, T, H) in `dtype`; conv_w (C, K), A_log and
+    dt_bias (H,) and an optional convolution history (N, C, K-1) in fp32."""
+    x: torch.Tensor
+    a: torch.Tensor
+    b: torch.Tensor
+    conv_w: torch.Tensor
+    A_log: torch.Tensor
+    dt_bias: torch.Tensor
+    hist: torch.Tensor | None
+    cu_seqlens: torch.Tensor | None
+    hk: int
+    dk: int
+    H: int
+    dv: int
+
+
+def make_prerule_inputs(*, B, T, H, hk, dk, dv, K=4, dtype="bf16", lengths=None, history=True,
+                        seed=0) -> PreruleInputs:
+    """Seeded raw projections, drawn in this order: packed lengths (if any), x ~ N(0,1),
+    a ~ N(0,1), b ~ N(0,1), conv_w ~ N(0, 1/K), A_log ~ U(0, log 16), dt_bias ~ N(0, 0.25),
+    history ~ N(0,1).  Values are rounded to `dtype` where the layer holds them in it."""
+    rng = np.random.default_rng(seed)
+    cu = None
+    if lengths is not None:
+        lengths = np.asarray(lengths, dtype=np.int64)
+        cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+        B, T = 1, int(cu[-1])
+    N = len(cu) - 1 if cu is not None else B
+    C = 2 * hk * dk + H * dv
+    x = _normal(rng, (B, T, C))
+    a = _normal(rng, (B, T, H))
+    b = _normal(rng, (B, T, H))
+    conv_w = (_normal(rng, (C, K)) / np.float32(np.sqrt(K))).astype(np.float32)
+    A_log = rng.uniform(0.0, np.log(16.0), size=H).astype(np.float32)
+    dt_bias = (rng.standard_normal(H) * 0.5).astype(np.float32)
+    hist = _normal(rng, (N, C, K - 1)) if history else None
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    t = lambda z: torch.from_numpy(z)
+    return PreruleInputs(x=t(x).to(td), a=t(a).to(td), b=t(b).to(td), conv_w=t(conv_w), A_log=t(A_log),
+                         dt_bias=t(dt_bias), hist=None if hist is None else t(hist),
+                         cu_seqlens=None if cu is None else t(cu), hk=hk, dk=dk, H=H, dv=dv)

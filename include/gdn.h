@@ -258,6 +258,47 @@ gdn_status gdn_decode_multi(const gdn_desc *d,
 gdn_status gdn_state_select(const gdn_desc *d, const float *step_states, const int32_t *accept,
                             float *state, gdn_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * gdn_prerule -- the layer's work before the recurrence, from its raw
+ * projections, producing the inputs of gdn_chunk_fwd / gdn_decode_step /
+ * gdn_decode_multi ("Attention, Part 4: Linear Attention, Gated DeltaNet and
+ * Hybrid Models", section 6, "Where alpha and beta come from" and the paragraph
+ * after it: short convolution, SiLU and length-1 queries and keys, beta =
+ * sigmoid(b), g = -exp(A_log) softplus(a + dt_bias); "From Traditional
+ * Attention to hybrid ones", "vLLM Storage": the convolution history kept per
+ * live sequence).
+ *
+ * For every token of every sequence and every channel c of the mixed projection
+ * x = [q heads (hk x d_k) | k heads (hk x d_k) | v heads (H x d_v)]:
+ *     y_c = SiLU( sum_{j<K} conv_w[c, j] * x_c(t - (K-1) + j) )
+ * (tap K-1 on the current token; inputs before the sequence's first token from
+ * conv_state_in, the sequence's last K-1 raw inputs oldest first, zeros if NULL);
+ * q, k = y / sqrt(|y|^2 + 1e-6) per head, v = y (written in d->dtype);
+ * beta = sigmoid(b), log_gate = -exp(A_log[h]) softplus(a + dt_bias[h]) (fp32).
+ * If conv_state_out != NULL it receives each sequence's last K-1 raw inputs
+ * (older history where the sequence is shorter); it may be conv_state_in.
+ *
+ *   d          B, T, H (value heads), hk, d_k, d_v, dtype; gate must be
+ *              GDN_GATE_HEAD (the formula is the per-head one)
+ *   x          (B, T, 2 hk d_k + H d_v) in d->dtype, 16-byte aligned
+ *   a, b       (B, T, H) in d->dtype
+ *   conv_w     (2 hk d_k + H d_v, K) fp32;  K in 1 .. 4
+ *   A_log, dt_bias (H) fp32
+ *   cu_seqlens / num_seqs  packed sequences as for gdn_chunk_fwd (B == 1), or
+ *              NULL: B sequences of T tokens (a decode step is T = 1)
+ *   conv_state_in, conv_state_out  (N, 2 hk d_k + H d_v, K-1) fp32, or NULL
+ *   q, k       (B, T, hk, d_k); v (B, T, H, d_v) -- 16-byte aligned
+ *   log_gate, beta (B, T, H) fp32
+ * Rows of a packed batch outside every sequence are not written.  Outputs must
+ * not overlap the inputs or each other.
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_prerule(const gdn_desc *d, const void *x, const void *a, const void *b,
+                       const float *conv_w, int32_t K, const float *A_log, const float *dt_bias,
+                       const int32_t *cu_seqlens, int32_t num_seqs,
+                       const float *conv_state_in, float *conv_state_out,
+                       void *q, void *k, void *v, float *log_gate, float *beta,
+                       gdn_stream_t stream);
+
 /* Static description of a status code. */
 const char *gdn_status_string(gdn_status s);
 

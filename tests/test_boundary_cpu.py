@@ -225,6 +225,36 @@ def test_state_select_validation(lib):
     assert sel(d, ss, acc, st) in (gdn.GDN_OK, gdn.GDN_ERR_CUDA)
 
 
+def _prerule(lib, d, p, K=4, cu=None, n=0):
+    # argument order: x, a, b, conv_w, A_log, dt_bias, state_in, state_out, q, k, v, log_gate, beta
+    return lib.gdn_prerule(ctypes.byref(d), p[0], p[1], p[2], p[3], K, p[4], p[5], cu, n, p[6], p[7], p[8], p[9],
+                           p[10], p[11], p[12], None)
+
+
+def test_prerule_validation(lib):
+    p = [_addr(i) for i in range(13)]
+    d = _desc(B=2, T=16, H=4, dk=64, dv=64)
+    assert _prerule(lib, d, p, K=0) == gdn.GDN_ERR_UNSUPPORTED
+    assert _prerule(lib, d, p, K=5) == gdn.GDN_ERR_UNSUPPORTED
+    assert _prerule(lib, _desc(B=2, T=16, H=4, dk=64, dv=64, gate=gdn.GDN_GATE_CHANNEL), p) == gdn.GDN_ERR_UNSUPPORTED
+    assert _prerule(lib, d, p, cu=_addr(13), n=2) == gdn.GDN_ERR_INVALID_ARG  # packed needs B == 1
+    q = list(p)
+    q[8] = None
+    assert _prerule(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[0] = _addr(0, 8)  # x not 16-byte aligned
+    assert _prerule(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[9] = _addr(0, 64)  # k inside x
+    assert _prerule(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[7] = _addr(6, 16)  # state_out partly over state_in
+    assert _prerule(lib, d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[7] = q[6]  # in place is fine
+    assert _prerule(lib, d, q) in (gdn.GDN_OK, gdn.GDN_ERR_CUDA)
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.gdn_status_string(s)
