@@ -24,16 +24,16 @@
 //                Gram matrix, the Q rows Q K^T); the unit-lower-triangular
 //                system is solved blockwise (16 x 16 diagonal blocks by forward
 //                substitution in fp32, off-diagonal blocks by tf32 warp MMAs);
-//                two MMAs give W^T and U^T.  The results are staged in shared
-//                memory as ready-made operand images and bulk-stored as one
-//                contiguous block per chunk-head.
+//                two MMAs give W^T and U^T.  The results are written as
+//                ready-made operand images into one contiguous block per
+//                chunk-head.
 //   gdn_scan_tc  one CTA per (sequence, head).  The fp32 state lives in
 //                registers (two threads per state row, 64 columns each); per
-//                chunk it is rounded to a bf16 operand in shared memory and four
-//                MMAs (S0 W^T, S0 Q^T, U' P^T, U'_w K) with fp32 accumulators in
-//                TMEM produce U', O and the state increment.  The next chunk's
-//                operands are prefetched (TMA + one bulk copy) into a second
-//                stage; full output tiles leave through a TMA store.
+//                chunk it is rounded to a bf16 A operand in TMEM and two MMA
+//                groups with fp32 accumulators in TMEM produce
+//                [S0 W^T | S0 Qs^T] and, from U' = U - W S0^T, U'^T [K~ | P^T]
+//                (the state increment and the intra-chunk output).  The next
+//                chunks' blocks are prefetched (bulk copies) into three stages.
 //
 // All tcgen05 MMAs are M = 128 (the 128 rows of the state, or the 64 K rows
 // stacked on the 64 Q rows), so accumulator rows map 1:1 onto TMEM lanes and
@@ -63,7 +63,7 @@ using namespace tc;
 //   [32K, 48K)  V tile
 //   [48K, 64K)  T (fp32)
 //   [64K, 68K)  per-warp 16 x 16 scratch of the blocked solve
-// The results (W image, U^T rows, P image, gate factors) are written straight
+// The results (W and Qs images, K~, P^T image, U^T rows, gate factor) are written straight
 // to the workspace block of the chunk-head.
 constexpr uint32_t kPrepTf = 49152, kPrepY = 65536;
 constexpr uint32_t kPrepSmem = kPrepY + 4096 + 1024;
@@ -82,7 +82,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     uint8_t *sm = align1024(smem_raw);
     __shared__ uint64_t bar_ld, bar_mma;
     __shared__ uint32_t tmem_base;
-    __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C];
+    __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C], s_w[C];
     __shared__ __align__(16) float s_b2[C];  // b in log2 units
 
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
@@ -94,6 +94,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     const int64_t ch = chunk * H + h;
     const int32_t tok0 = (int32_t)loc.start;
     uint8_t *blk = blocks + (size_t)ch * kTcBlock;
+    uint8_t *rest = blk + kBlkRest;
 
     // gate loads first: their latency overlaps the set-up and the TMA loads
     float g_in = 0.f, beta_in = 0.f;
@@ -142,13 +143,11 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     if (tid < C) {
         const bool in = tid < L;
         const float bl = s_b[L - 1], bi = s_b[tid];
-        float *fac = reinterpret_cast<float *>(blk + kBlkFac);
         s_b2[tid] = bi * 1.4426950408889634f;
         s_bg[tid] = s_beta[tid] * __expf(bi);
         s_sg[tid] = in ? scale * __expf(bi) : 0.f;
-        fac[kFacW + tid] = in ? __expf(bl - bi) : 0.f;
-        fac[kFacSG + tid] = s_sg[tid];
-        fac[kFacGL + tid] = tid == 0 ? __expf(bl) : 0.f;  // exp(b_L), then zero padding
+        s_w[tid] = in ? __expf(bl - bi) : 0.f;
+        if (tid == 0) reinterpret_cast<float *>(rest + kRestFac)[kFacGL] = __expf(bl);
     }
     __syncthreads();
 
@@ -164,24 +163,19 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         }
         mma_commit_warp(&bar_mma);
     }
-    // Qs = (scale * exp(b_i)) q_i, the rows of the Q tile rescaled (rows >= L: zero),
-    // written to the workspace with the tile's own byte layout.
+    // Qs = (scale * exp(b_i)) q_i and K~ = exp(b_L - b_j) k_j: the rows of the Q
+    // and K tiles rescaled (rows >= L: zero), written to the workspace with the
+    // tiles' own byte layout.
     if (ok) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int e = tid + kThreads * k;            // 16-byte chunk over both 8K blocks
             const int qb = e >> 9, i = (e & 511) >> 3;   // block, token row
             const uint32_t off = (uint32_t)((e & 511) << 4);
-            const uint4 src = *reinterpret_cast<const uint4 *>(sm + 8192 + qb * 16384 + off);
-            const float f = s_sg[i];
-            const uint32_t in[4] = {src.x, src.y, src.z, src.w};
-            uint32_t o4[4];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&in[w]);
-                o4[w] = pack_bf16(f * __low2float(b2), f * __high2float(b2));
-            }
-            *reinterpret_cast<uint4 *>(blk + kBlkWQ + 8192 + qb * 16384 + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            const uint4 qv = *reinterpret_cast<const uint4 *>(sm + 8192 + qb * 16384 + off);
+            const uint4 kv = *reinterpret_cast<const uint4 *>(sm + qb * 16384 + off);
+            *reinterpret_cast<uint4 *>(blk + 8192 + qb * 16384 + off) = scale8(qv, s_sg[i]);
+            *reinterpret_cast<uint4 *>(rest + kRestKt + qb * 8192 + off) = scale8(kv, s_w[i]);
         }
     }
     __syncthreads();  // every thread is done reading Q before A overwrites it
@@ -189,7 +183,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     tc_fence_after();
 
     // Epilogue 1: accumulator row r = qd*32 + lane, columns [32 hf, 32 hf + 32).
-    // Rows 0..63 (K K^T) -> A in fp32; rows 64..127 (Q K^T) -> P image (bf16).
+    // Rows 0..63 (K K^T) -> A in fp32; rows 64..127 (Q K^T) -> P^T image (bf16).
     if (ok) {
         const int r = qd * 32 + lane;
         const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
@@ -222,15 +216,23 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
                 *reinterpret_cast<float4 *>(sm + a_offset(i, 32 * hf + 4 * q)) =
                     make_float4(rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
         } else {
-            uint8_t *pimg = blk + kBlkP;
+            // P^T image (rows j, columns i), staged in the (still unused) T region:
+            // one column j per store instruction, 32 consecutive rows i per warp
+            __nv_bfloat16 *pt = reinterpret_cast<__nv_bfloat16 *>(sm + kPrepTf);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(pimg + sw128_offset(i, 4 * hf + q)) =
-                    make_uint4(pack_bf16(rr[8 * q], rr[8 * q + 1]), pack_bf16(rr[8 * q + 2], rr[8 * q + 3]),
-                               pack_bf16(rr[8 * q + 4], rr[8 * q + 5]), pack_bf16(rr[8 * q + 6], rr[8 * q + 7]));
+            for (int t = 0; t < 32; ++t) pt[img_offset(32 * hf + t, i) / 2] = __float2bfloat16_rn(rr[t]);
         }
     }
     tc_fence_before();
+    __syncthreads();
+    // the P^T image to the workspace, before the solve takes over its region
+    if (ok) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int e = tid + kThreads * k;
+            *reinterpret_cast<uint4 *>(rest + kRestPt + e * 16) = *reinterpret_cast<const uint4 *>(sm + kPrepTf + e * 16);
+        }
+    }
     __syncthreads();
 
     // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks.
@@ -296,36 +298,32 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
 // ===========================================================================
 // Scan
 // ===========================================================================
-// Shared memory (1024-aligned), three stages of per-chunk operands:
-//   [0, 32K)   [W rows | Qs rows] per 64-channel block: the N = 128 B operand
-//              of S0 [W ; Qs]^T (one bulk copy from the workspace block)
-//   [32K, 48K) K tile (TMA; the MN-major B operand of the state update)
-//   [48K, 72K) U^T rows, P image, gate factors (one bulk copy)
-// The operands the threads produce (S0 and U' in bf16) are written to TMEM
-// and used as A operands straight from there.
-// TMEM columns: [0,256) two buffers of [S0 W^T | S0 Qs^T + U' P^T] (the second
-// half is the chunk's output), [256,384) U'_w K, [384,448) S0, [448,480) U',
-// [480,512) U'_w.  The output of chunk c is read while chunk c+1's first MMAs run.
-constexpr uint32_t kStWQ = 0, kStK = 32768, kStRest = 49152, kStage = 75776;
-constexpr uint32_t kRestU = 0, kRestP = 16384, kRestFac = 24576;
-// bytes of the [U, P, factors] part of a block, and of one stage's copies
-template <bool KDA> constexpr uint32_t rest_bytes() {
-    return KDA ? (uint32_t)(kTcUt + kTcPImg + kTcFacKda) : (uint32_t)(kTcBlock - kTcWQ);
-}
-template <bool KDA> constexpr uint32_t stage_bytes() { return (uint32_t)kTcWQ + 16384 + rest_bytes<KDA>(); }
-static_assert(kStRest + rest_bytes<true>() <= kStage && kStRest + rest_bytes<false>() <= kStage, "stage layout");
+// Shared memory (1024-aligned), three stages of per-chunk operands, each the
+// chunk-head's workspace block as it is (two bulk copies):
+//   [0, 32K)      [W rows | Qs rows] per 64-channel block: the N = 128 B operand
+//                 of S0 [W ; Qs]^T
+//   [32K, 56K)    [K~ | P^T]: the N = 192 MN-major B operand of U'^T [K~ | P^T]
+//   [56K, 72K)    U^T rows;  [72K, 73K) gate factors
+// The operands the threads produce (S0 and U' in bf16) are written to TMEM and
+// used as A operands straight from there.
+// TMEM columns: [0,128) D1 = [S0 W^T | S0 Qs^T], [128,320) D2 = [U'^T K~ | U'^T P^T],
+// [320,384) S0, [384,416) U'.
+// A tcgen05.ld waits for the MMAs in flight, so every accumulator is read once
+// the chunk's MMAs are done (the output with the state increment), and the
+// output leaves from registers while the next chunk's first MMA group runs.
+constexpr uint32_t kStWQ = 0, kStRest = kBlkRest, kStage = (uint32_t)kTcBlock;
+static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled operands");
 constexpr int kStages = 3;
 constexpr uint32_t kScanSmem = kStages * kStage + 1024;
-constexpr uint32_t kTmD = 0, kTmAcc4 = 256, kTmAS = 384, kTmAUp = 448, kTmAUw = 480;
+constexpr uint32_t kTmD1 = 0, kTmD2 = 128, kTmAS = 320, kTmAU = 384;
 
 struct ScanBars {
     uint64_t full[kStages];
-    uint64_t mma[3];
+    uint64_t mma[2];
 };
 
-// KDA: per-channel gate.  The state-update operand is then K~ from the block
-// (instead of the K tile), U'_w = U', and the carried state is scaled per key
-// channel by exp(b_L).
+// KDA: per-channel gate (the carried state is then scaled per key channel by
+// exp(b_L) instead of one factor).
 // Sequence split of long fixed-length sequences (G >= 3 segments of `seg` chunks).
 // A segment's end state is an affine function of its start state,
 // S_end = S_start M_g + B_g.  Pass 1 runs, in parallel, segment 0 from the true
@@ -348,11 +346,10 @@ __device__ __forceinline__ float *split_state(const ScanSplit &sp, int64_t n, in
 // SPLIT: launched as a pass of the split scan (the block's work then comes from `sp`).
 template <bool KDA, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
-gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32_t *__restrict__ cu,
-            const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk,
-            int64_t max_chunks,
-            int64_t snap_stride, int64_t n_snap, const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out,
-            float *final_state, float *__restrict__ snaps, const ScanSplit sp, int *err) {
+gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T,
+            int64_t rows, int64_t H, int64_t max_chunks, int64_t snap_stride, int64_t n_snap,
+            const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out, float *final_state,
+            float *__restrict__ snaps, const ScanSplit sp, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     __shared__ ScanBars bars;
@@ -408,7 +405,7 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(&bars.full[i], 1);
-        for (int i = 0; i < 3; ++i) mbar_init(&bars.mma[i], 1);
+        for (int i = 0; i < 2; ++i) mbar_init(&bars.mma[i], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -425,18 +422,11 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
     auto issue_loads = [&](int64_t c) {
         const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
-        const uint8_t *blk = blocks + (size_t)((chunk0 + cb + c) * H + h) * (KDA ? kTcBlockKda : kTcBlock);
-        const int32_t tok = (int32_t)(start + (cb + c) * C);
+        const uint8_t *blk = blocks + (size_t)((chunk0 + cb + c) * H + h) * kTcBlock;
         uint64_t *bar = &bars.full[stage];
-        mbar_arrive_expect_tx(bar, stage_bytes<KDA>());
-        bulk_load(st + kStWQ, blk + kBlkWQ, (uint32_t)kTcWQ, bar);
-        if (KDA) {
-            bulk_load(st + kStK, blk + kBlkKt, (uint32_t)kTcKt, bar);
-        } else {
-            tma_load_3d(st + kStK, &mk, 0, (int32_t)(h / (H / Hk)), tok, bar);
-            tma_load_3d(st + kStK + 8192, &mk, 64, (int32_t)(h / (H / Hk)), tok, bar);
-        }
-        bulk_load(st + kStRest, blk + kBlkU, rest_bytes<KDA>(), bar);
+        mbar_arrive_expect_tx(bar, kStage);
+        bulk_load(st + kStWQ, blk, (uint32_t)kTcWQ, bar);
+        bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
     };
     if (tid == kLoader)
         for (int64_t c = 0; c < kStages && c < nchunks; ++c) issue_loads(c);
@@ -454,19 +444,13 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         for (int c = 0; c < 64; ++c) S[c] = (start_kind == kStartIdentity && 64 * hf + c == v) ? 1.f : 0.f;
     }
 
-    // Output of chunk `c` (tokens [32 hf, 32 hf + 32) of column v): waits for its last MMA.
-    auto emit_output = [&](int64_t c) -> bool {
-        const bool ok_w = mbar_wait(&bars.mma[2], (uint32_t)(c & 1));
-        tc_fence_after();
+    // Output of chunk c held in registers: o[t / 16][t % 16] = token 32 hf + t, channel v.
+    float o[2][16];
+    auto store_output = [&](int64_t c) {
         const int64_t ca = cb + c;
         const int L = (int)(len - ca * C < C ? len - ca * C : C);
-        float o[2][16];
-        const uint32_t dcol = kTmD + (uint32_t)(c & 1) * 128 + 64 + 32 * hf;
-        tmem_ld16(tm + lane_off + dcol, o[0]);
-        tmem_ld16(tm + lane_off + dcol + 16, o[1]);
-        tmem_wait_ld();
-        // 4 x 4 transposes among groups of 4 lanes (4 adjacent channels): afterwards
-        // lane j of a group holds those 4 channels of token 4 b + j -> one 8-byte store.
+        // 4 x 4 transposes among the quads of lanes (4 adjacent channels): afterwards
+        // lane j of a quad holds those 4 channels of token 4 b + j -> one 8-byte store.
         const int j4 = lane & 3;
         const int64_t tstride = H * D;
         __nv_bfloat16 *op = out + ((start + ca * C + 32 * hf + j4) * H + h) * D + (v - j4);
@@ -474,33 +458,19 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         for (int b = 0; b < 8; ++b) {
             float x0 = o[b >> 2][4 * (b & 3)], x1 = o[b >> 2][4 * (b & 3) + 1], x2 = o[b >> 2][4 * (b & 3) + 2],
                   x3 = o[b >> 2][4 * (b & 3) + 3];
-            {
-                const bool hi = lane & 1;
-                const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x1, 1);
-                const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x2 : x3, 1);
-                if (hi) { x0 = r0; x2 = r1; } else { x1 = r0; x3 = r1; }
-            }
-            {
-                const bool hi = lane & 2;
-                const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x2, 2);
-                const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x1 : x3, 2);
-                if (hi) { x0 = r0; x1 = r1; } else { x2 = r0; x3 = r1; }
-            }
+            quad_transpose(x0, x1, x2, x3, lane);
             if (32 * hf + 4 * b + j4 < L)
                 *reinterpret_cast<uint2 *>(op + (int64_t)(4 * b) * tstride) = make_uint2(pack_bf16(x0, x1), pack_bf16(x2, x3));
         }
-        return ok_w;
     };
 
-    const uint32_t id_wq = idesc_bf16(128, 128, 0, 0), id_k = idesc_bf16(128, 128, 0, 1),
-                   id_p = idesc_bf16(128, 64, 0, 0);
+    const uint32_t id_wq = idesc_bf16(128, 128, 0, 0), id_kp = idesc_bf16(128, emit ? 192 : 128, 0, 1);
     bool ok = true;
     for (int64_t c = 0; c < nchunks; ++c) {
         const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
         const uint32_t st_u = smem_u32(st);
         const uint32_t par = (uint32_t)(c & 1);
-        const uint32_t dbuf = kTmD + par * 128;
         const uint8_t *rest = st + kStRest;
         const float *fac = reinterpret_cast<const float *>(rest + kRestFac);
 
@@ -520,37 +490,33 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         __syncthreads();
         tc_fence_after();
 
-        // (b) D[buf] = S0 [W ; Qs]^T   (N = 128, K = 128): [U-correction | inter-chunk output]
+        // (b) D1 = S0 [W ; Qs]^T   (N = 128, K = 128): [U correction | inter-chunk output]
         if (warp == 0) {
             const uint64_t bwq = sdesc_sw128(st_u + kStWQ, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_ts(tm + dbuf, tm + kTmAS + kk * 8, bwq + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                mma_bf16_ts(tm + kTmD1, tm + kTmAS + kk * 8, bwq + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
                             id_wq, kk > 0);
             mma_commit_warp(&bars.mma[0]);
         }
-        // the previous chunk's output, while this chunk's MMAs run; after it every MMA of
-        // chunk c-1 has completed, so its stage can take chunk c+2
-        // (without outputs every MMA of chunk c-1 was waited for in its steps (c) and (e))
-        if (c >= 1 && emit) ok = emit_output(c - 1) && ok;
+        // the previous chunk's output, while these MMAs run; every MMA of chunk c-1
+        // has completed (step (e) waited for them), so its stage can take chunk c+2
+        if (c >= 1 && emit) store_output(c - 1);
         if (tid == kLoader && c >= 1 && c + kStages - 1 < nchunks) issue_loads(c + kStages - 1);
 
-        // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32) -> TMEM A operands U', U' * w
+        // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32) -> TMEM A operand
         ok = mbar_wait(&bars.mma[0], par) && ok;
         tc_fence_after();
         {
             float a0[16], a1[16];
-            tmem_ld16(tm + lane_off + dbuf + 32 * hf, a0);
-            tmem_ld16(tm + lane_off + dbuf + 32 * hf + 16, a1);
+            tmem_ld16(tm + lane_off + kTmD1 + 32 * hf, a0);
+            tmem_ld16(tm + lane_off + kTmD1 + 32 * hf + 16, a1);
             tmem_wait_ld();
-            uint32_t wu[16], ww[16];
+            uint32_t wu[16];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int cq = 4 * hf + q;  // 16-byte chunk = tokens 8 cq .. 8 cq + 7
                 const uint4 u8 = *reinterpret_cast<const uint4 *>(rest + kRestU + sw128_offset(v, cq));
-                const float4 wlo = *reinterpret_cast<const float4 *>(fac + kFacW + 8 * cq);
-                const float4 whi = *reinterpret_cast<const float4 *>(fac + kFacW + 8 * cq + 4);
-                const float wv[8] = {wlo.x, wlo.y, wlo.z, wlo.w, whi.x, whi.y, whi.z, whi.w};
                 const uint32_t uw32[4] = {u8.x, u8.y, u8.z, u8.w};
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
@@ -562,44 +528,42 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
                         up0 *= umul;
                         up1 *= umul;
                     }
-                    up0 -= acc_lo;
-                    up1 -= acc_hi;
-                    wu[4 * q + e / 2] = pack_bf16(up0, up1);
-                    ww[4 * q + e / 2] = pack_bf16(up0 * wv[e], up1 * wv[e + 1]);
+                    wu[4 * q + e / 2] = pack_bf16(up0 - acc_lo, up1 - acc_hi);
                 }
             }
-            tmem_st16u(tm + lane_off + kTmAUp + 16 * hf, wu);
-            tmem_st16u(tm + lane_off + kTmAUw + 16 * hf, ww);
+            tmem_st16u(tm + lane_off + kTmAU + 16 * hf, wu);
             tmem_wait_st();
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        // (d) acc4 = U'_w K (state increment; warp 0) and, from warp 1 at the same time,
-        // D[buf] output half += U' P^T
+        // (d) D2 = U'^T [K~ | P^T]   (N = 192, K = 64 tokens): [state increment | intra-chunk output]
         if (warp == 0) {
-            const uint64_t bk = sdesc_sw128(st_u + kStK, 8192, 1024);
+            const uint64_t bkp = sdesc_sw128(st_u + kStRest + kRestKt, 8192, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(tm + kTmAcc4, tm + kTmAUw + kk * 8, bk + (uint64_t)((kk * 2048) >> 4), id_k, kk > 0);
+                mma_bf16_ts(tm + kTmD2, tm + kTmAU + kk * 8, bkp + (uint64_t)((kk * 2048) >> 4), id_kp, kk > 0);
             mma_commit_warp(&bars.mma[1]);
-        } else if (warp == 1 && emit) {
-            const uint64_t bp = sdesc_sw128(st_u + kStRest + kRestP, 16, 1024);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(tm + dbuf + 64, tm + kTmAUp + kk * 8, bp + (uint64_t)((kk * 32) >> 4), id_p, 1);
-            mma_commit_warp(&bars.mma[2]);
         }
 
-        // (e) S = gam_L S0 + acc4 (columns [64 hf, 64 hf + 64)); per key channel for KDA
+        // (e) S = gam_L S0 + increment (columns [64 hf, 64 hf + 64); per key channel
+        // for KDA) and the output o = S0 Qs^T + U'^T P^T
         const float gl = fac[kFacGL];
         ok = mbar_wait(&bars.mma[1], par) && ok;
         tc_fence_after();
         {
-            float a[4][16];
+            float a[4][16], o2[2][16];
+            auto load_output = [&] {
 #pragma unroll
-            for (int c0 = 0; c0 < 4; ++c0) tmem_ld16(tm + lane_off + kTmAcc4 + 64 * hf + 16 * c0, a[c0]);
+                for (int q = 0; q < 2; ++q) {
+                    tmem_ld16(tm + lane_off + kTmD1 + 64 + 32 * hf + 16 * q, o[q]);
+                    tmem_ld16(tm + lane_off + kTmD2 + 128 + 32 * hf + 16 * q, o2[q]);
+                }
+            };
+#pragma unroll
+            for (int c0 = 0; c0 < 4; ++c0) tmem_ld16(tm + lane_off + kTmD2 + 64 * hf + 16 * c0, a[c0]);
+            if (emit && !KDA) load_output();  // (KDA: after the state update, for registers)
             tmem_wait_ld();
             if (KDA) {
                 const float4 *gl4 = reinterpret_cast<const float4 *>(fac + kFacGL + 64 * hf);
@@ -617,6 +581,16 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
 #pragma unroll
                     for (int t = 0; t < 16; ++t) S[16 * c0 + t] = gl * S[16 * c0 + t] + a[c0][t];
             }
+            if (emit) {
+                if (KDA) {
+                    load_output();
+                    tmem_wait_ld();
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) o[q][t] += o2[q][t];
+            }
         }
 
         // snapshot after n * stride tokens of the sequence
@@ -631,7 +605,7 @@ gdn_scan_tc(const __grid_constant__ CUtensorMap mk, const float *h0, const int32
         }
         if (__syncthreads_or(!ok)) break;
     }
-    if (ok && nchunks > 0 && emit) ok = emit_output(nchunks - 1) && ok;
+    if (ok && nchunks > 0 && emit) store_output(nchunks - 1);
     if (!ok && tid == 0) flag_error(err, 2);
     if (ok && s_end) {
 #pragma unroll
@@ -791,8 +765,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         auto kern = p.per_channel ? gdn_scan_tc<true, false> : gdn_scan_tc<false, false>;
         LaunchScope ls("gdn_scan_tc", s);
         kern<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
-            mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap,
-            blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
+            a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
         return check_launch("gdn_scan_tc");
     }
     // sequence split: pass 1, the chained start states, pass 2
@@ -803,7 +776,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         LaunchScope ls("gdn_scan_tc", s);
         kern<<<dim3((unsigned)(a.N * per1), (unsigned)p.H), kThreads, kScanSmem, s>>>(
-            mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+            a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
             (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
     }
     if ((st = check_launch("gdn_scan_tc")) != GDN_OK) return st;
@@ -816,7 +789,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         LaunchScope ls("gdn_scan_tc", s);
         kern<<<dim3((unsigned)(a.N * per2), (unsigned)p.H), kThreads, kScanSmem, s>>>(
-            mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+            a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
             (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
     }
     return check_launch("gdn_scan_tc");

@@ -47,7 +47,7 @@ namespace {
 //   [64K, 80K)  K * R (layout of a K tile, channel halves 8K apart); after the blocks:
 //               T (fp32)
 //   [80K, 96K)  after the blocks: the solve's scratch (4K) and T diag(beta) (8K at 88K)
-//   [96K, 104K) P image (bf16, K-major rows of 64 tokens)
+//   [96K, 104K) P^T image (bf16, rows = key tokens j, columns = query tokens i)
 constexpr uint32_t kSmKQ = 0, kSmB = 32768, kSmA = 32768, kSmV = 49152, kSmZ = 65536, kSmP = 98304;
 constexpr uint32_t kSmT = 65536, kSmY = 81920, kSmTp = 90112;
 constexpr uint32_t kSmem = kSmP + 8192 + 1024;
@@ -68,10 +68,6 @@ __device__ __forceinline__ uint32_t kq_chunk(int qk, int i, int cc) {
 // 8-channel chunk `cc` of row i of the K * R image.
 __device__ __forceinline__ uint32_t z_chunk(int i, int cc) {
     return (uint32_t)(kSmZ + (cc >> 3) * 8192 + i * 128 + (((cc & 7) ^ (i & 7)) << 4));
-}
-// bf16 pair (j, j+1), j even, of row i of the P image.
-__device__ __forceinline__ uint32_t p_pair(int i, int j) {
-    return (uint32_t)(i * 128 + (((j >> 3) ^ (i & 7)) << 4) + (j & 7) * 2);
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -157,10 +153,11 @@ __device__ __forceinline__ void ap_blocks(uint8_t *sm, const Factors &f, int p, 
             // P: causal (j <= i) and rows of the chunk only
             const bool k00 = i0 < L && (!diag || col <= i0), k01 = i0 < L && (!diag || col + 1 <= i0);
             const bool k10 = i1 < L && (!diag || col <= i1), k11 = i1 < L && (!diag || col + 1 <= i1);
-            *reinterpret_cast<uint32_t *>(sm + kSmP + p_pair(i0, col)) =
-                pack_bf16(k00 ? scale * cP[b][nt][0] : 0.f, k01 ? scale * cP[b][nt][1] : 0.f);
-            *reinterpret_cast<uint32_t *>(sm + kSmP + p_pair(i1, col)) =
-                pack_bf16(k10 ? scale * cP[b][nt][2] : 0.f, k11 ? scale * cP[b][nt][3] : 0.f);
+            __nv_bfloat16 *pt = reinterpret_cast<__nv_bfloat16 *>(sm + kSmP);  // P^T: element (j, i)
+            pt[img_offset(col, i0) / 2] = __float2bfloat16_rn(k00 ? scale * cP[b][nt][0] : 0.f);
+            pt[img_offset(col + 1, i0) / 2] = __float2bfloat16_rn(k01 ? scale * cP[b][nt][1] : 0.f);
+            pt[img_offset(col, i1) / 2] = __float2bfloat16_rn(k10 ? scale * cP[b][nt][2] : 0.f);
+            pt[img_offset(col + 1, i1) / 2] = __float2bfloat16_rn(k11 ? scale * cP[b][nt][3] : 0.f);
         }
     }
 }
@@ -235,8 +232,7 @@ __device__ __forceinline__ void diag_exact_store(uint8_t *sm, const DiagKeep &ke
         const bool first = it <= r;
         const int i = base + (first ? r : 15 - r), j = base + (first ? r - it : 16 - it);
         *reinterpret_cast<float *>(sm + kSmA + f32_offset(i, j)) = s_beta[i] * keep.a[k];
-        *reinterpret_cast<__nv_bfloat16 *>(sm + kSmP + p_pair(i, j & ~1) + (j & 1) * 2) =
-            __float2bfloat16_rn(i < L ? scale * keep.p[k] : 0.f);
+        *reinterpret_cast<__nv_bfloat16 *>(sm + kSmP + img_offset(j, i)) = __float2bfloat16_rn(i < L ? scale * keep.p[k] : 0.f);
     }
 }
 
@@ -260,7 +256,8 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, hf = warp >> 2;
     const int32_t tok0 = (int32_t)loc.start;
-    uint8_t *blk = blocks + (size_t)(chunk * H + h) * kTcBlockKda;
+    uint8_t *blk = blocks + (size_t)(chunk * H + h) * kTcBlock;
+    uint8_t *rest = blk + kBlkRest;
 
     const float beta_in = tid < L ? beta[(int64_t)(tok0 + tid) * H + h] : 0.f;
     if (tid == 0) {
@@ -381,18 +378,16 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                     kt[u] = in ? pack_bf16(kf[a] * ta, kf[b] * tb) : 0u;
                     qs[u] = in ? pack_bf16(scale * qf[a] * ga, scale * qf[b] * gb) : 0u;
                 }
-                *reinterpret_cast<uint4 *>(blk + kBlkKt + hc * 8192 + i * 128 + pc * 16) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
-                *reinterpret_cast<uint4 *>(blk + kBlkWQ + 8192 + hc * 16384 + i * 128 + pc * 16) =
+                *reinterpret_cast<uint4 *>(rest + kRestKt + hc * 8192 + i * 128 + pc * 16) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+                *reinterpret_cast<uint4 *>(blk + 8192 + hc * 16384 + i * 128 + pc * 16) =
                     make_uint4(qs[0], qs[1], qs[2], qs[3]);
                 // (no other thread reads this chunk of the tiles)
                 *reinterpret_cast<uint4 *>(sm + kSmKQ + so) = make_uint4(xk[0], xk[1], xk[2], xk[3]);
                 *reinterpret_cast<uint4 *>(sm + kSmKQ + so + 8192) = make_uint4(xq[0], xq[1], xq[2], xq[3]);
                 *reinterpret_cast<uint4 *>(sm + kSmZ + hc * 8192 + i * 128 + pc * 16) = make_uint4(zr[0], zr[1], zr[2], zr[3]);
             }
-            float *fac = reinterpret_cast<float *>(blk + kBlkFac);
+            float *fac = reinterpret_cast<float *>(rest + kRestFac);
             if (tid < D) fac[kFacGL + tid] = ex2(*reinterpret_cast<const float *>(sm + kSmB + b_off(Lm1, tid)));
-            else if (tid < D + C) fac[kFacW + tid - D] = tid - D < L ? 1.f : 0.f;
-            else if (tid < D + 2 * C) fac[kFacSG + tid - D - C] = 0.f;
         }
         fence_async_smem();  // the b region is taken over by the V tile (TMA) below
         __syncthreads();
@@ -416,10 +411,10 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     }
     __syncthreads();
 
-    // P image to the block; K * L -> K * Gam = K * L * exp(r_p) in place.
+    // P^T image to the block; K * L -> K * Gam = K * L * exp(r_p) in place.
     if (ok) {
         for (int e = tid; e < 512; e += kThreads)
-            *reinterpret_cast<uint4 *>(blk + kBlkP + e * 16) = *reinterpret_cast<const uint4 *>(sm + kSmP + e * 16);
+            *reinterpret_cast<uint4 *>(rest + kRestPt + e * 16) = *reinterpret_cast<const uint4 *>(sm + kSmP + e * 16);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int e = tid + kThreads * k;

@@ -107,7 +107,7 @@ ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed) {
     p.split_seg = 0;
     p.off_split = 0;
     if (p.tc) {
-        p.tc_block = p.per_channel ? kTcBlockKda : kTcBlock;
+        p.tc_block = kTcBlock;
         p.off_W = p.off_U = p.off_P = p.off_b = off;  // one block of tc_block bytes per chunk-head
         off = align_up(off + p.tc_block * (size_t)ch, 256);
         if (!packed && d.T > 0) {

@@ -80,19 +80,17 @@ gdn_status launch_chunk_simt(const ChunkPlan &p, const ChunkArgs &a, int dtype, 
 gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s);
 bool tc_eligible(const gdn_desc &d);
 
-// Per chunk-head workspace block of the tensor-core path (bytes):
+// Per chunk-head workspace block of the tensor-core path (bytes), both gate kinds:
 //   [W (channels 0-63) 8K][Qs (0-63) 8K][W (64-127) 8K][Qs (64-127) 8K]
-//   [U^T rows 16K][P image 8K][gate factors 768]
-// W and Qs = (scale * exp(b_i)) q_i are K-major operand images (rows = tokens)
-// laid out so that [W ; Qs] is one N = 128 operand; the scan copies the block
-// with two bulk copies.  The per-channel gate's block has 1 KB of gate
-// factors and adds K~ = K * exp(b_L - b) (16K, the layout of a K tile), the
-// operand of its state update:
-//   [W|Qs 32K][U^T rows 16K][P image 8K][gate factors 1K][K~ 16K]
-constexpr size_t kTcWQ = 32768, kTcUt = 128 * 128, kTcPImg = 64 * 128, kTcFac = 192 * 4;
-constexpr size_t kTcBlock = kTcWQ + kTcUt + kTcPImg + kTcFac;  // 58112
-constexpr size_t kTcFacKda = 256 * 4, kTcKt = 64 * 128 * 2;
-constexpr size_t kTcBlockKda = kTcWQ + kTcUt + kTcPImg + kTcFacKda + kTcKt;  // 74752
+//   [K~ 16K][P^T image 8K][U^T rows 16K][gate factors 1K]
+// W and Qs = scale Q * Gam are K-major operand images (rows = tokens) laid out
+// so that [W ; Qs] is one N = 128 operand.  K~ = K * exp(b_L - b) (the layout of
+// a K tile: rows = tokens, two 64-channel halves) followed by P^T (rows = key
+// tokens j, columns = query tokens i) is one N = 192 MN-major operand.  The scan
+// copies a block with two bulk copies.
+constexpr size_t kTcWQ = 32768, kTcKt = 64 * 128 * 2, kTcPImg = 64 * 128, kTcUt = 128 * 128, kTcFac = 1024;
+constexpr size_t kTcRest = kTcKt + kTcPImg + kTcUt + kTcFac;  // 41984
+constexpr size_t kTcBlock = kTcWQ + kTcRest;                  // 74752
 gdn_status launch_decode(const gdn_desc &d, const void *q, const void *k, const void *v,
                          const float *g, const float *beta, float *state, void *out,
                          cudaStream_t s);

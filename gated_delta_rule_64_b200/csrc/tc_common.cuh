@@ -18,14 +18,16 @@ constexpr int C = kChunk;  // 64 tokens per chunk
 constexpr int D = 128;     // d_k = d_v
 constexpr int kThreads = 256;
 
-// Offsets inside one workspace block (kTcBlock bytes for the per-head gate,
-// kTcBlockKda for the per-channel gate, whose block adds K~ at the end).
-constexpr uint32_t kBlkWQ = 0, kBlkU = 32768, kBlkP = 49152, kBlkFac = 57344;
-constexpr uint32_t kBlkKt = kBlkFac + (uint32_t)kTcFacKda;  // per-channel gate only
-// Gate factors (floats):
-//   per-head gate:    [0, 64) w_i = exp(b_L - b_i); [64, 128) scale exp(b_i); [128] exp(b_L)
-//   per-channel gate: [0, 64) w_i = 1 (0 past the chunk end); [128, 256) exp(b_L) per key channel
-constexpr int kFacW = 0, kFacSG = 64, kFacGL = 128;
+// Offsets inside one workspace block: [W ; Qs] images at 0, then the rest at
+// kBlkRest: K~, P^T image, U^T rows, gate factors.
+constexpr uint32_t kBlkRest = (uint32_t)kTcWQ;
+constexpr uint32_t kRestKt = 0, kRestPt = 16384, kRestU = 24576, kRestFac = 40960;
+static_assert(kRestPt == kTcKt && kRestU == kRestPt + kTcPImg && kRestFac == kRestU + kTcUt &&
+                  kRestFac + kTcFac == kTcRest,
+              "block layout");
+// Gate factors (floats): exp(b_L), at [0] for the per-head gate and per key
+// channel at [0, 128) for the per-channel gate.
+constexpr int kFacGL = 0;
 
 __device__ __forceinline__ void flag_error(int *err, int code) {
     if (err) atomicCAS(err, 0, code);
@@ -86,6 +88,42 @@ __device__ __forceinline__ void warp_store16(uint8_t *base, int r0, int c0, cons
         *reinterpret_cast<float *>(base + off(r0 + g + 8, col)) = sign * c[nt][2];
         *reinterpret_cast<float *>(base + off(r0 + g + 8, col + 1)) = sign * c[nt][3];
     }
+}
+
+// 4 x 4 transpose among the 4 lanes of a quad: lane j of the quad holds x[0..3]
+// = element (row r_j, columns c .. c+3) before, and (rows r_0 .. r_3, column
+// c + j) after (r_j = the quad's j-th lane's row).
+__device__ __forceinline__ void quad_transpose(float &x0, float &x1, float &x2, float &x3, int lane) {
+    {
+        const bool hi = lane & 1;
+        const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x1, 1);
+        const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x2 : x3, 1);
+        if (hi) { x0 = r0; x2 = r1; } else { x1 = r0; x3 = r1; }
+    }
+    {
+        const bool hi = lane & 2;
+        const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x2, 2);
+        const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x1 : x3, 2);
+        if (hi) { x0 = r0; x1 = r1; } else { x2 = r0; x3 = r1; }
+    }
+}
+
+// Eight bf16 values (one 16-byte chunk) times f, rounded back to bf16.
+__device__ __forceinline__ uint4 scale8(const uint4 &src, float f) {
+    const uint32_t in[4] = {src.x, src.y, src.z, src.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&in[w]);
+        o[w] = pack_bf16(f * __low2float(b2), f * __high2float(b2));
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Byte offset of the bf16 element (row, col) of a 64-column operand image with
+// 128-byte rows and the 128-byte swizzle.
+__device__ __forceinline__ uint32_t img_offset(int row, int col) {
+    return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2);
 }
 
 // T = (I + A)^-1 for the 64 x 64 strictly lower A of a chunk, in 16 x 16 blocks.
@@ -185,7 +223,7 @@ static __device__ __noinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, 
     tmem_ld16(taddr + 64, u0);
     tmem_ld16(taddr + 64 + 16, u1);
     tmem_wait_ld();
-    uint8_t *wimg = blk + kBlkWQ + (r >> 6) * 16384 + (r & 7) * 2;
+    uint8_t *wimg = blk + (r >> 6) * 16384 + (r & 7) * 2;
     const int wchunk = (r & 63) >> 3;
 #pragma unroll
     for (int t = 0; t < 32; ++t) {
@@ -193,7 +231,7 @@ static __device__ __noinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, 
         *reinterpret_cast<__nv_bfloat16 *>(wimg + i * 128 + ((wchunk ^ (i & 7)) << 4)) =
             __float2bfloat16_rn(t < 16 ? w0[t] : w1[t - 16]);
     }
-    uint8_t *urow = blk + kBlkU;
+    uint8_t *urow = blk + kBlkRest + kRestU;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const float *u = q < 2 ? u0 + 8 * q : u1 + 8 * (q - 2);

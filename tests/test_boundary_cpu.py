@@ -65,10 +65,10 @@ def test_workspace_size(lib):
         return n.value
     simt = 4 * 64 * (128 + 128 + 64 + 1)          # fp32 W, U, P and gate per chunk-head
     assert 6 * 3 * simt <= size(dtype=gdn.GDN_F32) < 6 * 3 * simt + 4096
-    tc = 32768 + 128 * 128 + 64 * 128 + 192 * 4  # [W;Qs] image, U^T rows, P image, gate factors
+    tc = 32768 + 64 * 128 * 2 + 64 * 128 + 128 * 128 + 1024  # [W;Qs] images, K~, P^T image, U^T rows, factors
     assert 6 * 3 * tc <= size() < 6 * 3 * tc + 4096
-    kda = tc + (1024 - 192 * 4) + 64 * 128 * 2  # per-channel gate: 1 KB of factors and K~
-    assert 6 * 3 * kda <= size(gate=gdn.GDN_GATE_CHANNEL) < 6 * 3 * kda + 4096
+    # the per-channel gate uses the same block
+    assert 6 * 3 * tc <= size(gate=gdn.GDN_GATE_CHANNEL) < 6 * 3 * tc + 4096
     assert size(dtype=gdn.GDN_F32, gate=gdn.GDN_GATE_CHANNEL) > size(dtype=gdn.GDN_F32)
     d = _desc()
     assert lib.gdn_chunk_workspace_size(ctypes.byref(d), 2, None) == gdn.GDN_ERR_INVALID_ARG
@@ -305,7 +305,7 @@ def test_split_scan_workspace(lib):
         d = _desc(**kw)
         assert lib.gdn_chunk_workspace_size(ctypes.byref(d), kw.get("B", 2), ctypes.byref(n)) == gdn.GDN_OK
         return n.value
-    blk = 32768 + 128 * 128 + 64 * 128 + 192 * 4
+    blk = 32768 + 64 * 128 * 2 + 64 * 128 + 128 * 128 + 1024
     # one sequence of 262144 tokens, 16 heads: 4096 chunks
     G, seg = _split_policy(1, 16, 4096)
     assert G >= 3 and (G - 1) * seg < 4096 <= G * seg
