@@ -409,6 +409,7 @@ gdn_status gdn_prerule(const gdn_desc *d, const void *x, const void *a, const vo
     const int64_t rows = d->B * d->T, Hk = qk_heads(*d);
     const int64_t C = 2 * Hk * d->dk + d->H * d->dv;
     if (rows == 0 && N == 0) return GDN_OK;
+    if (rows > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "more than 2^31 - 1 token rows");
     if (!x || !a || !b || !conv_w || !A_log || !dt_bias || !q || !k || !v || !log_gate || !beta)
         return fail(GDN_ERR_INVALID_ARG, "x, a, b, conv_w, A_log, dt_bias and the five outputs are required");
     const size_t el = d->dtype == GDN_F32 ? 4 : 2;

@@ -290,7 +290,9 @@ gdn_status gdn_state_select(const gdn_desc *d, const float *step_states, const i
  *   q, k       (B, T, hk, d_k); v (B, T, H, d_v) -- 16-byte aligned
  *   log_gate, beta (B, T, H) fp32
  * Rows of a packed batch outside every sequence are not written.  Outputs must
- * not overlap the inputs or each other.
+ * not overlap the inputs or each other.  GDN_ERR_UNSUPPORTED for more than
+ * 2^31 - 1 token rows.  SiLU is evaluated through the hardware tanh for bf16
+ * (relative error about 2^-11, below the rounding of the bf16 result).
  * ------------------------------------------------------------------------- */
 gdn_status gdn_prerule(const gdn_desc *d, const void *x, const void *a, const void *b,
                        const float *conv_w, int32_t K, const float *A_log, const float *dt_bias,
