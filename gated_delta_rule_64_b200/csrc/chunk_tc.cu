@@ -102,21 +102,10 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         g_in = g[(int64_t)(tok0 + tid) * H + h];
         beta_in = beta[(int64_t)(tok0 + tid) * H + h];
     }
-    if (tid == 0) {
+    if (tid == 0) {  // the tile loads first: their latency overlaps the rest of the set-up
         mbar_init(&bar_ld, 1);
         mbar_init(&bar_mma, 1);
         fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&tmem_base, 128);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tm = tmem_base;
-
-    if (tid == 0) {
         mbar_arrive_expect_tx(&bar_ld, 6 * 8192);
         const int32_t hq = (int32_t)(h / (H / Hk));  // query/key head of value head h
         tma_load_3d(sm + 0, &mk, 0, hq, tok0, &bar_ld);
@@ -126,6 +115,14 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         tma_load_3d(sm + 32768, &mv, 0, (int32_t)h, tok0, &bar_ld);
         tma_load_3d(sm + 40960, &mv, 64, (int32_t)h, tok0, &bar_ld);
     }
+    if (warp == 0) {
+        tmem_alloc(&tmem_base, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
     // Gates (rows >= L: beta = 0, g = 0): in-chunk inclusive cumsum of the log gate.
     if (tid < C) {
         s_beta[tid] = beta_in;
@@ -225,19 +222,17 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     }
     tc_fence_before();
     __syncthreads();
-    // the P^T image to the workspace, before the solve takes over its region
-    if (ok) {
+
+    // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks; warps 4-7 first copy the
+    // staged P^T image to the workspace (the solve writes its region after that).
+    uint8_t *Tf = sm + kPrepTf;
+    blocked_solve<kPrepTf, kPrepY>(sm, [](int i, int j) { return a_offset(i, j); }, ok, [&] {
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int e = tid + kThreads * k;
+        for (int k = 0; k < 4; ++k) {
+            const int e = tid - 128 + 128 * k;
             *reinterpret_cast<uint4 *>(rest + kRestPt + e * 16) = *reinterpret_cast<const uint4 *>(sm + kPrepTf + e * 16);
         }
-    }
-    __syncthreads();
-
-    // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks.
-    uint8_t *Tf = sm + kPrepTf;
-    blocked_solve<kPrepTf, kPrepY>(sm, [](int i, int j) { return a_offset(i, j); }, ok);
+    });
 
     // T' = T diag(beta gam), T'' = T diag(beta) as bf16 operand images (K-major rows i).
     if (ok) {

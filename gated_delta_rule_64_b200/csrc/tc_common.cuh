@@ -5,6 +5,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "chunk_common.cuh"
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
@@ -133,17 +135,24 @@ __device__ __forceinline__ uint32_t img_offset(int row, int col) {
 // TY is 4 KB of scratch.  Diagonal blocks: forward substitution in fp32 (one
 // column per lane); off-diagonal blocks by the block recurrence
 // T_pq = -T_pp sum_{q <= r < p} A_pr T_rq with tf32 warp MMAs.  Every thread
-// of the block calls it (it synchronises internally).
-template <uint32_t TF, uint32_t TY, typename OffA>
-__device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok) {
+// of the block calls it (it synchronises internally).  If `pre` is given, warps
+// 4-7 run it first, while warps 0-3 substitute; it may read shared memory in
+// [TF, TF + 12K) (the region of T's first 48 rows), which the solve writes only
+// after it (named barriers 1 and 2).
+struct NoPre {
+    __device__ __forceinline__ void operator()() const {}
+};
+template <uint32_t TF, uint32_t TY, typename OffA, typename Pre = NoPre>
+__device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok, Pre pre = Pre()) {
+    constexpr bool kPre = !std::is_same<Pre, NoPre>::value;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto offT = [](int i, int j) { return TF + f32_offset(i, j); };
     auto offY = [](int i, int j) { return TY + (uint32_t)i * 64u + (uint32_t)j * 4u; };  // 4 blocks, rows of 16
-    if (ok) {
-        if (warp < 4) {
-            // diagonal block p: column `col` of (I + A_pp)^-1 by forward substitution (fp32)
-            const int p = warp, col = lane & 15;
-            float x[16];
+    if (warp < 4) {
+        // diagonal block p: column `col` of (I + A_pp)^-1 by forward substitution (fp32)
+        const int p = warp, col = lane & 15;
+        float x[16];
+        if (ok) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 float acc = 0.f;
@@ -151,18 +160,25 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok) {
                 for (int j = 0; j < i; ++j) acc += *reinterpret_cast<const float *>(sm + offA(16 * p + i, 16 * p + j)) * x[j];
                 x[i] = (i == col) ? 1.f : -acc;
             }
-            if (lane < 16)
+        }
+        if (kPre) named_bar_sync(1, 256);  // warps 4-7 are done with `pre`
+        if (ok && lane < 16)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + offT(16 * p + i, 16 * p + col)) = x[i];
-        } else {
-            // zero the strictly upper off-diagonal blocks
+            for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + offT(16 * p + i, 16 * p + col)) = x[i];
+    } else {
+        if (kPre) {
+            if (ok) pre();
+            named_bar_sync(2, 128);    // all of warps 4-7 are done with `pre` ...
+            named_bar_arrive(1, 256);  // ... so warps 0-3 may write T
+        }
+        // zero the strictly upper off-diagonal blocks
+        if (ok)
             for (int e = tid - 128; e < 6 * 256; e += 128) {
                 const int b = e >> 8, w = e & 255;
                 const int pb = b < 3 ? 0 : (b < 5 ? 1 : 2);
                 const int qb = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
                 *reinterpret_cast<float *>(sm + offT(16 * pb + (w >> 4), 16 * qb + (w & 15))) = 0.f;
             }
-        }
     }
     __syncthreads();
     // level 1: T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
