@@ -133,10 +133,11 @@ __device__ __forceinline__ uint32_t img_offset(int row, int col) {
 // below their diagonal and the blocks below the block diagonal); T is written
 // in fp32 at byte offset TF of `sm` (f32_offset layout, upper blocks zeroed);
 // TY is 4 KB of scratch.  Diagonal blocks: forward substitution in fp32 (one
-// column per lane); off-diagonal blocks by the block recurrence
-// T_pq = -T_pp sum_{q <= r < p} A_pr T_rq with tf32 warp MMAs.  Every thread
-// of the block calls it (it synchronises internally).  If `pre` is given, warps
-// 4-7 run it first, while warps 0-3 substitute; it may read shared memory in
+// column per lane, two blocks per warp); off-diagonal blocks by the block
+// recurrence T_pq = -T_pp sum_{q <= r < p} A_pr T_rq with tf32 warp MMAs (the
+// first level by the warps that formed its diagonal blocks).  Every thread of
+// the block calls it (it synchronises internally).  If `pre` is given, warps 4-7
+// run it first, while warps 0-1 substitute; it may read shared memory in
 // [TF, TF + 12K) (the region of T's first 48 rows), which the solve writes only
 // after it (named barriers 1 and 2).
 struct NoPre {
@@ -148,9 +149,10 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok, P
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto offT = [](int i, int j) { return TF + f32_offset(i, j); };
     auto offY = [](int i, int j) { return TY + (uint32_t)i * 64u + (uint32_t)j * 4u; };  // 4 blocks, rows of 16
-    if (warp < 4) {
-        // diagonal block p: column `col` of (I + A_pp)^-1 by forward substitution (fp32)
-        const int p = warp, col = lane & 15;
+    if (warp < 2) {
+        // diagonal blocks 2 warp and 2 warp + 1 (lanes 0-15 and 16-31): column `col` of
+        // (I + A_pp)^-1 by forward substitution (fp32) ...
+        const int p = 2 * warp + (lane >> 4), col = lane & 15;
         float x[16];
         if (ok) {
 #pragma unroll
@@ -161,15 +163,28 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok, P
                 x[i] = (i == col) ? 1.f : -acc;
             }
         }
-        if (kPre) named_bar_sync(1, 256);  // warps 4-7 are done with `pre`
-        if (ok && lane < 16)
+        if (kPre) named_bar_sync(1, 192);  // warps 4-7 are done with `pre`
+        if (ok)
 #pragma unroll
             for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + offT(16 * p + i, 16 * p + col)) = x[i];
-    } else {
+        __syncwarp();
+        // ... then level 1: T_pq = -D_p (A_pq D_q) for (p, q) = (2 warp + 1, 2 warp)
+        if (ok) {
+            const int pp = 2 * warp + 1, q = 2 * warp;
+            float c[2][4];
+            const int xr[1] = {16 * pp}, xc[1] = {16 * q}, yr[1] = {16 * q}, yc[1] = {16 * q};
+            warp_gemm16(sm, 1, xr, xc, yr, yc, offA, offT, c);
+            warp_store16(sm, 16 * warp, 0, c, 1.f, offY);
+            __syncwarp();
+            const int xr2[1] = {16 * pp}, xc2[1] = {16 * pp}, yr2[1] = {16 * warp}, yc2[1] = {0};
+            warp_gemm16(sm, 1, xr2, xc2, yr2, yc2, offT, offY, c);
+            warp_store16(sm, 16 * pp, 16 * q, c, -1.f, offT);
+        }
+    } else if (warp >= 4) {
         if (kPre) {
             if (ok) pre();
             named_bar_sync(2, 128);    // all of warps 4-7 are done with `pre` ...
-            named_bar_arrive(1, 256);  // ... so warps 0-3 may write T
+            named_bar_arrive(1, 192);  // ... so warps 0-1 may write T
         }
         // zero the strictly upper off-diagonal blocks
         if (ok)
@@ -179,19 +194,6 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok, P
                 const int qb = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
                 *reinterpret_cast<float *>(sm + offT(16 * pb + (w >> 4), 16 * qb + (w & 15))) = 0.f;
             }
-    }
-    __syncthreads();
-    // level 1: T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
-    if (ok && warp < 2) {
-        const int p = 2 * warp + 1, q = 2 * warp;
-        float c[2][4];
-        const int xr[1] = {16 * p}, xc[1] = {16 * q}, yr[1] = {16 * q}, yc[1] = {16 * q};
-        warp_gemm16(sm, 1, xr, xc, yr, yc, offA, offT, c);
-        warp_store16(sm, 16 * warp, 0, c, 1.f, offY);
-        __syncwarp();
-        const int xr2[1] = {16 * p}, xc2[1] = {16 * p}, yr2[1] = {16 * warp}, yc2[1] = {0};
-        warp_gemm16(sm, 1, xr2, xc2, yr2, yc2, offT, offY, c);
-        warp_store16(sm, 16 * p, 16 * q, c, -1.f, offT);
     }
     __syncthreads();
     // level 2, step 1: Y_pq = sum_{r in {0,1}} A_pr T_rq for p in {2,3}, q in {0,1}
