@@ -12,7 +12,7 @@
 // ("From Traditional Attention to hybrid ones", section 5): decay, the delta
 // correction on the decayed state, then the read of the updated state.  Rows of
 // the d_v x d_k state evolve independently, so the block's threads keep the state
-// in registers (two or four threads per row) and apply the tokens to it in order:
+// in registers (a warp per eight rows, a lane per d_k/32 columns) and apply the tokens in order:
 // the state is read from HBM once for all tokens and written back at most once
 // (plus one copy per token when the caller asks for every step's state).
 #include "gdn_internal.cuh"
@@ -20,7 +20,8 @@
 namespace gdn {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 4;        // warps per block
+constexpr int kRowsPerWarp = 8;  // state rows of one warp (a block: 32 rows)
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -28,26 +29,58 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-// Shared memory per token t of the block's (sequence, head): a_t k_t, a_t q_t,
-// a_t, k_t (d_k each; q already scaled) and v_t (d_v); then beta_t and k_t . q_t.
-// The 256 threads split the state into TPR = 256 / d_v threads per row; thread
-// part p of a row holds the 16-byte column chunks p, p + TPR, p + 2 TPR, ... in
-// registers, so one warp instruction moves whole 32-byte sectors of 8 or 16 rows.
-// A token's two dot products are per-thread sums (four independent partial sums)
-// finished by log2(TPR) shuffles.
+// Sums over the 32 lanes of eight per-lane values x[0..7] (one per row), left
+// reduce-scattered: lane l returns the total of row (l >> 2) & 7.  Nine shuffles
+// instead of 40 for eight separate reductions.
+__device__ __forceinline__ float reduce8(const float (&x)[8], int lane) {
+    float a[4], b2[2];
+    const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = (u16 ? x[i + 4] : x[i]) + __shfl_xor_sync(0xffffffffu, u16 ? x[i] : x[i + 4], 16);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) b2[i] = (u8 ? a[i + 2] : a[i]) + __shfl_xor_sync(0xffffffffu, u8 ? a[i] : a[i + 2], 8);
+    float c = (u4 ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, u4 ? b2[0] : b2[1], 4);
+    c += __shfl_xor_sync(0xffffffffu, c, 2);
+    c += __shfl_xor_sync(0xffffffffu, c, 1);
+    return c;
+}
+
+template <int VEC> struct Vec4;
+template <> struct Vec4<4> {
+    static __device__ __forceinline__ void ld(const float *p, float (&x)[4]) {
+        const float4 t = __ldcs(reinterpret_cast<const float4 *>(p));
+        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+    }
+    static __device__ __forceinline__ void st(float *p, const float (&x)[4]) {
+        __stcs(reinterpret_cast<float4 *>(p), make_float4(x[0], x[1], x[2], x[3]));
+    }
+};
+template <> struct Vec4<2> {
+    static __device__ __forceinline__ void ld(const float *p, float (&x)[2]) {
+        const float2 t = __ldcs(reinterpret_cast<const float2 *>(p));
+        x[0] = t.x; x[1] = t.y;
+    }
+    static __device__ __forceinline__ void st(float *p, const float (&x)[2]) {
+        __stcs(reinterpret_cast<float2 *>(p), make_float2(x[0], x[1]));
+    }
+};
+
+// Warp w of block (unit, y) owns rows 32 y + 8 w .. + 7 of the unit's state; lane l
+// holds columns l VEC .. l VEC + VEC - 1 of those rows in registers (one
+// coalesced row per load / store instruction).  Per token the lane reads its
+// columns of k, q and the gate straight into registers (the same for all eight
+// rows), the eight rows' dot products are reduce-scattered over the warp, and each
+// row's correction d is broadcast back for the update.
 template <int DK, int DV, typename Tin, bool PER_CHANNEL>
-__global__ void __launch_bounds__(kWarps * 32, 2)
+__global__ void __launch_bounds__(kWarps * 32)
 gdn_decode_multi_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                         const float *__restrict__ g, const float *__restrict__ beta,
                         const int32_t *__restrict__ n_tokens, float *__restrict__ state, int commit,
                         Tin *__restrict__ out, float *__restrict__ step_states, int T, int64_t H, int64_t Hk,
                         float scale) {
-    constexpr int TPR = kWarps * 32 / DV, NCH = DK / 4 / TPR, VEC = DK / 32;  // NCH chunks per thread
-    extern __shared__ float4 dm_raw[];
-    float *sm = reinterpret_cast<float *>(dm_raw);
-    constexpr int per_tok = 4 * DK + DV;
-    float *s_beta = sm + (size_t)T * per_tok, *s_kq = s_beta + T;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int VEC = DK / 32;
+    static_assert(DV % (kWarps * kRowsPerWarp) == 0, "layout");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t unit = blockIdx.x, b = unit / H, h = unit % H;
     int n = T;
     if (n_tokens) {
@@ -55,79 +88,68 @@ gdn_decode_multi_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, co
         n = n < 0 ? 0 : (n > T ? T : n);
     }
     if (n == 0) return;
-
-    // stage the tokens' vectors (warp w takes tokens w, w + 8, ...)
-    for (int t = warp; t < n; t += kWarps) {
-        const int64_t tk = (b * T + t) * H + h;             // (b, t, h)
-        const int64_t tq = (b * T + t) * Hk + h / (H / Hk);  // its query/key head
-        float *st = sm + (size_t)t * per_tok;
-        float kq = 0.f;
+    const int row0 = (int)blockIdx.y * (kWarps * kRowsPerWarp) + warp * kRowsPerWarp;
+    float *S = state + (unit * DV + row0) * (int64_t)DK + lane * VEC;
+    float s[kRowsPerWarp][VEC];
 #pragma unroll
-        for (int c = 0; c < VEC; ++c) {
-            const int col = lane * VEC + c;
-            const float kc = to_f32<Tin>(k[tq * DK + col]);
-            const float qc = scale * to_f32<Tin>(q[tq * DK + col]);
-            const float a = expf(PER_CHANNEL ? g[tk * DK + col] : g[tk]);
-            st[col] = a * kc;
-            st[DK + col] = a * qc;
-            st[2 * DK + col] = a;
-            st[3 * DK + col] = kc;
-            kq += kc * qc;
-        }
-        for (int r = lane; r < DV; r += 32) st[4 * DK + r] = to_f32<Tin>(v[tk * DV + r]);
-        kq = warp_sum(kq);
-        if (lane == 0) {
-            s_beta[t] = beta[tk];
-            s_kq[t] = kq;
-        }
-    }
-
-    const int row = tid / TPR, part = tid % TPR;
-    float4 s[NCH];  // chunk j holds columns 4 (j TPR + part) .. + 3
-    float *S = state + (unit * DV + row) * (int64_t)DK + 4 * part;
-#pragma unroll
-    for (int j = 0; j < NCH; ++j) s[j] = *reinterpret_cast<const float4 *>(S + 4 * j * TPR);
-    __syncthreads();
+    for (int r = 0; r < kRowsPerWarp; ++r) Vec4<VEC>::ld(S + (int64_t)r * DK, s[r]);
+    const int R = (lane >> 2) & 7;  // the row whose reduced sums this lane receives
 
     for (int t = 0; t < n; ++t) {
-        const float *st = sm + (size_t)t * per_tok + 4 * part;
-        float y[4] = {0.f, 0.f, 0.f, 0.f}, z[4] = {0.f, 0.f, 0.f, 0.f};
+        const int64_t tk = (b * T + t) * H + h;             // (b, t, h)
+        const int64_t tq = (b * T + t) * Hk + h / (H / Hk);  // its query/key head
+        float kr[VEC], qr[VEC], a[VEC];
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) {
-            const float4 ak = *reinterpret_cast<const float4 *>(st + 4 * j * TPR);
-            const float4 aq = *reinterpret_cast<const float4 *>(st + DK + 4 * j * TPR);
-            y[0] = fmaf(s[j].x, ak.x, y[0]); y[1] = fmaf(s[j].y, ak.y, y[1]);
-            y[2] = fmaf(s[j].z, ak.z, y[2]); y[3] = fmaf(s[j].w, ak.w, y[3]);
-            z[0] = fmaf(s[j].x, aq.x, z[0]); z[1] = fmaf(s[j].y, aq.y, z[1]);
-            z[2] = fmaf(s[j].z, aq.z, z[2]); z[3] = fmaf(s[j].w, aq.w, z[3]);
+        for (int c = 0; c < VEC; ++c) {
+            kr[c] = to_f32<Tin>(k[tq * DK + lane * VEC + c]);
+            qr[c] = scale * to_f32<Tin>(q[tq * DK + lane * VEC + c]);
         }
-        float yy = (y[0] + y[1]) + (y[2] + y[3]), zz = (z[0] + z[1]) + (z[2] + z[3]);
+        if (PER_CHANNEL) {
 #pragma unroll
-        for (int o = 1; o < TPR; o <<= 1) {
-            yy += __shfl_xor_sync(0xffffffffu, yy, o);
-            zz += __shfl_xor_sync(0xffffffffu, zz, o);
+            for (int c = 0; c < VEC; ++c) a[c] = expf(g[tk * DK + lane * VEC + c]);
+        } else {
+            const float al = expf(g[tk]);
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) a[c] = al;
         }
-        const float d = s_beta[t] * (st[4 * DK - 4 * part + row] - yy);
-        const int64_t tk = (b * T + t) * H + h;
-        if (part == 0) out[tk * DV + row] = from_f32<Tin>(zz + d * s_kq[t]);
+        const float vb = lane < kRowsPerWarp ? to_f32<Tin>(v[tk * DV + row0 + lane]) : 0.f;
+        const float bt = beta[tk];
+        float kq = 0.f;
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) {
-            const float4 a = *reinterpret_cast<const float4 *>(st + 2 * DK + 4 * j * TPR);
-            const float4 kk = *reinterpret_cast<const float4 *>(st + 3 * DK + 4 * j * TPR);
-            s[j].x = fmaf(a.x, s[j].x, d * kk.x);
-            s[j].y = fmaf(a.y, s[j].y, d * kk.y);
-            s[j].z = fmaf(a.z, s[j].z, d * kk.z);
-            s[j].w = fmaf(a.w, s[j].w, d * kk.w);
+        for (int c = 0; c < VEC; ++c) kq = fmaf(kr[c], qr[c], kq);
+        kq = warp_sum(kq);
+        // what the decayed state predicts for k, and its read by q, for the eight rows
+        float yp[kRowsPerWarp], zp[kRowsPerWarp];
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            float y = 0.f, z = 0.f;
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) {
+                const float sa = s[r][c] * a[c];
+                y = fmaf(sa, kr[c], y);
+                z = fmaf(sa, qr[c], z);
+            }
+            yp[r] = y;
+            zp[r] = z;
+        }
+        const float y = reduce8(yp, lane), z = reduce8(zp, lane);
+        const float d = bt * (__shfl_sync(0xffffffffu, vb, R) - y);
+        if ((lane & 3) == 0) out[tk * DV + row0 + R] = from_f32<Tin>(z + d * kq);
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const float dr = __shfl_sync(0xffffffffu, d, 4 * r);
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) s[r][c] = fmaf(a[c], s[r][c], dr * kr[c]);
         }
         if (step_states) {
-            float *p = step_states + (tk * DV + row) * (int64_t)DK + 4 * part;
+            float *p = step_states + (tk * DV + row0) * (int64_t)DK + lane * VEC;
 #pragma unroll
-            for (int j = 0; j < NCH; ++j) *reinterpret_cast<float4 *>(p + 4 * j * TPR) = s[j];
+            for (int r = 0; r < kRowsPerWarp; ++r) Vec4<VEC>::st(p + (int64_t)r * DK, s[r]);
         }
     }
     if (commit) {
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) *reinterpret_cast<float4 *>(S + 4 * j * TPR) = s[j];
+        for (int r = 0; r < kRowsPerWarp; ++r) Vec4<VEC>::st(S + (int64_t)r * DK, s[r]);
     }
 }
 
@@ -150,17 +172,13 @@ gdn_status launch_multi(const gdn_desc &d, const void *q, const void *k, const v
                         float *step_states, cudaStream_t s) {
     const int64_t units = d.B * d.H;
     if (units > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "too many (sequence, head) pairs");
-    const size_t smem = ((size_t)d.T * (4 * DK + DV) + 2 * (size_t)d.T) * sizeof(float);
     auto kern = d.gate == GDN_GATE_CHANNEL ? gdn_decode_multi_kernel<DK, DV, Tin, true>
                                            : gdn_decode_multi_kernel<DK, DV, Tin, false>;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return check_launch("gdn_decode_multi attributes");
     {
         LaunchScope ls("gdn_decode_multi_kernel", s);
-        kern<<<(unsigned)units, kWarps * 32, smem, s>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta,
-                                                        n_tokens, state, commit, (Tin *)out, step_states,
-                                                        (int)d.T, d.H, qk_heads(d), d.scale);
+        kern<<<dim3((unsigned)units, (unsigned)(DV / (kWarps * kRowsPerWarp))), kWarps * 32, 0, s>>>(
+            (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, n_tokens, state, commit, (Tin *)out, step_states,
+            (int)d.T, d.H, qk_heads(d), d.scale);
     }
     return check_launch("gdn_decode_multi_kernel");
 }
