@@ -15,62 +15,15 @@
 // in registers (a warp per eight rows, a lane per d_k/32 columns) and apply the tokens in order:
 // the state is read from HBM once for all tokens and written back at most once
 // (plus one copy per token when the caller asks for every step's state).
-#include "gdn_internal.cuh"
+#include "decode_rows.cuh"
 
 namespace gdn {
 namespace {
 
-constexpr int kWarps = 4;        // warps per block
-constexpr int kRowsPerWarp = 8;  // state rows of one warp (a block: 32 rows)
+using dec::kRowsPerWarp;
+using dec::kWarps;
 
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
-// Sums over the 32 lanes of eight per-lane values x[0..7] (one per row), left
-// reduce-scattered: lane l returns the total of row (l >> 2) & 7.  Nine shuffles
-// instead of 40 for eight separate reductions.
-__device__ __forceinline__ float reduce8(const float (&x)[8], int lane) {
-    float a[4], b2[2];
-    const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = (u16 ? x[i + 4] : x[i]) + __shfl_xor_sync(0xffffffffu, u16 ? x[i] : x[i + 4], 16);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) b2[i] = (u8 ? a[i + 2] : a[i]) + __shfl_xor_sync(0xffffffffu, u8 ? a[i] : a[i + 2], 8);
-    float c = (u4 ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, u4 ? b2[0] : b2[1], 4);
-    c += __shfl_xor_sync(0xffffffffu, c, 2);
-    c += __shfl_xor_sync(0xffffffffu, c, 1);
-    return c;
-}
-
-template <int VEC> struct Vec4;
-template <> struct Vec4<4> {
-    static __device__ __forceinline__ void ld(const float *p, float (&x)[4]) {
-        const float4 t = __ldcs(reinterpret_cast<const float4 *>(p));
-        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
-    }
-    static __device__ __forceinline__ void st(float *p, const float (&x)[4]) {
-        __stcs(reinterpret_cast<float4 *>(p), make_float4(x[0], x[1], x[2], x[3]));
-    }
-};
-template <> struct Vec4<2> {
-    static __device__ __forceinline__ void ld(const float *p, float (&x)[2]) {
-        const float2 t = __ldcs(reinterpret_cast<const float2 *>(p));
-        x[0] = t.x; x[1] = t.y;
-    }
-    static __device__ __forceinline__ void st(float *p, const float (&x)[2]) {
-        __stcs(reinterpret_cast<float2 *>(p), make_float2(x[0], x[1]));
-    }
-};
-
-// Warp w of block (unit, y) owns rows 32 y + 8 w .. + 7 of the unit's state; lane l
-// holds columns l VEC .. l VEC + VEC - 1 of those rows in registers (one
-// coalesced row per load / store instruction).  Per token the lane reads its
-// columns of k, q and the gate straight into registers (the same for all eight
-// rows), the eight rows' dot products are reduce-scattered over the warp, and each
-// row's correction d is broadcast back for the update.
+// See decode_rows: a warp per eight state rows, a lane per d_k / 32 columns.
 template <int DK, int DV, typename Tin, bool PER_CHANNEL>
 __global__ void __launch_bounds__(kWarps * 32)
 gdn_decode_multi_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
@@ -78,79 +31,14 @@ gdn_decode_multi_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, co
                         const int32_t *__restrict__ n_tokens, float *__restrict__ state, int commit,
                         Tin *__restrict__ out, float *__restrict__ step_states, int T, int64_t H, int64_t Hk,
                         float scale) {
-    constexpr int VEC = DK / 32;
-    static_assert(DV % (kWarps * kRowsPerWarp) == 0, "layout");
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t unit = blockIdx.x, b = unit / H, h = unit % H;
     int n = T;
     if (n_tokens) {
-        n = n_tokens[b];
+        n = n_tokens[blockIdx.x / H];
         n = n < 0 ? 0 : (n > T ? T : n);
     }
     if (n == 0) return;
-    const int row0 = (int)blockIdx.y * (kWarps * kRowsPerWarp) + warp * kRowsPerWarp;
-    float *S = state + (unit * DV + row0) * (int64_t)DK + lane * VEC;
-    float s[kRowsPerWarp][VEC];
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) Vec4<VEC>::ld(S + (int64_t)r * DK, s[r]);
-    const int R = (lane >> 2) & 7;  // the row whose reduced sums this lane receives
-
-    for (int t = 0; t < n; ++t) {
-        const int64_t tk = (b * T + t) * H + h;             // (b, t, h)
-        const int64_t tq = (b * T + t) * Hk + h / (H / Hk);  // its query/key head
-        float kr[VEC], qr[VEC], a[VEC];
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) {
-            kr[c] = to_f32<Tin>(k[tq * DK + lane * VEC + c]);
-            qr[c] = scale * to_f32<Tin>(q[tq * DK + lane * VEC + c]);
-        }
-        if (PER_CHANNEL) {
-#pragma unroll
-            for (int c = 0; c < VEC; ++c) a[c] = expf(g[tk * DK + lane * VEC + c]);
-        } else {
-            const float al = expf(g[tk]);
-#pragma unroll
-            for (int c = 0; c < VEC; ++c) a[c] = al;
-        }
-        const float vb = lane < kRowsPerWarp ? to_f32<Tin>(v[tk * DV + row0 + lane]) : 0.f;
-        const float bt = beta[tk];
-        float kq = 0.f;
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) kq = fmaf(kr[c], qr[c], kq);
-        kq = warp_sum(kq);
-        // what the decayed state predicts for k, and its read by q, for the eight rows
-        float yp[kRowsPerWarp], zp[kRowsPerWarp];
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) {
-            float y = 0.f, z = 0.f;
-#pragma unroll
-            for (int c = 0; c < VEC; ++c) {
-                const float sa = s[r][c] * a[c];
-                y = fmaf(sa, kr[c], y);
-                z = fmaf(sa, qr[c], z);
-            }
-            yp[r] = y;
-            zp[r] = z;
-        }
-        const float y = reduce8(yp, lane), z = reduce8(zp, lane);
-        const float d = bt * (__shfl_sync(0xffffffffu, vb, R) - y);
-        if ((lane & 3) == 0) out[tk * DV + row0 + R] = from_f32<Tin>(z + d * kq);
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) {
-            const float dr = __shfl_sync(0xffffffffu, d, 4 * r);
-#pragma unroll
-            for (int c = 0; c < VEC; ++c) s[r][c] = fmaf(a[c], s[r][c], dr * kr[c]);
-        }
-        if (step_states) {
-            float *p = step_states + (tk * DV + row0) * (int64_t)DK + lane * VEC;
-#pragma unroll
-            for (int r = 0; r < kRowsPerWarp; ++r) Vec4<VEC>::st(p + (int64_t)r * DK, s[r]);
-        }
-    }
-    if (commit) {
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) Vec4<VEC>::st(S + (int64_t)r * DK, s[r]);
-    }
+    dec::decode_rows<DK, DV, Tin, PER_CHANNEL>(q, k, v, g, beta, state, commit != 0, out, step_states, n, T, H, Hk,
+                                               scale);
 }
 
 // state[b, h] = step_states[b, accept[b] - 1, h] where accept[b] > 0.
