@@ -243,6 +243,10 @@ def traffic_for(kernel: str):
         return None
     if kernel_source_hash(os.path.join(ROOT, rec["source"]), kernel) != rec["sha256"]:
         return None
+    for dep, sha in rec.get("deps", {}).items():  # files the kernel's code comes from, hashed whole
+        path = os.path.join(ROOT, dep)
+        if not os.path.exists(path) or hashlib.sha256(open(path, "rb").read()).hexdigest() != sha:
+            return None
     return float(rec["bytes_per_launch"])
 
 
