@@ -193,9 +193,9 @@ def _decode_gpu(x):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("per_channel", [False, True])
-@pytest.mark.parametrize("d", [64, 128])
-def test_decode_steps(dtype, per_channel, d):
-    w = DECODE.replace(B=6, H=3, dk=d, dv=d, decode_steps=20, dtype=dtype, per_channel=per_channel, seed=20)
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64), (64, 128)])
+def test_decode_steps(dtype, per_channel, dk, dv):
+    w = DECODE.replace(B=6, H=3, dk=dk, dv=dv, decode_steps=20, dtype=dtype, per_channel=per_channel, seed=20)
     x = make_inputs(w)
     o, s = _decode_gpu(x)
     o_ref, s_ref, _ = _decode_oracle(x)
@@ -226,9 +226,9 @@ def test_decode_continues_prefill():
 # Multi-token decode (speculative verify) and rollback
 # ---------------------------------------------------------------------------
 
-def _multi_inputs(dtype, per_channel, d, B=5, T=6, H=3, seed=30):
-    w = DECODE.replace(B=B, H=H, dk=d, dv=d, decode_steps=0, T=T, dtype=dtype, per_channel=per_channel,
-                       h0_std=0.1, seed=seed)
+def _multi_inputs(dtype, per_channel, d, B=5, T=6, H=3, seed=30, dv=None):
+    w = DECODE.replace(B=B, H=H, dk=d, dv=d if dv is None else dv, decode_steps=0, T=T, dtype=dtype,
+                       per_channel=per_channel, h0_std=0.1, seed=seed)
     return make_inputs(w)
 
 
@@ -251,9 +251,9 @@ def _multi_oracle(x, n):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("per_channel", [False, True])
-@pytest.mark.parametrize("d", [64, 128])
-def test_decode_multi_commit(dtype, per_channel, d):
-    x = _multi_inputs(dtype, per_channel, d)
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64), (64, 128)])
+def test_decode_multi_commit(dtype, per_channel, dk, dv):
+    x = _multi_inputs(dtype, per_channel, dk, dv=dv)
     dx = to_dev(x)
     st = dx.h0.clone()
     out, steps = gdn.gdn_decode_multi(dx.q, dx.k, dx.v, dx.g, dx.beta, st, commit=True, step_states=True)
