@@ -460,7 +460,9 @@ SPEC_K = 4  # draft tokens per sequence in the speculative-decoding measurement
 def run_prerule(args) -> int:
     """The work before the recurrence (gdn_prerule: short convolution + SiLU, q/k length,
     gates) on the prefill workload's shape, with the convolution history read and
-    written, then the same followed by the chunked prefill (the layer core)."""
+    written, then the same followed by the chunked prefill (the layer core); and a
+    decode step from raw projections on the decode workload's shape, fused
+    (gdn_decode_step_prerule) and as gdn_prerule followed by gdn_decode_step."""
     import torch
 
     from gated_delta_rule_64_b200 import gdn
@@ -486,6 +488,22 @@ def run_prerule(args) -> int:
                                                                       conv_state_out=hist, stream=stream),
                                                      h0, final_state=h0, workspace=ws, stream=stream),
     }
+    # a decode step from raw projections on the decode workload's shape (256 sequences x
+    # 32 heads, one token each): fused (gdn_decode_step_prerule) against gdn_prerule
+    # followed by gdn_decode_step
+    from gated_delta_rule_64_b200.inputs import DECODE
+    wd = DECODE
+    pd = make_prerule_inputs(B=wd.B, T=1, H=wd.H, hk=wd.H, dk=wd.dk, dv=wd.dv, dtype=wd.dtype, seed=wd.seed)
+    dx, da, db, dcw, dal, ddt, dhist = (d(t) for t in (pd.x[:, 0], pd.a[:, 0], pd.b[:, 0], pd.conv_w, pd.A_log,
+                                                       pd.dt_bias, pd.hist))
+    dstate = torch.zeros((wd.B, wd.H, wd.dv, wd.dk), dtype=torch.float32, device="cuda")
+    dout = torch.empty((wd.B, wd.H, wd.dv), dtype=dx.dtype, device="cuda")
+    modes["decode: fused pre-rule + step"] = lambda: gdn.gdn_decode_step_prerule(
+        dx, da, db, dcw, dal, ddt, dhist, dstate, hk=wd.H, dk=wd.dk, H=wd.H, dv=wd.dv, out=dout, stream=stream)
+    modes["decode: pre-rule, then step"] = lambda: gdn.gdn_decode_step(
+        *gdn.gdn_prerule(dx[:, None], da[:, None], db[:, None], dcw, dal, ddt, hk=wd.H, dk=wd.dk, H=wd.H, dv=wd.dv,
+                         conv_state_in=dhist, conv_state_out=dhist, stream=stream), dstate, out=dout, stream=stream)
+    tokens = {"decode: fused pre-rule + step": wd.B, "decode: pre-rule, then step": wd.B}
     el = x.element_size()
     pre_bytes = B * T * (C * el + 2 * w.H * el) + 2 * B * C * (K - 1) * 4 + B * T * C * el + B * T * w.H * 8
     clocks = ClockSampler(0)
@@ -507,7 +525,7 @@ def run_prerule(args) -> int:
         gdn.profile_enable(False)
         kern = gdn.profile_read()
         ms = e0.elapsed_time(e1) / args.steps
-        res[name] = {"ms_per_step": ms, "tokens_per_s": B * T / (ms * 1e-3),
+        res[name] = {"ms_per_step": ms, "tokens_per_s": tokens.get(name, B * T) / (ms * 1e-3),
                      "kernels_us": {n: t / max(1, c) * 1e3 for n, (c, t) in kern.items()}}
     pre_us = res["prerule"]["kernels_us"].get("gdn_prerule_kernel", 0.0) + \
         res["prerule"]["kernels_us"].get("gdn_prerule_history", 0.0)

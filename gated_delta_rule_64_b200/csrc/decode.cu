@@ -18,7 +18,8 @@ __global__ void __launch_bounds__(dec::kWarps * 32)
 gdn_decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                   const float *__restrict__ g, const float *__restrict__ beta, float *__restrict__ state,
                   Tin *__restrict__ out, int64_t H, int64_t Hk, float scale) {
-    dec::decode_rows<DK, DV, Tin, PER_CHANNEL>(q, k, v, g, beta, state, true, out, nullptr, 1, 1, H, Hk, scale);
+    const dec::ArraySrc<DK, DV, Tin, PER_CHANNEL> src{q, k, v, g, beta, Hk, scale};
+    dec::decode_rows<DK, DV, Tin>(src, state, true, out, nullptr, 1, 1, H);
 }
 
 template <int DK, int DV, typename Tin>

@@ -37,8 +37,8 @@ gdn_decode_multi_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, co
         n = n < 0 ? 0 : (n > T ? T : n);
     }
     if (n == 0) return;
-    dec::decode_rows<DK, DV, Tin, PER_CHANNEL>(q, k, v, g, beta, state, commit != 0, out, step_states, n, T, H, Hk,
-                                               scale);
+    const dec::ArraySrc<DK, DV, Tin, PER_CHANNEL> src{q, k, v, g, beta, Hk, scale};
+    dec::decode_rows<DK, DV, Tin>(src, state, commit != 0, out, step_states, n, T, H);
 }
 
 // state[b, h] = step_states[b, accept[b] - 1, h] where accept[b] > 0.

@@ -63,35 +63,21 @@ template <> struct Vec4<2> {
     }
 };
 
-// Warp w of block (unit, y) owns rows 32 y + 8 w .. + 7 of the unit's state; lane l
-// holds columns l VEC .. l VEC + VEC - 1 of those rows in registers (one
-// coalesced row per load / store instruction).  Per token the lane reads its
-// columns of k, q and the gate straight into registers (the same for all eight
-// rows), the eight rows' dot products are reduce-scattered over the warp, and
-// each row's correction d is broadcast back for the update.
-//   tokens n (<= T) of unit = b H + h, inputs laid out (B, T, H or Hk, d);
-//   commit: write the state back; step_states: (B, T, H, d_v, d_k) or nullptr.
+// Where a token's vectors come from: the q, k, v, gate and beta arrays.
+// token() gives lane l's columns l VEC .. l VEC + VEC - 1 of k and of scale * q and
+// the decay a = exp(g) on them, v of row row0 + l (lanes 0 .. 7) and beta.
 template <int DK, int DV, typename Tin, bool PER_CHANNEL>
-__device__ __forceinline__ void decode_rows(const Tin *__restrict__ q, const Tin *__restrict__ k,
-                                            const Tin *__restrict__ v, const float *__restrict__ g,
-                                            const float *__restrict__ beta, float *__restrict__ state, bool commit,
-                                            Tin *__restrict__ out, float *__restrict__ step_states, int n, int T,
-                                            int64_t H, int64_t Hk, float scale) {
-    constexpr int VEC = DK / 32;
-    static_assert(DV % (kWarps * kRowsPerWarp) == 0, "layout");
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t unit = blockIdx.x, b = unit / H, h = unit % H;
-    const int row0 = (int)blockIdx.y * (kWarps * kRowsPerWarp) + warp * kRowsPerWarp;
-    float *S = state + (unit * DV + row0) * (int64_t)DK + lane * VEC;
-    float s[kRowsPerWarp][VEC];
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) Vec4<VEC>::ld(S + (int64_t)r * DK, s[r]);
-    const int R = (lane >> 2) & 7;  // the row whose reduced sums this lane receives
-
-    for (int t = 0; t < n; ++t) {
+struct ArraySrc {
+    const Tin *q, *k, *v;
+    const float *g, *beta;
+    int64_t Hk;
+    float scale;
+    template <int VEC>
+    __device__ __forceinline__ void token(int64_t b, int t, int T, int64_t H, int64_t h, int row0, int lane,
+                                          float (&kr)[VEC], float (&qr)[VEC], float (&a)[VEC], float &vb,
+                                          float &bt) const {
         const int64_t tk = (b * T + t) * H + h;             // (b, t, h)
         const int64_t tq = (b * T + t) * Hk + h / (H / Hk);  // its query/key head
-        float kr[VEC], qr[VEC], a[VEC];
 #pragma unroll
         for (int c = 0; c < VEC; ++c) {
             kr[c] = to_f32<Tin>(k[tq * DK + lane * VEC + c]);
@@ -105,8 +91,39 @@ __device__ __forceinline__ void decode_rows(const Tin *__restrict__ q, const Tin
 #pragma unroll
             for (int c = 0; c < VEC; ++c) a[c] = al;
         }
-        const float vb = lane < kRowsPerWarp ? to_f32<Tin>(v[tk * DV + row0 + lane]) : 0.f;
-        const float bt = beta[tk];
+        vb = lane < 8 ? to_f32<Tin>(v[tk * DV + row0 + lane]) : 0.f;
+        bt = beta[tk];
+    }
+};
+
+// Warp w of block (unit, y) owns rows 8 (y W + w) .. + 7 of the unit's state (W warps
+// per block; the decode kernels use 4, i.e. 32 rows per block); lane l
+// holds columns l VEC .. l VEC + VEC - 1 of those rows in registers (one
+// coalesced row per load / store instruction).  Per token the lane takes its
+// columns of k, q and the decay from `src` straight into registers (the same for
+// all eight rows), the eight rows' dot products are reduce-scattered over the
+// warp, and each row's correction d is broadcast back for the update.
+//   tokens n (<= T) of unit = b H + h, outputs laid out (B, T, H, d_v);
+//   commit: write the state back; step_states: (B, T, H, d_v, d_k) or nullptr.
+template <int DK, int DV, typename Tin, typename Src>
+__device__ __forceinline__ void decode_rows(const Src &src, float *__restrict__ state, bool commit,
+                                            Tin *__restrict__ out, float *__restrict__ step_states, int n, int T,
+                                            int64_t H) {
+    constexpr int VEC = DK / 32;
+    static_assert(DV % (kWarps * kRowsPerWarp) == 0, "layout");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t unit = blockIdx.x, b = unit / H, h = unit % H;
+    const int row0 = ((int)blockIdx.y * (int)(blockDim.x >> 5) + warp) * kRowsPerWarp;  // eight rows per warp
+    float *S = state + (unit * DV + row0) * (int64_t)DK + lane * VEC;
+    float s[kRowsPerWarp][VEC];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) Vec4<VEC>::ld(S + (int64_t)r * DK, s[r]);
+    const int R = (lane >> 2) & 7;  // the row whose reduced sums this lane receives
+
+    for (int t = 0; t < n; ++t) {
+        const int64_t tk = (b * T + t) * H + h;  // (b, t, h)
+        float kr[VEC], qr[VEC], a[VEC], vb, bt;
+        src.template token<VEC>(b, t, T, H, h, row0, lane, kr, qr, a, vb, bt);
         float kq = 0.f;
 #pragma unroll
         for (int c = 0; c < VEC; ++c) kq = fmaf(kr[c], qr[c], kq);

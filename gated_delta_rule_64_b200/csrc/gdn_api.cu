@@ -354,6 +354,59 @@ gdn_status gdn_decode_step(const gdn_desc *d, const void *q, const void *k, cons
     return launch_decode(*d, q, k, v, log_gate, beta, state, out, (cudaStream_t)stream);
 }
 
+gdn_status gdn_decode_step_prerule(const gdn_desc *d, const void *x, const void *a, const void *b,
+                                   const float *conv_w, int32_t K, const float *A_log, const float *dt_bias,
+                                   float *conv_state, float *state, void *out, gdn_stream_t stream) {
+    g_last_error[0] = 0;
+    gdn_status st = check_desc(d);
+    if (st != GDN_OK) return st;
+    if (d->T != 1) return fail(GDN_ERR_INVALID_ARG, "decode needs T == 1 (got %lld)", (long long)d->T);
+    if (d->gate != GDN_GATE_HEAD)
+        return fail(GDN_ERR_UNSUPPORTED, "the pre-rule gate formula is the per-head one");
+    if (K < 1 || K > 4) return fail(GDN_ERR_UNSUPPORTED, "convolution width %d (1 .. 4 supported)", K);
+    if (d->B == 0) return GDN_OK;
+    if (!x || !a || !b || !conv_w || !A_log || !dt_bias || !state || !out)
+        return fail(GDN_ERR_INVALID_ARG, "x, a, b, conv_w, A_log, dt_bias, state and out are required");
+    const size_t el = d->dtype == GDN_F32 ? 4 : 2;
+    if (!aligned16(state) || !aligned16(out)) return fail(GDN_ERR_INVALID_ARG, "state and out must be 16-byte aligned");
+    if (((uintptr_t)x % el) || ((uintptr_t)a % el) || ((uintptr_t)b % el) || !aligned4(conv_w) || !aligned4(A_log) ||
+        !aligned4(dt_bias) || (conv_state && !aligned4(conv_state)))
+        return fail(GDN_ERR_INVALID_ARG, "x, a, b: element-aligned; conv_w, A_log, dt_bias, conv_state: 4-byte aligned");
+    const int64_t Hk = qk_heads(*d), C = 2 * Hk * d->dk + d->H * d->dv;
+    const Range outs[] = {range_of(out, (size_t)d->B * d->H * d->dv * el),
+                          range_of(state, (size_t)d->B * d->H * d->dv * d->dk * 4),
+                          range_of(conv_state, conv_state ? (size_t)d->B * C * (K - 1) * 4 : 0)};
+    const Range ins[] = {range_of(x, (size_t)d->B * C * el), range_of(a, (size_t)d->B * d->H * el),
+                         range_of(b, (size_t)d->B * d->H * el), range_of(conv_w, (size_t)C * K * 4),
+                         range_of(A_log, (size_t)d->H * 4), range_of(dt_bias, (size_t)d->H * 4)};
+    for (int i = 0; i < 3; ++i) {
+        for (const Range &r : ins)
+            if (overlaps(outs[i], r)) return fail(GDN_ERR_INVALID_ARG, "an output overlaps an input");
+        for (int j = i + 1; j < 3; ++j)
+            if (overlaps(outs[i], outs[j])) return fail(GDN_ERR_INVALID_ARG, "outputs overlap");
+    }
+    PreruleArgs p{};
+    p.dtype = d->dtype;
+    p.K = K;
+    p.T = 1;
+    p.N = d->B;
+    p.rows = d->B;
+    p.H = d->H;
+    p.Hk = Hk;
+    p.dk = d->dk;
+    p.dv = d->dv;
+    p.x = x;
+    p.a = a;
+    p.b = b;
+    p.conv_w = conv_w;
+    p.A_log = A_log;
+    p.dt_bias = dt_bias;
+    p.cu_seqlens = nullptr;
+    p.hist_in = conv_state;
+    p.hist_out = conv_state;
+    return launch_decode_prerule(*d, p, state, out, (cudaStream_t)stream);
+}
+
 gdn_status gdn_decode_multi(const gdn_desc *d, const void *q, const void *k, const void *v,
                             const float *log_gate, const float *beta, const int32_t *n_tokens, float *state,
                             int32_t commit, void *out, float *step_states, gdn_stream_t stream) {

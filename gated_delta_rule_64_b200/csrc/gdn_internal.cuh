@@ -114,6 +114,12 @@ struct PreruleArgs {
     float *g, *beta;
 };
 gdn_status launch_prerule(const PreruleArgs &a, cudaStream_t s);
+// Only the convolution history update of launch_prerule (hist_in -> hist_out, in place
+// allowed), for the leading `channels` channels of every row (< 0: all).
+gdn_status launch_prerule_history(const PreruleArgs &a, int64_t channels, cudaStream_t s);
+// A decode step from the raw projections (one token per sequence, T = 1): the pre-rule
+// work for the token in registers, then the recurrence; the history is updated after.
+gdn_status launch_decode_prerule(const gdn_desc &d, const PreruleArgs &a, float *state, void *out, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Device helpers

@@ -272,9 +272,10 @@ gdn_prerule_kernel(const Tin *__restrict__ x, const Tin *__restrict__ a, const T
 // hist_out may be hist_in.
 template <typename Tin, int K>
 __global__ void gdn_prerule_history(const Tin *__restrict__ x, const int32_t *__restrict__ cu, int64_t N, int64_t T,
-                                    int64_t C, const float *hist_in, float *hist_out) {
+                                    int64_t C, int64_t Cn, const float *hist_in, float *hist_out) {
+    // channels [0, Cn) of rows of C channels
     const int64_t n = blockIdx.x, ch = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;
-    if (ch >= C || K < 2) return;
+    if (ch >= Cn || K < 2) return;
     int64_t start, len;
     if (cu) {
         start = cu[n];
@@ -324,7 +325,7 @@ gdn_status launch_k(const PreruleArgs &a, cudaStream_t s) {
     {
         LaunchScope ls("gdn_prerule_history", s);
         gdn_prerule_history<Tin, K><<<dim3((unsigned)a.N, (unsigned)((C + 255) / 256)), 256, 0, s>>>(
-            (const Tin *)a.x, a.cu_seqlens, a.N, a.T, C, a.hist_in, a.hist_out);
+            (const Tin *)a.x, a.cu_seqlens, a.N, a.T, C, C, a.hist_in, a.hist_out);
     }
     return check_launch("gdn_prerule_history");
 }
@@ -344,6 +345,34 @@ gdn_status launch_t(const PreruleArgs &a, cudaStream_t s) {
 
 gdn_status launch_prerule(const PreruleArgs &a, cudaStream_t s) {
     return a.dtype == GDN_BF16 ? launch_t<__nv_bfloat16>(a, s) : launch_t<float>(a, s);
+}
+
+namespace {
+template <typename Tin, int K>
+gdn_status launch_history_k(const PreruleArgs &a, int64_t channels, cudaStream_t s) {
+    const int64_t C = 2 * a.Hk * a.dk + a.H * a.dv, Cn = channels < 0 || channels > C ? C : channels;
+    if (!a.hist_out || K < 2 || a.N == 0 || Cn == 0) return GDN_OK;
+    {
+        LaunchScope ls("gdn_prerule_history", s);
+        gdn_prerule_history<Tin, K><<<dim3((unsigned)a.N, (unsigned)((Cn + 255) / 256)), 256, 0, s>>>(
+            (const Tin *)a.x, a.cu_seqlens, a.N, a.T, C, Cn, a.hist_in, a.hist_out);
+    }
+    return check_launch("gdn_prerule_history");
+}
+template <typename Tin>
+gdn_status launch_history_t(const PreruleArgs &a, int64_t channels, cudaStream_t s) {
+    switch (a.K) {
+        case 2: return launch_history_k<Tin, 2>(a, channels, s);
+        case 3: return launch_history_k<Tin, 3>(a, channels, s);
+        case 4: return launch_history_k<Tin, 4>(a, channels, s);
+        default: return GDN_OK;  // K = 1 keeps no history
+    }
+}
+}  // namespace
+
+gdn_status launch_prerule_history(const PreruleArgs &a, int64_t channels, cudaStream_t s) {
+    return a.dtype == GDN_BF16 ? launch_history_t<__nv_bfloat16>(a, channels, s)
+                               : launch_history_t<float>(a, channels, s);
 }
 
 }  // namespace gdn

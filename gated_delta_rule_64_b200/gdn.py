@@ -25,8 +25,8 @@ GDN_F32, GDN_BF16 = 0, 1
 GDN_GATE_HEAD, GDN_GATE_CHANNEL = 0, 1
 
 EXPORTED = ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
-            "gdn_decode_multi", "gdn_state_select", "gdn_prerule", "gdn_status_string", "gdn_last_error",
-            "gdn_profile_enable", "gdn_profile_read")
+            "gdn_decode_multi", "gdn_state_select", "gdn_prerule", "gdn_decode_step_prerule", "gdn_status_string",
+            "gdn_last_error", "gdn_profile_enable", "gdn_profile_read")
 
 
 class GdnDesc(ctypes.Structure):
@@ -68,6 +68,7 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_decode_multi.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
         lib.gdn_state_select.argtypes = [dp, vp, vp, vp, vp]
         lib.gdn_prerule.argtypes = [dp, vp, vp, vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.gdn_decode_step_prerule.argtypes = [dp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]
         lib.gdn_status_string.argtypes = [ctypes.c_int]
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_last_error.argtypes = []
@@ -75,8 +76,8 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_profile_enable.argtypes = [ctypes.c_int]
         lib.gdn_profile_read.argtypes = [ctypes.POINTER(GdnKernelTime), i32, ctypes.POINTER(i32)]
         for name in ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
-                     "gdn_decode_multi", "gdn_state_select", "gdn_prerule", "gdn_profile_enable",
-                     "gdn_profile_read"):
+                     "gdn_decode_multi", "gdn_state_select", "gdn_prerule", "gdn_decode_step_prerule",
+                     "gdn_profile_enable", "gdn_profile_read"):
             getattr(lib, name).restype = ctypes.c_int
         if path == LIB_PATH:
             _lib = lib
@@ -262,6 +263,24 @@ def gdn_prerule(x, a, b, conv_w, A_log, dt_bias, *, hk, dk, H, dv, cu_seqlens=No
                          _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _stream(stream))
     _check(lib, st)
     return q, k, v, g, beta
+
+
+def gdn_decode_step_prerule(x, a, b, conv_w, A_log, dt_bias, conv_state, state, *, hk, dk, H, dv, scale=1.0,
+                            out=None, stream=None):
+    """One decode step from the raw projections: x (B,2*hk*dk+H*dv) (or (B,1,C)); a, b (B,H)
+    (or (B,1,H)) in x's dtype; conv_w (C,K), A_log, dt_bias (H,) fp32; conv_state (B,C,K-1) fp32
+    or None, updated in place; state (B,H,dv,dk) fp32, updated in place.  Returns out (B,H,dv)."""
+    lib = load_library()
+    _need_cuda(x, a, b, conv_w, A_log, dt_bias, conv_state, state)
+    B = x.shape[0]
+    K = conv_w.shape[1]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=x.dtype, device=x.device)
+    d = make_desc(B, 1, H, dk, dv, _dtype_code(x), False, scale, hk)
+    _check(lib, lib.gdn_decode_step_prerule(ctypes.byref(d), _ptr(x), _ptr(a), _ptr(b), _ptr(conv_w), int(K),
+                                            _ptr(A_log), _ptr(dt_bias), _ptr(conv_state), _ptr(state), _ptr(out),
+                                            _stream(stream)))
+    return out
 
 
 def gdn_state_select(step_states, accept, state, *, stream=None):

@@ -302,6 +302,31 @@ gdn_status gdn_prerule(const gdn_desc *d, const void *x, const void *a, const vo
                        gdn_stream_t stream);
 
 /* Static description of a status code. */
+/* -------------------------------------------------------------------------
+ * gdn_decode_step_prerule -- one decode step from the layer's raw projections:
+ * for every sequence's new token, the work of gdn_prerule (short causal
+ * convolution with the sequence's history, SiLU, length-1 q and k, beta =
+ * sigmoid(b), g = -exp(A_log) softplus(a + dt_bias); "Attention, Part 4: Linear
+ * Attention, Gated DeltaNet and Hybrid Models", section 6) and then the step of
+ * gdn_decode_step ("From Traditional Attention to hybrid ones", section 5), in
+ * one kernel: q, k, v, g and beta stay in registers (fp32).  The convolution
+ * history is then shifted by a second small kernel (so it is updated in place).
+ *
+ *   d          B sequences, T == 1, H (value heads), hk, d_k, d_v, dtype, scale;
+ *              gate must be GDN_GATE_HEAD
+ *   x          (B, 2 hk d_k + H d_v) raw mixed projection in d->dtype
+ *   a, b       (B, H) in d->dtype;  conv_w (2 hk d_k + H d_v, K) fp32, K in 1 .. 4
+ *   A_log, dt_bias (H) fp32
+ *   conv_state (B, 2 hk d_k + H d_v, K-1) fp32, the last K-1 raw inputs (oldest
+ *              first), updated in place; NULL: zero history, none kept
+ *   state      (B, H, d_v, d_k) fp32, updated in place; out (B, H, d_v) in d->dtype
+ * state and out 16-byte aligned; outputs must not overlap the inputs or each
+ * other.  Errors as gdn_decode_step.
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_decode_step_prerule(const gdn_desc *d, const void *x, const void *a, const void *b,
+                                   const float *conv_w, int32_t K, const float *A_log, const float *dt_bias,
+                                   float *conv_state, float *state, void *out, gdn_stream_t stream);
+
 const char *gdn_status_string(gdn_status s);
 
 /* One-line reason for the most recent failed call on this thread ("" if none). */

@@ -255,6 +255,32 @@ def test_prerule_validation(lib):
     assert _prerule(lib, d, q) in (gdn.GDN_OK, gdn.GDN_ERR_CUDA)
 
 
+def test_fused_decode_validation(lib):
+    """gdn_decode_step_prerule: T == 1, the per-head gate, K in 1..4, required pointers,
+    alignment and overlap checks, before any launch."""
+    call = lambda d, p, K=4: lib.gdn_decode_step_prerule(ctypes.byref(d), p[0], p[1], p[2], p[3], K, p[4], p[5],
+                                                         p[6], p[7], p[8], None)
+    p = [_addr(i) for i in range(9)]
+    d = _desc(B=2, T=1, H=4, dk=64, dv=64)
+    assert call(_desc(B=2, T=2, H=4, dk=64, dv=64), p) == gdn.GDN_ERR_INVALID_ARG
+    assert call(_desc(B=2, T=1, H=4, dk=64, dv=64, gate=gdn.GDN_GATE_CHANNEL), p) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(d, p, K=0) == gdn.GDN_ERR_UNSUPPORTED and call(d, p, K=5) == gdn.GDN_ERR_UNSUPPORTED
+    for i in (0, 1, 2, 3, 4, 5, 7, 8):  # every pointer but conv_state is required
+        q = list(p)
+        q[i] = None
+        assert call(d, q) == gdn.GDN_ERR_INVALID_ARG, i
+    q = list(p)
+    q[7] = _addr(7, 8)  # state not 16-byte aligned
+    assert call(d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[8] = _addr(0, 64)  # out inside x
+    assert call(d, q) == gdn.GDN_ERR_INVALID_ARG
+    q = list(p)
+    q[6] = _addr(7, 256)  # conv_state over the state
+    assert call(d, q) == gdn.GDN_ERR_INVALID_ARG
+    assert call(_desc(B=0, T=1, H=4, dk=64, dv=64), p) == gdn.GDN_OK
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.gdn_status_string(s)

@@ -104,3 +104,72 @@ def test_layer_core_end_to_end():
     o_ref, f_ref, _ = oracle.gated_delta_rule(rep(bf(rq)), rep(bf(rk)), bf(rv), torch.from_numpy(rg).float(),
                                               torch.from_numpy(rb).float())
     assert rel_l2(out, o_ref) <= 2e-2 and rel_l2(fin, f_ref) <= 1e-2
+
+
+# ---------------------------------------------------------------------------
+# gdn_decode_step_prerule: the pre-rule work and the decode step in one kernel
+# ---------------------------------------------------------------------------
+
+def _fused_decode_case(dtype, d, K, hk, H, T=6, history=True, seed=60):
+    pi = make_prerule_inputs(B=5, T=T, H=H, hk=hk, dk=d, dv=d, K=K, dtype=dtype, history=history, seed=seed)
+    rng = np.random.default_rng(seed + 1000)
+    h0 = rng.normal(0.0, 0.02, size=(5, H, d, d)).astype(np.float32)
+    dev = lambda t: t.cuda().contiguous()
+    conv = dev(pi.hist) if pi.hist is not None else None
+    state = torch.from_numpy(h0).cuda()
+    outs = []
+    for t in range(T):
+        outs.append(gdn.gdn_decode_step_prerule(dev(pi.x[:, t]), dev(pi.a[:, t]), dev(pi.b[:, t]), dev(pi.conv_w),
+                                                dev(pi.A_log), dev(pi.dt_bias), conv, state, hk=hk, dk=d, H=H,
+                                                dv=d))
+    torch.cuda.synchronize()
+    # oracle: the pre-rule work over the T tokens, then the recurrence (q/k heads repeated
+    # for the value heads that share them)
+    rq, rk, rv, rg, rb, rhist = _oracle(pi)
+    rep = lambda z: np.repeat(z, H // hk, axis=2)
+    o_ref, f_ref, _ = oracle.gated_delta_rule(rep(rq), rep(rk), rv, rg, rb, h0)
+    return torch.stack(outs, 1), state, conv, o_ref, f_ref, rhist
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("K", [4, 2])
+@pytest.mark.parametrize("hk", [2, 4])  # shared query/key heads (history moved by a second kernel) or not
+def test_fused_decode_steps(dtype, d, K, hk):
+    out, state, conv, o_ref, f_ref, rhist = _fused_decode_case(dtype, d, K, hk=hk, H=4, seed=60 + K)
+    tol_o, tol_s = (1e-4, 1e-4) if dtype == "f32" else (2e-2, 1e-2)
+    assert rel_l2(out, o_ref) <= tol_o
+    assert rel_l2(state, f_ref) <= tol_s
+    assert np.array_equal(conv.cpu().double().numpy(), rhist)  # the history: raw inputs, copied exactly
+
+
+def test_fused_decode_without_history_and_k1():
+    # without a history every step sees zeros before its token: one step equals a
+    # one-token sequence with no history
+    out, state, conv, o_ref, f_ref, _ = _fused_decode_case("bf16", 128, 4, hk=1, H=2, T=1, history=False, seed=66)
+    assert conv is None
+    assert rel_l2(out, o_ref) <= 2e-2 and rel_l2(state, f_ref) <= 1e-2
+    out, state, conv, o_ref, f_ref, _ = _fused_decode_case("f32", 64, 1, hk=2, H=2, seed=67)  # no history kept
+    assert rel_l2(out, o_ref) <= 1e-4 and rel_l2(state, f_ref) <= 1e-4
+
+
+def test_fused_decode_equals_prerule_then_decode():
+    """The fused step and gdn_prerule followed by gdn_decode_step agree (fp32 inputs:
+    the unfused path stores q, k, v in fp32 too)."""
+    pi = make_prerule_inputs(B=4, T=1, H=4, hk=2, dk=128, dv=128, K=4, dtype="f32", seed=68)
+    rng = np.random.default_rng(69)
+    h0 = torch.from_numpy(rng.normal(0.0, 0.02, size=(4, 4, 128, 128)).astype(np.float32)).cuda()
+    dev = lambda t: t.cuda().contiguous()
+    s1, s2 = h0.clone(), h0.clone()
+    c1, c2 = dev(pi.hist), dev(pi.hist)
+    o1 = gdn.gdn_decode_step_prerule(dev(pi.x[:, 0]), dev(pi.a[:, 0]), dev(pi.b[:, 0]), dev(pi.conv_w),
+                                     dev(pi.A_log), dev(pi.dt_bias), c1, s1, hk=2, dk=128, H=4, dv=128)
+    q, k, v, g, beta = gdn.gdn_prerule(dev(pi.x), dev(pi.a), dev(pi.b), dev(pi.conv_w), dev(pi.A_log),
+                                       dev(pi.dt_bias), hk=2, dk=128, H=4, dv=128, conv_state_in=c2,
+                                       conv_state_out=c2)
+    rep = lambda z: z.repeat_interleave(2, dim=2)
+    o2 = gdn.gdn_decode_step(rep(q), rep(k), v, g, beta, s2)
+    torch.cuda.synchronize()
+    assert rel_l2(o1, o2.reshape(o1.shape).cpu().double().numpy()) <= 1e-5
+    assert rel_l2(s1, s2.cpu().double().numpy()) <= 1e-5
+    assert torch.equal(c1, c2)
