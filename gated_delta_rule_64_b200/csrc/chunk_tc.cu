@@ -598,7 +598,10 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
                     *reinterpret_cast<float4 *>(dst + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
             }
         }
-        if (__syncthreads_or(!ok)) break;
+        if (__syncthreads_or(!ok)) {  // a wait gave up: every thread leaves as failed
+            ok = false;
+            break;
+        }
     }
     if (ok && nchunks > 0 && emit) store_output(nchunks - 1);
     if (!ok && tid == 0) flag_error(err, 2);
