@@ -339,8 +339,17 @@ __device__ __forceinline__ float *split_state(const ScanSplit &sp, int64_t n, in
 }
 
 // SPLIT: launched as a pass of the split scan (the block's work then comes from `sp`).
+// Per-head gate, unsplit: kThreads + 32 threads; warps 0-7 hold the state and warp 8
+// issues the MMAs and the copies, so the state warps spend the MMA groups storing
+// the previous chunk's output.  A ninth warp puts three warps on one SM sub-partition,
+// which caps a thread at 168 registers; the per-channel and split scans need more,
+// so there warp 0 issues the MMAs and warp 4 the copies.
 template <bool KDA, bool SPLIT>
-__global__ void __launch_bounds__(kThreads, 1)
+constexpr int scan_threads() {
+    return KDA || SPLIT ? kThreads : kThreads + 32;
+}
+template <bool KDA, bool SPLIT>
+__global__ void __launch_bounds__(scan_threads<KDA, SPLIT>(), 1)
 gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T,
             int64_t rows, int64_t H, int64_t max_chunks, int64_t snap_stride, int64_t n_snap,
             const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out, float *final_state,
@@ -353,6 +362,9 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, hf = warp >> 2;
     const int v = qd * 32 + lane;  // state row; this thread holds columns [64 hf, 64 hf + 64)
+    constexpr bool WS = scan_threads<KDA, SPLIT>() > kThreads;  // a warp of its own issues the MMAs and copies
+    constexpr int kIssuer = WS ? kThreads / 32 : 0;
+    const bool holds_rows = !WS || tid < kThreads;  // this thread holds part of the state
 
     // This block's work: sequence n, chunks [cb, ce) of it, its start state and
     // where its end state goes (both D x D fp32 states of this (sequence, head)).
@@ -413,7 +425,7 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
     const uint32_t tm = tmem_base;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
 
-    constexpr int kLoader = 128;  // warp 4 lane 0 issues the copies (warp 0 issues the MMAs)
+    constexpr int kLoader = WS ? kThreads : 128;  // lane 0 of the issuing warp, else warp 4 lane 0
     auto issue_loads = [&](int64_t c) {
         const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
@@ -428,7 +440,10 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
 
     float S[64];
     const int64_t srow = (int64_t)v * D + 64 * hf;  // this thread's part of a state
-    if (start_kind == kStartGiven && s_init) {
+    if (!holds_rows) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) S[c] = 0.f;
+    } else if (start_kind == kStartGiven && s_init) {
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
             const float4 t = *reinterpret_cast<const float4 *>(s_init + srow + c);
@@ -439,9 +454,10 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
         for (int c = 0; c < 64; ++c) S[c] = (start_kind == kStartIdentity && 64 * hf + c == v) ? 1.f : 0.f;
     }
 
-    // Output of chunk c held in registers: o[t / 16][t % 16] = token 32 hf + t, channel v.
+    // Output of chunk c held in registers: o[t / 16][t % 16] = token 32 hf + t, channel v;
+    // stored in two halves (tokens 32 hf + 16 half ..), one during each MMA group.
     float o[2][16];
-    auto store_output = [&](int64_t c) {
+    auto store_output = [&](int64_t c, int half) {
         const int64_t ca = cb + c;
         const int L = (int)(len - ca * C < C ? len - ca * C : C);
         // 4 x 4 transposes among the quads of lanes (4 adjacent channels): afterwards
@@ -450,7 +466,8 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
         const int64_t tstride = H * D;
         __nv_bfloat16 *op = out + ((start + ca * C + 32 * hf + j4) * H + h) * D + (v - j4);
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
+        for (int bb = 0; bb < 4; ++bb) {
+            const int b = 4 * half + bb;
             float x0 = o[b >> 2][4 * (b & 3)], x1 = o[b >> 2][4 * (b & 3) + 1], x2 = o[b >> 2][4 * (b & 3) + 2],
                   x3 = o[b >> 2][4 * (b & 3) + 3];
             quad_transpose(x0, x1, x2, x3, lane);
@@ -470,7 +487,7 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
         const float *fac = reinterpret_cast<const float *>(rest + kRestFac);
 
         // (a) S0 -> bf16 pairs -> TMEM A operand (this thread: 32 columns of its row)
-        {
+        if (holds_rows) {
             uint32_t w[16];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -482,11 +499,18 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
         }
         ok = mbar_wait(&bars.full[stage], (uint32_t)((c / kStages) & 1)) && ok;
         tc_fence_before();
-        __syncthreads();
+        if (WS) {
+            if (__syncthreads_or(!ok)) {  // a wait gave up: every thread leaves as failed
+                ok = false;
+                break;
+            }
+        } else {
+            __syncthreads();
+        }
         tc_fence_after();
 
         // (b) D1 = S0 [W ; Qs]^T   (N = 128, K = 128): [U correction | inter-chunk output]
-        if (warp == 0) {
+        if (warp == kIssuer) {
             const uint64_t bwq = sdesc_sw128(st_u + kStWQ, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
@@ -494,10 +518,22 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
                             id_wq, kk > 0);
             mma_commit_warp(&bars.mma[0]);
         }
-        // the previous chunk's output, while these MMAs run; every MMA of chunk c-1
-        // has completed (step (e) waited for them), so its stage can take chunk c+2
-        if (c >= 1 && emit) store_output(c - 1);
+        // every MMA of chunk c-1 has completed (step (e) waited for them), so its
+        // stage can take chunk c+2
         if (tid == kLoader && c >= 1 && c + kStages - 1 < nchunks) issue_loads(c + kStages - 1);
+        if (WS && warp == kIssuer) {
+            // (d) once every row's U' is in TMEM (named barrier 1)
+            named_bar_sync(1, kThreads + 32);
+            tc_fence_after();
+            const uint64_t bkp = sdesc_sw128(st_u + kStRest + kRestKt, 8192, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(tm + kTmD2, tm + kTmAU + kk * 8, bkp + (uint64_t)((kk * 2048) >> 4), id_kp, kk > 0);
+            mma_commit_warp(&bars.mma[1]);
+            continue;
+        }
+        // the first half of the previous chunk's output, while these MMAs run
+        if (c >= 1 && emit) store_output(c - 1, 0);
 
         // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32) -> TMEM A operand
         ok = mbar_wait(&bars.mma[0], par) && ok;
@@ -530,17 +566,24 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
             tmem_wait_st();
         }
         tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        if (WS) {
+            named_bar_arrive(1, kThreads + 32);  // the issuing warp waits for these
+        } else {
+            __syncthreads();
+            tc_fence_after();
+        }
 
         // (d) D2 = U'^T [K~ | P^T]   (N = 192, K = 64 tokens): [state increment | intra-chunk output]
-        if (warp == 0) {
+        if (!WS && warp == 0) {
             const uint64_t bkp = sdesc_sw128(st_u + kStRest + kRestKt, 8192, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ts(tm + kTmD2, tm + kTmAU + kk * 8, bkp + (uint64_t)((kk * 2048) >> 4), id_kp, kk > 0);
             mma_commit_warp(&bars.mma[1]);
         }
+
+        // the second half of the previous chunk's output, while these MMAs run
+        if (c >= 1 && emit) store_output(c - 1, 1);
 
         // (e) S = gam_L S0 + increment (columns [64 hf, 64 hf + 64); per key channel
         // for KDA) and the output o = S0 Qs^T + U'^T P^T
@@ -598,14 +641,18 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
                     *reinterpret_cast<float4 *>(dst + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
             }
         }
-        if (__syncthreads_or(!ok)) {  // a wait gave up: every thread leaves as failed
+        if (!WS && __syncthreads_or(!ok)) {  // a wait gave up: every thread leaves as failed
             ok = false;
             break;
         }
     }
-    if (ok && nchunks > 0 && emit) store_output(nchunks - 1);
+    if (WS) ok = !__syncthreads_or(!ok);  // the last chunk's waits
+    if (ok && nchunks > 0 && emit && holds_rows) {
+        store_output(nchunks - 1, 0);
+        store_output(nchunks - 1, 1);
+    }
     if (!ok && tid == 0) flag_error(err, 2);
-    if (ok && s_end) {
+    if (ok && s_end && holds_rows) {
 #pragma unroll
         for (int cc = 0; cc < 64; cc += 4)
             *reinterpret_cast<float4 *>(s_end + srow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
@@ -759,21 +806,23 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         }
     }
     ScanSplit sp{1, 0, 0, nullptr};
+    const int scan_block = p.per_channel ? scan_threads<true, false>() : scan_threads<false, false>();
     if (p.split_G < 3) {
         auto kern = p.per_channel ? gdn_scan_tc<true, false> : gdn_scan_tc<false, false>;
         LaunchScope ls("gdn_scan_tc", s);
-        kern<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kScanSmem, s>>>(
+        kern<<<dim3((unsigned)a.N, (unsigned)p.H), scan_block, kScanSmem, s>>>(
             a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
         return check_launch("gdn_scan_tc");
     }
     // sequence split: pass 1, the chained start states, pass 2
+    const int split_block = p.per_channel ? scan_threads<true, true>() : scan_threads<false, true>();
     auto kern = p.per_channel ? gdn_scan_tc<true, true> : gdn_scan_tc<false, true>;
     sp = ScanSplit{p.split_G, p.split_seg, 1, reinterpret_cast<float *>(a.ws + p.off_split)};
     const int64_t per1 = 1 + 2 * (int64_t)(p.split_G - 2), per2 = p.split_G - 1;
     if (a.N * per1 > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
     {
         LaunchScope ls("gdn_scan_tc", s);
-        kern<<<dim3((unsigned)(a.N * per1), (unsigned)p.H), kThreads, kScanSmem, s>>>(
+        kern<<<dim3((unsigned)(a.N * per1), (unsigned)p.H), split_block, kScanSmem, s>>>(
             a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
             (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
     }
@@ -786,7 +835,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     sp.pass = 2;
     {
         LaunchScope ls("gdn_scan_tc", s);
-        kern<<<dim3((unsigned)(a.N * per2), (unsigned)p.H), kThreads, kScanSmem, s>>>(
+        kern<<<dim3((unsigned)(a.N * per2), (unsigned)p.H), split_block, kScanSmem, s>>>(
             a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
             (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
     }
