@@ -34,6 +34,9 @@
 //                [S0 W^T | S0 Qs^T] and, from U' = U - W S0^T, U'^T [K~ | P^T]
 //                (the state increment and the intra-chunk output).  The next
 //                chunks' blocks are prefetched (bulk copies) into three stages.
+//                A ninth warp issues the MMAs and copies (per-head gate, no
+//                sequence split), so the eight state warps store the previous
+//                chunk's output while the MMA groups run.
 //
 // All tcgen05 MMAs are M = 128 (the 128 rows of the state, or the 64 K rows
 // stacked on the 64 Q rows), so accumulator rows map 1:1 onto TMEM lanes and
