@@ -59,6 +59,26 @@ def test_packed_sequences(dtype, per_channel):
     check(make_inputs(w, lengths=lengths))
 
 
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_packed_stage_ring(per_channel):
+    # bf16 (tensor-core path): sequences of 4 to 9 chunks with ragged tails, so the
+    # scan's three operand stages wrap several times and the copy issued ahead of
+    # each chunk meets every stage, next to empty and one-token sequences
+    lengths = [257, 0, 449, 1, 320, 575, 193]
+    w = SMALL.replace(per_channel=per_channel, seed=21)
+    check(make_inputs(w, lengths=lengths))
+
+
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_zero_length_bf16_copies_initial_state(per_channel):
+    x = make_inputs(SMALL.replace(T=0, per_channel=per_channel, seed=22))
+    dx = to_dev(x)
+    out, fin, _ = gdn.gdn_chunk_fwd(dx.q, dx.k, dx.v, dx.g, dx.beta, dx.h0)
+    torch.cuda.synchronize()
+    assert out.numel() == 0
+    assert torch.equal(fin.cpu(), x.h0)
+
+
 def test_packed_equals_separate_runs():
     lengths = [70, 129, 3]
     x = make_inputs(SMALL.replace(seed=6), lengths=lengths)
