@@ -57,7 +57,7 @@ typedef struct CUstream_st *gdn_stream_t; /* same type as cudaStream_t */
 typedef enum gdn_status {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARG = 1, /* a size, pointer, alignment or flag is wrong      */
-    GDN_ERR_UNSUPPORTED = 2, /* valid request this build does not implement      */
+    GDN_ERR_UNSUPPORTED = 2, /* valid request the library does not implement     */
     GDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required       */
     GDN_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed             */
     GDN_ERR_TIMEOUT = 5,     /* reserved: a bounded device-side wait ran out     */
