@@ -75,6 +75,39 @@ __global__ void gdn_chunk_table(const int32_t *__restrict__ cu, int64_t N, int64
         __syncthreads();
     }
     if (threadIdx.x == 0) off[N] = (int32_t)running;
+
+    // The sequences by decreasing chunk count (ties by index), after the offsets: the
+    // scan's blocks start longest first, so the long sequences do not end up in a
+    // last wave.  Bitonic sort of (count, ~index) keys in shared memory, for up to
+    // 2 x blockDim.x sequences; larger batches keep their own order.
+    __shared__ uint64_t key[2048];
+    int32_t *order = off + N + 1;
+    const int64_t P2 = N <= 1 ? 1 : (int64_t)1 << (64 - __clzll((unsigned long long)(N - 1)));
+    if (N > 2 * (int64_t)blockDim.x || P2 > 2048) {
+        for (int64_t i = threadIdx.x; i < N; i += blockDim.x) order[i] = (int32_t)i;
+        return;
+    }
+    __syncthreads();  // off[] complete
+    for (int64_t i = threadIdx.x; i < P2; i += blockDim.x)
+        key[i] = i < N ? ((uint64_t)(uint32_t)(off[i + 1] - off[i]) << 32) | (uint32_t)~(uint32_t)i : 0ull;
+    __syncthreads();
+    for (int64_t k = 2; k <= P2; k <<= 1) {
+        for (int64_t j = k >> 1; j > 0; j >>= 1) {
+            for (int64_t i = threadIdx.x; i < P2; i += blockDim.x) {
+                const int64_t ij = i ^ j;
+                if (ij > i) {
+                    const uint64_t a = key[i], b = key[ij];
+                    const bool down = (i & k) == 0;  // this run sorts in decreasing order
+                    if (down ? a < b : a > b) {
+                        key[i] = b;
+                        key[ij] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int64_t i = threadIdx.x; i < N; i += blockDim.x) order[i] = (int32_t)~(uint32_t)(key[i] & 0xffffffffu);
 }
 
 template <typename Tin, int DK, int DV, bool PC>

@@ -361,7 +361,16 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
     uint8_t *sm = align1024(smem_raw);
     __shared__ ScanBars bars;
     __shared__ uint32_t tmem_base;
-    const int64_t h = blockIdx.y;
+    // Packed batches: blocks in launch order take the sequences longest first (the
+    // order the chunk table wrote after the chunk offsets), all heads of one
+    // sequence after another, so the long sequences start in the first wave.
+    int64_t n = blockIdx.x;
+    int h = (int)blockIdx.y;
+    if (!SPLIT && cu) {
+        const int id = (int)(blockIdx.y * gridDim.x + blockIdx.x);  // < N H, checked at launch
+        n = off[N + 1 + id / (int)H];
+        h = id % (int)H;
+    }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, hf = warp >> 2;
     const int v = qd * 32 + lane;  // state row; this thread holds columns [64 hf, 64 hf + 64)
@@ -372,7 +381,7 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
     // This block's work: sequence n, chunks [cb, ce) of it, its start state and
     // where its end state goes (both D x D fp32 states of this (sequence, head)).
     enum { kStartGiven, kStartZero, kStartIdentity };
-    int64_t n = blockIdx.x, g = 0;
+    int64_t g = 0;
     int start_kind = kStartGiven;
     bool emit_rt = true;
     if (SPLIT) {
@@ -811,6 +820,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     ScanSplit sp{1, 0, 0, nullptr};
     const int scan_block = p.per_channel ? scan_threads<true, false>() : scan_threads<false, false>();
     if (p.split_G < 3) {
+        if (a.N * p.H > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
         auto kern = p.per_channel ? gdn_scan_tc<true, false> : gdn_scan_tc<false, false>;
         LaunchScope ls("gdn_scan_tc", s);
         kern<<<dim3((unsigned)a.N, (unsigned)p.H), scan_block, kScanSmem, s>>>(

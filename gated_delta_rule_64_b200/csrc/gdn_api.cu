@@ -102,7 +102,7 @@ ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed) {
     const int64_t ch = p.max_chunks * p.H;
     size_t off = 0;
     p.off_chunk_offsets = off;
-    off = align_up(off + sizeof(int32_t) * (size_t)(p.N + 1), 256);
+    off = align_up(off + sizeof(int32_t) * (size_t)(2 * p.N + 1), 256);
     p.split_G = 1;
     p.split_seg = 0;
     p.off_split = 0;

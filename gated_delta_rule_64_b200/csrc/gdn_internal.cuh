@@ -44,7 +44,8 @@ struct ChunkPlan {
     int32_t split_G;     // tensor-core path, fixed-length sequences: segments per sequence (1: none)
     int32_t split_seg;   // chunks per segment
     // byte offsets into the workspace
-    size_t off_chunk_offsets;  // int32 (N+1): first global chunk index of each sequence
+    size_t off_chunk_offsets;  // int32 (N+1): first global chunk index of each sequence, then
+                               // int32 (N): the sequences by decreasing chunk count (packed batches)
     size_t off_W, off_U, off_P, off_b;
     size_t off_split;    // [N][G][3][H][d_v][d_k] fp32 segment maps and start states
     size_t total;

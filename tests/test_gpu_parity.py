@@ -79,6 +79,33 @@ def test_zero_length_bf16_copies_initial_state(per_channel):
     assert torch.equal(fin.cpu(), x.h0)
 
 
+@pytest.mark.parametrize("n_seqs", [1, 3, 8, 37, 1000, 2049])
+def test_packed_sequence_order(n_seqs):
+    # the chunk table that a packed call writes at the start of its workspace: the
+    # first global chunk of every sequence, then the sequences by decreasing chunk
+    # count (ties in index order) that the scan's blocks take in launch order;
+    # batches of more than 2048 sequences keep their own order
+    rng = np.random.default_rng(n_seqs)
+    lengths = rng.integers(0, 300, size=n_seqs)
+    lengths[rng.random(n_seqs) < 0.2] = 64 * rng.integers(0, 4)  # ties, empty sequences
+    w = Workload("order", B=1, T=0, H=1, dk=128, dv=128, dtype="bf16", h0_std=0.0, seed=n_seqs)
+    x = make_inputs(w, lengths=[int(v) for v in lengths])
+    dx = to_dev(x)
+    nbytes = gdn.gdn_chunk_workspace_size(1, int(lengths.sum()), 1, 128, 128, n_seqs)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    gdn.gdn_chunk_fwd(dx.q, dx.k, dx.v, dx.g, dx.beta, None, dx.cu_seqlens, workspace=ws)
+    torch.cuda.synchronize()
+    table = ws[: 4 * (2 * n_seqs + 1)].cpu().view(torch.int32).numpy().astype(np.int64)
+    off, order = table[: n_seqs + 1], table[n_seqs + 1:]
+    chunks = (lengths + 63) // 64
+    assert off[0] == 0 and np.array_equal(np.diff(off), chunks)
+    if n_seqs > 2048:
+        assert np.array_equal(order, np.arange(n_seqs))
+    else:
+        expect = sorted(range(n_seqs), key=lambda i: (-chunks[i], i))
+        assert np.array_equal(order, expect)
+
+
 def test_packed_equals_separate_runs():
     lengths = [70, 129, 3]
     x = make_inputs(SMALL.replace(seed=6), lengths=lengths)
