@@ -268,8 +268,17 @@ gdn_scan_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const float 
               const float *__restrict__ bg, Tin *__restrict__ out, float *final_state, float *__restrict__ snaps) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto &sm = *reinterpret_cast<ScanSmem<DK, PC> *>(smem_raw);
-    const int64_t n = blockIdx.x, h = blockIdx.y;
-    const int r0 = blockIdx.z * kScanRows;
+    // packed batches: blocks in launch order take the sequences longest first (the
+    // order the chunk table wrote after the chunk offsets)
+    int64_t n = blockIdx.x, h = blockIdx.y, zb = blockIdx.z;
+    if (cu) {
+        const int64_t per = (int64_t)gridDim.y * gridDim.z;
+        const int64_t id = blockIdx.x + (int64_t)gridDim.x * (blockIdx.y + (int64_t)gridDim.y * blockIdx.z);
+        n = off[N + 1 + id / per];
+        h = (id % per) % gridDim.y;
+        zb = (id % per) / gridDim.y;
+    }
+    const int r0 = (int)zb * kScanRows;
     const int tid = threadIdx.x;
     const int64_t state_off = ((n * H + h) * DV + r0) * (int64_t)DK;
 
