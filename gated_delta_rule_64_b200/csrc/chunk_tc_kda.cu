@@ -25,6 +25,12 @@
 //             factor is >= 1: fine as long as the block's decay is moderate
 //             (2^64 at most); otherwise the block is formed term by term from
 //             exp(b_i - b_j) on the CUDA cores.
+// Most chunks decay moderately: with m = b at row 31 and every channel's
+// b_0 - m and m - b_63 at most 2^kSpanFast, the factors E+_i = exp(b_i - m) and
+// E-_j = exp(m - b_j) stay far inside the bf16 range, exp(b_i - b_j) = E+_i E-_j,
+// and the whole of A and P is one tensor-core product [K * E+ ; Q * E+] (K * E-)^T
+// (tcgen05, M = 128, N = 64, K = 128), as in the per-head kernel; the entries above
+// the diagonal, which may overflow, are never used.  Other chunks take the blocks.
 // The triangular solve and the W / U tensor-core products are those of the
 // per-head kernel.
 #include <string.h>
@@ -56,6 +62,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // product of scaled operands: its middle factor reaches 2^kSpanMax (far inside
 // the bf16 / fp32 range).
 constexpr float kSpanMax = 64.f;
+// Largest decay on either side of row 31 (log2 units) for the one-product form.
+constexpr float kSpanFast = 60.f;
 
 // Element (token i, channel c) of the gate / b tile.
 __device__ __forceinline__ uint32_t b_off(int i, int c) {
@@ -292,6 +300,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     // largest decay inside any 16-token block decides how the diagonal blocks
     // are formed.
     bool ok = mbar_wait(&bar_g, 0);
+    bool fast = false;  // A and P as one product
     const int c_own = tid & 127, half = tid >> 7;
     {
         float vals[32];
@@ -306,7 +315,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             if (half == 0) s_tot[c_own] = vals[31];
         }
         __syncthreads();
-        bool wide = false;
+        bool wide = false, narrow = true;
         if (ok) {
             const float base = half ? s_tot[c_own] : 0.f;
 #pragma unroll
@@ -321,8 +330,17 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             fct.sp[2 * half][c_own] = ex2(r0 - e0);
             fct.sp[2 * half + 1][c_own] = ex2(e0 - e1);
             wide = (r0 - e0 > kSpanMax) || (e0 - e1 > kSpanMax);
+            // half 1: r0 = b at row 31 (= m), e1 = b at row 63
+            if (half) narrow = -r0 <= kSpanFast && r0 - e1 <= kSpanFast;
         }
         const bool any_wide = __syncthreads_or(wide);  // uniform over the block
+        fast = !__syncthreads_or(!narrow);
+        // one product: K * Gam = (K * E+) exp(m), for the pass after A and P
+        if (ok && fast && tid < D) {
+            const float em = ex2(*reinterpret_cast<const float *>(sm + kSmB + b_off(31, tid)));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) fct.rp[q][tid] = em;
+        }
         // exp(r_p - e_q) for (p, q) = (2, 0), (3, 0), (3, 1)
         if (ok && tid < D) {
             const float e0 = *reinterpret_cast<const float *>(sm + kSmB + b_off(15, tid));
@@ -354,15 +372,25 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                 unpack8(*reinterpret_cast<const uint4 *>(sm + kSmKQ + so), kf);
                 unpack8(*reinterpret_cast<const uint4 *>(sm + kSmKQ + so + 8192), qf);
                 ld_f8(sm, i, c8, bi);
-                ld_f8(sm, 16 * p + 15, c8, ee);
                 ld_f8(sm, Lm1, c8, bl);
-                if (p > 0) ld_f8(sm, 16 * p - 1, c8, rr);
-                else
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) rr[u] = 0.f;
                 float er[8];  // exp(r_p): Gam_i = L_i exp(r_p), both factors <= 1
-                *reinterpret_cast<float4 *>(er) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8);
-                *reinterpret_cast<float4 *>(er + 4) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8 + 4);
+                if (fast) {
+                    // one product: L -> E+ = exp(b - m), R -> E- = exp(m - b), Gam = E+ exp(m)
+                    ld_f8(sm, 31, c8, ee);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        rr[u] = ee[u];
+                        er[u] = ex2(ee[u]);
+                    }
+                } else {
+                    ld_f8(sm, 16 * p + 15, c8, ee);
+                    if (p > 0) ld_f8(sm, 16 * p - 1, c8, rr);
+                    else
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) rr[u] = 0.f;
+                    *reinterpret_cast<float4 *>(er) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8);
+                    *reinterpret_cast<float4 *>(er + 4) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8 + 4);
+                }
                 uint32_t xk[4], xq[4], zr[4], kt[4], qs[4];
                 const bool in = i < L;
 #pragma unroll
@@ -401,7 +429,52 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         // (p, q0, nq) per warp, one hex digit each, with the diagonal blocks (10
         // blocks) or without them (6), spread so that warps w and w + 4 (which
         // share a scheduler) hold at most 3 blocks between them.
-        if (ok) {
+        if (fast) {
+            // [K * E+ ; Q * E+] (K * E-)^T: rows 0..63 give beta_i A_ij, rows 64..127 P_ij
+            if (warp == 0 && __all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                const uint64_t da = sdesc_sw128(smem_u32(sm + kSmKQ), 16, 1024), dz = sdesc_sw128(smem_u32(sm + kSmZ), 16, 1024);
+                const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tm, da + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                dz + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id, kk > 0);
+                mma_commit_warp(&bar_mma);
+            }
+            ok = ok && mbar_wait(&bar_mma, 0);
+            tc_fence_after();
+            if (ok) {
+                // accumulator row r = qd*32 + lane, columns [32 hf, 32 hf + 32); only the
+                // entries below (A) or on and below (P) the diagonal are kept
+                const int r = qd * 32 + lane;
+                const bool is_a = r < C;
+                const int i = is_a ? r : r - C;
+                float v0[16], v1[16];
+                const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
+                tmem_ld16(taddr, v0);
+                tmem_ld16(taddr + 16, v1);
+                tmem_wait_ld();
+                const float pre = is_a ? s_beta[i] : scale;
+                float rr[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const int j = 32 * hf + t;
+                    const bool keep = i < L && (is_a ? j < i : j <= i);
+                    rr[t] = keep ? pre * (t < 16 ? v0[t] : v1[t - 16]) : 0.f;
+                }
+                if (is_a) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<float4 *>(sm + kSmA + f32_offset(i, 32 * hf + 4 * q)) =
+                            make_float4(rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
+                } else {
+                    __nv_bfloat16 *pt = reinterpret_cast<__nv_bfloat16 *>(sm + kSmP);  // P^T: element (j, i)
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) pt[img_offset(32 * hf + t, i) / 2] = __float2bfloat16_rn(rr[t]);
+                }
+            }
+            tc_fence_before();  // the W / U products later reuse these TMEM columns
+        } else if (ok) {
             if (any_wide) diag_exact_store(sm, keep, L, scale, s_beta);
             const uint32_t P = any_wide ? 0x00100233u : 0x01102233u, Q0 = any_wide ? 0x00000020u : 0x01002020u,
                            NQ = any_wide ? 0x00100212u : 0x01111222u;
@@ -471,7 +544,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm + 64, dv + ((kk * 2048) >> 4), dt + ((kk * 32) >> 4), id, kk > 0);
         mma_commit_warp(&bar_mma);
     }
-    ok = ok && mbar_wait(&bar_mma, 0);
+    ok = ok && mbar_wait(&bar_mma, fast ? 1 : 0);
     tc_fence_after();
     if (ok) {
         store_wu(tm, blk, qd, hf, lane);
