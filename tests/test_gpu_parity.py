@@ -189,6 +189,20 @@ def test_extreme_gates_per_channel(dtype):
     check(_with_gates(x, g))
 
 
+def test_per_channel_gate_strength_by_chunk():
+    """Per-channel gates whose strength changes from chunk to chunk, so one launch
+    forms A and P in every way the prep has: chunk 0 ordinary gates and chunk 3
+    g = -1.2 per token (one product; 55 of the 60 log2 units it allows), chunk 1
+    g = -1.5 (blocks: 69 units), chunk 2 g = -80 on every fourth channel (blocks
+    with the diagonal blocks term by term), chunk 4 ordinary again."""
+    x = make_inputs(SMALL.replace(T=320, H=2, per_channel=True, seed=23))
+    g = x.g.clone()
+    g[:, 64:128] = -1.5
+    g[:, 128:192, :, ::4] = -80.0
+    g[:, 192:256] = -1.2
+    check(_with_gates(x, g))
+
+
 @pytest.mark.parametrize("gate_mu", [2.0, 6.0])
 def test_strong_per_channel_gates(gate_mu):
     """Strong decays on every channel (alpha ~ e^-2 .. e^-6 per token): in-chunk
