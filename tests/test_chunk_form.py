@@ -43,3 +43,68 @@ def test_chunk_form_long_memory_gates():
     o, s = chunk_forward(q, k, v, g, beta, S0, C=64)
     assert np.max(np.abs(o - o_ref[0, :, 0])) <= 1e-12 * max(1, np.abs(o_ref).max())
     assert np.max(np.abs(s - s_ref[0, 0])) <= 1e-12 * max(1, np.abs(s_ref).max())
+
+
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_segment_end_state_is_affine_in_its_start(per_channel):
+    """The sequence split rests on this: over a run of chunks the end state is
+    S_end = S_start M + B, with B the end state from a zero start and M the end state
+    from the identity start with the writes dropped (v = 0; d_v = d_k)."""
+    d = 10
+    q, k, v, g, beta, _ = _problem(31, 230, d, d, per_channel)
+    X = np.random.default_rng(32).standard_normal((d, d))
+    _, S_x = chunk_forward(q, k, v, g, beta, X, C=64)
+    _, B = chunk_forward(q, k, v, g, beta, np.zeros((d, d)), C=64)
+    _, M = chunk_forward(q, k, np.zeros_like(v), g, beta, np.eye(d), C=64)
+    assert np.max(np.abs(S_x - (X @ M + B))) <= 1e-12 * max(1, np.abs(S_x).max())
+
+
+def test_one_group_form_of_a_chunk():
+    """Substituting U' = U - W S0^T, one product [S0 | U^T] [[-W^T K~, -W^T P^T, Qs^T],
+    [K~, P^T, 0]] gives the state increment S - gam_L S0 and the output in two parts
+    (the one-MMA-group form of a chunk, worked out as an alternative to the two groups)."""
+    C, dk, dv = 64, 12, 9
+    q, k, v, g, beta, S0 = _problem(34, C, dk, dv, False)
+    o_ref, s_ref = chunk_forward(q, k, v, g, beta, S0, C=C)
+    b = np.cumsum(g)
+    Gam = np.exp(b)
+    Kd, Ki = k * Gam[:, None], k / Gam[:, None]
+    A = np.tril(beta[:, None] * (Kd @ Ki.T), -1)
+    Tinv = np.linalg.inv(np.eye(C) + A)
+    W, U = Tinv @ (beta[:, None] * Kd), Tinv @ (beta[:, None] * v)
+    Qs = q * Gam[:, None]
+    P = np.tril(Qs @ Ki.T)
+    Kt = k * np.exp(b[-1] - b)[:, None]
+    top = np.hstack([-W.T @ Kt, -W.T @ P.T, Qs.T])           # d_k x (d_k + 2 C)
+    bottom = np.hstack([Kt, P.T, np.zeros((C, C))])         # C x (d_k + 2 C)
+    D = np.hstack([S0, U.T]) @ np.vstack([top, bottom])      # d_v x (d_k + 2 C)
+    s = Gam[-1] * S0 + D[:, :dk]
+    o = (D[:, dk:dk + C] + D[:, dk + C:]).T
+    assert np.max(np.abs(s - s_ref)) <= 1e-12 * max(1, np.abs(s_ref).max())
+    assert np.max(np.abs(o - o_ref)) <= 1e-12 * max(1, np.abs(o_ref).max())
+
+
+@pytest.mark.parametrize("L", [64, 40, 17])
+def test_per_channel_blocks_as_one_product(L):
+    """The per-channel prep forms A and P as one product when the decays are
+    moderate: with m = b at row 31 (b constant after row L - 1), E+_i = exp(b_i - m),
+    E-_j = exp(m - b_j), beta_i (K*E+)(K*E-)^T below the diagonal is A and
+    (Q*E+)(K*E-)^T on and below it is P; the entries above are dropped by selection."""
+    dk = 16
+    q, k, _, g, beta, _ = _problem(36 + L, 64, dk, 4, True, gate_mu=0.5)
+    g[L:] = 0.0
+    beta[L:] = 0.0
+    b = np.cumsum(g, axis=0)
+    dec = np.exp(b[:, None, :] - b[None, :, :])               # exp(b_i - b_j) per channel
+    A_def = np.tril(beta[:, None] * np.einsum("ic,jc,ijc->ij", k, k, dec), -1)
+    P_def = np.tril(np.einsum("ic,jc,ijc->ij", q, k, dec))
+    m = b[31]
+    Ep, Em = np.exp(b - m), np.exp(m - b)
+    full_a = beta[:, None] * ((k * Ep) @ (k * Em).T)
+    full_p = (q * Ep) @ (k * Em).T
+    i, j = np.indices((64, 64))
+    A = np.where((j < i) & (i < L), full_a, 0.0)
+    P = np.where((j <= i) & (i < L), full_p, 0.0)
+    P_def[L:] = 0.0
+    assert np.max(np.abs(A - A_def)) <= 1e-12 * max(1, np.abs(A_def).max())
+    assert np.max(np.abs(P - P_def)) <= 1e-12 * max(1, np.abs(P_def).max())
