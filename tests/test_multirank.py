@@ -7,7 +7,6 @@ per-rank batches."""
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
