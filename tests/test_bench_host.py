@@ -1,0 +1,73 @@
+"""Host logic of bench.py (CPU): the recorded ncu traffic of a kernel is reported
+only while the kernel's source text and the files it depends on are unchanged."""
+import hashlib
+import importlib.util
+import json
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+KERNEL = """// a comment
+template <int N>
+__global__ void __launch_bounds__(128) my_kernel(float *x) {
+    x[threadIdx.x] = N;
+}
+
+__global__ void other(float *x) { x[0] = 1.f; }
+"""
+
+
+def _tree(tmp_path, kernel_src, dep_text):
+    (tmp_path / "profiles").mkdir(exist_ok=True)
+    (tmp_path / "k.cu").write_text(kernel_src)
+    (tmp_path / "dep.cuh").write_text(dep_text)
+    return tmp_path
+
+
+def test_traffic_follows_the_kernel_source(bench, tmp_path, monkeypatch):
+    root = _tree(tmp_path, KERNEL, "// helpers v1\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    sha = bench.kernel_source_hash(str(root / "k.cu"), "my_kernel")
+    assert sha is not None
+    rec = {"my_kernel": {"source": "k.cu", "sha256": sha, "bytes_per_launch": 1234.0,
+                         "deps": {"dep.cuh": hashlib.sha256(b"// helpers v1\n").hexdigest()}}}
+    (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.traffic_for("my_kernel") == 1234.0
+    assert bench.traffic_for("missing_kernel") is None
+
+    # text outside the kernel (a comment, another kernel) does not matter
+    (root / "k.cu").write_text(KERNEL.replace("// a comment", "// another comment").replace("1.f", "2.f"))
+    assert bench.traffic_for("my_kernel") == 1234.0
+    # the kernel's own text does, launch bounds included
+    (root / "k.cu").write_text(KERNEL.replace("x[threadIdx.x] = N;", "x[threadIdx.x] = 2 * N;"))
+    assert bench.traffic_for("my_kernel") is None
+    (root / "k.cu").write_text(KERNEL.replace("__launch_bounds__(128)", "__launch_bounds__(256)"))
+    assert bench.traffic_for("my_kernel") is None
+    # and so does every file the kernel's code comes from
+    (root / "k.cu").write_text(KERNEL)
+    assert bench.traffic_for("my_kernel") == 1234.0
+    (root / "dep.cuh").write_text("// helpers v2\n")
+    assert bench.traffic_for("my_kernel") is None
+
+
+def test_committed_records_name_existing_kernels(bench):
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        records = json.load(f)
+    for name, rec in records.items():
+        assert os.path.exists(os.path.join(ROOT, rec["source"])), name
+        assert bench.kernel_source_hash(os.path.join(ROOT, rec["source"]), name) is not None, name
+        assert rec["bytes_per_launch"] > 0 and rec["ncu"].startswith("ncu "), name
+        assert "--clock-control none" in rec["ncu"], name
+        for dep in rec.get("deps", {}):
+            assert os.path.exists(os.path.join(ROOT, dep)), (name, dep)
