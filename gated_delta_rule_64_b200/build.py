@@ -1,9 +1,13 @@
 """Build the C-ABI library libgdn.so (sm_100a) in-tree with nvcc.
 
-    python -m gated_delta_rule_64_b200.build [--force] [--verbose]
+    python -m gated_delta_rule_64_b200.build [--force] [--verbose] [--checked]
 
 Every ``csrc/*.cu`` file is compiled for sm_100a only and linked into
 ``gated_delta_rule_64_b200/libgdn.so``; the header is ``include/gdn.h``.
+``--checked`` builds ``libgdn_checked.so`` instead, with -DGDN_CHECKED: the
+chunked-prefill kernels then check the ranges they derive from the sizes they
+are given and report a failed check in the call's status word (for tests; the
+Python binding loads it when GDN_LIBRARY names it).
 """
 from __future__ import annotations
 
@@ -19,6 +23,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgdn.so")
+LIB_CHECKED = os.path.join(PKG, "libgdn_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2",
@@ -40,17 +45,20 @@ def deps() -> list[str]:
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "gdn.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and up_to_date():
-        return LIB
-    objdir = os.path.join(PKG, "_build")
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(lib):
+        return lib
+    if checked:
+        extra = ["-DGDN_CHECKED"] + list(extra or [])
+    objdir = os.path.join(PKG, "_build_checked" if checked else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     for src in sources():
@@ -60,13 +68,13 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main(argv=None):
@@ -74,9 +82,10 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem use per kernel")
+    ap.add_argument("--checked", action="store_true", help="build the bounds-checked libgdn_checked.so")
     a = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if a.ptxas_v else None
-    print(build(force=a.force or a.ptxas_v, verbose=a.verbose, extra=extra))
+    print(build(force=a.force or a.ptxas_v, verbose=a.verbose, extra=extra, checked=a.checked))
 
 
 if __name__ == "__main__":

@@ -8,6 +8,22 @@
 
 namespace gdn {
 
+// Bounds-checked builds (compiled with -DGDN_CHECKED): the chunked-prefill kernels
+// check the sequence, head and token range each block derives from the sizes the
+// host passed against those sizes before touching memory; a failed check records
+// GDN_DEV_BOUNDS in the call's status word and the block does nothing.  In the
+// ordinary build the checks compile away.
+#ifdef GDN_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+__device__ __forceinline__ bool in_bounds(bool cond, int *err) {
+    if (!kChecked) return true;
+    if (!cond && err) atomicCAS(err, 0, (int)GDN_DEV_BOUNDS);
+    return cond;
+}
+
 // Token range of the chunk `chunk` (global index), or false when the index is
 // past the last chunk.  Offsets from cu_seqlens are clamped into [0, rows].
 struct ChunkLoc {

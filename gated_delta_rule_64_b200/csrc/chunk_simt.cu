@@ -127,12 +127,13 @@ gdn_prep_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
               const float *__restrict__ g, const float *__restrict__ beta, const int32_t *__restrict__ cu,
               const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk,
               float scale, float *__restrict__ Wg, float *__restrict__ Ug, float *__restrict__ Pg,
-              float *__restrict__ bg) {
+              float *__restrict__ bg, int *err) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto &sm = *reinterpret_cast<PrepSmem<Tin, DK, DV, PC> *>(smem_raw);
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
     ChunkLoc loc;
     if (!locate_chunk(chunk, cu, off, N, T, rows, loc)) return;
+    if (!in_bounds(loc.start >= 0 && loc.start + loc.len <= rows && h < H && H % Hk == 0, err)) return;
     const int L = (int)loc.len;
     const int tid = threadIdx.x;
     const int64_t ch = chunk * H + h;  // chunk-head index into the workspace
@@ -265,7 +266,8 @@ gdn_scan_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const float 
               int64_t rows, int64_t H, int64_t Hk, int64_t max_chunks, float scale, int64_t snap_stride,
               int64_t n_snap,
               const float *__restrict__ Wg, const float *__restrict__ Ug, const float *__restrict__ Pg,
-              const float *__restrict__ bg, Tin *__restrict__ out, float *final_state, float *__restrict__ snaps) {
+              const float *__restrict__ bg, Tin *__restrict__ out, float *final_state, float *__restrict__ snaps,
+              int *err) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto &sm = *reinterpret_cast<ScanSmem<DK, PC> *>(smem_raw);
     // packed batches: blocks in launch order take the sequences longest first (the
@@ -280,6 +282,7 @@ gdn_scan_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const float 
     }
     const int r0 = (int)zb * kScanRows;
     const int tid = threadIdx.x;
+    if (!in_bounds(n >= 0 && n < N && h >= 0 && h < H && r0 + kScanRows <= DV, err)) return;
     const int64_t state_off = ((n * H + h) * DV + r0) * (int64_t)DK;
 
     for (int idx = tid; idx < kScanRows * DK; idx += kScanThreads)
@@ -287,6 +290,7 @@ gdn_scan_simt(const Tin *__restrict__ q, const Tin *__restrict__ k, const float 
 
     int64_t start, len;
     seq_bounds(cu, n, T, rows, start, len);
+    if (!in_bounds(start >= 0 && start + len <= rows, err)) return;
     const int64_t nchunks = (len + C - 1) / C;
     const int64_t chunk0 = cu ? (int64_t)off[n] : n * ((T + C - 1) / C);
 
@@ -384,10 +388,11 @@ gdn_status launch_typed(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s) 
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return check_launch("gdn_prep_simt attributes");
         if (p.max_chunks > 0x7fffffffLL || p.H > 65535) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
+        log_launch("gdn_prep_simt", dim3((unsigned)p.max_chunks, (unsigned)p.H), dim3(kPrepThreads), smem);
         LaunchScope ls("gdn_prep_simt", s);
         kern<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kPrepThreads, smem, s>>>(
             (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows,
-            p.H, a.Hk, a.scale, W, U, P, b);
+            p.H, a.Hk, a.scale, W, U, P, b, a.status);
     }
     st = check_launch("gdn_prep_simt");
     if (st != GDN_OK) return st;
@@ -397,10 +402,11 @@ gdn_status launch_typed(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s) 
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return check_launch("gdn_scan_simt attributes");
         if (a.N > 0x7fffffffLL || p.H > 65535) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
+        log_launch("gdn_scan_simt", dim3((unsigned)a.N, (unsigned)p.H, DV / kScanRows), dim3(kScanThreads), smem);
         LaunchScope ls("gdn_scan_simt", s);
         kern<<<dim3((unsigned)a.N, (unsigned)p.H, DV / kScanRows), kScanThreads, smem, s>>>(
             (const Tin *)a.q, (const Tin *)a.k, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, p.max_chunks,
-            a.scale, a.snapshot_stride, a.n_snap, W, U, P, b, (Tin *)a.out, a.final_state, a.snapshots);
+            a.scale, a.snapshot_stride, a.n_snap, W, U, P, b, (Tin *)a.out, a.final_state, a.snapshots, a.status);
     }
     return check_launch("gdn_scan_simt");
 }

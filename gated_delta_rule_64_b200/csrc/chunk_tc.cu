@@ -83,7 +83,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
             int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    __shared__ uint64_t bar_ld, bar_mma;
+    __shared__ uint64_t bar_ld, bar_mma, bar_drain;
     __shared__ uint32_t tmem_base;
     __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C], s_w[C];
     __shared__ __align__(16) float s_b2[C];  // b in log2 units
@@ -91,6 +91,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
     ChunkLoc loc;
     if (!locate_chunk(chunk, cu, off, N, T, rows, loc)) return;
+    if (!in_bounds(loc.start >= 0 && loc.start + loc.len <= rows && h < H && H % Hk == 0, err)) return;
     const int L = (int)loc.len;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, hf = warp >> 2;
@@ -108,6 +109,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     if (tid == 0) {  // the tile loads first: their latency overlaps the rest of the set-up
         mbar_init(&bar_ld, 1);
         mbar_init(&bar_mma, 1);
+        mbar_init(&bar_drain, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(&bar_ld, 6 * 8192);
         const int32_t hq = (int32_t)(h / (H / Hk));  // query/key head of value head h
@@ -166,7 +168,11 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     // Qs = (scale * exp(b_i)) q_i and K~ = exp(b_L - b_j) k_j: the rows of the Q
     // and K tiles rescaled (rows >= L: zero), written to the workspace with the
     // tiles' own byte layout.
+    // The same pass sums |k_i|^2 for the decay bound: thread (row tid / 8, 16-byte
+    // chunk tid % 8) sees rows tid / 8 and 32 + tid / 8 in both channel halves.
+    bool bad = false;  // a token of the chunk outside the decay bound's range
     if (ok) {
+        float k2[2] = {0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int e = tid + kThreads * k;            // 16-byte chunk over both 8K blocks
@@ -176,6 +182,16 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
             const uint4 kv = *reinterpret_cast<const uint4 *>(sm + qb * 16384 + off);
             *reinterpret_cast<uint4 *>(blk + 8192 + qb * 16384 + off) = scale8(qv, s_sg[i]);
             *reinterpret_cast<uint4 *>(rest + kRestKt + qb * 8192 + off) = scale8(kv, s_w[i]);
+            k2[k & 1] += sum_sq8(kv);
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            float x = k2[r];
+            x += __shfl_xor_sync(0xffffffffu, x, 1);
+            x += __shfl_xor_sync(0xffffffffu, x, 2);
+            x += __shfl_xor_sync(0xffffffffu, x, 4);
+            const int i = 32 * r + (tid >> 3);
+            bad = bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * x <= kBetaK2Max));
         }
     }
     __syncthreads();  // every thread is done reading Q before A overwrites it
@@ -224,7 +240,9 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         }
     }
     tc_fence_before();
-    __syncthreads();
+    // (and a gate above 0, outside the documented range, leaves the chunk without a bound)
+    const bool any_bad = __syncthreads_or(bad || (tid < L && !(g_in <= 0.f)));
+    if (tid == 0) reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = any_bad ? kLamNone : s_b2[L - 1];
 
     // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks; warps 4-7 first copy the
     // staged P^T image to the workspace (the solve writes its region after that).
@@ -283,13 +301,21 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     // Epilogue 2: thread row r is channel r of W^T and U^T, tokens [32 hf, 32 hf + 32).
     // W goes out as a K-major operand image (rows = tokens, two 64-channel
     // blocks), U^T as 128-byte-swizzled rows (row = channel).
-    if (ok) {
-        store_wu(tm, blk, qd, hf, lane);
-    } else if (tid == 0) {
-        flag_error(err, 1);
-    }
+    if (ok) store_wu(tm, blk, qd, hf, lane);
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(!ok)) {
+        // A wait gave up: record it, then wait (bounded) for the tile copies and for
+        // every MMA issued before the TMEM columns are freed.
+        if (tid == 0) {
+            flag_error(err, GDN_DEV_TIMEOUT_PREP);
+            mbar_wait(&bar_ld, 0);
+        }
+        if (warp == 0) {
+            mma_commit_warp(&bar_drain);
+            mbar_wait(&bar_drain, 0);
+        }
+        __syncthreads();
+    }
     if (warp == 0) tmem_dealloc(tm, 128);
 }
 
@@ -318,49 +344,69 @@ constexpr uint32_t kTmD1 = 0, kTmD2 = 128, kTmAS = 320, kTmAU = 384;
 struct ScanBars {
     uint64_t full[kStages];
     uint64_t mma[2];
+    uint64_t drain;  // after a failed wait: every MMA issued has completed
 };
 
 // KDA: per-channel gate (the carried state is then scaled per key channel by
 // exp(b_L) instead of one factor).
-// Sequence split of long fixed-length sequences (G >= 3 segments of `seg` chunks).
+// Sequence split of long fixed-length sequences (G >= 2 segments of `seg` chunks).
 // A segment's end state is an affine function of its start state,
-// S_end = S_start M_g + B_g.  Pass 1 runs, in parallel, segment 0 from the true
-// initial state (outputs included) and every middle segment twice: from zero
-// (giving B_g) and from the identity with the writes U dropped (giving M_g; the
-// state has d_k rows then, which needs d_v = d_k).  gdn_seg_combine chains the
-// maps into the start state of every segment; pass 2 runs segments 1 .. G-1 from
-// those, with outputs, snapshots and the final state.
+// S_end = S_start M_g + B_g, and the weight of S_start in whatever the segment
+// computes after its first m chunks is at most 2^(lam_0 + .. + lam_{m-1}) times
+// |S_start| (the chunks' decay bounds, kFacLam).  Pass 1 runs all segments at
+// once: segment 0 from the true initial state, every other one from a zero
+// start.  A zero-start segment writes the outputs and snapshots of the chunks
+// where that sum is below kLamDrop (there they equal the true ones to fp32
+// precision), its end state B_g, and m_g: the chunks before that point, or all
+// of them when the sum never gets there.  Only in that last case does the start
+// state reach the segment's end, and only then is the transition M_g formed,
+// from the identity with the writes dropped (the state then has d_k rows, which
+// needs d_v = d_k); those blocks come after all others in the grid and leave at
+// once when M_g is not needed.  gdn_seg_combine chains the start states,
+// S_{g+1} = S_g M_g + B_g (B_g where M_g was not needed), and pass 2 reruns the
+// first m_g chunks of every segment g >= 1 from its true start state.  With gates
+// that forget within a few chunks (every workload here) pass 2 is a few chunks
+// long; with gates that keep the state alive it reruns whole segments.
 struct ScanSplit {
-    int32_t G;      // segments per sequence; 1: no split
-    int32_t seg;    // chunks per segment
-    int32_t pass;   // 1 or 2 (with G >= 3)
-    float *states;  // [N][G][3][H][D][D] fp32: B_g, M_g and the start state of segment g
+    int32_t G;       // segments per sequence; 1: no split
+    int32_t seg;     // chunks per segment
+    int32_t pass;    // 1 or 2 (with G >= 2)
+    float *states;   // [N][G][3][H][D][D] fp32: B_g, M_g and the true start state S_g of segment g
+    int32_t *rec;    // [2][N][G][H] int32: m_g, and 1 where M_g was formed
 };
 __device__ __forceinline__ float *split_state(const ScanSplit &sp, int64_t n, int64_t g, int slot, int64_t H,
                                               int64_t h) {
     return sp.states + ((((n * sp.G + g) * 3 + slot) * H + h) * (int64_t)D) * D;
 }
+__device__ __forceinline__ int32_t *split_rec(const ScanSplit &sp, int which, int64_t N, int64_t n, int64_t g,
+                                              int64_t H, int64_t h) {
+    return sp.rec + ((which * N + n) * sp.G + g) * H + h;
+}
 
-// SPLIT: launched as a pass of the split scan (the block's work then comes from `sp`).
-// Per-head gate, unsplit: kThreads + 32 threads; warps 0-7 hold the state and warp 8
-// issues the MMAs and the copies, so the state warps spend the MMA groups storing
-// the previous chunk's output.  A ninth warp puts three warps on one SM sub-partition,
-// which caps a thread at 168 registers; the per-channel and split scans need more,
-// so there warp 0 issues the MMAs and warp 4 the copies.
+// SPLIT: launched as a pass of the split scan (1-D grid; the block's work comes from `sp`).
+// Per-head gate: kThreads + 32 threads; warps 0-7 hold the state and warp 8 issues
+// the MMAs and the copies, so the state warps spend the MMA groups storing the
+// previous chunk's output.  A ninth warp puts three warps on one SM sub-partition,
+// which caps a thread at 168 registers (gdn_scan_tc).  The per-channel scan needs
+// more, so there warp 0 issues the MMAs and warp 4 the copies (gdn_scan_kda_tc).
 template <bool KDA, bool SPLIT>
 constexpr int scan_threads() {
-    return KDA || SPLIT ? kThreads : kThreads + 32;
+    return KDA ? kThreads : kThreads + 32;
 }
+#define GDN_SCAN_PARAMS                                                                                              \
+    const float *h0, const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T,          \
+        int64_t rows, int64_t H, int64_t max_chunks, int64_t snap_stride, int64_t n_snap,                            \
+        const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out, float *final_state,                     \
+        float *__restrict__ snaps, const ScanSplit sp, int *err
+#define GDN_SCAN_ARGS h0, cu, off, N, T, rows, H, max_chunks, snap_stride, n_snap, blocks, out, final_state, snaps, sp, err
+
 template <bool KDA, bool SPLIT>
-__global__ void __launch_bounds__(scan_threads<KDA, SPLIT>(), 1)
-gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T,
-            int64_t rows, int64_t H, int64_t max_chunks, int64_t snap_stride, int64_t n_snap,
-            const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out, float *final_state,
-            float *__restrict__ snaps, const ScanSplit sp, int *err) {
+__device__ __forceinline__ void scan_body(GDN_SCAN_PARAMS) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     __shared__ ScanBars bars;
     __shared__ uint32_t tmem_base;
+    __shared__ float s_red[scan_threads<KDA, SPLIT>() / 32];
     // Packed batches: blocks in launch order take the sequences longest first (the
     // order the chunk table wrote after the chunk offsets), all heads of one
     // sequence after another, so the long sequences start in the first wave.
@@ -378,53 +424,92 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
     constexpr int kIssuer = WS ? kThreads / 32 : 0;
     const bool holds_rows = !WS || tid < kThreads;  // this thread holds part of the state
 
-    // This block's work: sequence n, chunks [cb, ce) of it, its start state and
-    // where its end state goes (both D x D fp32 states of this (sequence, head)).
+    // This block's work: sequence n, chunks [cb, cb + nchunks) of it (a segment of the
+    // split scan), its start state and where its end state goes.
     enum { kStartGiven, kStartZero, kStartIdentity };
     int64_t g = 0;
     int start_kind = kStartGiven;
-    bool emit_rt = true;
+    bool spec = false;      // zero start: outputs only where the start state no longer matters
+    bool emit_any = true;   // false: a transition map (no outputs)
     if (SPLIT) {
+        const int64_t id = blockIdx.x, nh_all = N * H;
+        int64_t nh;
         if (sp.pass == 1) {
-            const int64_t per = 1 + 2 * (sp.G - 2), i = n % per;
-            n /= per;
-            if (i > 0) {
-                g = 1 + (i - 1) / 2;
-                start_kind = ((i - 1) & 1) ? kStartIdentity : kStartZero;
-                emit_rt = false;
+            if (id < nh_all * sp.G) {
+                nh = id / sp.G;
+                g = id % sp.G;
+                if (g > 0) {
+                    start_kind = kStartZero;
+                    spec = true;
+                }
+            } else {
+                const int64_t j = id - nh_all * sp.G;
+                nh = j / (sp.G - 2);
+                g = 1 + j % (sp.G - 2);
+                start_kind = kStartIdentity;
+                emit_any = false;
             }
         } else {
-            const int64_t per = sp.G - 1;
-            g = 1 + n % per;
-            n /= per;
+            nh = id / (sp.G - 1);
+            g = 1 + id % (sp.G - 1);
         }
+        n = nh / H;
+        h = (int)(nh % H);
     }
     const int64_t sh = (n * H + h) * (int64_t)D * D;  // this (sequence, head)'s state in h0 / final_state
     const float *s_init = h0 ? h0 + sh : nullptr;     // kStartGiven: this state (nullptr: zero)
     float *s_end = final_state ? final_state + sh : nullptr;
     if (SPLIT) {
         if (sp.pass == 1)
-            s_end = g == 0 ? split_state(sp, n, 1, 2, H, h) : split_state(sp, n, g, start_kind == kStartZero ? 0 : 1, H, h);
-        else {
+            s_end = g == 0 ? split_state(sp, n, 1, 2, H, h) : split_state(sp, n, g, spec ? 0 : 1, H, h);
+        else
             s_init = split_state(sp, n, g, 2, H, h);
-            if (g != sp.G - 1) s_end = nullptr;
-        }
     }
 
     int64_t start, len;
     seq_bounds(cu, n, T, rows, start, len);
     int64_t ntot = (len + C - 1) / C;
     const int64_t chunk0 = cu ? (int64_t)off[n] : n * ((T + C - 1) / C);
+    if (!in_bounds(n >= 0 && n < N && h >= 0 && h < H && start >= 0 && start + len <= rows && chunk0 >= 0 &&
+                       (!SPLIT || (g >= 0 && g < sp.G)),
+                   err))
+        return;
     if (chunk0 + ntot > max_chunks) ntot = max_chunks > chunk0 ? max_chunks - chunk0 : 0;
     const int64_t cb = SPLIT ? g * sp.seg : 0;
     const int64_t ce = SPLIT && g < sp.G - 1 ? (cb + sp.seg < ntot ? cb + sp.seg : ntot) : ntot;
-    const int64_t nchunks = ce > cb ? ce - cb : 0;  // chunks of this block; chunk i is cb + i of the sequence
-    const bool emit = !SPLIT || emit_rt;
-    const float umul = SPLIT && start_kind == kStartIdentity ? 0.f : 1.f;
+    const int64_t nchunks = ce > cb ? ce - cb : 0;  // chunks of the segment; chunk i is cb + i of the sequence
+    int64_t nrun = nchunks;                         // chunks this block runs
+    const bool ident = SPLIT && start_kind == kStartIdentity;
+    const auto block_of = [&](int64_t c) { return blocks + (size_t)((chunk0 + cb + c) * H + h) * kTcBlock; };
+
+    if (ident) {
+        // The transition of the segment is needed only where the decay bound of the
+        // whole segment does not reach kLamDrop (a margin of 1 covers the order of
+        // the sum, which the zero-start block forms chunk by chunk).
+        float part = 0.f;
+        for (int64_t c = tid; c < nchunks; c += blockDim.x)
+            part += reinterpret_cast<const float *>(block_of(c) + kBlkRest + kRestFac)[kFacLam];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) s_red[warp] = part;
+        __syncthreads();
+        float tot = 0.f;
+        for (int w = 0; w < (int)(blockDim.x / 32); ++w) tot += s_red[w];
+        const bool need = !(tot < kLamDrop - 1.f);  // (NaN: needed)
+        if (tid == 0) *split_rec(sp, 1, N, n, g, H, h) = need ? 1 : 0;
+        if (!need) return;
+    }
+    if (SPLIT && sp.pass == 2) {
+        const int32_t m = *split_rec(sp, 0, N, n, g, H, h);
+        nrun = m < 0 ? 0 : (m < nchunks ? m : nchunks);
+        // the final state comes from here only when the whole last segment is rerun
+        s_end = (g == sp.G - 1 && nrun == nchunks && final_state) ? final_state + sh : nullptr;
+    }
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(&bars.full[i], 1);
         for (int i = 0; i < 2; ++i) mbar_init(&bars.mma[i], 1);
+        mbar_init(&bars.drain, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -438,17 +523,27 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
 
     constexpr int kLoader = WS ? kThreads : 128;  // lane 0 of the issuing warp, else warp 4 lane 0
+    int64_t issued = 0;                           // (loader) chunks whose copies are issued
     auto issue_loads = [&](int64_t c) {
         const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
-        const uint8_t *blk = blocks + (size_t)((chunk0 + cb + c) * H + h) * kTcBlock;
+        const uint8_t *blk = block_of(c);
         uint64_t *bar = &bars.full[stage];
-        mbar_arrive_expect_tx(bar, kStage);
-        bulk_load(st + kStWQ, blk, (uint32_t)kTcWQ, bar);
-        bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
+        if (ident) {  // a transition map reads W, K~ and the factors only
+            mbar_arrive_expect_tx(bar, (uint32_t)(2 * 8192 + kTcKt + kTcFac));
+            bulk_load(st + kStWQ, blk, 8192u, bar);
+            bulk_load(st + kStWQ + 16384, blk + 16384, 8192u, bar);
+            bulk_load(st + kStRest + kRestKt, blk + kBlkRest + kRestKt, (uint32_t)kTcKt, bar);
+            bulk_load(st + kStRest + kRestFac, blk + kBlkRest + kRestFac, (uint32_t)kTcFac, bar);
+        } else {
+            mbar_arrive_expect_tx(bar, kStage);
+            bulk_load(st + kStWQ, blk, (uint32_t)kTcWQ, bar);
+            bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
+        }
+        issued = c + 1;
     };
     if (tid == kLoader)
-        for (int64_t c = 0; c < kStages && c < nchunks; ++c) issue_loads(c);
+        for (int64_t c = 0; c < kStages && c < nrun; ++c) issue_loads(c);
 
     float S[64];
     const int64_t srow = (int64_t)v * D + 64 * hf;  // this thread's part of a state
@@ -463,7 +558,7 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
         }
     } else {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) S[c] = (start_kind == kStartIdentity && 64 * hf + c == v) ? 1.f : 0.f;
+        for (int c = 0; c < 64; ++c) S[c] = (ident && 64 * hf + c == v) ? 1.f : 0.f;
     }
 
     // Output of chunk c held in registers: o[t / 16][t % 16] = token 32 hf + t, channel v;
@@ -488,9 +583,14 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
         }
     };
 
-    const uint32_t id_wq = idesc_bf16(128, 128, 0, 0), id_kp = idesc_bf16(128, emit ? 192 : 128, 0, 1);
+    // Decay bound summed over the chunks run so far (zero-start segments) and the
+    // first chunk from which the start state no longer matters.
+    float lam = 0.f;
+    int64_t m_first = nchunks;
+    bool emit_prev = false;  // chunk c - 1 has an output to store
     bool ok = true;
-    for (int64_t c = 0; c < nchunks; ++c) {
+    int64_t c = 0;
+    for (; c < nrun; ++c) {
         const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
         const uint32_t st_u = smem_u32(st);
@@ -520,10 +620,17 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
             __syncthreads();
         }
         tc_fence_after();
+        // does this chunk write outputs, and its snapshot?
+        const float lam_next = lam + fac[kFacLam];
+        const bool emit = spec ? lam < kLamDrop : emit_any;
+        const bool emit_state = spec ? lam_next < kLamDrop : emit_any;
+        if (spec && emit && m_first == nchunks) m_first = c;
 
         // (b) D1 = S0 [W ; Qs]^T   (N = 128, K = 128): [U correction | inter-chunk output]
+        //     (N = 64, W only, for a chunk without outputs)
         if (warp == kIssuer) {
             const uint64_t bwq = sdesc_sw128(st_u + kStWQ, 16, 1024);
+            const uint32_t id_wq = idesc_bf16(128, emit ? 128 : 64, 0, 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
                 mma_bf16_ts(tm + kTmD1, tm + kTmAS + kk * 8, bwq + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
@@ -532,7 +639,8 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
         }
         // every MMA of chunk c-1 has completed (step (e) waited for them), so its
         // stage can take chunk c+2
-        if (tid == kLoader && c >= 1 && c + kStages - 1 < nchunks) issue_loads(c + kStages - 1);
+        if (tid == kLoader && c >= 1 && c + kStages - 1 < nrun) issue_loads(c + kStages - 1);
+        const uint32_t id_kp = idesc_bf16(128, emit ? 192 : 128, 0, 1);
         if (WS && warp == kIssuer) {
             // (d) once every row's U' is in TMEM (named barrier 1)
             named_bar_sync(1, kThreads + 32);
@@ -542,12 +650,15 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ts(tm + kTmD2, tm + kTmAU + kk * 8, bkp + (uint64_t)((kk * 2048) >> 4), id_kp, kk > 0);
             mma_commit_warp(&bars.mma[1]);
+            lam = lam_next;
+            emit_prev = emit;
             continue;
         }
         // the first half of the previous chunk's output, while these MMAs run
-        if (c >= 1 && emit) store_output(c - 1, 0);
+        if (c >= 1 && emit_prev) store_output(c - 1, 0);
 
         // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32) -> TMEM A operand
+        //     (a transition map drops the writes: U' = -S0 W^T)
         ok = mbar_wait(&bars.mma[0], par) && ok;
         tc_fence_after();
         {
@@ -559,19 +670,15 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int cq = 4 * hf + q;  // 16-byte chunk = tokens 8 cq .. 8 cq + 7
-                const uint4 u8 = *reinterpret_cast<const uint4 *>(rest + kRestU + sw128_offset(v, cq));
+                uint4 u8 = make_uint4(0u, 0u, 0u, 0u);
+                if (!ident) u8 = *reinterpret_cast<const uint4 *>(rest + kRestU + sw128_offset(v, cq));
                 const uint32_t uw32[4] = {u8.x, u8.y, u8.z, u8.w};
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
                     const float acc_lo = (q < 2 ? a0[8 * q + e] : a1[8 * (q - 2) + e]);
                     const float acc_hi = (q < 2 ? a0[8 * q + e + 1] : a1[8 * (q - 2) + e + 1]);
-                    float up0 = __low2float(u2), up1 = __high2float(u2);
-                    if (SPLIT) {
-                        up0 *= umul;
-                        up1 *= umul;
-                    }
-                    wu[4 * q + e / 2] = pack_bf16(up0 - acc_lo, up1 - acc_hi);
+                    wu[4 * q + e / 2] = pack_bf16(__low2float(u2) - acc_lo, __high2float(u2) - acc_hi);
                 }
             }
             tmem_st16u(tm + lane_off + kTmAU + 16 * hf, wu);
@@ -595,7 +702,7 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
         }
 
         // the second half of the previous chunk's output, while these MMAs run
-        if (c >= 1 && emit) store_output(c - 1, 1);
+        if (c >= 1 && emit_prev) store_output(c - 1, 1);
 
         // (e) S = gam_L S0 + increment (columns [64 hf, 64 hf + 64); per key channel
         // for KDA) and the output o = S0 Qs^T + U'^T P^T
@@ -611,9 +718,11 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
                     tmem_ld16(tm + lane_off + kTmD2 + 128 + 32 * hf + 16 * q, o2[q]);
                 }
             };
+            // (the output columns are read whether or not this chunk writes them: a
+            // value that is sometimes kept would stay live across the whole chunk)
 #pragma unroll
             for (int c0 = 0; c0 < 4; ++c0) tmem_ld16(tm + lane_off + kTmD2 + 64 * hf + 16 * c0, a[c0]);
-            if (emit && !KDA) load_output();  // (KDA: after the state update, for registers)
+            if (!KDA) load_output();  // (KDA: after the state update, for registers)
             tmem_wait_ld();
             if (KDA) {
                 const float4 *gl4 = reinterpret_cast<const float4 *>(fac + kFacGL + 64 * hf);
@@ -631,20 +740,18 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
 #pragma unroll
                     for (int t = 0; t < 16; ++t) S[16 * c0 + t] = gl * S[16 * c0 + t] + a[c0][t];
             }
-            if (emit) {
-                if (KDA) {
-                    load_output();
-                    tmem_wait_ld();
-                }
-#pragma unroll
-                for (int q = 0; q < 2; ++q)
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) o[q][t] += o2[q][t];
+            if (KDA) {
+                load_output();
+                tmem_wait_ld();
             }
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+#pragma unroll
+                for (int t = 0; t < 16; ++t) o[q][t] += o2[q][t];
         }
 
         // snapshot after n * stride tokens of the sequence
-        if (emit && snaps && snap_stride > 0 && ((cb + c + 1) * C) % snap_stride == 0 && (cb + c + 1) * C <= len) {
+        if (emit_state && snaps && snap_stride > 0 && ((cb + c + 1) * C) % snap_stride == 0 && (cb + c + 1) * C <= len) {
             const int64_t s = (cb + c + 1) * C / snap_stride - 1;
             if (s < n_snap) {
                 float *dst = snaps + (((n * n_snap + s) * H + h) * D + v) * (int64_t)D + 64 * hf;
@@ -653,36 +760,66 @@ gdn_scan_tc(const float *h0, const int32_t *__restrict__ cu, const int32_t *__re
                     *reinterpret_cast<float4 *>(dst + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
             }
         }
+        lam = lam_next;
+        emit_prev = emit;
         if (!WS && __syncthreads_or(!ok)) {  // a wait gave up: every thread leaves as failed
             ok = false;
             break;
         }
     }
     if (WS) ok = !__syncthreads_or(!ok);  // the last chunk's waits
-    if (ok && nchunks > 0 && emit && holds_rows) {
-        store_output(nchunks - 1, 0);
-        store_output(nchunks - 1, 1);
+    if (ok && nrun > 0 && emit_prev && holds_rows) {
+        store_output(nrun - 1, 0);
+        store_output(nrun - 1, 1);
     }
-    if (!ok && tid == 0) flag_error(err, 2);
-    if (ok && s_end && holds_rows) {
+    if (!ok) {
+        // A wait gave up: record it, then wait (bounded) for the copies still in
+        // flight and for every MMA issued, before the shared memory and the TMEM
+        // columns are given back.
+        if (tid == 0) flag_error(err, GDN_DEV_TIMEOUT_SCAN);
+        if (tid == kLoader)
+            for (int64_t j = c; j < issued; ++j) mbar_wait(&bars.full[j % kStages], (uint32_t)((j / kStages) & 1));
+        if (warp == kIssuer) {
+            mma_commit_warp(&bars.drain);
+            mbar_wait(&bars.drain, 0);
+        }
+    }
+    float *s_end2 = nullptr;  // a zero-start last segment whose end no longer depends on its start
+    if (SPLIT && spec) {
+        const bool exact_end = lam < kLamDrop;
+        if (ok && tid == 0) *split_rec(sp, 0, N, n, g, H, h) = (int32_t)(exact_end ? m_first : nchunks);
+        if (exact_end && g == sp.G - 1 && final_state) s_end2 = final_state + sh;
+    }
+    if (ok && holds_rows) {
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 4)
-            *reinterpret_cast<float4 *>(s_end + srow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
+        for (int k = 0; k < 2; ++k) {
+            float *dst = k ? s_end2 : s_end;
+            if (!dst) continue;
+#pragma unroll
+            for (int cc = 0; cc < 64; cc += 4)
+                *reinterpret_cast<float4 *>(dst + srow + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
+        }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
 }
 
+template <bool SPLIT>
+__global__ void __maxnreg__(168) gdn_scan_tc(GDN_SCAN_PARAMS) { scan_body<false, SPLIT>(GDN_SCAN_ARGS); }
+template <bool SPLIT>
+__global__ void __launch_bounds__(kThreads, 1) gdn_scan_kda_tc(GDN_SCAN_PARAMS) { scan_body<true, SPLIT>(GDN_SCAN_ARGS); }
+
 // Start states of the segments: S_{g+1} = S_g M_g + B_g for g = 1 .. G-2 (S_1
-// comes from pass 1), one block per (sequence, head), fp32 on the CUDA cores.
+// comes from pass 1; S_{g+1} = B_g where M_g was not formed), one block per
+// (sequence, head), fp32 on the CUDA cores.
 // Thread t computes a 4-row x 16-column tile (rows 4 (t % 32) .., columns
 // 16 (t / 32) ..), so every value loaded from shared memory feeds 4 or 16 FMAs.
 // S_g is kept transposed (column k = row of St) so the 4 row values of a k are
 // one 16-byte load.
 constexpr uint32_t kCombSmem = (uint32_t)(2 * D * D) * 4;
 
-__global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit sp, int64_t H) {
+__global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit sp, int64_t N, int64_t H) {
     extern __shared__ float4 comb_raw[];
     float *St = reinterpret_cast<float *>(comb_raw);  // S_g transposed: St[k][v]
     float *Ms = St + D * D;                             // M_g: Ms[k][c]
@@ -701,7 +838,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit s
     }
     for (int g = 1; g <= sp.G - 2; ++g) {
         const float *M = split_state(sp, n, g, 1, H, h), *B = split_state(sp, n, g, 0, H, h);
-        for (int e = tid; e < D * D / 4; e += kThreads) reinterpret_cast<float4 *>(Ms)[e] = reinterpret_cast<const float4 *>(M)[e];
+        const bool with_m = *split_rec(sp, 1, N, n, g, H, h) != 0;  // uniform over the block
+        if (with_m)
+            for (int e = tid; e < D * D / 4; e += kThreads)
+                reinterpret_cast<float4 *>(Ms)[e] = reinterpret_cast<const float4 *>(M)[e];
         float acc[4][16];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -711,17 +851,19 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit s
                 acc[i][c] = b4.x; acc[i][c + 1] = b4.y; acc[i][c + 2] = b4.z; acc[i][c + 3] = b4.w;
             }
         __syncthreads();
+        if (with_m) {
 #pragma unroll 2
-        for (int k = 0; k < D; ++k) {
-            const float4 s4 = *reinterpret_cast<const float4 *>(St + k * D + r0);
-            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-            float mv[16];
+            for (int k = 0; k < D; ++k) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(St + k * D + r0);
+                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+                float mv[16];
 #pragma unroll
-            for (int c = 0; c < 16; c += 4) *reinterpret_cast<float4 *>(mv + c) = *reinterpret_cast<const float4 *>(Ms + k * D + c0 + c);
+                for (int c = 0; c < 16; c += 4) *reinterpret_cast<float4 *>(mv + c) = *reinterpret_cast<const float4 *>(Ms + k * D + c0 + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int c = 0; c < 16; ++c) acc[i][c] = fmaf(sv[i], mv[c], acc[i][c]);
+                    for (int c = 0; c < 16; ++c) acc[i][c] = fmaf(sv[i], mv[c], acc[i][c]);
+            }
         }
         __syncthreads();  // every read of S_g and M_g is done
         float *dst = split_state(sp, n, g + 1, 2, H, h);
@@ -797,8 +939,8 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
         attr_err = cudaFuncSetAttribute(gdn_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrepSmem);
-        const void *scans[4] = {(const void *)gdn_scan_tc<false, false>, (const void *)gdn_scan_tc<false, true>,
-                                (const void *)gdn_scan_tc<true, false>, (const void *)gdn_scan_tc<true, true>};
+        const void *scans[4] = {(const void *)gdn_scan_tc<false>, (const void *)gdn_scan_tc<true>,
+                                (const void *)gdn_scan_kda_tc<false>, (const void *)gdn_scan_kda_tc<true>};
         for (const void *k : scans)
             if (attr_err == cudaSuccess)
                 attr_err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
@@ -811,64 +953,89 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         if (p.per_channel) {
             if ((st = tc::launch_prep_kda(mq, mk, mv, mg, p, a, off, blocks, s)) != GDN_OK) return st;
         } else {
+            const dim3 grid((unsigned)p.max_chunks, (unsigned)p.H);
+            log_launch("gdn_prep_tc", grid, dim3(kThreads), kPrepSmem);
             LaunchScope ls("gdn_prep_tc", s);
-            gdn_prep_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kPrepSmem, s>>>(
-                mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, nullptr);
+            gdn_prep_tc<<<grid, kThreads, kPrepSmem, s>>>(mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows,
+                                                          p.H, a.Hk, a.scale, blocks, a.status);
             if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
         }
     }
-    ScanSplit sp{1, 0, 0, nullptr};
+    ScanSplit sp{1, 0, 0, nullptr, nullptr};
     const int scan_block = p.per_channel ? scan_threads<true, false>() : scan_threads<false, false>();
-    if (p.split_G < 3) {
+    if (p.split_G < 2) {
         if (a.N * p.H > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
-        auto kern = p.per_channel ? gdn_scan_tc<true, false> : gdn_scan_tc<false, false>;
-        LaunchScope ls("gdn_scan_tc", s);
-        kern<<<dim3((unsigned)a.N, (unsigned)p.H), scan_block, kScanSmem, s>>>(
-            a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks, (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
+        auto kern = p.per_channel ? gdn_scan_kda_tc<false> : gdn_scan_tc<false>;
+        const dim3 grid((unsigned)a.N, (unsigned)p.H);
+        log_launch(p.per_channel ? "gdn_scan_kda_tc" : "gdn_scan_tc", grid, dim3(scan_block), kScanSmem);
+        LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc" : "gdn_scan_tc", s);
+        kern<<<grid, scan_block, kScanSmem, s>>>(a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks,
+                                                 a.snapshot_stride, a.n_snap, blocks, (__nv_bfloat16 *)a.out,
+                                                 a.final_state, a.snapshots, sp, a.status);
         return check_launch("gdn_scan_tc");
     }
-    // sequence split: pass 1, the chained start states, pass 2
+    // sequence split: pass 1 (every segment, then the transition maps), the chained
+    // start states (G >= 3), pass 2 (the leading chunks of segments 1 .. G-1)
     const int split_block = p.per_channel ? scan_threads<true, true>() : scan_threads<false, true>();
-    auto kern = p.per_channel ? gdn_scan_tc<true, true> : gdn_scan_tc<false, true>;
-    sp = ScanSplit{p.split_G, p.split_seg, 1, reinterpret_cast<float *>(a.ws + p.off_split)};
-    const int64_t per1 = 1 + 2 * (int64_t)(p.split_G - 2), per2 = p.split_G - 1;
-    if (a.N * per1 > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
+    auto kern = p.per_channel ? gdn_scan_kda_tc<true> : gdn_scan_tc<true>;
+    float *states = reinterpret_cast<float *>(a.ws + p.off_split);
+    sp = ScanSplit{p.split_G, p.split_seg, 1, states,
+                   reinterpret_cast<int32_t *>(states + (size_t)a.N * p.split_G * 3 * p.H * p.dv * p.dk)};
+    const int64_t nh = a.N * p.H, grid1 = nh * (2 * (int64_t)p.split_G - 2), grid2 = nh * (p.split_G - 1);
+    if (grid1 > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
     {
-        LaunchScope ls("gdn_scan_tc", s);
-        kern<<<dim3((unsigned)(a.N * per1), (unsigned)p.H), split_block, kScanSmem, s>>>(
-            a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
-            (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
+        log_launch("gdn_scan_tc (pass 1)", dim3((unsigned)grid1), dim3(split_block), kScanSmem);
+        LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 1)" : "gdn_scan_tc (pass 1)", s);
+        kern<<<(unsigned)grid1, split_block, kScanSmem, s>>>(a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H,
+                                                             p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+                                                             (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp,
+                                                             a.status);
     }
     if ((st = check_launch("gdn_scan_tc")) != GDN_OK) return st;
-    {
+    if (p.split_G >= 3) {
+        const dim3 grid((unsigned)a.N, (unsigned)p.H);
+        log_launch("gdn_seg_combine", grid, dim3(kThreads), kCombSmem);
         LaunchScope ls("gdn_seg_combine", s);
-        gdn_seg_combine<<<dim3((unsigned)a.N, (unsigned)p.H), kThreads, kCombSmem, s>>>(sp, p.H);
+        gdn_seg_combine<<<grid, kThreads, kCombSmem, s>>>(sp, a.N, p.H);
+        if ((st = check_launch("gdn_seg_combine")) != GDN_OK) return st;
     }
-    if ((st = check_launch("gdn_seg_combine")) != GDN_OK) return st;
     sp.pass = 2;
     {
-        LaunchScope ls("gdn_scan_tc", s);
-        kern<<<dim3((unsigned)(a.N * per2), (unsigned)p.H), split_block, kScanSmem, s>>>(
-            a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H, p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
-            (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, nullptr);
+        log_launch("gdn_scan_tc (pass 2)", dim3((unsigned)grid2), dim3(split_block), kScanSmem);
+        LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 2)" : "gdn_scan_tc (pass 2)", s);
+        kern<<<(unsigned)grid2, split_block, kScanSmem, s>>>(a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H,
+                                                             p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+                                                             (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp,
+                                                             a.status);
     }
     return check_launch("gdn_scan_tc");
 }
 
 SplitChoice choose_split(int64_t N, int64_t H, int64_t nch, int sms) {
     SplitChoice best{1, (int32_t)nch};
-    if (sms <= 0 || nch < 96) return best;
-    auto waves = [sms](int64_t ctas) { return (ctas + sms - 1) / sms; };
-    // cost in chunk steps of one block; a combine step costs about 4
-    double best_cost = (double)waves(N * H) * nch;
-    for (int64_t G = 3; G <= 128; ++G) {
+    if (sms <= 0 || nch < 64) return best;
+    auto waves = [sms](int64_t ctas) { return (double)((ctas + sms - 1) / sms); };
+    // Costs in chunk steps of one block.  An extra launch costs about 4, a combine
+    // step about 4 with a transition map and 0.5 without.  With gates that forget
+    // within a few chunks pass 1 is the whole cost apart from a short pass 2
+    // (kRerun chunks, a guess); with gates that keep the state alive pass 1 also
+    // forms the transition maps and pass 2 reruns whole segments.  The split is
+    // chosen for the first case, as long as the second stays within 1.3 times the
+    // unsplit scan.
+    constexpr double kRerun = 16.0;
+    const double unsplit = waves(N * H) * (double)nch;
+    double best_cost = 0.95 * unsplit;
+    for (int64_t G = 2; G <= 128; ++G) {
         const int64_t seg = (nch + G - 1) / G;
         if (seg < 32) break;
         const int64_t Gr = (nch + seg - 1) / seg;  // no empty segments
-        if (Gr < 3) continue;
-        const double cost = (double)(waves(N * H * (1 + 2 * (Gr - 2))) + waves(N * H * (Gr - 1))) * seg + 4.0 * (Gr - 2);
-        if (cost < 0.98 * best_cost) {
-            best_cost = cost;
+        if (Gr < 2) continue;
+        const double comb = Gr >= 3 ? 4.0 : 0.0;
+        const double fast = waves(N * H * Gr) * seg + (seg < kRerun ? seg : kRerun) + 4.0 + comb + 0.5 * (Gr - 2);
+        const double slow = waves(N * H * (2 * Gr - 2)) * seg + waves(N * H * (Gr - 1)) * seg + 4.0 + comb +
+                            4.0 * (Gr - 2);
+        if (fast < best_cost && slow <= 1.3 * unsplit) {
+            best_cost = fast;
             best = SplitChoice{(int32_t)Gr, (int32_t)seg};
         }
     }

@@ -252,14 +252,15 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                 int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    __shared__ uint64_t bar_g, bar_ld, bar_v, bar_mma;
+    __shared__ uint64_t bar_g, bar_ld, bar_v, bar_mma, bar_drain;
     __shared__ uint32_t tmem_base;
-    __shared__ float s_beta[C], s_tot[D];
+    __shared__ float s_beta[C], s_tot[D], s_lam[kThreads / 32];
     __shared__ __align__(16) Factors fct;
 
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
     ChunkLoc loc;
     if (!locate_chunk(chunk, cu, off, N, T, rows, loc)) return;
+    if (!in_bounds(loc.start >= 0 && loc.start + loc.len <= rows && h < H && H % Hk == 0, err)) return;
     const int L = (int)loc.len;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, hf = warp >> 2;
@@ -273,6 +274,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         mbar_init(&bar_ld, 1);
         mbar_init(&bar_v, 1);
         mbar_init(&bar_mma, 1);
+        mbar_init(&bar_drain, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(&bar_g, 4 * 8192);
 #pragma unroll
@@ -302,6 +304,27 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     bool ok = mbar_wait(&bar_g, 0);
     bool fast = false;  // A and P as one product
     const int c_own = tid & 127, half = tid >> 7;
+    bool gate_bad = false;  // a gate above 0 (outside the documented range): no decay bound
+    {
+        // decay bound of the chunk: the sum over its tokens of the largest gate over the
+        // channels (thread: token tid / 4, channels 32 (tid % 4) ..); before the tile
+        // becomes b in place
+        float gmax = -INFINITY;
+        if (ok && (tid >> 2) < L) {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const float4 f = *reinterpret_cast<const float4 *>(sm + kSmB + (tid & 3) * 8192 + (tid >> 2) * 128 + ch * 16);
+                gmax = fmaxf(gmax, fmaxf(fmaxf(f.x, f.y), fmaxf(f.z, f.w)));
+            }
+        }
+        gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 1));
+        gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 2));
+        gate_bad = (tid >> 2) < L && !(gmax <= 0.f);
+        float lsum = ((tid & 3) == 0 && (tid >> 2) < L) ? gmax : 0.f;
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+        if (lane == 0) s_lam[warp] = lsum;
+    }
     {
         float vals[32];
         if (ok) {
@@ -351,6 +374,26 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             fct.d[2][tid] = ex2(r3 - e1);
         }
         ok = mbar_wait(&bar_ld, 0) && ok;
+        // |k_i|^2 of every token (thread: token tid / 4, channels 32 (tid % 4) ..): is its
+        // write a contraction?  Read before the factor pass rescales K in place.
+        bool bad = false;
+        {
+            float k2 = 0.f;
+            if (ok) {
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float kf[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + kSmKQ + kq_chunk(0, tid >> 2, 4 * (tid & 3) + cc)), kf);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) k2 = fmaf(kf[u], kf[u], k2);
+                }
+            }
+            k2 += __shfl_xor_sync(0xffffffffu, k2, 1);
+            k2 += __shfl_xor_sync(0xffffffffu, k2, 2);
+            const int i = tid >> 2;
+            bad = gate_bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * k2 <= kBetaK2Max));
+        }
+        const bool any_bad = __syncthreads_or(bad);
         // exact diagonal blocks need the raw tiles and b: before the factor pass
         DiagKeep keep = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
         if (any_wide) {
@@ -416,6 +459,12 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             }
             float *fac = reinterpret_cast<float *>(rest + kRestFac);
             if (tid < D) fac[kFacGL + tid] = ex2(*reinterpret_cast<const float *>(sm + kSmB + b_off(Lm1, tid)));
+            if (tid == 0) {
+                float lam = 0.f;
+#pragma unroll
+                for (int w = 0; w < kThreads / 32; ++w) lam += s_lam[w];
+                fac[kFacLam] = any_bad ? kLamNone : lam * kLog2e;
+            }
         }
         fence_async_smem();  // the b region is taken over by the V tile (TMA) below
         __syncthreads();
@@ -546,13 +595,23 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     }
     ok = ok && mbar_wait(&bar_mma, fast ? 1 : 0);
     tc_fence_after();
-    if (ok) {
-        store_wu(tm, blk, qd, hf, lane);
-    } else if (tid == 0) {
-        flag_error(err, 1);
-    }
+    if (ok) store_wu(tm, blk, qd, hf, lane);
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(!ok)) {
+        // A wait gave up: record it, then wait (bounded) for the tile copies and for
+        // every MMA issued before the TMEM columns are freed.
+        if (tid == 0) {
+            flag_error(err, GDN_DEV_TIMEOUT_PREP);
+            mbar_wait(&bar_g, 0);
+            mbar_wait(&bar_ld, 0);
+            mbar_wait(&bar_v, 0);
+        }
+        if (warp == 0) {
+            mma_commit_warp(&bar_drain);
+            mbar_wait(&bar_drain, 0);
+        }
+        __syncthreads();
+    }
     if (warp == 0) tmem_dealloc(tm, 128);
 }
 
@@ -567,9 +626,10 @@ gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const C
         attr = cudaFuncSetAttribute(gdn_prep_kda_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     });
     if (attr != cudaSuccess) return fail(GDN_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(attr));
+    log_launch("gdn_prep_kda_tc", dim3((unsigned)p.max_chunks, (unsigned)p.H), dim3(kThreads), kSmem);
     LaunchScope ls("gdn_prep_kda_tc", s);
     gdn_prep_kda_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kSmem, s>>>(
-        mq, mk, mv, mg, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, nullptr);
+        mq, mk, mv, mg, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, a.status);
     return check_launch("gdn_prep_kda_tc");
 }
 

@@ -3,6 +3,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -31,6 +32,16 @@ gdn_status check_launch(const char *what) {
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     return GDN_OK;
+}
+
+void log_launch(const char *name, dim3 grid, dim3 block, size_t smem) {
+    static const bool on = [] {
+        const char *e = getenv("GDN_LOG");
+        return e && e[0] && strcmp(e, "0") != 0;
+    }();
+    if (on)
+        fprintf(stderr, "gdn: launch %s grid (%u, %u, %u) block (%u, %u, %u) smem %zu\n", name, grid.x, grid.y, grid.z,
+                block.x, block.y, block.z, smem);
 }
 
 // ---------------------------------------------------------------------------
@@ -101,6 +112,8 @@ ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed) {
     p.tc = tc_eligible(d) && p.rows < (1LL << 31);
     const int64_t ch = p.max_chunks * p.H;
     size_t off = 0;
+    p.off_status = off;
+    off += kStatusBytes;
     p.off_chunk_offsets = off;
     off = align_up(off + sizeof(int32_t) * (size_t)(2 * p.N + 1), 256);
     p.split_G = 1;
@@ -118,11 +131,13 @@ ChunkPlan make_plan(const gdn_desc &d, int64_t num_seqs, bool packed) {
                 sms = 148;
             }
             const SplitChoice sc = choose_split(p.N, p.H, (d.T + kChunk - 1) / kChunk, sms);
-            if (sc.G >= 3) {
+            if (sc.G >= 2) {
                 p.split_G = sc.G;
                 p.split_seg = sc.seg;
                 p.off_split = off;
-                off = align_up(off + sizeof(float) * (size_t)p.N * sc.G * 3 * p.H * p.dv * p.dk, 256);
+                off = align_up(off + sizeof(float) * (size_t)p.N * sc.G * 3 * p.H * p.dv * p.dk +
+                                   sizeof(int32_t) * 2 * (size_t)p.N * sc.G * p.H,
+                               256);
             }
         }
     } else {
@@ -310,6 +325,11 @@ gdn_status gdn_chunk_fwd(const gdn_desc *d, const void *q, const void *k, const 
         return fail(GDN_ERR_WORKSPACE, "workspace has %zu bytes, need %zu", workspace_bytes, p.total);
 
     ChunkArgs a{};
+    a.status = reinterpret_cast<int *>(reinterpret_cast<char *>(workspace) + p.off_status);
+    {
+        const cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(int32_t), (cudaStream_t)stream);
+        if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "status word: %s", cudaGetErrorString(e));
+    }
     a.q = q; a.k = k; a.v = v; a.g = log_gate; a.beta = beta; a.h0 = initial_state;
     a.cu_seqlens = cu_seqlens;
     a.T = d->T;
@@ -324,6 +344,21 @@ gdn_status gdn_chunk_fwd(const gdn_desc *d, const void *q, const void *k, const 
     a.snapshots = snapshots;
     a.ws = (char *)workspace;
     return p.tc ? launch_chunk_tc(p, a, (cudaStream_t)stream) : launch_chunk_simt(p, a, d->dtype, (cudaStream_t)stream);
+}
+
+gdn_status gdn_chunk_status(const void *workspace, gdn_stream_t stream, int32_t *device_code) {
+    g_last_error[0] = 0;
+    if (!workspace || !device_code) return fail(GDN_ERR_INVALID_ARG, "workspace and device_code are required");
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    int32_t code = 0;
+    if (e == cudaSuccess) e = cudaMemcpy(&code, workspace, sizeof code, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    *device_code = code;
+    if (code == GDN_DEV_OK) return GDN_OK;
+    if (code == GDN_DEV_TIMEOUT_PREP || code == GDN_DEV_TIMEOUT_SCAN)
+        return fail(GDN_ERR_TIMEOUT, "a device-side wait gave up (%s)",
+                    code == GDN_DEV_TIMEOUT_PREP ? "chunk-local kernel" : "scan");
+    return fail(GDN_ERR_INTERNAL, "device status %d", (int)code);
 }
 
 gdn_status gdn_decode_step(const gdn_desc *d, const void *q, const void *k, const void *v,

@@ -29,6 +29,9 @@ gdn_status fail(gdn_status st, const char *fmt, ...);
 // Map the result of a launch to a status.
 gdn_status check_launch(const char *what);
 
+// One line per launch on stderr when GDN_LOG=1 (the grid, block and shared memory).
+void log_launch(const char *name, dim3 grid, dim3 block, size_t smem);
+
 // ---------------------------------------------------------------------------
 // Workspace of the chunked forward pass.
 // ---------------------------------------------------------------------------
@@ -44,12 +47,15 @@ struct ChunkPlan {
     int32_t split_G;     // tensor-core path, fixed-length sequences: segments per sequence (1: none)
     int32_t split_seg;   // chunks per segment
     // byte offsets into the workspace
+    size_t off_status;         // int32 device status word (kStatusBytes reserved), zeroed by every call
     size_t off_chunk_offsets;  // int32 (N+1): first global chunk index of each sequence, then
                                // int32 (N): the sequences by decreasing chunk count (packed batches)
     size_t off_W, off_U, off_P, off_b;
-    size_t off_split;    // [N][G][3][H][d_v][d_k] fp32 segment maps and start states
+    size_t off_split;    // [N][G][3][H][d_v][d_k] fp32 segment maps and start states, then the
+                         // int32 [N][G][H] segment records (see ScanSplit)
     size_t total;
 };
+constexpr size_t kStatusBytes = 256;  // the status word's slot at the start of the workspace
 
 // Segments per sequence for the split scan of N fixed-length sequences of
 // `nch` chunks on `sms` multiprocessors (G = 1: no split).
@@ -74,6 +80,7 @@ struct ChunkArgs {
     void *out;
     float *final_state, *snapshots;
     char *ws;
+    int *status;                // device status word (workspace offset off_status)
 };
 
 gdn_status launch_chunk_table(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t s);

@@ -13,7 +13,10 @@
 namespace gdn {
 namespace sm100 {
 
-constexpr uint32_t kSpinLimit = 1u << 26;  // ~ seconds of polling; only reached on a bug
+#ifndef GDN_SPIN_LIMIT
+#define GDN_SPIN_LIMIT (1u << 26)
+#endif
+constexpr uint32_t kSpinLimit = GDN_SPIN_LIMIT;  // ~ seconds of polling; only reached on a bug
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -35,10 +38,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Wait until the phase with parity `parity` has completed.  Returns false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Wait until the phase with parity `parity` has completed.  Returns false after
+// `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = kSpinLimit) {
     const uint32_t a = smem_u32(bar);
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    for (uint32_t i = 0; i < limit; ++i) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"

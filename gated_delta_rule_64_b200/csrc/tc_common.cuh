@@ -28,8 +28,22 @@ static_assert(kRestPt == kTcKt && kRestU == kRestPt + kTcPImg && kRestFac == kRe
                   kRestFac + kTcFac == kTcRest,
               "block layout");
 // Gate factors (floats): exp(b_L), at [0] for the per-head gate and per key
-// channel at [0, 128) for the per-channel gate.
-constexpr int kFacGL = 0;
+// channel at [0, 128) for the per-channel gate; at [kFacLam] a bound on how much
+// the chunk can shrink a state, in log2 units (below).
+constexpr int kFacGL = 0, kFacLam = 128;
+
+// Decay bound of a chunk.  One token maps a state S to S D_t (I - beta_t k_t k_t^T)
+// (+ a write that does not depend on S).  When 0 <= beta_t |k_t|^2 <= 2 the
+// factor (I - beta_t k_t k_t^T) has spectral norm <= 1, so the chunk shrinks the
+// part of the state that came from before it by at least prod_t max_c alpha_{t,c}:
+// lam = sum_t max_c g_{t,c} log2(e) (for one gate per head, b_L log2(e)).  A chunk
+// with a token outside that range gets kLamNone (no bound).  Summed over chunks,
+// lam bounds the weight of a start state in everything computed after them; below
+// kLamDrop (2^-126, the end of the fp32 normal range, where an fp32 product of
+// the transitions flushes to zero as well) the start state no longer matters.
+constexpr float kLamNone = 1e30f;
+constexpr float kLamDrop = -126.f;
+constexpr float kBetaK2Max = 1.999f;  // beta |k|^2 bound, with room for rounding of |k|^2
 
 __device__ __forceinline__ void flag_error(int *err, int code) {
     if (err) atomicCAS(err, 0, code);
@@ -120,6 +134,19 @@ __device__ __forceinline__ uint4 scale8(const uint4 &src, float f) {
         o[w] = pack_bf16(f * __low2float(b2), f * __high2float(b2));
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Sum of the squares of eight bf16 values (one 16-byte chunk), in fp32.
+__device__ __forceinline__ float sum_sq8(const uint4 &src) {
+    const uint32_t in[4] = {src.x, src.y, src.z, src.w};
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&in[w]);
+        s = fmaf(__low2float(b2), __low2float(b2), s);
+        s = fmaf(__high2float(b2), __high2float(b2), s);
+    }
+    return s;
 }
 
 // Byte offset of the bf16 element (row, col) of a 64-column operand image with

@@ -17,16 +17,20 @@ import threading
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libgdn.so")
+# GDN_LIBRARY may name another build of the library (the bounds-checked one, for tests).
+LIB_PATH = os.environ.get("GDN_LIBRARY") or os.path.join(_PKG, "libgdn.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, \
     GDN_ERR_INTERNAL = range(7)
 GDN_F32, GDN_BF16 = 0, 1
 GDN_GATE_HEAD, GDN_GATE_CHANNEL = 0, 1
 
-EXPORTED = ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
-            "gdn_decode_multi", "gdn_state_select", "gdn_prerule", "gdn_decode_step_prerule", "gdn_status_string",
-            "gdn_last_error", "gdn_profile_enable", "gdn_profile_read")
+GDN_DEV_OK, GDN_DEV_TIMEOUT_PREP, GDN_DEV_TIMEOUT_SCAN, GDN_DEV_BOUNDS = 0, 1, 2, 16
+
+EXPORTED = ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_status", "gdn_chunk_fwd_static",
+            "gdn_chunk_status_static", "gdn_decode_step", "gdn_decode_multi", "gdn_state_select", "gdn_prerule",
+            "gdn_decode_step_prerule", "gdn_status_string", "gdn_last_error", "gdn_profile_enable",
+            "gdn_profile_read")
 
 
 class GdnDesc(ctypes.Structure):
@@ -64,6 +68,8 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_chunk_workspace_size.argtypes = [dp, i32, ctypes.POINTER(sz)]
         lib.gdn_chunk_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp, sz, vp]
         lib.gdn_chunk_fwd_static.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp]
+        lib.gdn_chunk_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
+        lib.gdn_chunk_status_static.argtypes = [vp, ctypes.POINTER(i32)]
         lib.gdn_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn_decode_multi.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
         lib.gdn_state_select.argtypes = [dp, vp, vp, vp, vp]
@@ -75,7 +81,8 @@ def load_library(path: str = LIB_PATH):
         lib.gdn_last_error.restype = ctypes.c_char_p
         lib.gdn_profile_enable.argtypes = [ctypes.c_int]
         lib.gdn_profile_read.argtypes = [ctypes.POINTER(GdnKernelTime), i32, ctypes.POINTER(i32)]
-        for name in ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_static", "gdn_decode_step",
+        for name in ("gdn_chunk_workspace_size", "gdn_chunk_fwd", "gdn_chunk_status", "gdn_chunk_status_static",
+                     "gdn_chunk_fwd_static", "gdn_decode_step",
                      "gdn_decode_multi", "gdn_state_select", "gdn_prerule", "gdn_decode_step_prerule",
                      "gdn_profile_enable", "gdn_profile_read"):
             getattr(lib, name).restype = ctypes.c_int
@@ -167,6 +174,29 @@ def gdn_chunk_fwd(q, k, v, log_gate, beta, initial_state=None, cu_seqlens=None, 
                            workspace.numel() * workspace.element_size(), _stream(stream))
     _check(lib, st)
     return out, final_state, snapshots
+
+
+def gdn_chunk_status(workspace, stream=None):
+    """Device status of the last gdn_chunk_fwd call that used `workspace` on `stream`
+    (waits for the stream): (status, device_code); status GDN_OK, GDN_ERR_TIMEOUT
+    or GDN_ERR_INTERNAL, device_code one of the GDN_DEV_* codes."""
+    lib = load_library()
+    _need_cuda(workspace)
+    code = ctypes.c_int32(-1)
+    st = lib.gdn_chunk_status(_ptr(workspace), _stream(stream), ctypes.byref(code))
+    if st == GDN_ERR_CUDA or st == GDN_ERR_INVALID_ARG:
+        _check(lib, st)
+    return st, int(code.value)
+
+
+def gdn_chunk_status_static(stream=None):
+    """gdn_chunk_status for gdn_chunk_fwd_static (its built-in scratch on the current device)."""
+    lib = load_library()
+    code = ctypes.c_int32(-1)
+    st = lib.gdn_chunk_status_static(_stream(stream), ctypes.byref(code))
+    if st == GDN_ERR_CUDA or st == GDN_ERR_INVALID_ARG:
+        _check(lib, st)
+    return st, int(code.value)
 
 
 def gdn_chunk_fwd_static(q, k, v, log_gate, beta, initial_state=None, cu_seqlens=None, *, scale=1.0,

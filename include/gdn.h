@@ -60,9 +60,25 @@ typedef enum gdn_status {
     GDN_ERR_UNSUPPORTED = 2, /* valid request the library does not implement     */
     GDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required       */
     GDN_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed             */
-    GDN_ERR_TIMEOUT = 5,     /* reserved: a bounded device-side wait ran out     */
+    GDN_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (gdn_chunk_status) */
     GDN_ERR_INTERNAL = 6     /* a device-side consistency check failed           */
 } gdn_status;
+
+/* Device status codes of the chunked prefill: the int32 at byte 0 of the
+ * workspace (or of the built-in scratch of gdn_chunk_fwd_static).  Every
+ * gdn_chunk_fwd call zeroes it on its stream before its kernels run; a kernel
+ * that gives up a bounded wait (on a tile copy or a tensor-core commit) writes
+ * its code there, waits (again bounded) for its copies and products in
+ * flight, frees its tensor memory and returns without trapping.  The first
+ * code written wins.  Read it with gdn_chunk_status. */
+typedef enum gdn_device_code {
+    GDN_DEV_OK = 0,
+    GDN_DEV_TIMEOUT_PREP = 1, /* the chunk-local kernel gave up a wait          */
+    GDN_DEV_TIMEOUT_SCAN = 2, /* the sequential scan gave up a wait             */
+    GDN_DEV_BOUNDS = 16       /* bounds-checked builds only: an index left the
+                                 range the descriptor gives (the access was
+                                 skipped)                                       */
+} gdn_device_code;
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
@@ -134,7 +150,9 @@ gdn_status gdn_chunk_workspace_size(const gdn_desc *d, int32_t num_seqs, size_t 
  *                  snapshot_stride > 0
  *   workspace      device scratch of at least gdn_chunk_workspace_size bytes,
  *                  256-byte aligned; contents on entry do not matter and are
- *                  clobbered.  Two calls in flight at once need two workspaces.
+ *                  clobbered.  Its first 4 bytes hold the call's device status
+ *                  (gdn_chunk_status).  Two calls in flight at once need two
+ *                  workspaces.
  *   stream         CUDA stream
  * ------------------------------------------------------------------------- */
 gdn_status gdn_chunk_fwd(const gdn_desc *d,
@@ -146,6 +164,20 @@ gdn_status gdn_chunk_fwd(const gdn_desc *d,
                          void *out, float *final_state, float *snapshots,
                          void *workspace, size_t workspace_bytes,
                          gdn_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * gdn_chunk_status -- the device status of the last gdn_chunk_fwd call that
+ * used `workspace` on `stream`.
+ *
+ * Waits for `stream` (cudaStreamSynchronize), then reads the int32 status
+ * word at byte 0 of the workspace (one 4-byte device-to-host copy) into
+ * *device_code (a gdn_device_code).  Returns GDN_OK when it is zero,
+ * GDN_ERR_TIMEOUT for a timeout code, GDN_ERR_INTERNAL for a bounds code, and
+ * GDN_ERR_CUDA when the wait or the copy fails.  Not for use during stream
+ * capture (it synchronises).  The outputs of a call whose status is not
+ * GDN_OK are incomplete.
+ * ------------------------------------------------------------------------- */
+gdn_status gdn_chunk_status(const void *workspace, gdn_stream_t stream, int32_t *device_code);
 
 /* ---------------------------------------------------------------------------
  * gdn_chunk_fwd_static -- gdn_chunk_fwd without a caller-provided workspace.
@@ -177,6 +209,10 @@ gdn_status gdn_chunk_fwd_static(const gdn_desc *d,
                                 int64_t snapshot_stride,
                                 void *out, float *final_state, float *snapshots,
                                 gdn_stream_t stream);
+
+/* gdn_chunk_status for gdn_chunk_fwd_static: the status word in the built-in
+ * scratch of the current device (same waits and return values). */
+gdn_status gdn_chunk_status_static(gdn_stream_t stream, int32_t *device_code);
 
 /* ---------------------------------------------------------------------------
  * gdn_decode_step -- one token of every live sequence, state updated in place.
@@ -349,6 +385,10 @@ gdn_status gdn_profile_enable(int on);
 /* Writes up to `cap` entries and stores the number of distinct kernels seen in
  * *count (which may exceed cap). */
 gdn_status gdn_profile_read(gdn_kernel_time *entries, int32_t cap, int32_t *count);
+
+/* Launch log.  With the environment variable GDN_LOG=1 (read once, at the first
+ * launch), every kernel launch of the chunked prefill prints one line to
+ * stderr: the kernel, its grid, block and dynamic shared memory. */
 
 #ifdef __cplusplus
 }

@@ -65,3 +65,13 @@ def check(x: Inputs, *, scale=1.0, snapshot_stride=0, heads=None):
             f.write(f"{os.environ.get('PYTEST_CURRENT_TEST', '?').split(' ')[0]}\t{eo:.3e}\t{ef:.3e}\t{es:.3e}\n")
     assert eo <= tol_o and ef <= tol_s and es <= tol_s, f"rel-L2 out {eo:.2e} state {ef:.2e} snaps {es:.2e}"
     return eo, ef, es
+
+
+def check_against_oracle(x: Inputs, out, fin, *, scale=1.0):
+    """Outputs and final states of a GPU call on `x` against the oracle."""
+    torch.cuda.synchronize()
+    o_ref, f_ref, _ = run_oracle(x, scale=scale)
+    tol_o, tol_s = tolerances(x.q.dtype)
+    eo, ef = rel_l2(out, o_ref), rel_l2(fin, f_ref)
+    assert eo <= tol_o and ef <= tol_s, f"rel-L2 out {eo:.2e} state {ef:.2e}"
+    return eo, ef

@@ -303,22 +303,29 @@ def test_python_binding_refuses_cpu_tensors(lib):
 
 
 def _split_policy(N, H, nch, sms=148):
-    """Segments per sequence the split scan picks (restated from the host code's
-    cost model: blocks waves x chunks per segment, plus 4 chunk steps per combine)."""
+    """Segments per sequence the split scan picks, restated from the host code's cost
+    model (chunk steps of one block): with gates that forget, waves of pass 1 x chunks
+    per segment plus a short pass 2 and the launches; chosen as long as gates that
+    keep the state alive (transition maps in pass 1, whole segments in pass 2) cost
+    at most 1.3 times the unsplit scan."""
     waves = lambda ctas: -(-ctas // sms)
-    best, best_cost = (1, nch), waves(N * H) * nch
-    if nch < 96:
+    best = (1, nch)
+    if nch < 64:
         return best
-    for G in range(3, 129):
+    unsplit = waves(N * H) * nch
+    best_cost = 0.95 * unsplit
+    for G in range(2, 129):
         seg = -(-nch // G)
         if seg < 32:
             break
         Gr = -(-nch // seg)
-        if Gr < 3:
+        if Gr < 2:
             continue
-        cost = (waves(N * H * (1 + 2 * (Gr - 2))) + waves(N * H * (Gr - 1))) * seg + 4.0 * (Gr - 2)
-        if cost < 0.98 * best_cost:
-            best, best_cost = (Gr, seg), cost
+        comb = 4.0 if Gr >= 3 else 0.0
+        fast = waves(N * H * Gr) * seg + min(seg, 16.0) + 4.0 + comb + 0.5 * (Gr - 2)
+        slow = waves(N * H * (2 * Gr - 2)) * seg + waves(N * H * (Gr - 1)) * seg + 4.0 + comb + 4.0 * (Gr - 2)
+        if fast < best_cost and slow <= 1.3 * unsplit:
+            best, best_cost = (Gr, seg), fast
     return best
 
 
@@ -332,13 +339,23 @@ def test_split_scan_workspace(lib):
         assert lib.gdn_chunk_workspace_size(ctypes.byref(d), kw.get("B", 2), ctypes.byref(n)) == gdn.GDN_OK
         return n.value
     blk = 32768 + 64 * 128 * 2 + 64 * 128 + 128 * 128 + 1024
-    # one sequence of 262144 tokens, 16 heads: 4096 chunks
+    up = lambda x: -(-x // 256) * 256
+    state = 128 * 128 * 4
+
+    def expect(N, H, nch, G):
+        # status slot, chunk table, blocks, then (split) the segment states and records
+        head = 256 + up(4 * (2 * N + 1))
+        fixed = head + N * nch * H * blk + (up(N * G * 3 * H * state + 4 * 2 * N * G * H) if G >= 2 else 0)
+        packed = head + (N * nch + N) * H * blk
+        return max(fixed, packed)
+    # one sequence of 262144 tokens, 16 heads: 4096 chunks, split so one wave holds pass 1
     G, seg = _split_policy(1, 16, 4096)
-    assert G >= 3 and (G - 1) * seg < 4096 <= G * seg
-    fixed = 256 + 4096 * 16 * blk + 1 * G * 3 * 16 * 128 * 128 * 4
-    packed = 256 + (262144 // 64 + 1) * 16 * blk
+    assert G >= 3 and (G - 1) * seg < 4096 <= G * seg and 16 * G <= 148
     got = size(B=1, T=262144, H=16)
-    assert max(fixed, packed) <= got < max(fixed, packed) + 1024
-    # the prefill workload (64 (sequence, head) pairs of 64 chunks) runs unsplit
-    assert _split_policy(4, 16, 64) == (1, 64)
-    assert size(B=4, T=4096, H=16) < 256 + (4 * 4096 // 64 + 4) * 16 * blk + 1024
+    assert expect(1, 16, 4096, G) <= got < expect(1, 16, 4096, G) + 1024
+    # the prefill workload (64 (sequence, head) pairs of 64 chunks): two segments
+    assert _split_policy(4, 16, 64) == (2, 32)
+    got = size(B=4, T=4096, H=16)
+    assert expect(4, 16, 64, 2) <= got < expect(4, 16, 64, 2) + 1024
+    # many pairs: no split
+    assert _split_policy(64, 16, 64) == (1, 64)

@@ -108,3 +108,40 @@ def test_per_channel_blocks_as_one_product(L):
     P_def[L:] = 0.0
     assert np.max(np.abs(A - A_def)) <= 1e-12 * max(1, np.abs(A_def).max())
     assert np.max(np.abs(P - P_def)) <= 1e-12 * max(1, np.abs(P_def).max())
+
+
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_decay_bound_of_a_chunk(per_channel):
+    """The split scan drops a segment's start state once the summed decay bound of the
+    chunks before falls below 2^-126.  The bound: with 0 <= beta_t |k_t|^2 <= 2 every
+    factor (I - beta_t k_t k_t^T) is a contraction, so the homogeneous map of a run
+    of tokens (the writes dropped) has spectral norm <= prod_t max_c alpha_{t,c}; the
+    kernels store log2 of that product per chunk.  Checked in fp64 on runs of 64
+    tokens with keys of length up to sqrt(2) and beta up to 1, and with beta = 1."""
+    d = 16
+    r = np.random.default_rng(33)
+    for trial in range(20):
+        q, k, v, g, beta, _ = _problem(40 + trial, 64, d, d, per_channel, gate_mu=-5.0)
+        k = k * r.uniform(0.2, np.sqrt(2.0), size=(64, 1))  # |k|^2 up to 2 with beta <= 1
+        if trial % 2:
+            beta = np.ones_like(beta)
+            k = k / np.linalg.norm(k, axis=1, keepdims=True)
+        _, M = chunk_forward(q, k, np.zeros_like(v), g, beta, np.eye(d), C=64)  # the map S0 -> S0 M
+        gmax = g if g.ndim == 1 else g.max(axis=1)
+        bound = np.exp(gmax.sum())
+        assert np.linalg.norm(M, 2) <= bound * (1 + 1e-12), (np.linalg.norm(M, 2), bound)
+
+
+def test_zero_start_outputs_after_the_bound_match():
+    """A run whose summed decay bound falls below 2^-126: from there on its outputs and
+    state from a zero start equal those from the true start to far below fp32
+    resolution (the split scan takes them from the zero-start pass)."""
+    q, k, v, g, beta, S0 = _problem(51, 640, 16, 16, False, gate_mu=1.0)  # strong decay
+    lam = np.cumsum(g) / np.log(2.0)
+    m = int(np.argmax(lam < -126.0))
+    assert 0 < m < 600
+    o_true, s_true = chunk_forward(q, k, v, g, beta, S0 * 100.0, C=64)
+    o_zero, s_zero = chunk_forward(q, k, v, g, beta, np.zeros_like(S0), C=64)
+    scale = np.abs(o_true).max()
+    assert np.max(np.abs(o_true[m + 1:] - o_zero[m + 1:])) <= 2.0 ** -100 * scale
+    assert np.max(np.abs(s_true - s_zero)) <= 2.0 ** -100 * max(1.0, np.abs(s_true).max())
