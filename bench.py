@@ -2,23 +2,31 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step is one chunked-prefill pass (gdn_chunk_fwd) over the prefill workload
-B=4, T=4096, H=16, d_k=d_v=128 (bf16 q/k/v, fp32 gates and states, chunk 64).
-`value` is prefill tokens/s over all ranks (every rank runs its own batch: weak
-scaling, no collective on the data path), timed with CUDA events around
-exactly K steps after W warm-up steps, max over ranks.  The inputs (~280 MB)
-are larger than L2, so no explicit flush is done between steps.
+One step is one chunked-prefill pass (gdn_chunk_fwd) over the long single-sequence
+workload: one sequence of T=262,144 tokens, H=16 heads, d_k=d_v=128 (bf16 q/k/v,
+fp32 gates and states, chunk 64), zero initial state, a state snapshot every 8,192
+tokens (32 of them) and the final state.  `value` is prefill tokens/s over all
+ranks (every rank runs its own sequence: weak scaling, no collective on the data
+path), timed with CUDA events around exactly K steps after W warm-up steps, max
+over ranks.  The inputs (~3.2 GB) are larger than L2, so no explicit flush is
+done between steps.
 
 The same line carries:
   e2e          the same metric with host (pinned) inputs copied in and the
-               outputs copied back inside the timed region (consecutive steps
-               pipelined over three streams: in, compute, out);
-  roofline     for the dominant kernel, from the library's own per-kernel event
-               timer in the timed region;
+               outputs (o, final state, snapshots) copied back inside the timed
+               region (consecutive steps pipelined over three streams);
+  roofline     HBM roofline of the step (algorithmic bytes over the summed
+               device time of its kernels, from the library's own per-kernel
+               event timer in the timed region), its tensor-core counterpart,
+               and per kernel its time, share and recorded DRAM traffic;
+  prefill_b4   the same for the prefill workload B=4, T=4096, H=16;
+  kda_packed   the same for the per-channel-gate workload (8 packed sequences
+               of 512..16384 tokens, H=32);
   decode       decode tokens/s on 256 sequences x 32 heads (state updated in
                place, 64 steps per pass) with its own roofline;
-  cpu_baseline the fp64 oracle on a bounded sample, on this host's cores;
-  clocks       SM clocks sampled with nvidia-smi during the timed region.
+  cpu_baseline the fp64 oracle on a bounded sample of the headline workload,
+               on this host's cores (one thread per head);
+  clocks       SM clocks sampled with nvidia-smi during the headline's timed region.
 
 --impl reference times the oracle (the CPU reference of the method) instead.
 """
@@ -154,9 +162,11 @@ def rank_seed(base: int, rank: int) -> int:
 # ---------------------------------------------------------------------------
 # Oracle (CPU baseline / reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample(tokens_per_seq: int, seed: int = 1):
-    from gated_delta_rule_64_b200.inputs import PREFILL_BF16, make_inputs
-    w = PREFILL_BF16.replace(T=tokens_per_seq, seed=seed)
+def oracle_sample(tokens_per_seq: int):
+    """The first `tokens_per_seq` tokens of the long single-sequence workload (all 16
+    heads; its zero initial state), drawn as the full workload would be."""
+    from gated_delta_rule_64_b200.inputs import LONG_SNAPSHOTS, make_inputs
+    w = LONG_SNAPSHOTS.replace(T=tokens_per_seq, snapshot_stride=0)
     return w, make_inputs(w)
 
 
@@ -167,45 +177,52 @@ def time_oracle(x, n_threads):
     return time.perf_counter() - t
 
 
-def cpu_baseline(target_s: float = 12.0):
+def oracle_threads() -> int:
+    """Threads the oracle uses on this host: one per (sequence, head) unit at most."""
     import oracle
-    cores = oracle.host_threads()
-    w, x = oracle_sample(64)
+    return max(1, min(oracle.host_threads(), 16))
+
+
+def sample_tokens(budget_s: float, cores: int) -> int:
+    """Tokens of the long sequence the oracle gets through in about `budget_s` seconds."""
+    _, x = oracle_sample(256)
+    per_tok = time_oracle(x, cores) / 256
+    return int(max(256, min(262144, budget_s / per_tok)) // 64 * 64)
+
+
+def cpu_baseline(target_s: float = 12.0):
+    cores = oracle_threads()
+    T = sample_tokens(target_s, cores)
+    _, x = oracle_sample(T)
     dt = time_oracle(x, cores)
-    per_tok = dt / (w.B * 64)
-    T = int(max(64, min(4096, (target_s / per_tok) / w.B)) // 64 * 64)
-    w, x = oracle_sample(T)
-    dt = time_oracle(x, cores)
-    tokens = w.B * T
-    return {"value": tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"prefill workload B=4 H=16 d=128 bf16, first {T} of 4096 tokens per sequence "
-                      f"({tokens} tokens x 16 heads), fp64 token loop, {dt:.1f} s"}
+    return {"value": T / dt, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+            "sample": f"long single-sequence workload (T=262144, H=16, d=128, bf16 inputs): its first {T} tokens, "
+                      f"all 16 heads, fp64 token loop, one thread per head, {dt:.1f} s"}
 
 
 def run_reference(args):
     rank, world, _ = env_rank()
     if rank != 0:
         return 0
-    import oracle
-    cores = oracle.host_threads()
+    from gated_delta_rule_64_b200.inputs import LONG_SNAPSHOTS
+    cores = oracle_threads()
     budget = 150.0
-    w, x = oracle_sample(64)
-    per_tok = time_oracle(x, cores) / (w.B * 64)
-    T = int(max(64, min(4096, budget / max(1, args.steps + args.warmup) / per_tok / w.B)) // 64 * 64)
-    w, x = oracle_sample(T)
+    T = sample_tokens(budget / max(1, args.steps + args.warmup), cores)
+    _, x = oracle_sample(T)
     for _ in range(args.warmup):
         time_oracle(x, cores)
     times = [time_oracle(x, cores) for _ in range(args.steps)]
     dt = sum(times) / len(times)
-    value = w.B * T / dt
+    value = T / dt
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "prefill B4 T4096 H16 d128 bf16 (bounded sample per step)", "global_batch": 4,
-                   "seq_len": 4096, "parallelism": "replicas only: oracle on rank 0", "sample_tokens_per_seq": T},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"first {T} tokens of each of the 4 sequences, all 16 heads, per step"},
+        "config": {"workload": LONG_SNAPSHOTS.name + " (bounded sample per step)", "global_batch": 1,
+                   "seq_len": LONG_SNAPSHOTS.T, "parallelism": "replicas only: oracle on rank 0",
+                   "sample_tokens": T},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+                         "sample": f"first {T} tokens of the sequence, all 16 heads, per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -232,13 +249,14 @@ def kernel_source_hash(path: str, name: str):
     return hashlib.sha256(text[start:end].encode()).hexdigest()
 
 
-def traffic_for(kernel: str):
-    """ncu DRAM bytes (read + write) per launch recorded in profiles/traffic.json for
-    `kernel` on the benchmark workload, or None when the kernel's source changed."""
+def traffic_for(kernel: str, workload: str):
+    """ncu DRAM bytes (read + write) per launch of `kernel` on `workload`, as recorded in
+    profiles/traffic.json ({workload: {kernel: record}}), or None when there is no
+    record or the kernel's source (or a file it depends on) changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    rec = json.load(open(p)).get(kernel)
+    rec = json.load(open(p)).get(workload, {}).get(kernel)
     if not rec:
         return None
     if kernel_source_hash(os.path.join(ROOT, rec["source"]), kernel) != rec["sha256"]:
@@ -250,152 +268,194 @@ def traffic_for(kernel: str):
     return float(rec["bytes_per_launch"])
 
 
-def run_gpu(args):
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def alg_work(x, w):
+    """Algorithmic bytes and flops of one chunked-prefill pass over inputs `x` of workload `w`:
+    q, k, v read and o written once (their dtype), the fp32 gate (per head or per key
+    channel) and beta read once, the initial state read (when given), the final state
+    and the snapshots written once; flops per head-token as in the chunkwise form."""
+    el = x.q.element_size()
+    H, dk, dv = x.v.shape[2], x.q.shape[3], x.v.shape[3]
+    N = x.n_seqs
+    n_snap = (x.q.shape[1] // w.snapshot_stride) if w.snapshot_stride else 0
+    head_tokens = x.tokens() * H
+    per_ht = (2 * dk + 2 * dv) * el + 4 * (dk if w.per_channel else 1) + 4
+    states = ((1 if x.h0 is not None else 0) + 1 + n_snap) * N * H * dv * dk * 4
+    return head_tokens * per_ht + states, head_tokens * PREFILL_FLOPS_PER_HEAD_TOKEN
+
+
+def time_chunked(w, args, rank, world, dev, pk, *, clocks=None, e2e=False):
+    """Time K chunked-prefill steps of workload `w` (every rank its own seeded batch),
+    with the library's per-kernel event timer on; optionally the end-to-end metric
+    through host buffers.  Returns (result dict, device tensors kept for nothing)."""
     import torch
     import torch.distributed as dist
 
     from gated_delta_rule_64_b200 import gdn
-    from gated_delta_rule_64_b200.inputs import DECODE, PREFILL_BF16, make_inputs
+    from gated_delta_rule_64_b200.inputs import make_inputs
 
-    rank, world, local = env_rank()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    gdn.load_library()
-    pk = peaks()
+    w = w.replace(seed=rank_seed(w.seed, rank))
+    x = make_inputs(w)
+    d = lambda t: None if t is None else t.to(dev).contiguous()
+    q, k, v, g, beta, h0, cu = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0), d(x.cu_seqlens)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = x.n_seqs
+    n_snap = T // w.snapshot_stride if w.snapshot_stride else 0
+    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    fin = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    snaps = torch.empty((N, n_snap, H, dv, dk), dtype=torch.float32, device=dev) if n_snap else None
+    ws = torch.empty(gdn.gdn_chunk_workspace_size(B, T, H, dk, dv, N, dtype=q.dtype, per_channel=w.per_channel),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(bufs=None, s=stream):
+        bq, bk, bv, bg, bb, bh0, bout, bfin, bsn, bws = bufs or (q, k, v, g, beta, h0, out, fin, snaps, ws)
+        gdn.gdn_chunk_fwd(bq, bk, bv, bg, bb, bh0, cu, snapshot_stride=w.snapshot_stride, out=bout,
+                          final_state=bfin, snapshots=bsn, workspace=bws, stream=s)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    # ---------------- prefill ----------------
-    w = PREFILL_BF16.replace(seed=rank_seed(PREFILL_BF16.seed, rank))
-    x = make_inputs(w)
-    d = lambda t: t.to(dev).contiguous()
-    q, k, v, g, beta, h0 = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
-    fin = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
-    ws = torch.empty(gdn.gdn_chunk_workspace_size(B, T, H, dk, dv, B, dtype=q.dtype), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        gdn.gdn_chunk_fwd(q, k, v, g, beta, h0, out=out, final_state=fin, workspace=ws, stream=stream)
-
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-
-    clocks = ClockSampler(local)
-    clocks.start()
+    st, code = gdn.gdn_chunk_status(ws)
+    if st != gdn.GDN_OK:
+        raise RuntimeError(f"{w.name}: device status {code}")
     gdn.profile_read()
     gdn.profile_enable(True)
     barrier()
     torch.cuda.synchronize()
-    clocks.mark_begin()
+    if clocks:
+        clocks.mark_begin()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    clocks.mark_end()
+    if clocks:
+        clocks.mark_end()
     barrier()
     gdn.profile_enable(False)
     kernels = gdn.profile_read()
-    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    ms_step = ms_total / args.steps
-    tokens_all = B * T * world
-    value = tokens_all / (ms_step * 1e-3)
+    ms_step = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    tokens = x.tokens()
+    value = tokens * world / (ms_step * 1e-3)
 
-    # Roofline of the prefill step.  The step is two kernels (chunk-local prep of
-    # every chunk in parallel, then the in-order scan); neither moves the path's
-    # algorithmic bytes on its own, so the HBM roofline is taken over both.
-    head_tokens = B * T * H
-    alg_bytes = head_tokens * PREFILL_BYTES_PER_HEAD_TOKEN + 2 * B * H * STATE_BYTES
-    alg_flops = head_tokens * PREFILL_FLOPS_PER_HEAD_TOKEN
-    per_launch = {n: t / max(1, c) * 1e-3 for n, (c, t) in kernels.items()}
-    step_kernel_s = sum(per_launch.values()) or ms_step * 1e-3
-    achieved = alg_bytes / step_kernel_s / 1e9
-    traffics = [traffic_for(n) for n in per_launch]
-    traffic = sum(traffics) if traffics and all(t is not None for t in traffics) else None
-    top_name = max(per_launch, key=per_launch.get) if per_launch else "none"
+    # Roofline of the step.  The chunked prefill is two to four kernels (chunk-local
+    # work on every chunk in parallel, then the ordered scan in one or two passes);
+    # none of them moves the path's algorithmic bytes on its own, so the HBM roofline
+    # is taken over the step: algorithmic bytes / summed kernel time.
+    alg_bytes, alg_flops = alg_work(x, w)
+    per_step = {n: t / args.steps * 1e-3 for n, (c, t) in kernels.items()}  # seconds per step, per kernel
+    launches = {n: c / args.steps for n, (c, t) in kernels.items()}
+    step_s = sum(per_step.values()) or ms_step * 1e-3
+    achieved = alg_bytes / step_s / 1e9
+    traffics = {n: traffic_for(n, w.name) for n in per_step}
+    traffic = (sum(traffics[n] * launches[n] for n in per_step)
+               if traffics and all(t is not None for t in traffics.values()) else None)
+    top = max(per_step, key=per_step.get) if per_step else "none"
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                "kernel": " + ".join(sorted(per_launch)) + " (one prefill step)",
+                "scope": "one prefill step: algorithmic bytes / summed kernel time (" + " + ".join(sorted(per_step))
+                         + ")",
                 "algorithmic_bytes": alg_bytes, "peak_source": f"{pk['source']} hbm_gbs (burst copy)",
-                "tensor": {"achieved_tflops": alg_flops / step_kernel_s / 1e12, "peak": pk["bf16_tflops"],
-                           "frac": alg_flops / step_kernel_s / 1e12 / pk["bf16_tflops"]},
-                "kernels": {n: {"us_per_launch": per_launch[n] * 1e6, "share": per_launch[n] / step_kernel_s,
-                                "traffic": traffic_for(n)} for n in per_launch},
-                "dominant_kernel": top_name}
-    launches = sum(c for c, _ in kernels.values())
+                "tensor": {"algorithmic_flops": alg_flops, "achieved_tflops": alg_flops / step_s / 1e12,
+                           "peak": pk["bf16_tflops"], "frac": alg_flops / step_s / 1e12 / pk["bf16_tflops"],
+                           "peak_source": f"{pk['source']} bf16_tflops (burst)"},
+                "kernels": {n: {"launches_per_step": launches[n], "us_per_step": per_step[n] * 1e6,
+                                "share": per_step[n] / step_s, "traffic_per_launch": traffics[n]}
+                            for n in per_step},
+                "dominant_kernel": top}
+    res = {"value": value, "unit": UNIT, "ms_per_step": ms_step, "tokens_per_step": tokens * world,
+           "config": {"workload": w.name, "sequences": N, "tokens": tokens, "heads": H, "d_k": dk, "d_v": dv,
+                      "per_channel_gate": w.per_channel, "snapshot_stride": w.snapshot_stride, "chunk": 64},
+           "roofline": roofline, "gpu_launches": sum(c for c, _ in kernels.values())}
 
-    # ---------------- e2e through the public API with host buffers ----------------
-    # Every step copies its inputs in from pinned host memory, runs gdn_chunk_fwd and
-    # copies its output and final state back.  Three streams and two device buffer
-    # sets pipeline consecutive steps: step s+1's inputs go in while step s computes
-    # and step s-1's results come out (PCIe runs both directions at once).
-    pin = lambda t: t.pin_memory()
-    hq, hk, hv, hg, hb, hh0 = pin(x.q), pin(x.k), pin(x.v), pin(x.g), pin(x.beta), pin(x.h0)
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hfin = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hh0))
-    d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
-    bufs = [(q, k, v, g, beta, h0, out, fin, ws)]
-    bufs.append(tuple(torch.empty_like(t) for t in bufs[0]))
-    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = lambda: torch.cuda.Event()
-    freed = [None, None]  # per buffer set: its last device->host copy (the set is reusable after it)
+    if e2e:
+        # Every step copies its inputs in from pinned host memory, runs gdn_chunk_fwd and
+        # copies its outputs (o, final state, snapshots) back.  Three streams and two
+        # device buffer sets pipeline consecutive steps: step s+1's inputs go in while
+        # step s computes and step s-1's results come out (PCIe runs both ways at once).
+        pin = lambda t: None if t is None else t.pin_memory()
+        hin = [pin(t) for t in (x.q, x.k, x.v, x.g, x.beta, x.h0)]
+        hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (out, fin, snaps) if t is not None]
+        h2d = sum(t.numel() * t.element_size() for t in hin if t is not None)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        sets = [(q, k, v, g, beta, h0, out, fin, snaps, ws)]
+        sets.append(tuple(None if t is None else torch.empty_like(t) for t in sets[0]))
+        s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        freed = [None, None]
 
-    def e2e_step(i):
-        bq, bk, bv, bg, bb, bh0, bout, bfin, bws = bufs[i & 1]
-        if freed[i & 1] is not None:
-            s_in.wait_event(freed[i & 1])
-        with torch.cuda.stream(s_in):
-            for src, dst in ((hq, bq), (hk, bk), (hv, bv), (hg, bg), (hb, bb), (hh0, bh0)):
-                dst.copy_(src, non_blocking=True)
-        landed = ev()
-        landed.record(s_in)
-        s_comp.wait_event(landed)
-        gdn.gdn_chunk_fwd(bq, bk, bv, bg, bb, bh0, out=bout, final_state=bfin, workspace=bws, stream=s_comp)
-        done = ev()
-        done.record(s_comp)
-        s_out.wait_event(done)
-        with torch.cuda.stream(s_out):
-            hout.copy_(bout, non_blocking=True)
-            hfin.copy_(bfin, non_blocking=True)
-        freed[i & 1] = ev()
-        freed[i & 1].record(s_out)
+        def e2e_step(i):
+            b = sets[i & 1]
+            if freed[i & 1] is not None:
+                s_in.wait_event(freed[i & 1])
+            with torch.cuda.stream(s_in):
+                for src, dst in zip(hin, b[:6]):
+                    if src is not None:
+                        dst.copy_(src, non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(s_in)
+            s_comp.wait_event(landed)
+            step(b, s_comp)
+            done = torch.cuda.Event()
+            done.record(s_comp)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                for src, dst in zip([t for t in b[6:9] if t is not None], hout):
+                    dst.copy_(src, non_blocking=True)
+            freed[i & 1] = torch.cuda.Event()
+            freed[i & 1].record(s_out)
 
-    e2e_steps = max(3, min(args.steps, 20))
-    for i in range(2):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    e1.record(s_out)  # after the last step's copies back, which follow every earlier step's work
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
-    e2e = {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
-           "pipelined": "3 streams, 2 buffer sets: step s+1 in, step s compute, step s-1 out"}
-    del q, k, v, g, beta, h0, out, fin, ws, hq, hk, hv, hg, hb, hh0, hout, hfin, bufs
+        n_e2e = max(3, min(args.steps, 10))
+        for i in range(2):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(s_in)
+        for i in range(n_e2e):
+            e2e_step(i)
+        e1.record(s_out)  # after the last step's copies back, which follow every earlier step's work
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n_e2e
+        res["e2e"] = {"value": tokens * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e,
+                      "pipelined": "3 streams, 2 buffer sets: step s+1 in, step s compute, step s-1 out"}
+        del sets, hin, hout
+    del q, k, v, g, beta, h0, cu, out, fin, snaps, ws
     torch.cuda.empty_cache()
+    return res
 
-    # ---------------- decode ----------------
+
+def time_decode(args, rank, world, dev, pk):
+    import torch
+
+    from gated_delta_rule_64_b200 import gdn
+    from gated_delta_rule_64_b200.inputs import DECODE, make_inputs
+
     wd = DECODE.replace(seed=rank_seed(DECODE.seed, rank))
     xd = make_inputs(wd)
+    d = lambda t: t.to(dev).contiguous()
     dq, dk_, dv_, dg, db = (d(t) for t in (xd.q, xd.k, xd.v, xd.g, xd.beta))
     state = d(xd.h0)
     steps_d = xd.q.shape[0]
     dout = torch.empty((steps_d,) + tuple(xd.v.shape[1:]), dtype=dq.dtype, device=dev)
+    stream = torch.cuda.current_stream()
 
     def decode_pass():
         for s in range(steps_d):
@@ -406,45 +466,78 @@ def run_gpu(args):
     passes = max(2, min(10, args.steps // 10 + 1))
     gdn.profile_read()
     gdn.profile_enable(True)
-    barrier()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(passes):
         decode_pass()
     e1.record(stream)
     torch.cuda.synchronize()
     gdn.profile_enable(False)
-    dk_times = gdn.profile_read()
+    times = gdn.profile_read()
     dms = max_over_ranks(e0.elapsed_time(e1), world, dev) / (passes * steps_d)
     nseq = xd.q.shape[1]
-    dec_units = nseq * xd.q.shape[3]
-    dname, (dl, dt_ms) = max(dk_times.items(), key=lambda kv: kv[1][1])
-    d_per_launch = dt_ms / dl * 1e-3
-    d_ach = dec_units * DECODE_BYTES_PER_UNIT / d_per_launch / 1e9
-    decode = {"metric": "decode tokens/s", "value": nseq * world / (dms * 1e-3), "unit": UNIT,
-              "ms_per_step": dms, "config": {"workload": wd.name, "sequences": nseq, "heads": xd.q.shape[3],
-                                             "state": "fp32 in HBM, updated in place"},
-              "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                           "frac": d_ach / pk["hbm_gbs"], "traffic": traffic_for(dname), "kernel": dname,
-                           "peak_source": f"{pk['source']} hbm_gbs"},
-              "gpu_launches": sum(c for c, _ in dk_times.values())}
+    units = nseq * xd.q.shape[3]
+    name, (launches, total_ms) = max(times.items(), key=lambda kv: kv[1][1])
+    per_launch = total_ms / launches * 1e-3
+    ach = units * DECODE_BYTES_PER_UNIT / per_launch / 1e9
     del dq, dk_, dv_, dg, db, state, dout
+    torch.cuda.empty_cache()
+    return {"metric": "decode tokens/s", "value": nseq * world / (dms * 1e-3), "unit": UNIT, "ms_per_step": dms,
+            "config": {"workload": wd.name, "sequences": nseq, "heads": xd.q.shape[3],
+                       "state": "fp32 in HBM, updated in place"},
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"], "traffic": traffic_for(name, wd.name), "kernel": name,
+                         "algorithmic_bytes_per_launch": units * DECODE_BYTES_PER_UNIT,
+                         "peak_source": f"{pk['source']} hbm_gbs (burst copy)"},
+            "gpu_launches": sum(c for c, _ in times.values())}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from gated_delta_rule_64_b200 import gdn
+    from gated_delta_rule_64_b200.inputs import KDA_PACKED, LONG_SNAPSHOTS, PREFILL_BF16
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    gdn.load_library()
+    pk = peaks()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    head = time_chunked(LONG_SNAPSHOTS, args, rank, world, dev, pk, clocks=clocks, e2e=True)
     clk = clocks.stop()
+    others = {}
+    if not args.headline_only:
+        others["prefill_b4"] = time_chunked(PREFILL_BF16, args, rank, world, dev, pk)
+        others["kda_packed"] = time_chunked(KDA_PACKED, args, rank, world, dev, pk)
+        others["decode"] = time_decode(args, rank, world, dev, pk)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline()
 
     if rank == 0:
+        cfg = dict(head["config"])
+        cfg.update({"global_batch": cfg["sequences"] * world, "seq_len": LONG_SNAPSHOTS.T,
+                    "parallelism": f"dp{world} (independent sequences per rank)" if world > 1 else "single GPU",
+                    "l2": "inputs larger than L2 (no flush)"})
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "global_batch": B * world, "seq_len": T, "heads": H, "d_k": dk, "d_v": dv,
-                       "chunk": 64, "parallelism": f"dp{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (no flush)"},
-            "roofline": roofline, "decode": decode, "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
-            "gpu_launches": launches,
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "roofline": head["roofline"], "cpu_baseline": cpu, "clocks": clk, "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"],
         }
+        line.update(others)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -612,72 +705,23 @@ def run_spec(args) -> int:
 
 
 def run_secondary(args) -> int:
-    """Time one of the other chunked workloads (the parity configurations) the way the
-    headline line times the prefill workload; prints one JSON line of its own."""
+    """Time one of the other chunked workloads the way the headline line times its
+    workload; prints one JSON line of its own (one GPU)."""
     import torch
 
     from gated_delta_rule_64_b200 import gdn, inputs
 
     w = getattr(inputs, SECONDARY[args.workload])
     torch.cuda.set_device(0)
+    gdn.load_library()
     pk = peaks()
-    x = inputs.make_inputs(w)
-    d = lambda t: None if t is None else t.cuda().contiguous()
-    q, k, v, g, beta, h0, cu = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0), d(x.cu_seqlens)
-    N = x.n_seqs
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    rows = B * T
-    out = torch.empty_like(v)
-    fin = torch.empty((N, H, dv, dk), dtype=torch.float32, device="cuda")
-    n_snap = T // w.snapshot_stride if w.snapshot_stride else 0
-    snaps = torch.empty((N, n_snap, H, dv, dk), dtype=torch.float32, device="cuda") if n_snap else None
-    ws = torch.empty(gdn.gdn_chunk_workspace_size(B, T, H, dk, dv, N, dtype=q.dtype, per_channel=w.per_channel),
-                     dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
-
-    def step():
-        gdn.gdn_chunk_fwd(q, k, v, g, beta, h0, cu, snapshot_stride=w.snapshot_stride, out=out, final_state=fin,
-                          snapshots=snaps, workspace=ws, stream=stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
     clocks = ClockSampler(0)
     clocks.start()
-    gdn.profile_read()
-    gdn.profile_enable(True)
-    clocks.mark_begin()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    clocks.mark_end()
-    gdn.profile_enable(False)
-    kernels = gdn.profile_read()
-    clk = clocks.stop()
-    ms_step = e0.elapsed_time(e1) / args.steps
-    tokens = x.tokens()
-    el = q.element_size()
-    gate_per_tok = 4 * (dk if w.per_channel else 1)
-    alg_bytes = (tokens * H * ((2 * dk + 2 * dv) * el + gate_per_tok + 4)
-                 + (2 if h0 is not None else 1) * N * H * STATE_BYTES + n_snap * N * H * STATE_BYTES)
-    per_launch = {n: t / max(1, c) * 1e-3 for n, (c, t) in kernels.items()}
-    step_s = sum(per_launch.values()) or ms_step * 1e-3
-    achieved = alg_bytes / step_s / 1e9
-    line = {"metric": "chunked prefill tokens/s (secondary workload)", "value": tokens / (ms_step * 1e-3),
-            "unit": UNIT, "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup,
-            "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "tokens": tokens, "sequences": N, "heads": H, "d_k": dk, "d_v": dv,
-                       "per_channel_gate": w.per_channel, "snapshot_stride": w.snapshot_stride},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": alg_bytes,
-                         "kernels": {n: {"us_per_launch": per_launch[n] * 1e6, "share": per_launch[n] / step_s}
-                                     for n in per_launch}},
-            "gpu_launches": sum(c for c, _ in kernels.values()), "clocks": clk}
-    print(json.dumps(line), flush=True)
+    res = time_chunked(w, args, 0, 1, torch.device("cuda", 0), pk, clocks=clocks)
+    res.update({"metric": "chunked prefill tokens/s (secondary workload)", "steps": args.steps,
+                "warmup": args.warmup, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+                "clocks": clocks.stop()})
+    print(json.dumps(res), flush=True)
     return 0
 
 
@@ -685,14 +729,18 @@ def run_profile(which: str) -> int:
     import torch
 
     from gated_delta_rule_64_b200 import gdn
-    from gated_delta_rule_64_b200.inputs import DECODE, KDA_PACKED, PREFILL_BF16, make_inputs
+    from gated_delta_rule_64_b200.inputs import DECODE, KDA_PACKED, LONG_SNAPSHOTS, PREFILL_BF16, make_inputs
     d = lambda t: None if t is None else t.cuda()
-    if which in ("prefill", "kda-small"):
-        # kda-small: the per-channel packed workload on 8 of its 32 heads (about 1.5 GB on the device)
-        x = make_inputs(PREFILL_BF16) if which == "prefill" else make_inputs(KDA_PACKED, heads=8)
+    if which != "decode":
+        # kda-small: the per-channel packed workload on 8 of its 32 heads (about 1.5 GB on the
+        # device); long-small: the first 32768 tokens of the long sequence (about 1 GB)
+        x = {"prefill": lambda: make_inputs(PREFILL_BF16), "kda-small": lambda: make_inputs(KDA_PACKED, heads=8),
+             "long": lambda: make_inputs(LONG_SNAPSHOTS),
+             "long-small": lambda: make_inputs(LONG_SNAPSHOTS.replace(T=32768))}[which]()
         q, k, v, g, b, h0, cu = d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.h0), d(x.cu_seqlens)
+        stride = 8192 if which.startswith("long") else 0
         for _ in range(3):
-            gdn.gdn_chunk_fwd(q, k, v, g, b, h0, cu)
+            gdn.gdn_chunk_fwd(q, k, v, g, b, h0, cu, snapshot_stride=stride)
     else:
         x = make_inputs(DECODE.replace(decode_steps=3))
         st = d(x.h0)
@@ -709,7 +757,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "decode", "kda-small"],
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the headline workload (no prefill-B4 / per-channel / decode objects)")
+    ap.add_argument("--profile", choices=["prefill", "decode", "kda-small", "long", "long-small"],
                     help="run three calls of one workload and exit (for ncu captures; prints nothing to time)")
     ap.add_argument("--workload", choices=["prefill"] + sorted(SECONDARY), default="prefill",
                     help="prefill (default): the headline line; kda / long / tiny: time that chunked "
