@@ -63,12 +63,14 @@ using namespace tc;
 //               After that MMA the Q rows hold A (fp32; rows 0-31 | 32-63),
 //               then T diag(beta gam) at [8K,16K) and T diag(beta) at [24K,32K)
 //               (bf16 operand images).
-//   [32K, 48K)  V tile
-//   [48K, 64K)  T (fp32)
-//   [64K, 68K)  per-warp 16 x 16 scratch of the blocked solve
+//   [32K, 48K)  the P^T image (staged, before the solve), then T (fp32), then
+//               the V tile: V is prefetched into L2 at the start and loaded
+//               here once T has become the bf16 images above
+//   [48K, 52K)  per-warp 16 x 16 scratch of the blocked solve
 // The results (W and Qs images, K~, P^T image, U^T rows, gate factor) are written straight
-// to the workspace block of the chunk-head.
-constexpr uint32_t kPrepTf = 49152, kPrepY = 65536;
+// to the workspace block of the chunk-head.  About 54 KB of shared memory and 64
+// registers a thread let four blocks share an SM.
+constexpr uint32_t kPrepTf = 32768, kPrepV = 32768, kPrepY = 49152;
 constexpr uint32_t kPrepSmem = kPrepY + 4096 + 1024;
 
 __device__ __forceinline__ uint32_t a_offset(int i, int j) {
@@ -76,14 +78,15 @@ __device__ __forceinline__ uint32_t a_offset(int i, int j) {
     return (i < 32 ? 8192u : 24576u) + f32_offset(i & 31, j);
 }
 
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 4)
 gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
             const __grid_constant__ CUtensorMap mv, const float *__restrict__ g, const float *__restrict__ beta,
             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
             int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    __shared__ uint64_t bar_ld, bar_mma, bar_drain;
+    // (one barrier per commit: a waiter two phases behind could not tell them apart)
+    __shared__ uint64_t bar_ld, bar_v, bar_mma, bar_w, bar_u, bar_drain;
     __shared__ uint32_t tmem_base;
     __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C], s_w[C];
     __shared__ __align__(16) float s_b2[C];  // b in log2 units
@@ -108,17 +111,20 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     }
     if (tid == 0) {  // the tile loads first: their latency overlaps the rest of the set-up
         mbar_init(&bar_ld, 1);
+        mbar_init(&bar_v, 1);
         mbar_init(&bar_mma, 1);
+        mbar_init(&bar_w, 1);
+        mbar_init(&bar_u, 1);
         mbar_init(&bar_drain, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&bar_ld, 6 * 8192);
+        mbar_arrive_expect_tx(&bar_ld, 4 * 8192);
         const int32_t hq = (int32_t)(h / (H / Hk));  // query/key head of value head h
         tma_load_3d(sm + 0, &mk, 0, hq, tok0, &bar_ld);
         tma_load_3d(sm + 16384, &mk, 64, hq, tok0, &bar_ld);
         tma_load_3d(sm + 8192, &mq, 0, hq, tok0, &bar_ld);
         tma_load_3d(sm + 24576, &mq, 64, hq, tok0, &bar_ld);
-        tma_load_3d(sm + 32768, &mv, 0, (int32_t)h, tok0, &bar_ld);
-        tma_load_3d(sm + 40960, &mv, 64, (int32_t)h, tok0, &bar_ld);
+        tma_prefetch_3d(&mv, 0, (int32_t)h, tok0);  // loaded after the solve
+        tma_prefetch_3d(&mv, 64, (int32_t)h, tok0);
     }
     if (warp == 0) {
         tmem_alloc(&tmem_base, 128);
@@ -149,7 +155,9 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         s_bg[tid] = s_beta[tid] * __expf(bi);
         s_sg[tid] = in ? scale * __expf(bi) : 0.f;
         s_w[tid] = in ? __expf(bl - bi) : 0.f;
-        if (tid == 0) reinterpret_cast<float *>(rest + kRestFac)[kFacGL] = __expf(bl);
+        float *fac = reinterpret_cast<float *>(rest + kRestFac);
+        fac[kFacQs + tid] = s_sg[tid];  // the scan scales its output by these (it reads Q itself)
+        if (tid == 0) fac[kFacGL] = __expf(bl);
     }
     __syncthreads();
 
@@ -165,9 +173,9 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         }
         mma_commit_warp(&bar_mma);
     }
-    // Qs = (scale * exp(b_i)) q_i and K~ = exp(b_L - b_j) k_j: the rows of the Q
-    // and K tiles rescaled (rows >= L: zero), written to the workspace with the
-    // tiles' own byte layout.
+    // K~ = exp(b_L - b_j) k_j: the rows of the K tile rescaled (rows >= L: zero),
+    // written to the workspace with the tile's own byte layout.  (The query side
+    // needs no image: the scan reads Q and scales its output by scale exp(b_i).)
     // The same pass sums |k_i|^2 for the decay bound: thread (row tid / 8, 16-byte
     // chunk tid % 8) sees rows tid / 8 and 32 + tid / 8 in both channel halves.
     bool bad = false;  // a token of the chunk outside the decay bound's range
@@ -178,9 +186,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
             const int e = tid + kThreads * k;            // 16-byte chunk over both 8K blocks
             const int qb = e >> 9, i = (e & 511) >> 3;   // block, token row
             const uint32_t off = (uint32_t)((e & 511) << 4);
-            const uint4 qv = *reinterpret_cast<const uint4 *>(sm + 8192 + qb * 16384 + off);
             const uint4 kv = *reinterpret_cast<const uint4 *>(sm + qb * 16384 + off);
-            *reinterpret_cast<uint4 *>(blk + 8192 + qb * 16384 + off) = scale8(qv, s_sg[i]);
             *reinterpret_cast<uint4 *>(rest + kRestKt + qb * 8192 + off) = scale8(kv, s_w[i]);
             k2[k & 1] += sum_sq8(kv);
         }
@@ -247,7 +253,8 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks; warps 4-7 first copy the
     // staged P^T image to the workspace (the solve writes its region after that).
     uint8_t *Tf = sm + kPrepTf;
-    blocked_solve<kPrepTf, kPrepY>(sm, [](int i, int j) { return a_offset(i, j); }, ok, [&] {
+    blocked_solve<kPrepTf, kPrepY>(sm, [](int i, int j) { return a_offset(i, j); },
+                                   [](int i) { return (i < 32 ? 8192u : 24576u) + (uint32_t)(i & 31) * 256u; }, ok, [&] {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int e = tid - 128 + 128 * k;
@@ -279,29 +286,47 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
             st_shared_v4(tpp + o, pack_bf16(b[0], b[1]), pack_bf16(b[2], b[3]), pack_bf16(b[4], b[5]), pack_bf16(b[6], b[7]));
         }
     }
-    fence_async_smem();
+    fence_async_smem();  // (T's region is taken over by the V tile below)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    // W^T = K^T T'^T (M = d_k), U^T = V^T T''^T (M = d_v); K = 64 tokens.
-    if (warp == 0 && __all_sync(0xffffffffu, ok)) {
-        const uint64_t dk = sdesc_sw128(smem_u32(sm), 16384, 1024), dv = sdesc_sw128(smem_u32(sm + 32768), 8192, 1024),
-                       dtp = sdesc_sw128(smem_u32(sm + 8192), 16, 1024), dtpp = sdesc_sw128(smem_u32(sm + 24576), 16, 1024);
-        const uint32_t id = idesc_bf16(128, 64, 1, 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm, dk + ((kk * 2048) >> 4), dtp + ((kk * 32) >> 4), id, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm + 64, dv + ((kk * 2048) >> 4), dtpp + ((kk * 32) >> 4), id, kk > 0);
-        mma_commit_warp(&bar_mma);
+    // W^T = K^T T'^T (M = d_k) now; U^T = V^T T''^T (M = d_v) once V is in; K = 64 tokens.
+    bool v_issued = false;
+    if (tid == 0 && ok) {
+        mbar_arrive_expect_tx(&bar_v, 2 * 8192);
+        tma_load_3d(sm + kPrepV, &mv, 0, (int32_t)h, tok0, &bar_v);
+        tma_load_3d(sm + kPrepV + 8192, &mv, 64, (int32_t)h, tok0, &bar_v);
+        v_issued = true;
     }
-    ok = ok && mbar_wait(&bar_mma, 1);
-    tc_fence_after();
+    const uint32_t id_wu = idesc_bf16(128, 64, 1, 0);
+    if (warp == 0 && __all_sync(0xffffffffu, ok)) {
+        const uint64_t dk = sdesc_sw128(smem_u32(sm), 16384, 1024), dtp = sdesc_sw128(smem_u32(sm + 8192), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm, dk + ((kk * 2048) >> 4), dtp + ((kk * 32) >> 4), id_wu, kk > 0);
+        mma_commit_warp(&bar_w);
+        const bool vok = mbar_wait(&bar_v, 0);
+        ok = vok;  // (warp 0 reports a V wait that gave up)
+        if (__all_sync(0xffffffffu, vok)) {
+            tc_fence_after();
+            const uint64_t dv = sdesc_sw128(smem_u32(sm + kPrepV), 8192, 1024),
+                           dtpp = sdesc_sw128(smem_u32(sm + 24576), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tm + 64, dv + ((kk * 2048) >> 4), dtpp + ((kk * 32) >> 4), id_wu, kk > 0);
+        }
+        mma_commit_warp(&bar_u);  // (after a failed V wait this tracks no new product: U is garbage, ok is false)
+    }
 
     // Epilogue 2: thread row r is channel r of W^T and U^T, tokens [32 hf, 32 hf + 32).
     // W goes out as a K-major operand image (rows = tokens, two 64-channel
-    // blocks), U^T as 128-byte-swizzled rows (row = channel).
-    if (ok) store_wu(tm, blk, qd, hf, lane);
+    // blocks) while U^T is formed, then U^T as 128-byte-swizzled rows (row = channel).
+    ok = ok && mbar_wait(&bar_w, 0);
+    tc_fence_after();
+    if (ok) store_w(tm, blk, qd, hf, lane);
+    ok = ok && mbar_wait(&bar_u, 0);
+    tc_fence_after();
+    if (ok) store_u(tm, blk, qd, hf, lane);
     tc_fence_before();
     if (__syncthreads_or(!ok)) {
         // A wait gave up: record it, then wait (bounded) for the tile copies and for
@@ -309,6 +334,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         if (tid == 0) {
             flag_error(err, GDN_DEV_TIMEOUT_PREP);
             mbar_wait(&bar_ld, 0);
+            if (v_issued) mbar_wait(&bar_v, 0);
         }
         if (warp == 0) {
             mma_commit_warp(&bar_drain);
@@ -384,24 +410,31 @@ __device__ __forceinline__ int32_t *split_rec(const ScanSplit &sp, int which, in
 }
 
 // SPLIT: launched as a pass of the split scan (1-D grid; the block's work comes from `sp`).
-// Per-head gate: kThreads + 32 threads; warps 0-7 hold the state and warp 8 issues
-// the MMAs and the copies, so the state warps spend the MMA groups storing the
+// Per-head gate, unsplit: kThreads + 32 threads; warps 0-7 hold the state and warp 8
+// issues the MMAs and the copies, so the state warps spend the MMA groups storing the
 // previous chunk's output.  A ninth warp puts three warps on one SM sub-partition,
-// which caps a thread at 168 registers (gdn_scan_tc).  The per-channel scan needs
-// more, so there warp 0 issues the MMAs and warp 4 the copies (gdn_scan_kda_tc).
+// which caps a thread at 168 registers (gdn_scan_tc).  The split and per-channel
+// scans need more, so there warp 0 issues the MMAs and warp 4 the copies
+// (gdn_scan_split_tc, gdn_scan_kda_tc).
 template <bool KDA, bool SPLIT>
 constexpr int scan_threads() {
-    return KDA ? kThreads : kThreads + 32;
+    return KDA || SPLIT ? kThreads : kThreads + 32;
 }
 #define GDN_SCAN_PARAMS                                                                                              \
-    const float *h0, const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T,          \
-        int64_t rows, int64_t H, int64_t max_chunks, int64_t snap_stride, int64_t n_snap,                            \
-        const uint8_t *__restrict__ blocks, __nv_bfloat16 *__restrict__ out, float *final_state,                     \
-        float *__restrict__ snaps, const ScanSplit sp, int *err
-#define GDN_SCAN_ARGS h0, cu, off, N, T, rows, H, max_chunks, snap_stride, n_snap, blocks, out, final_state, snaps, sp, err
+    const __grid_constant__ CUtensorMap mq, const float *h0, const int32_t *__restrict__ cu,                          \
+        const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk,                  \
+        int64_t max_chunks, int64_t snap_stride, int64_t n_snap, const uint8_t *__restrict__ blocks,                  \
+        __nv_bfloat16 *__restrict__ out, float *final_state, float *__restrict__ snaps, const ScanSplit sp, int *err
+#define GDN_SCAN_ARGS \
+    mq, h0, cu, off, N, T, rows, H, Hk, max_chunks, snap_stride, n_snap, blocks, out, final_state, snaps, sp, err
 
 template <bool KDA, bool SPLIT>
-__device__ __forceinline__ void scan_body(GDN_SCAN_PARAMS) {
+__device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0, const int32_t *__restrict__ cu,
+                                          const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
+                                          int64_t H, int64_t Hk, int64_t max_chunks, int64_t snap_stride,
+                                          int64_t n_snap, const uint8_t *__restrict__ blocks,
+                                          __nv_bfloat16 *__restrict__ out, float *final_state,
+                                          float *__restrict__ snaps, const ScanSplit sp, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     __shared__ ScanBars bars;
@@ -524,6 +557,12 @@ __device__ __forceinline__ void scan_body(GDN_SCAN_PARAMS) {
 
     constexpr int kLoader = WS ? kThreads : 128;  // lane 0 of the issuing warp, else warp 4 lane 0
     int64_t issued = 0;                           // (loader) chunks whose copies are issued
+    // (one gate per head) the Q tile of chunk c: token rows q_row0 + 64 c, query/key head hq
+    int32_t q_row0 = 0, hq = 0;
+    if (!KDA && tid == kLoader) {
+        q_row0 = (int32_t)(start + cb * C);
+        hq = (int32_t)(h / (H / Hk));
+    }
     auto issue_loads = [&](int64_t c) {
         const int stage = (int)(c % kStages);
         uint8_t *st = sm + stage * kStage;
@@ -535,9 +574,17 @@ __device__ __forceinline__ void scan_body(GDN_SCAN_PARAMS) {
             bulk_load(st + kStWQ + 16384, blk + 16384, 8192u, bar);
             bulk_load(st + kStRest + kRestKt, blk + kBlkRest + kRestKt, (uint32_t)kTcKt, bar);
             bulk_load(st + kStRest + kRestFac, blk + kBlkRest + kRestFac, (uint32_t)kTcFac, bar);
-        } else {
+        } else if (KDA) {
             mbar_arrive_expect_tx(bar, kStage);
             bulk_load(st + kStWQ, blk, (uint32_t)kTcWQ, bar);
+            bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
+        } else {  // one gate per head: the Q tile itself next to W (the output is scaled later)
+            mbar_arrive_expect_tx(bar, kStage);
+            const int32_t row0 = q_row0 + (int32_t)c * C;
+            bulk_load(st + kStWQ, blk, 8192u, bar);
+            bulk_load(st + kStWQ + 16384, blk + 16384, 8192u, bar);
+            tma_load_3d(st + kStWQ + 8192, &mq, 0, hq, row0, bar);
+            tma_load_3d(st + kStWQ + 24576, &mq, 64, hq, row0, bar);
             bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
         }
         issued = c + 1;
@@ -743,11 +790,23 @@ __device__ __forceinline__ void scan_body(GDN_SCAN_PARAMS) {
             if (KDA) {
                 load_output();
                 tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) o[q][t] += o2[q][t];
+            } else {  // S0 Q^T scaled per token by scale exp(b_i)
+                const float4 *sg4 = reinterpret_cast<const float4 *>(fac + kFacQs + 32 * hf);
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+#pragma unroll
+                    for (int t4 = 0; t4 < 4; ++t4) {
+                        const float4 f = sg4[4 * q + t4];
+                        o[q][4 * t4] = fmaf(o[q][4 * t4], f.x, o2[q][4 * t4]);
+                        o[q][4 * t4 + 1] = fmaf(o[q][4 * t4 + 1], f.y, o2[q][4 * t4 + 1]);
+                        o[q][4 * t4 + 2] = fmaf(o[q][4 * t4 + 2], f.z, o2[q][4 * t4 + 2]);
+                        o[q][4 * t4 + 3] = fmaf(o[q][4 * t4 + 3], f.w, o2[q][4 * t4 + 3]);
+                    }
             }
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
-#pragma unroll
-                for (int t = 0; t < 16; ++t) o[q][t] += o2[q][t];
         }
 
         // snapshot after n * stride tokens of the sequence
@@ -805,8 +864,8 @@ __device__ __forceinline__ void scan_body(GDN_SCAN_PARAMS) {
     if (warp == 0) tmem_dealloc(tm, 512);
 }
 
-template <bool SPLIT>
-__global__ void __maxnreg__(168) gdn_scan_tc(GDN_SCAN_PARAMS) { scan_body<false, SPLIT>(GDN_SCAN_ARGS); }
+__global__ void __maxnreg__(168) gdn_scan_tc(GDN_SCAN_PARAMS) { scan_body<false, false>(GDN_SCAN_ARGS); }
+__global__ void __launch_bounds__(kThreads, 1) gdn_scan_split_tc(GDN_SCAN_PARAMS) { scan_body<false, true>(GDN_SCAN_ARGS); }
 template <bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) gdn_scan_kda_tc(GDN_SCAN_PARAMS) { scan_body<true, SPLIT>(GDN_SCAN_ARGS); }
 
@@ -939,7 +998,10 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
         attr_err = cudaFuncSetAttribute(gdn_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrepSmem);
-        const void *scans[4] = {(const void *)gdn_scan_tc<false>, (const void *)gdn_scan_tc<true>,
+        // four blocks per SM need the whole shared-memory carveout
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(gdn_prep_tc, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        const void *scans[4] = {(const void *)gdn_scan_tc, (const void *)gdn_scan_split_tc,
                                 (const void *)gdn_scan_kda_tc<false>, (const void *)gdn_scan_kda_tc<true>};
         for (const void *k : scans)
             if (attr_err == cudaSuccess)
@@ -965,29 +1027,30 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     const int scan_block = p.per_channel ? scan_threads<true, false>() : scan_threads<false, false>();
     if (p.split_G < 2) {
         if (a.N * p.H > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
-        auto kern = p.per_channel ? gdn_scan_kda_tc<false> : gdn_scan_tc<false>;
+        auto kern = p.per_channel ? gdn_scan_kda_tc<false> : gdn_scan_tc;
         const dim3 grid((unsigned)a.N, (unsigned)p.H);
         log_launch(p.per_channel ? "gdn_scan_kda_tc" : "gdn_scan_tc", grid, dim3(scan_block), kScanSmem);
         LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc" : "gdn_scan_tc", s);
-        kern<<<grid, scan_block, kScanSmem, s>>>(a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, p.max_chunks,
-                                                 a.snapshot_stride, a.n_snap, blocks, (__nv_bfloat16 *)a.out,
-                                                 a.final_state, a.snapshots, sp, a.status);
+        kern<<<grid, scan_block, kScanSmem, s>>>(mq, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk,
+                                                 p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+                                                 (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, a.status);
         return check_launch("gdn_scan_tc");
     }
     // sequence split: pass 1 (every segment, then the transition maps), the chained
     // start states (G >= 3), pass 2 (the leading chunks of segments 1 .. G-1)
     const int split_block = p.per_channel ? scan_threads<true, true>() : scan_threads<false, true>();
-    auto kern = p.per_channel ? gdn_scan_kda_tc<true> : gdn_scan_tc<true>;
+    auto kern = p.per_channel ? gdn_scan_kda_tc<true> : gdn_scan_split_tc;
     float *states = reinterpret_cast<float *>(a.ws + p.off_split);
     sp = ScanSplit{p.split_G, p.split_seg, 1, states,
                    reinterpret_cast<int32_t *>(states + (size_t)a.N * p.split_G * 3 * p.H * p.dv * p.dk)};
     const int64_t nh = a.N * p.H, grid1 = nh * (2 * (int64_t)p.split_G - 2), grid2 = nh * (p.split_G - 1);
     if (grid1 > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
     {
-        log_launch("gdn_scan_tc (pass 1)", dim3((unsigned)grid1), dim3(split_block), kScanSmem);
-        LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 1)" : "gdn_scan_tc (pass 1)", s);
-        kern<<<(unsigned)grid1, split_block, kScanSmem, s>>>(a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H,
-                                                             p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+        log_launch("gdn_scan (pass 1)", dim3((unsigned)grid1), dim3(split_block), kScanSmem);
+        LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 1)" : "gdn_scan_split_tc (pass 1)", s);
+        kern<<<(unsigned)grid1, split_block, kScanSmem, s>>>(mq, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
+                                                             p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap,
+                                                             blocks,
                                                              (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp,
                                                              a.status);
     }
@@ -1001,10 +1064,11 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     }
     sp.pass = 2;
     {
-        log_launch("gdn_scan_tc (pass 2)", dim3((unsigned)grid2), dim3(split_block), kScanSmem);
-        LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 2)" : "gdn_scan_tc (pass 2)", s);
-        kern<<<(unsigned)grid2, split_block, kScanSmem, s>>>(a.h0, nullptr, nullptr, a.N, a.T, p.rows, p.H,
-                                                             p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
+        log_launch("gdn_scan (pass 2)", dim3((unsigned)grid2), dim3(split_block), kScanSmem);
+        LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 2)" : "gdn_scan_split_tc (pass 2)", s);
+        kern<<<(unsigned)grid2, split_block, kScanSmem, s>>>(mq, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
+                                                             p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap,
+                                                             blocks,
                                                              (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp,
                                                              a.status);
     }

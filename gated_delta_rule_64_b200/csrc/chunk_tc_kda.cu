@@ -555,7 +555,8 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     __syncthreads();
 
     // T = (I + A)^-1 into the (now free) K * R region.
-    blocked_solve<kSmT, kSmY>(sm, [](int i, int j) { return kSmA + f32_offset(i, j); }, ok);
+    blocked_solve<kSmT, kSmY>(sm, [](int i, int j) { return kSmA + f32_offset(i, j); },
+                              [](int i) { return kSmA + (uint32_t)i * 256u; }, ok);
 
     // T'' = T diag(beta) as a bf16 operand image (K-major rows i).
     if (ok) {

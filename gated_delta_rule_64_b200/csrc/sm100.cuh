@@ -14,9 +14,9 @@ namespace gdn {
 namespace sm100 {
 
 #ifndef GDN_SPIN_LIMIT
-#define GDN_SPIN_LIMIT (1u << 26)
+#define GDN_SPIN_LIMIT (1u << 22)
 #endif
-constexpr uint32_t kSpinLimit = GDN_SPIN_LIMIT;  // ~ seconds of polling; only reached on a bug
+constexpr uint32_t kSpinLimit = GDN_SPIN_LIMIT;  // tens of milliseconds of polling: only reached on a bug
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -73,6 +73,13 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         "[%5];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
+}
+// Prefetch a tile into L2 (no shared memory destination, no completion tracking).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int32_t x, int32_t y, int32_t z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
 }
 // Plain bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

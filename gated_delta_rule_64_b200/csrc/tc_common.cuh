@@ -31,6 +31,9 @@ static_assert(kRestPt == kTcKt && kRestU == kRestPt + kTcPImg && kRestFac == kRe
 // channel at [0, 128) for the per-channel gate; at [kFacLam] a bound on how much
 // the chunk can shrink a state, in log2 units (below).
 constexpr int kFacGL = 0, kFacLam = 128;
+// One gate per head: scale exp(b_i) per token at [kFacQs, kFacQs + 64) (the scan
+// scales its S0 Q^T output columns by them).
+constexpr int kFacQs = 192;
 
 // Decay bound of a chunk.  One token maps a state S to S D_t (I - beta_t k_t k_t^T)
 // (+ a write that does not depend on S).  When 0 <= beta_t |k_t|^2 <= 2 the
@@ -170,8 +173,10 @@ __device__ __forceinline__ uint32_t img_offset(int row, int col) {
 struct NoPre {
     __device__ __forceinline__ void operator()() const {}
 };
-template <uint32_t TF, uint32_t TY, typename OffA, typename Pre = NoPre>
-__device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok, Pre pre = Pre()) {
+// rowA(i) is the byte offset of row i of A, whose element (i, j) sits at
+// rowA(i) + f32_offset(0, j) with row i's swizzle (the f32_offset layout per row).
+template <uint32_t TF, uint32_t TY, typename OffA, typename RowA, typename Pre = NoPre>
+__device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, RowA rowA, bool ok, Pre pre = Pre()) {
     constexpr bool kPre = !std::is_same<Pre, NoPre>::value;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto offT = [](int i, int j) { return TF + f32_offset(i, j); };
@@ -180,20 +185,34 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok, P
         // diagonal blocks 2 warp and 2 warp + 1 (lanes 0-15 and 16-31): column `col` of
         // (I + A_pp)^-1 by forward substitution (fp32) ...
         const int p = 2 * warp + (lane >> 4), col = lane & 15;
+        // Element (16p + i, 16p + j) of the f32_offset layout, i, j < 16: row 16p + i,
+        // then the 16-byte chunk ((4p + j / 4) ^ i) = (4p ^ (i & 12)) + ((j / 4) ^ (i & 3))
+        // (disjoint bits): one run-time term per row, the rest a constant.
+        uint32_t xv[4], cv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            xv[k] = ((uint32_t)(4 * p) ^ (uint32_t)(4 * k)) << 4;
+            cv[k] = ((uint32_t)(col >> 2) ^ (uint32_t)k) << 4;
+        }
         float x[16];
         if (ok) {
+            const uint8_t *a0 = sm + rowA(16 * p);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
+                const uint8_t *row = a0 + i * 256 + xv[i >> 2];
                 float acc = 0.f;
 #pragma unroll
-                for (int j = 0; j < i; ++j) acc += *reinterpret_cast<const float *>(sm + offA(16 * p + i, 16 * p + j)) * x[j];
+                for (int j = 0; j < i; ++j)
+                    acc += *reinterpret_cast<const float *>(row + ((((j >> 2) ^ (i & 3)) << 4) + (j & 3) * 4)) * x[j];
                 x[i] = (i == col) ? 1.f : -acc;
             }
         }
         if (kPre) named_bar_sync(1, 192);  // warps 4-7 are done with `pre`
-        if (ok)
+        if (ok) {
+            uint8_t *t0 = sm + TF + (uint32_t)(16 * p) * 256u + (uint32_t)(col & 3) * 4u;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + offT(16 * p + i, 16 * p + col)) = x[i];
+            for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(t0 + i * 256 + xv[i >> 2] + cv[i & 3]) = x[i];
+        }
         __syncwarp();
         // ... then level 1: T_pq = -D_p (A_pq D_q) for (p, q) = (2 warp + 1, 2 warp)
         if (ok) {
@@ -258,15 +277,13 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, bool ok, P
 // (lane = channel, column = token).  Thread row r = qd*32 + lane writes
 // tokens [32 hf, 32 hf + 32): W as a K-major operand image (rows = tokens, two
 // 64-channel blocks), U^T as 128-byte-swizzled rows (row = channel).
-// (Kept out of line: inlined, it pushes the per-head prep kernel past its register budget.)
-static __device__ __noinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
+// (Kept out of line: inlined, they push the per-head prep kernel past its register budget.)
+static __device__ __noinline__ void store_w(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
     const int r = qd * 32 + lane;
     const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
-    float w0[16], w1[16], u0[16], u1[16];
+    float w0[16], w1[16];
     tmem_ld16(taddr, w0);
     tmem_ld16(taddr + 16, w1);
-    tmem_ld16(taddr + 64, u0);
-    tmem_ld16(taddr + 64 + 16, u1);
     tmem_wait_ld();
     uint8_t *wimg = blk + (r >> 6) * 16384 + (r & 7) * 2;
     const int wchunk = (r & 63) >> 3;
@@ -276,6 +293,14 @@ static __device__ __noinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, 
         *reinterpret_cast<__nv_bfloat16 *>(wimg + i * 128 + ((wchunk ^ (i & 7)) << 4)) =
             __float2bfloat16_rn(t < 16 ? w0[t] : w1[t - 16]);
     }
+}
+static __device__ __noinline__ void store_u(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
+    const int r = qd * 32 + lane;
+    const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
+    float u0[16], u1[16];
+    tmem_ld16(taddr + 64, u0);
+    tmem_ld16(taddr + 64 + 16, u1);
+    tmem_wait_ld();
     uint8_t *urow = blk + kBlkRest + kRestU;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -283,6 +308,10 @@ static __device__ __noinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, 
         *reinterpret_cast<uint4 *>(urow + sw128_offset(r, 4 * hf + q)) =
             make_uint4(pack_bf16(u[0], u[1]), pack_bf16(u[2], u[3]), pack_bf16(u[4], u[5]), pack_bf16(u[6], u[7]));
     }
+}
+static __device__ __forceinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
+    store_w(tm, blk, qd, hf, lane);
+    store_u(tm, blk, qd, hf, lane);
 }
 
 // Prep kernel of the per-channel gate (its own translation unit).
