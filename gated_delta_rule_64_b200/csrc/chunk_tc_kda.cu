@@ -374,26 +374,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             fct.d[2][tid] = ex2(r3 - e1);
         }
         ok = mbar_wait(&bar_ld, 0) && ok;
-        // |k_i|^2 of every token (thread: token tid / 4, channels 32 (tid % 4) ..): is its
-        // write a contraction?  Read before the factor pass rescales K in place.
-        bool bad = false;
-        {
-            float k2 = 0.f;
-            if (ok) {
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float kf[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + kSmKQ + kq_chunk(0, tid >> 2, 4 * (tid & 3) + cc)), kf);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) k2 = fmaf(kf[u], kf[u], k2);
-                }
-            }
-            k2 += __shfl_xor_sync(0xffffffffu, k2, 1);
-            k2 += __shfl_xor_sync(0xffffffffu, k2, 2);
-            const int i = tid >> 2;
-            bad = gate_bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * k2 <= kBetaK2Max));
-        }
-        const bool any_bad = __syncthreads_or(bad);
+        bool bad = gate_bad;  // a token outside the decay bound's range (|k_i|^2 below)
         // exact diagonal blocks need the raw tiles and b: before the factor pass
         DiagKeep keep = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
         if (any_wide) {
@@ -403,8 +384,11 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
 
         // Factor pass over (token, 8-channel) chunks: K * L and Q * L in place,
         // K * R to its image; Qs = scale Q * Gam and K~ = K * exp(b_L - b) to the block.
+        // The same pass sums |k_i|^2 for the decay bound: thread (row tid / 8, 16-byte
+        // chunk tid % 8) sees rows tid / 8 and 32 + tid / 8 in both channel halves.
         if (ok) {
             const int Lm1 = L - 1;
+            float k2a = 0.f, k2b = 0.f;  // rows tid / 8 and 32 + tid / 8
 #pragma unroll 1
             for (int k = 0; k < 4; ++k) {
                 const int e = tid + kThreads * k;
@@ -434,6 +418,10 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                     *reinterpret_cast<float4 *>(er) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8);
                     *reinterpret_cast<float4 *>(er + 4) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8 + 4);
                 }
+                float ss = 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) ss = fmaf(kf[u], kf[u], ss);
+                if (k & 1) k2b += ss; else k2a += ss;
                 uint32_t xk[4], xq[4], zr[4], kt[4], qs[4];
                 const bool in = i < L;
 #pragma unroll
@@ -457,17 +445,26 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                 *reinterpret_cast<uint4 *>(sm + kSmKQ + so + 8192) = make_uint4(xq[0], xq[1], xq[2], xq[3]);
                 *reinterpret_cast<uint4 *>(sm + kSmZ + hc * 8192 + i * 128 + pc * 16) = make_uint4(zr[0], zr[1], zr[2], zr[3]);
             }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float x = r ? k2b : k2a;
+                x += __shfl_xor_sync(0xffffffffu, x, 1);
+                x += __shfl_xor_sync(0xffffffffu, x, 2);
+                x += __shfl_xor_sync(0xffffffffu, x, 4);
+                const int i = 32 * r + (tid >> 3);
+                bad = bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * x <= kBetaK2Max));
+            }
             float *fac = reinterpret_cast<float *>(rest + kRestFac);
             if (tid < D) fac[kFacGL + tid] = ex2(*reinterpret_cast<const float *>(sm + kSmB + b_off(Lm1, tid)));
-            if (tid == 0) {
-                float lam = 0.f;
-#pragma unroll
-                for (int w = 0; w < kThreads / 32; ++w) lam += s_lam[w];
-                fac[kFacLam] = any_bad ? kLamNone : lam * kLog2e;
-            }
         }
         fence_async_smem();  // the b region is taken over by the V tile (TMA) below
-        __syncthreads();
+        const bool any_bad = __syncthreads_or(bad);
+        if (tid == 0) {
+            float lam = 0.f;
+#pragma unroll
+            for (int w = 0; w < kThreads / 32; ++w) lam += s_lam[w];
+            reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = any_bad ? kLamNone : lam * kLog2e;
+        }
         if (tid == 0) {
             mbar_arrive_expect_tx(&bar_v, 2 * 8192);
             tma_load_3d(sm + kSmV, &mv, 0, (int32_t)h, tok0, &bar_v);
