@@ -495,8 +495,9 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
     if (SPLIT) {
         if (sp.pass == 1)
             s_end = g == 0 ? split_state(sp, n, 1, 2, H, h) : split_state(sp, n, g, spec ? 0 : 1, H, h);
-        else
-            s_init = split_state(sp, n, g, 2, H, h);
+        else  // S_g, or B_{g-1} itself where M_{g-1} was not formed (gdn_seg_combine wrote nothing)
+            s_init = (g >= 2 && *split_rec(sp, 1, N, n, g - 1, H, h) == 0) ? split_state(sp, n, g - 1, 0, H, h)
+                                                                           : split_state(sp, n, g, 2, H, h);
     }
 
     int64_t start, len;
@@ -869,9 +870,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_scan_split_tc(GDN_SCAN_PARAMS
 template <bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) gdn_scan_kda_tc(GDN_SCAN_PARAMS) { scan_body<true, SPLIT>(GDN_SCAN_ARGS); }
 
-// Start states of the segments: S_{g+1} = S_g M_g + B_g for g = 1 .. G-2 (S_1
-// comes from pass 1; S_{g+1} = B_g where M_g was not formed), one block per
-// (sequence, head), fp32 on the CUDA cores.
+// Start states of the segments: S_{g+1} = S_g M_g + B_g for g = 1 .. G-2 where M_g
+// was formed (S_1 comes from pass 1; where M_g was not formed the start of segment
+// g+1 is B_g itself, which pass 2 reads from where pass 1 left it), one block per
+// (sequence, head), fp32 on the CUDA cores.  S_g is S_1, the result of the previous
+// step, or B_{g-1}.
 // Thread t computes a 4-row x 16-column tile (rows 4 (t % 32) .., columns
 // 16 (t / 32) ..), so every value loaded from shared memory feeds 4 or 16 FMAs.
 // S_g is kept transposed (column k = row of St) so the 4 row values of a k are
@@ -884,23 +887,29 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit s
     float *Ms = St + D * D;                             // M_g: Ms[k][c]
     const int64_t n = blockIdx.x, h = blockIdx.y;
     const int tid = threadIdx.x, r0 = 4 * (tid & 31), c0 = 16 * (tid >> 5);
-    {
-        const float *s1 = split_state(sp, n, 1, 2, H, h);
+    auto load_st = [&](const float *src) {  // St = src^T
         for (int e = tid; e < D * D / 4; e += kThreads) {  // lanes take consecutive rows v
             const int v = e & 127, c4 = e >> 7;
-            const float4 x = *reinterpret_cast<const float4 *>(s1 + v * D + 4 * c4);
+            const float4 x = *reinterpret_cast<const float4 *>(src + v * D + 4 * c4);
             St[(4 * c4) * D + v] = x.x;
             St[(4 * c4 + 1) * D + v] = x.y;
             St[(4 * c4 + 2) * D + v] = x.z;
             St[(4 * c4 + 3) * D + v] = x.w;
         }
-    }
+    };
+    bool have = false;  // St holds S_g
     for (int g = 1; g <= sp.G - 2; ++g) {
+        if (*split_rec(sp, 1, N, n, g, H, h) == 0) {  // uniform over the block
+            have = false;
+            continue;
+        }
+        if (!have) {
+            __syncthreads();
+            load_st(g == 1 ? split_state(sp, n, 1, 2, H, h) : split_state(sp, n, g - 1, 0, H, h));
+        }
         const float *M = split_state(sp, n, g, 1, H, h), *B = split_state(sp, n, g, 0, H, h);
-        const bool with_m = *split_rec(sp, 1, N, n, g, H, h) != 0;  // uniform over the block
-        if (with_m)
-            for (int e = tid; e < D * D / 4; e += kThreads)
-                reinterpret_cast<float4 *>(Ms)[e] = reinterpret_cast<const float4 *>(M)[e];
+        for (int e = tid; e < D * D / 4; e += kThreads)
+            reinterpret_cast<float4 *>(Ms)[e] = reinterpret_cast<const float4 *>(M)[e];
         float acc[4][16];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -910,19 +919,17 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit s
                 acc[i][c] = b4.x; acc[i][c + 1] = b4.y; acc[i][c + 2] = b4.z; acc[i][c + 3] = b4.w;
             }
         __syncthreads();
-        if (with_m) {
 #pragma unroll 2
-            for (int k = 0; k < D; ++k) {
-                const float4 s4 = *reinterpret_cast<const float4 *>(St + k * D + r0);
-                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-                float mv[16];
+        for (int k = 0; k < D; ++k) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(St + k * D + r0);
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+            float mv[16];
 #pragma unroll
-                for (int c = 0; c < 16; c += 4) *reinterpret_cast<float4 *>(mv + c) = *reinterpret_cast<const float4 *>(Ms + k * D + c0 + c);
+            for (int c = 0; c < 16; c += 4) *reinterpret_cast<float4 *>(mv + c) = *reinterpret_cast<const float4 *>(Ms + k * D + c0 + c);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) acc[i][c] = fmaf(sv[i], mv[c], acc[i][c]);
-            }
+                for (int c = 0; c < 16; ++c) acc[i][c] = fmaf(sv[i], mv[c], acc[i][c]);
         }
         __syncthreads();  // every read of S_g and M_g is done
         float *dst = split_state(sp, n, g + 1, 2, H, h);
@@ -935,6 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seg_combine(const ScanSplit s
 #pragma unroll
             for (int c = 0; c < 16; ++c) St[(c0 + c) * D + r0 + i] = acc[i][c];
         }
+        have = true;
     }
 }
 
