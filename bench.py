@@ -259,7 +259,8 @@ def traffic_for(kernel: str, workload: str):
     rec = json.load(open(p)).get(workload, {}).get(kernel)
     if not rec:
         return None
-    if kernel_source_hash(os.path.join(ROOT, rec["source"]), kernel) != rec["sha256"]:
+    # (`kernel` is the library's timer label; the record names the __global__ function)
+    if kernel_source_hash(os.path.join(ROOT, rec["source"]), rec.get("function", kernel)) != rec["sha256"]:
         return None
     for dep, sha in rec.get("deps", {}).items():  # files the kernel's code comes from, hashed whole
         path = os.path.join(ROOT, dep)
