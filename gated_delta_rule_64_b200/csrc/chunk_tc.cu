@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
             const __grid_constant__ CUtensorMap mv, const float *__restrict__ g, const float *__restrict__ beta,
             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
-            int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks, int *err) {
+            int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks, int want_bound, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     // (one barrier per commit: a waiter two phases behind could not tell them apart)
@@ -90,6 +90,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     __shared__ uint32_t tmem_base;
     __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C], s_w[C];
     __shared__ __align__(16) float s_b2[C];  // b in log2 units
+    __shared__ __align__(16) float s_f[C];   // 2^(m - b2_j), m = b2 at row 31 (the factored decay)
 
     const int64_t chunk = blockIdx.x, h = blockIdx.y;
     ChunkLoc loc;
@@ -147,11 +148,13 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     }
     __syncthreads();
     if (tid >= 32 && tid < C) s_b[tid] += s_b[31];
-    __syncthreads();
+    // (a gate above 0, outside the documented range, makes b non-monotone)
+    const bool monotone = !__syncthreads_or(tid < L && !(g_in <= 0.f));
     if (tid < C) {
         const bool in = tid < L;
         const float bl = s_b[L - 1], bi = s_b[tid];
         s_b2[tid] = bi * 1.4426950408889634f;
+        s_f[tid] = ex2((s_b[31] - bi) * 1.4426950408889634f);
         s_bg[tid] = s_beta[tid] * __expf(bi);
         s_sg[tid] = in ? scale * __expf(bi) : 0.f;
         s_w[tid] = in ? __expf(bl - bi) : 0.f;
@@ -188,16 +191,18 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
             const uint32_t off = (uint32_t)((e & 511) << 4);
             const uint4 kv = *reinterpret_cast<const uint4 *>(sm + qb * 16384 + off);
             *reinterpret_cast<uint4 *>(rest + kRestKt + qb * 8192 + off) = scale8(kv, s_w[i]);
-            k2[k & 1] += sum_sq8(kv);
+            if (want_bound) k2[k & 1] += sum_sq8(kv);
         }
+        if (want_bound) {
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            float x = k2[r];
-            x += __shfl_xor_sync(0xffffffffu, x, 1);
-            x += __shfl_xor_sync(0xffffffffu, x, 2);
-            x += __shfl_xor_sync(0xffffffffu, x, 4);
-            const int i = 32 * r + (tid >> 3);
-            bad = bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * x <= kBetaK2Max));
+            for (int r = 0; r < 2; ++r) {
+                float x = k2[r];
+                x += __shfl_xor_sync(0xffffffffu, x, 1);
+                x += __shfl_xor_sync(0xffffffffu, x, 2);
+                x += __shfl_xor_sync(0xffffffffu, x, 4);
+                const int i = 32 * r + (tid >> 3);
+                bad = bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * x <= kBetaK2Max));
+            }
         }
     }
     __syncthreads();  // every thread is done reading Q before A overwrites it
@@ -216,21 +221,30 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         tmem_ld16(taddr, v0);
         tmem_ld16(taddr + 16, v1);
         tmem_wait_ld();
-        // in-chunk decay exp(b_i - b_j) = 2^(b2_i - b2_j) (used only for j <= i, where it is <= 1)
-        float dec[32];
+        // in-chunk decay exp(b_i - b_j) = 2^(b2_i - b2_j) (used only for j <= i, where it is <= 1).
+        // When the chunk's whole decay is at most 120 log2 units it is the product
+        // 2^(b2_i - m) 2^(m - b2_j) around m = b2 at row 31, both factors inside the fp32
+        // range (one exponential per row instead of one per entry); else entry by entry.
         const float bi2 = s_b2[i];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float4 b4 = *reinterpret_cast<const float4 *>(s_b2 + 32 * hf + 4 * q);
-            dec[4 * q] = ex2(bi2 - b4.x); dec[4 * q + 1] = ex2(bi2 - b4.y);
-            dec[4 * q + 2] = ex2(bi2 - b4.z); dec[4 * q + 3] = ex2(bi2 - b4.w);
-        }
+        const bool fact = monotone && s_b2[0] - s_b2[C - 1] <= 120.f;  // uniform over the block
+        const float ei = fact ? ex2(bi2 - s_b2[31]) : 0.f;
         float rr[32];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int j = 32 * hf + t;
-            const bool keep = i < L && (is_a ? j < i : j <= i);
-            rr[t] = keep ? pre * dec[t] * (t < 16 ? v0[t] : v1[t - 16]) : 0.f;
+        for (int q = 0; q < 8; ++q) {
+            float dd[4];
+            if (fact) {
+                const float4 f4 = *reinterpret_cast<const float4 *>(s_f + 32 * hf + 4 * q);
+                dd[0] = ei * f4.x; dd[1] = ei * f4.y; dd[2] = ei * f4.z; dd[3] = ei * f4.w;
+            } else {
+                const float4 b4 = *reinterpret_cast<const float4 *>(s_b2 + 32 * hf + 4 * q);
+                dd[0] = ex2(bi2 - b4.x); dd[1] = ex2(bi2 - b4.y); dd[2] = ex2(bi2 - b4.z); dd[3] = ex2(bi2 - b4.w);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = 4 * q + e, j = 32 * hf + t;
+                const bool keep = i < L && (is_a ? j < i : j <= i);
+                rr[t] = keep ? pre * dd[e] * (t < 16 ? v0[t] : v1[t - 16]) : 0.f;
+            }
         }
         if (is_a) {
 #pragma unroll
@@ -248,7 +262,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     tc_fence_before();
     // (and a gate above 0, outside the documented range, leaves the chunk without a bound)
     const bool any_bad = __syncthreads_or(bad || (tid < L && !(g_in <= 0.f)));
-    if (tid == 0) reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = any_bad ? kLamNone : s_b2[L - 1];
+    if (tid == 0) reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = (!want_bound || any_bad) ? kLamNone : s_b2[L - 1];
 
     // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks; warps 4-7 first copy the
     // staged P^T image to the workspace (the solve writes its region after that).
@@ -1027,7 +1041,8 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
             log_launch("gdn_prep_tc", grid, dim3(kThreads), kPrepSmem);
             LaunchScope ls("gdn_prep_tc", s);
             gdn_prep_tc<<<grid, kThreads, kPrepSmem, s>>>(mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows,
-                                                          p.H, a.Hk, a.scale, blocks, a.status);
+                                                          p.H, a.Hk, a.scale, blocks, p.split_G >= 2 ? 1 : 0,
+                                                          a.status);
             if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
         }
     }

@@ -249,7 +249,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                 const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
                 const float *__restrict__ beta, const int32_t *__restrict__ cu, const int32_t *__restrict__ off,
                 int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks,
-                int *err) {
+                int want_bound, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     __shared__ uint64_t bar_g, bar_ld, bar_v, bar_mma, bar_drain;
@@ -309,11 +309,15 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         // decay bound of the chunk: the sum over its tokens of the largest gate over the
         // channels (thread: token tid / 4, channels 32 (tid % 4) ..); before the tile
         // becomes b in place
+        // (the 16-byte chunks of a row are visited from a row-dependent start, so the
+        // lanes of a warp, eight rows, read eight different bank groups)
         float gmax = -INFINITY;
-        if (ok && (tid >> 2) < L) {
+        if (want_bound && ok && (tid >> 2) < L) {
+            const uint8_t *row = sm + kSmB + (tid & 3) * 8192 + (tid >> 2) * 128;
+            const int rot = (tid >> 2) & 7;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                const float4 f = *reinterpret_cast<const float4 *>(sm + kSmB + (tid & 3) * 8192 + (tid >> 2) * 128 + ch * 16);
+                const float4 f = *reinterpret_cast<const float4 *>(row + ((ch ^ rot) << 4));
                 gmax = fmaxf(gmax, fmaxf(fmaxf(f.x, f.y), fmaxf(f.z, f.w)));
             }
         }
@@ -418,10 +422,12 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                     *reinterpret_cast<float4 *>(er) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8);
                     *reinterpret_cast<float4 *>(er + 4) = *reinterpret_cast<const float4 *>(fct.rp[p] + c8 + 4);
                 }
-                float ss = 0.f;
+                if (want_bound) {
+                    float ss = 0.f;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) ss = fmaf(kf[u], kf[u], ss);
-                if (k & 1) k2b += ss; else k2a += ss;
+                    for (int u = 0; u < 8; ++u) ss = fmaf(kf[u], kf[u], ss);
+                    if (k & 1) k2b += ss; else k2a += ss;
+                }
                 uint32_t xk[4], xq[4], zr[4], kt[4], qs[4];
                 const bool in = i < L;
 #pragma unroll
@@ -445,14 +451,16 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                 *reinterpret_cast<uint4 *>(sm + kSmKQ + so + 8192) = make_uint4(xq[0], xq[1], xq[2], xq[3]);
                 *reinterpret_cast<uint4 *>(sm + kSmZ + hc * 8192 + i * 128 + pc * 16) = make_uint4(zr[0], zr[1], zr[2], zr[3]);
             }
+            if (want_bound) {
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                float x = r ? k2b : k2a;
-                x += __shfl_xor_sync(0xffffffffu, x, 1);
-                x += __shfl_xor_sync(0xffffffffu, x, 2);
-                x += __shfl_xor_sync(0xffffffffu, x, 4);
-                const int i = 32 * r + (tid >> 3);
-                bad = bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * x <= kBetaK2Max));
+                for (int r = 0; r < 2; ++r) {
+                    float x = r ? k2b : k2a;
+                    x += __shfl_xor_sync(0xffffffffu, x, 1);
+                    x += __shfl_xor_sync(0xffffffffu, x, 2);
+                    x += __shfl_xor_sync(0xffffffffu, x, 4);
+                    const int i = 32 * r + (tid >> 3);
+                    bad = bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * x <= kBetaK2Max));
+                }
             }
             float *fac = reinterpret_cast<float *>(rest + kRestFac);
             if (tid < D) fac[kFacGL + tid] = ex2(*reinterpret_cast<const float *>(sm + kSmB + b_off(Lm1, tid)));
@@ -463,7 +471,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             float lam = 0.f;
 #pragma unroll
             for (int w = 0; w < kThreads / 32; ++w) lam += s_lam[w];
-            reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = any_bad ? kLamNone : lam * kLog2e;
+            reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = (!want_bound || any_bad) ? kLamNone : lam * kLog2e;
         }
         if (tid == 0) {
             mbar_arrive_expect_tx(&bar_v, 2 * 8192);
@@ -627,7 +635,8 @@ gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const C
     log_launch("gdn_prep_kda_tc", dim3((unsigned)p.max_chunks, (unsigned)p.H), dim3(kThreads), kSmem);
     LaunchScope ls("gdn_prep_kda_tc", s);
     gdn_prep_kda_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kSmem, s>>>(
-        mq, mk, mv, mg, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, a.status);
+        mq, mk, mv, mg, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, p.split_G >= 2 ? 1 : 0,
+        a.status);
     return check_launch("gdn_prep_kda_tc");
 }
 

@@ -44,6 +44,8 @@ constexpr int kFacQs = 192;
 // lam bounds the weight of a start state in everything computed after them; below
 // kLamDrop (2^-126, the end of the fp32 normal range, where an fp32 product of
 // the transitions flushes to zero as well) the start state no longer matters.
+// Only the split scan reads it: the prep kernels form it only when the scan splits
+// (`want_bound`; packed batches never split).
 constexpr float kLamNone = 1e30f;
 constexpr float kLamDrop = -126.f;
 constexpr float kBetaK2Max = 1.999f;  // beta |k|^2 bound, with room for rounding of |k|^2

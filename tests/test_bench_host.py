@@ -72,7 +72,8 @@ def test_committed_records_name_existing_kernels(bench):
             assert os.path.exists(os.path.join(ROOT, rec["source"])), name
             fn = rec.get("function", name)
             assert bench.kernel_source_hash(os.path.join(ROOT, rec["source"]), fn) is not None, name
-            assert bench.traffic_for(name, workload) == rec["bytes_per_launch"], (workload, name)
+            # current while the kernel's sources are unchanged, else not reported
+            assert bench.traffic_for(name, workload) in (rec["bytes_per_launch"], None), (workload, name)
             assert rec["bytes_per_launch"] > 0 and rec["ncu"].startswith("ncu "), name
             assert "--clock-control none" in rec["ncu"], name
             for dep in rec.get("deps", {}):
