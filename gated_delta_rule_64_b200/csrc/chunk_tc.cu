@@ -25,13 +25,13 @@
 //                system is solved blockwise (16 x 16 diagonal blocks by forward
 //                substitution in fp32, off-diagonal blocks by tf32 warp MMAs);
 //                two MMAs give W^T and U^T.  The results are written as
-//                ready-made operand images into one contiguous block per
-//                chunk-head.
+//                ready-made operand images (16-byte stores of 128-byte swizzled
+//                rows) into one contiguous block per chunk-head.
 //   gdn_scan_tc  one CTA per (sequence, head).  The fp32 state lives in
 //                registers (two threads per state row, 64 columns each); per
 //                chunk it is rounded to a bf16 A operand in TMEM and two MMA
 //                groups with fp32 accumulators in TMEM produce
-//                [S0 W^T | S0 Qs^T] and, from U' = U - W S0^T, U'^T [K~ | P^T]
+//                [S0 W^T | S0 Q^T] and, from U' = U - W S0^T, [U'^T K~ | U'^T P^T]
 //                (the state increment and the intra-chunk output).  The next
 //                chunks' blocks are prefetched (bulk copies) into three stages.
 //                A ninth warp issues the MMAs and copies (per-head gate, no
@@ -63,11 +63,10 @@ using namespace tc;
 //               After that MMA the Q rows hold A (fp32; rows 0-31 | 32-63),
 //               then T diag(beta gam) at [8K,16K) and T diag(beta) at [24K,32K)
 //               (bf16 operand images).
-//   [32K, 48K)  the P^T image (staged, before the solve), then T (fp32), then
-//               the V tile: V is prefetched into L2 at the start and loaded
-//               here once T has become the bf16 images above
+//   [32K, 48K)  T (fp32), then the V tile: V is prefetched into L2 at the start
+//               and loaded here once T has become the bf16 images above
 //   [48K, 52K)  per-warp 16 x 16 scratch of the blocked solve
-// The results (W and Qs images, K~, P^T image, U^T rows, gate factor) are written straight
+// The results (W^T rows, K~, P rows, U^T rows, gate factors) are written straight
 // to the workspace block of the chunk-head.  About 54 KB of shared memory and 64
 // registers a thread let four blocks share an SM.
 constexpr uint32_t kPrepTf = 32768, kPrepV = 32768, kPrepY = 49152;
@@ -210,7 +209,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     tc_fence_after();
 
     // Epilogue 1: accumulator row r = qd*32 + lane, columns [32 hf, 32 hf + 32).
-    // Rows 0..63 (K K^T) -> A in fp32; rows 64..127 (Q K^T) -> P^T image (bf16).
+    // Rows 0..63 (K K^T) -> A in fp32; rows 64..127 (Q K^T) -> P rows (bf16).
     if (ok) {
         const int r = qd * 32 + lane;
         const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
@@ -252,11 +251,12 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
                 *reinterpret_cast<float4 *>(sm + a_offset(i, 32 * hf + 4 * q)) =
                     make_float4(rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
         } else {
-            // P^T image (rows j, columns i), staged in the (still unused) T region:
-            // one column j per store instruction, 32 consecutive rows i per warp
-            __nv_bfloat16 *pt = reinterpret_cast<__nv_bfloat16 *>(sm + kPrepTf);
+            // P row i (key tokens j = 32 hf ..) straight to the block: four 16-byte chunks
 #pragma unroll
-            for (int t = 0; t < 32; ++t) pt[img_offset(32 * hf + t, i) / 2] = __float2bfloat16_rn(rr[t]);
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(rest + kRestP + sw128_offset(i, 4 * hf + q)) =
+                    make_uint4(pack_bf16(rr[8 * q], rr[8 * q + 1]), pack_bf16(rr[8 * q + 2], rr[8 * q + 3]),
+                               pack_bf16(rr[8 * q + 4], rr[8 * q + 5]), pack_bf16(rr[8 * q + 6], rr[8 * q + 7]));
         }
     }
     tc_fence_before();
@@ -264,25 +264,21 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     const bool any_bad = __syncthreads_or(bad || (tid < L && !(g_in <= 0.f)));
     if (tid == 0) reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = (!want_bound || any_bad) ? kLamNone : s_b2[L - 1];
 
-    // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks; warps 4-7 first copy the
-    // staged P^T image to the workspace (the solve writes its region after that).
+    // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks.
     uint8_t *Tf = sm + kPrepTf;
     blocked_solve<kPrepTf, kPrepY>(sm, [](int i, int j) { return a_offset(i, j); },
-                                   [](int i) { return (i < 32 ? 8192u : 24576u) + (uint32_t)(i & 31) * 256u; }, ok, [&] {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int e = tid - 128 + 128 * k;
-            *reinterpret_cast<uint4 *>(rest + kRestPt + e * 16) = *reinterpret_cast<const uint4 *>(sm + kPrepTf + e * 16);
-        }
-    });
+                                   [](int i) { return (i < 32 ? 8192u : 24576u) + (uint32_t)(i & 31) * 256u; }, ok);
 
-    // T' = T diag(beta gam), T'' = T diag(beta) as bf16 operand images (K-major rows i).
+    // T' = T diag(beta gam), T'' = T diag(beta) as bf16 operand images (K-major rows i);
+    // the blocks of T above its block diagonal are zero (the solve leaves them unwritten).
     if (ok) {
         const int i = tid >> 2, j0 = (tid & 3) * 16;
+        const bool upper = (tid & 3) > (i >> 4);
         float tv[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float4 f = *reinterpret_cast<const float4 *>(Tf + f32_offset(i, j0 + 4 * q));
+            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!upper) f = *reinterpret_cast<const float4 *>(Tf + f32_offset(i, j0 + 4 * q));
             tv[4 * q] = f.x; tv[4 * q + 1] = f.y; tv[4 * q + 2] = f.z; tv[4 * q + 3] = f.w;
         }
         const uint32_t tp = smem_u32(sm + 8192), tpp = smem_u32(sm + 24576);
@@ -363,19 +359,21 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
 // Scan
 // ===========================================================================
 // Shared memory (1024-aligned), three stages of per-chunk operands, each the
-// chunk-head's workspace block as it is (two bulk copies):
-//   [0, 32K)      [W rows | Qs rows] per 64-channel block: the N = 128 B operand
-//                 of S0 [W ; Qs]^T
-//   [32K, 56K)    [K~ | P^T]: the N = 192 MN-major B operand of U'^T [K~ | P^T]
+// chunk-head's workspace block as it is (two bulk copies; with one gate per head
+// the Q tile comes from q itself, by TMA, where the block holds Qs):
+//   [0, 16K)      W^T rows: the MN-major B operand of S0 W^T (N = 64)
+//   [16K, 32K)    Q or Qs, two 64-channel halves: the K-major B operand of S0 Q^T
+//   [32K, 48K)    K~: the MN-major B operand of U'^T K~ (N = 128)
+//   [48K, 56K)    P rows: the K-major B operand of U'^T P^T (N = 64)
 //   [56K, 72K)    U^T rows;  [72K, 73K) gate factors
 // The operands the threads produce (S0 and U' in bf16) are written to TMEM and
 // used as A operands straight from there.
-// TMEM columns: [0,128) D1 = [S0 W^T | S0 Qs^T], [128,320) D2 = [U'^T K~ | U'^T P^T],
+// TMEM columns: [0,128) D1 = [S0 W^T | S0 Q^T], [128,320) D2 = [U'^T K~ | U'^T P^T],
 // [320,384) S0, [384,416) U'.
 // A tcgen05.ld waits for the MMAs in flight, so every accumulator is read once
 // the chunk's MMAs are done (the output with the state increment), and the
 // output leaves from registers while the next chunk's first MMA group runs.
-constexpr uint32_t kStWQ = 0, kStRest = kBlkRest, kStage = (uint32_t)kTcBlock;
+constexpr uint32_t kStW = kBlkW, kStQ = kBlkQs, kStRest = kBlkRest, kStage = (uint32_t)kTcBlock;
 static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled operands");
 constexpr int kStages = 3;
 constexpr uint32_t kScanSmem = kStages * kStage + 1024;
@@ -383,8 +381,8 @@ constexpr uint32_t kTmD1 = 0, kTmD2 = 128, kTmAS = 320, kTmAU = 384;
 
 struct ScanBars {
     uint64_t full[kStages];
-    uint64_t mma[2];
-    uint64_t drain;  // after a failed wait: every MMA issued has completed
+    uint64_t mma[3];  // per chunk: S0 W^T done; U'^T K~ done; every product of the chunk done
+    uint64_t drain;   // after a failed wait: every MMA issued has completed
 };
 
 // KDA: per-channel gate (the carried state is then scaled per key channel by
@@ -556,7 +554,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(&bars.full[i], 1);
-        for (int i = 0; i < 2; ++i) mbar_init(&bars.mma[i], 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bars.mma[i], 1);
         mbar_init(&bars.drain, 1);
         fence_mbar_init();
     }
@@ -583,23 +581,21 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
         uint8_t *st = sm + stage * kStage;
         const uint8_t *blk = block_of(c);
         uint64_t *bar = &bars.full[stage];
-        if (ident) {  // a transition map reads W, K~ and the factors only
-            mbar_arrive_expect_tx(bar, (uint32_t)(2 * 8192 + kTcKt + kTcFac));
-            bulk_load(st + kStWQ, blk, 8192u, bar);
-            bulk_load(st + kStWQ + 16384, blk + 16384, 8192u, bar);
+        if (ident) {  // a transition map reads W^T, K~ and the factors only
+            mbar_arrive_expect_tx(bar, (uint32_t)(16384 + kTcKt + kTcFac));
+            bulk_load(st + kStW, blk + kBlkW, 16384u, bar);
             bulk_load(st + kStRest + kRestKt, blk + kBlkRest + kRestKt, (uint32_t)kTcKt, bar);
             bulk_load(st + kStRest + kRestFac, blk + kBlkRest + kRestFac, (uint32_t)kTcFac, bar);
         } else if (KDA) {
             mbar_arrive_expect_tx(bar, kStage);
-            bulk_load(st + kStWQ, blk, (uint32_t)kTcWQ, bar);
+            bulk_load(st, blk, (uint32_t)kTcWQ, bar);
             bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
-        } else {  // one gate per head: the Q tile itself next to W (the output is scaled later)
+        } else {  // one gate per head: the Q tile itself (the output is scaled later)
             mbar_arrive_expect_tx(bar, kStage);
             const int32_t row0 = q_row0 + (int32_t)c * C;
-            bulk_load(st + kStWQ, blk, 8192u, bar);
-            bulk_load(st + kStWQ + 16384, blk + 16384, 8192u, bar);
-            tma_load_3d(st + kStWQ + 8192, &mq, 0, hq, row0, bar);
-            tma_load_3d(st + kStWQ + 24576, &mq, 64, hq, row0, bar);
+            bulk_load(st + kStW, blk + kBlkW, 16384u, bar);
+            tma_load_3d(st + kStQ, &mq, 0, hq, row0, bar);
+            tma_load_3d(st + kStQ + 8192, &mq, 64, hq, row0, bar);
             bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
         }
         issued = c + 1;
@@ -688,30 +684,48 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
         const bool emit_state = spec ? lam_next < kLamDrop : emit_any;
         if (spec && emit && m_first == nchunks) m_first = c;
 
-        // (b) D1 = S0 [W ; Qs]^T   (N = 128, K = 128): [U correction | inter-chunk output]
-        //     (N = 64, W only, for a chunk without outputs)
+        // (b) D1 = [S0 W^T | S0 Q^T]   (N = 64 + 64, K = 128): [U correction | inter-chunk
+        //     output] (S0 W^T only, for a chunk without outputs).  S0 W^T is committed
+        //     on its own: U' needs only it, and is formed while S0 Q^T runs.
         if (warp == kIssuer) {
-            const uint64_t bwq = sdesc_sw128(st_u + kStWQ, 16, 1024);
-            const uint32_t id_wq = idesc_bf16(128, emit ? 128 : 64, 0, 0);
+            const uint64_t bw = sdesc_sw128(st_u + kStW, 8192, 1024), bq = sdesc_sw128(st_u + kStQ, 16, 1024);
+            const uint32_t id_w = idesc_bf16(128, 64, 0, 1), id_q = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_ts(tm + kTmD1, tm + kTmAS + kk * 8, bwq + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                            id_wq, kk > 0);
+                mma_bf16_ts(tm + kTmD1, tm + kTmAS + kk * 8, bw + (uint64_t)((kk * 2048) >> 4), id_w, kk > 0);
             mma_commit_warp(&bars.mma[0]);
+            if (emit)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tm + kTmD1 + 64, tm + kTmAS + kk * 8,
+                                bq + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_q, kk > 0);
         }
         // every MMA of chunk c-1 has completed (step (e) waited for them), so its
         // stage can take chunk c+2
         if (tid == kLoader && c >= 1 && c + kStages - 1 < nrun) issue_loads(c + kStages - 1);
-        const uint32_t id_kp = idesc_bf16(128, emit ? 192 : 128, 0, 1);
+        // (d) D2 = [U'^T K~ | U'^T P^T]   (N = 128 + 64, K = 64 tokens): [state increment |
+        //     intra-chunk output] (the increment only, for a chunk without outputs).  The
+        //     increment is committed on its own (the state is updated while U'^T P^T
+        //     runs), then every product of the chunk.
+        auto issue_d2 = [&] {
+            const uint64_t bk = sdesc_sw128(st_u + kStRest + kRestKt, 8192, 1024),
+                           bp = sdesc_sw128(st_u + kStRest + kRestP, 16, 1024);
+            const uint32_t id_k = idesc_bf16(128, 128, 0, 1), id_p = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(tm + kTmD2, tm + kTmAU + kk * 8, bk + (uint64_t)((kk * 2048) >> 4), id_k, kk > 0);
+            mma_commit_warp(&bars.mma[1]);
+            if (emit)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(tm + kTmD2 + 128, tm + kTmAU + kk * 8, bp + (uint64_t)((kk * 32) >> 4), id_p, kk > 0);
+            mma_commit_warp(&bars.mma[2]);
+        };
         if (WS && warp == kIssuer) {
             // (d) once every row's U' is in TMEM (named barrier 1)
             named_bar_sync(1, kThreads + 32);
             tc_fence_after();
-            const uint64_t bkp = sdesc_sw128(st_u + kStRest + kRestKt, 8192, 1024);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(tm + kTmD2, tm + kTmAU + kk * 8, bkp + (uint64_t)((kk * 2048) >> 4), id_kp, kk > 0);
-            mma_commit_warp(&bars.mma[1]);
+            issue_d2();
             lam = lam_next;
             emit_prev = emit;
             continue;
@@ -754,37 +768,22 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
             tc_fence_after();
         }
 
-        // (d) D2 = U'^T [K~ | P^T]   (N = 192, K = 64 tokens): [state increment | intra-chunk output]
-        if (!WS && warp == 0) {
-            const uint64_t bkp = sdesc_sw128(st_u + kStRest + kRestKt, 8192, 1024);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(tm + kTmD2, tm + kTmAU + kk * 8, bkp + (uint64_t)((kk * 2048) >> 4), id_kp, kk > 0);
-            mma_commit_warp(&bars.mma[1]);
-        }
+        // (d)
+        if (!WS && warp == 0) issue_d2();
 
         // the second half of the previous chunk's output, while these MMAs run
         if (c >= 1 && emit_prev) store_output(c - 1, 1);
 
         // (e) S = gam_L S0 + increment (columns [64 hf, 64 hf + 64); per key channel
-        // for KDA) and the output o = S0 Qs^T + U'^T P^T
+        // for KDA) and the output o = S0 Qs^T + U'^T P^T (one gate per head: Qs^T = Q^T
+        // scaled per token)
         const float gl = fac[kFacGL];
         ok = mbar_wait(&bars.mma[1], par) && ok;
         tc_fence_after();
         {
-            float a[4][16], o2[2][16];
-            auto load_output = [&] {
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    tmem_ld16(tm + lane_off + kTmD1 + 64 + 32 * hf + 16 * q, o[q]);
-                    tmem_ld16(tm + lane_off + kTmD2 + 128 + 32 * hf + 16 * q, o2[q]);
-                }
-            };
-            // (the output columns are read whether or not this chunk writes them: a
-            // value that is sometimes kept would stay live across the whole chunk)
+            float a[4][16];
 #pragma unroll
             for (int c0 = 0; c0 < 4; ++c0) tmem_ld16(tm + lane_off + kTmD2 + 64 * hf + 16 * c0, a[c0]);
-            if (!KDA) load_output();  // (KDA: after the state update, for registers)
             tmem_wait_ld();
             if (KDA) {
                 const float4 *gl4 = reinterpret_cast<const float4 *>(fac + kFacGL + 64 * hf);
@@ -802,9 +801,20 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
 #pragma unroll
                     for (int t = 0; t < 16; ++t) S[16 * c0 + t] = gl * S[16 * c0 + t] + a[c0][t];
             }
+        }
+        ok = mbar_wait(&bars.mma[2], par) && ok;
+        tc_fence_after();
+        {
+            // (the output columns are read whether or not this chunk writes them: a
+            // value that is sometimes kept would stay live across the whole chunk)
+            float o2[2][16];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                tmem_ld16(tm + lane_off + kTmD1 + 64 + 32 * hf + 16 * q, o[q]);
+                tmem_ld16(tm + lane_off + kTmD2 + 128 + 32 * hf + 16 * q, o2[q]);
+            }
+            tmem_wait_ld();
             if (KDA) {
-                load_output();
-                tmem_wait_ld();
 #pragma unroll
                 for (int q = 0; q < 2; ++q)
 #pragma unroll

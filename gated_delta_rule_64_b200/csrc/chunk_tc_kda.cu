@@ -53,7 +53,7 @@ namespace {
 //   [64K, 80K)  K * R (layout of a K tile, channel halves 8K apart); after the blocks:
 //               T (fp32)
 //   [80K, 96K)  after the blocks: the solve's scratch (4K) and T diag(beta) (8K at 88K)
-//   [96K, 104K) P^T image (bf16, rows = key tokens j, columns = query tokens i)
+//   [96K, 104K) P rows (bf16, row = query token i, 64 key tokens j, 128-byte swizzle)
 constexpr uint32_t kSmKQ = 0, kSmB = 32768, kSmA = 32768, kSmV = 49152, kSmZ = 65536, kSmP = 98304;
 constexpr uint32_t kSmT = 65536, kSmY = 81920, kSmTp = 90112;
 constexpr uint32_t kSmem = kSmP + 8192 + 1024;
@@ -161,11 +161,11 @@ __device__ __forceinline__ void ap_blocks(uint8_t *sm, const Factors &f, int p, 
             // P: causal (j <= i) and rows of the chunk only
             const bool k00 = i0 < L && (!diag || col <= i0), k01 = i0 < L && (!diag || col + 1 <= i0);
             const bool k10 = i1 < L && (!diag || col <= i1), k11 = i1 < L && (!diag || col + 1 <= i1);
-            __nv_bfloat16 *pt = reinterpret_cast<__nv_bfloat16 *>(sm + kSmP);  // P^T: element (j, i)
-            pt[img_offset(col, i0) / 2] = __float2bfloat16_rn(k00 ? scale * cP[b][nt][0] : 0.f);
-            pt[img_offset(col + 1, i0) / 2] = __float2bfloat16_rn(k01 ? scale * cP[b][nt][1] : 0.f);
-            pt[img_offset(col, i1) / 2] = __float2bfloat16_rn(k10 ? scale * cP[b][nt][2] : 0.f);
-            pt[img_offset(col + 1, i1) / 2] = __float2bfloat16_rn(k11 ? scale * cP[b][nt][3] : 0.f);
+            // P rows: the pair of columns (col, col + 1) of rows i0 and i1, one 4-byte store each
+            *reinterpret_cast<uint32_t *>(sm + kSmP + img_offset(i0, col)) =
+                pack_bf16(k00 ? scale * cP[b][nt][0] : 0.f, k01 ? scale * cP[b][nt][1] : 0.f);
+            *reinterpret_cast<uint32_t *>(sm + kSmP + img_offset(i1, col)) =
+                pack_bf16(k10 ? scale * cP[b][nt][2] : 0.f, k11 ? scale * cP[b][nt][3] : 0.f);
         }
     }
 }
@@ -240,7 +240,7 @@ __device__ __forceinline__ void diag_exact_store(uint8_t *sm, const DiagKeep &ke
         const bool first = it <= r;
         const int i = base + (first ? r : 15 - r), j = base + (first ? r - it : 16 - it);
         *reinterpret_cast<float *>(sm + kSmA + f32_offset(i, j)) = s_beta[i] * keep.a[k];
-        *reinterpret_cast<__nv_bfloat16 *>(sm + kSmP + img_offset(j, i)) = __float2bfloat16_rn(i < L ? scale * keep.p[k] : 0.f);
+        *reinterpret_cast<__nv_bfloat16 *>(sm + kSmP + img_offset(i, j)) = __float2bfloat16_rn(i < L ? scale * keep.p[k] : 0.f);
     }
 }
 
@@ -444,7 +444,7 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                     qs[u] = in ? pack_bf16(scale * qf[a] * ga, scale * qf[b] * gb) : 0u;
                 }
                 *reinterpret_cast<uint4 *>(rest + kRestKt + hc * 8192 + i * 128 + pc * 16) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
-                *reinterpret_cast<uint4 *>(blk + 8192 + hc * 16384 + i * 128 + pc * 16) =
+                *reinterpret_cast<uint4 *>(blk + kBlkQs + hc * 8192 + i * 128 + pc * 16) =
                     make_uint4(qs[0], qs[1], qs[2], qs[3]);
                 // (no other thread reads this chunk of the tiles)
                 *reinterpret_cast<uint4 *>(sm + kSmKQ + so) = make_uint4(xk[0], xk[1], xk[2], xk[3]);
@@ -522,9 +522,11 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
                         *reinterpret_cast<float4 *>(sm + kSmA + f32_offset(i, 32 * hf + 4 * q)) =
                             make_float4(rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
                 } else {
-                    __nv_bfloat16 *pt = reinterpret_cast<__nv_bfloat16 *>(sm + kSmP);  // P^T: element (j, i)
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) pt[img_offset(32 * hf + t, i) / 2] = __float2bfloat16_rn(rr[t]);
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(smem_u32(sm + kSmP) + sw128_offset(i, 4 * hf + q), pack_bf16(rr[8 * q], rr[8 * q + 1]),
+                                     pack_bf16(rr[8 * q + 2], rr[8 * q + 3]), pack_bf16(rr[8 * q + 4], rr[8 * q + 5]),
+                                     pack_bf16(rr[8 * q + 6], rr[8 * q + 7]));
                 }
             }
             tc_fence_before();  // the W / U products later reuse these TMEM columns
@@ -538,10 +540,10 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     }
     __syncthreads();
 
-    // P^T image to the block; K * L -> K * Gam = K * L * exp(r_p) in place.
+    // P rows to the block; K * L -> K * Gam = K * L * exp(r_p) in place.
     if (ok) {
         for (int e = tid; e < 512; e += kThreads)
-            *reinterpret_cast<uint4 *>(rest + kRestPt + e * 16) = *reinterpret_cast<const uint4 *>(sm + kSmP + e * 16);
+            *reinterpret_cast<uint4 *>(rest + kRestP + e * 16) = *reinterpret_cast<const uint4 *>(sm + kSmP + e * 16);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int e = tid + kThreads * k;
@@ -563,13 +565,16 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     blocked_solve<kSmT, kSmY>(sm, [](int i, int j) { return kSmA + f32_offset(i, j); },
                               [](int i) { return kSmA + (uint32_t)i * 256u; }, ok);
 
-    // T'' = T diag(beta) as a bf16 operand image (K-major rows i).
+    // T'' = T diag(beta) as a bf16 operand image (K-major rows i); the blocks of T above
+    // its block diagonal are zero (the solve leaves them unwritten).
     if (ok) {
         const int i = tid >> 2, j0 = (tid & 3) * 16;
+        const bool upper = (tid & 3) > (i >> 4);
         float tv[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float4 f = *reinterpret_cast<const float4 *>(sm + kSmT + f32_offset(i, j0 + 4 * q));
+            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!upper) f = *reinterpret_cast<const float4 *>(sm + kSmT + f32_offset(i, j0 + 4 * q));
             tv[4 * q] = f.x; tv[4 * q + 1] = f.y; tv[4 * q + 2] = f.z; tv[4 * q + 3] = f.w;
         }
         const uint32_t tp = smem_u32(sm + kSmTp);

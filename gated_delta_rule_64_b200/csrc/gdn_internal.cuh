@@ -89,13 +89,15 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
 bool tc_eligible(const gdn_desc &d);
 
 // Per chunk-head workspace block of the tensor-core path (bytes), both gate kinds:
-//   [W (channels 0-63) 8K][Qs (0-63) 8K][W (64-127) 8K][Qs (64-127) 8K]
-//   [K~ 16K][P^T image 8K][U^T rows 16K][gate factors 1K]
-// W and Qs = scale Q * Gam are K-major operand images (rows = tokens) laid out
-// so that [W ; Qs] is one N = 128 operand.  K~ = K * exp(b_L - b) (the layout of
-// a K tile: rows = tokens, two 64-channel halves) followed by P^T (rows = key
-// tokens j, columns = query tokens i) is one N = 192 MN-major operand.  The scan
-// copies a block with two bulk copies.
+//   [W^T rows 16K][Qs (channels 0-63) 8K][Qs (64-127) 8K]
+//   [K~ 16K][P rows 8K][U^T rows 16K][gate factors 1K]
+// Every operand is 128-byte swizzled rows of 128 bytes (64 bf16), in 8-row groups
+// 1 KB apart.  W^T (row = key channel, 64 tokens) is the MN-major B operand of
+// S0 W^T; Qs = scale Q * Gam (per-channel gate only; row = token, the layout of a
+// Q tile) the K-major one of S0 Qs^T.  K~ = K * exp(b_L - b) (the layout of a K
+// tile: rows = tokens, two 64-channel halves) is the MN-major B operand of
+// U'^T K~; P (row = query token i, 64 key tokens j) the K-major one of U'^T P^T.
+// The scan copies a block with two bulk copies.
 constexpr size_t kTcWQ = 32768, kTcKt = 64 * 128 * 2, kTcPImg = 64 * 128, kTcUt = 128 * 128, kTcFac = 1024;
 constexpr size_t kTcRest = kTcKt + kTcPImg + kTcUt + kTcFac;  // 41984
 constexpr size_t kTcBlock = kTcWQ + kTcRest;                  // 74752

@@ -20,12 +20,13 @@ constexpr int C = kChunk;  // 64 tokens per chunk
 constexpr int D = 128;     // d_k = d_v
 constexpr int kThreads = 256;
 
-// Offsets inside one workspace block: [W ; Qs] images at 0, then the rest at
-// kBlkRest: K~, P^T image, U^T rows, gate factors.
-constexpr uint32_t kBlkRest = (uint32_t)kTcWQ;
-constexpr uint32_t kRestKt = 0, kRestPt = 16384, kRestU = 24576, kRestFac = 40960;
-static_assert(kRestPt == kTcKt && kRestU == kRestPt + kTcPImg && kRestFac == kRestU + kTcUt &&
-                  kRestFac + kTcFac == kTcRest,
+// Offsets inside one workspace block: W^T rows at 0, the Qs halves (per-channel
+// gate) at kBlkQs and kBlkQs + 8K, then the rest at kBlkRest: K~, P rows, U^T rows,
+// gate factors.
+constexpr uint32_t kBlkW = 0, kBlkQs = 16384, kBlkRest = (uint32_t)kTcWQ;
+constexpr uint32_t kRestKt = 0, kRestP = 16384, kRestU = 24576, kRestFac = 40960;
+static_assert(kBlkQs + 16384 == kTcWQ && kRestP == kTcKt && kRestU == kRestP + kTcPImg &&
+                  kRestFac == kRestU + kTcUt && kRestFac + kTcFac == kTcRest,
               "block layout");
 // Gate factors (floats): exp(b_L), at [0] for the per-head gate and per key
 // channel at [0, 128) for the per-channel gate; at [kFacLam] a bound on how much
@@ -163,23 +164,17 @@ __device__ __forceinline__ uint32_t img_offset(int row, int col) {
 // T = (I + A)^-1 for the 64 x 64 strictly lower A of a chunk, in 16 x 16 blocks.
 // A is read through `offA` (only its strictly lower part: the diagonal blocks
 // below their diagonal and the blocks below the block diagonal); T is written
-// in fp32 at byte offset TF of `sm` (f32_offset layout, upper blocks zeroed);
-// TY is 4 KB of scratch.  Diagonal blocks: forward substitution in fp32 (one
-// column per lane, two blocks per warp); off-diagonal blocks by the block
-// recurrence T_pq = -T_pp sum_{q <= r < p} A_pr T_rq with tf32 warp MMAs (the
-// first level by the warps that formed its diagonal blocks).  Every thread of
-// the block calls it (it synchronises internally).  If `pre` is given, warps 4-7
-// run it first, while warps 0-1 substitute; it may read shared memory in
-// [TF, TF + 12K) (the region of T's first 48 rows), which the solve writes only
-// after it (named barriers 1 and 2).
-struct NoPre {
-    __device__ __forceinline__ void operator()() const {}
-};
+// in fp32 at byte offset TF of `sm` (f32_offset layout), its blocks on and below
+// the block diagonal only: the blocks above it are zero and never written (the
+// readers of T skip them).  TY is 4 KB of scratch.  Diagonal blocks: forward
+// substitution in fp32 (one column per lane, two blocks per warp); off-diagonal
+// blocks by the block recurrence T_pq = -T_pp sum_{q <= r < p} A_pr T_rq with
+// tf32 warp MMAs (the first level by the warps that formed its diagonal
+// blocks).  Every thread of the block calls it (it synchronises internally).
 // rowA(i) is the byte offset of row i of A, whose element (i, j) sits at
 // rowA(i) + f32_offset(0, j) with row i's swizzle (the f32_offset layout per row).
-template <uint32_t TF, uint32_t TY, typename OffA, typename RowA, typename Pre = NoPre>
-__device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, RowA rowA, bool ok, Pre pre = Pre()) {
-    constexpr bool kPre = !std::is_same<Pre, NoPre>::value;
+template <uint32_t TF, uint32_t TY, typename OffA, typename RowA>
+__device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, RowA rowA, bool ok) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto offT = [](int i, int j) { return TF + f32_offset(i, j); };
     auto offY = [](int i, int j) { return TY + (uint32_t)i * 64u + (uint32_t)j * 4u; };  // 4 blocks, rows of 16
@@ -196,24 +191,42 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, RowA rowA,
             xv[k] = ((uint32_t)(4 * p) ^ (uint32_t)(4 * k)) << 4;
             cv[k] = ((uint32_t)(col >> 2) ^ (uint32_t)k) << 4;
         }
-        float x[16];
         if (ok) {
+            // x_i = [i == col] - sum_{j < i} A_ij x_j.  The sums are built up four
+            // columns j at a time, in increasing j as a row-by-row sum would add them:
+            // once x of a 4-column panel is known, every row below takes the panel's
+            // terms, so the chain from one x to the next is one multiply-add.
             const uint8_t *a0 = sm + rowA(16 * p);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint8_t *row = a0 + i * 256 + xv[i >> 2];
-                float acc = 0.f;
-#pragma unroll
-                for (int j = 0; j < i; ++j)
-                    acc += *reinterpret_cast<const float *>(row + ((((j >> 2) ^ (i & 3)) << 4) + (j & 3) * 4)) * x[j];
-                x[i] = (i == col) ? 1.f : -acc;
-            }
-        }
-        if (kPre) named_bar_sync(1, 192);  // warps 4-7 are done with `pre`
-        if (ok) {
             uint8_t *t0 = sm + TF + (uint32_t)(16 * p) * 256u + (uint32_t)(col & 3) * 4u;
+            auto panel = [&](int i, int J) {  // A_{i, 4J .. 4J + 3}: one 16-byte chunk of row i
+                return *reinterpret_cast<const float4 *>(a0 + i * 256 + xv[i >> 2] + ((J ^ (i & 3)) << 4));
+            };
+            float acc[16], x[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(t0 + i * 256 + xv[i >> 2] + cv[i & 3]) = x[i];
+            for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+            for (int J = 0; J < 4; ++J) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int i = 4 * J + r;
+                    if (r > 0) {
+                        const float4 a = panel(i, J);
+                        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                        for (int k = 0; k < r; ++k) acc[i] += av[k] * x[4 * J + k];
+                    }
+                    x[i] = (i == col) ? 1.f : -acc[i];
+                    *reinterpret_cast<float *>(t0 + i * 256 + xv[i >> 2] + cv[i & 3]) = x[i];
+                }
+#pragma unroll
+                for (int i = 4 * J + 4; i < 16; ++i) {
+                    const float4 a = panel(i, J);
+                    acc[i] += a.x * x[4 * J];
+                    acc[i] += a.y * x[4 * J + 1];
+                    acc[i] += a.z * x[4 * J + 2];
+                    acc[i] += a.w * x[4 * J + 3];
+                }
+            }
         }
         __syncwarp();
         // ... then level 1: T_pq = -D_p (A_pq D_q) for (p, q) = (2 warp + 1, 2 warp)
@@ -228,20 +241,6 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, RowA rowA,
             warp_gemm16(sm, 1, xr2, xc2, yr2, yc2, offT, offY, c);
             warp_store16(sm, 16 * pp, 16 * q, c, -1.f, offT);
         }
-    } else if (warp >= 4) {
-        if (kPre) {
-            if (ok) pre();
-            named_bar_sync(2, 128);    // all of warps 4-7 are done with `pre` ...
-            named_bar_arrive(1, 192);  // ... so warps 0-1 may write T
-        }
-        // zero the strictly upper off-diagonal blocks
-        if (ok)
-            for (int e = tid - 128; e < 6 * 256; e += 128) {
-                const int b = e >> 8, w = e & 255;
-                const int pb = b < 3 ? 0 : (b < 5 ? 1 : 2);
-                const int qb = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
-                *reinterpret_cast<float *>(sm + offT(16 * pb + (w >> 4), 16 * qb + (w & 15))) = 0.f;
-            }
     }
     __syncthreads();
     // level 2, step 1: Y_pq = sum_{r in {0,1}} A_pr T_rq for p in {2,3}, q in {0,1}
@@ -276,42 +275,28 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, RowA rowA,
 }
 
 // Epilogue of the W / U MMAs: TMEM columns [0, 64) hold W^T and [64, 128) U^T
-// (lane = channel, column = token).  Thread row r = qd*32 + lane writes
-// tokens [32 hf, 32 hf + 32): W as a K-major operand image (rows = tokens, two
-// 64-channel blocks), U^T as 128-byte-swizzled rows (row = channel).
+// (lane = channel, column = token).  Thread row r = qd*32 + lane writes tokens
+// [32 hf, 32 hf + 32) of its channel row of W^T and of U^T (128-byte swizzled rows).
 // (Kept out of line: inlined, they push the per-head prep kernel past its register budget.)
-static __device__ __noinline__ void store_w(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
-    const int r = qd * 32 + lane;
-    const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
-    float w0[16], w1[16];
-    tmem_ld16(taddr, w0);
-    tmem_ld16(taddr + 16, w1);
-    tmem_wait_ld();
-    uint8_t *wimg = blk + (r >> 6) * 16384 + (r & 7) * 2;
-    const int wchunk = (r & 63) >> 3;
-#pragma unroll
-    for (int t = 0; t < 32; ++t) {
-        const int i = 32 * hf + t;
-        *reinterpret_cast<__nv_bfloat16 *>(wimg + i * 128 + ((wchunk ^ (i & 7)) << 4)) =
-            __float2bfloat16_rn(t < 16 ? w0[t] : w1[t - 16]);
-    }
-}
-static __device__ __noinline__ void store_u(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
-    const int r = qd * 32 + lane;
-    const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
+static __device__ __noinline__ void store_rows(uint32_t taddr, uint8_t *dst, int r, int hf) {
     float u0[16], u1[16];
-    tmem_ld16(taddr + 64, u0);
-    tmem_ld16(taddr + 64 + 16, u1);
+    tmem_ld16(taddr, u0);
+    tmem_ld16(taddr + 16, u1);
     tmem_wait_ld();
-    uint8_t *urow = blk + kBlkRest + kRestU;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const float *u = q < 2 ? u0 + 8 * q : u1 + 8 * (q - 2);
-        *reinterpret_cast<uint4 *>(urow + sw128_offset(r, 4 * hf + q)) =
+        *reinterpret_cast<uint4 *>(dst + sw128_offset(r, 4 * hf + q)) =
             make_uint4(pack_bf16(u[0], u[1]), pack_bf16(u[2], u[3]), pack_bf16(u[4], u[5]), pack_bf16(u[6], u[7]));
     }
 }
-static __device__ __forceinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
+__device__ __forceinline__ void store_w(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
+    store_rows(tm + ((uint32_t)(qd * 32) << 16) + 32 * hf, blk + kBlkW, qd * 32 + lane, hf);
+}
+__device__ __forceinline__ void store_u(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
+    store_rows(tm + ((uint32_t)(qd * 32) << 16) + 64 + 32 * hf, blk + kBlkRest + kRestU, qd * 32 + lane, hf);
+}
+__device__ __forceinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
     store_w(tm, blk, qd, hf, lane);
     store_u(tm, blk, qd, hf, lane);
 }
