@@ -31,9 +31,11 @@
 //                registers (two threads per state row, 64 columns each); per
 //                chunk it is rounded to a bf16 A operand in TMEM and two MMA
 //                groups with fp32 accumulators in TMEM produce
-//                [S0 W^T | S0 Q^T] and, from U' = U - W S0^T, [U'^T K~ | U'^T P^T]
-//                (the state increment and the intra-chunk output).  The next
-//                chunks' blocks are prefetched (bulk copies) into three stages.
+//                [S0 W^T | S0 Q^T] and, from U' = U - W S0^T,
+//                [(diag(w) U')^T K | U'^T P^T] with w_j = exp(b_L - b_j) (the
+//                state increment and the intra-chunk output).  The next chunks'
+//                blocks are prefetched (bulk copies; Q and K tiles by TMA) into
+//                three stages.
 //                A ninth warp issues the MMAs and copies (per-head gate, no
 //                sequence split), so the eight state warps store the previous
 //                chunk's output while the MMA groups run.
@@ -87,7 +89,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     // (one barrier per commit: a waiter two phases behind could not tell them apart)
     __shared__ uint64_t bar_ld, bar_v, bar_mma, bar_w, bar_u, bar_drain;
     __shared__ uint32_t tmem_base;
-    __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C], s_w[C];
+    __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C];
     __shared__ __align__(16) float s_b2[C];  // b in log2 units
     __shared__ __align__(16) float s_f[C];   // 2^(m - b2_j), m = b2 at row 31 (the factored decay)
 
@@ -156,9 +158,9 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         s_f[tid] = ex2((s_b[31] - bi) * 1.4426950408889634f);
         s_bg[tid] = s_beta[tid] * __expf(bi);
         s_sg[tid] = in ? scale * __expf(bi) : 0.f;
-        s_w[tid] = in ? __expf(bl - bi) : 0.f;
         float *fac = reinterpret_cast<float *>(rest + kRestFac);
         fac[kFacQs + tid] = s_sg[tid];  // the scan scales its output by these (it reads Q itself)
+        fac[kFacW + tid] = in ? __expf(bl - bi) : 0.f;  // and its U' rows by these (it reads K itself)
         if (tid == 0) fac[kFacGL] = __expf(bl);
     }
     __syncthreads();
@@ -175,41 +177,12 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         }
         mma_commit_warp(&bar_mma);
     }
-    // K~ = exp(b_L - b_j) k_j: the rows of the K tile rescaled (rows >= L: zero),
-    // written to the workspace with the tile's own byte layout.  (The query side
-    // needs no image: the scan reads Q and scales its output by scale exp(b_i).)
-    // The same pass sums |k_i|^2 for the decay bound: thread (row tid / 8, 16-byte
-    // chunk tid % 8) sees rows tid / 8 and 32 + tid / 8 in both channel halves.
-    bool bad = false;  // a token of the chunk outside the decay bound's range
-    if (ok) {
-        float k2[2] = {0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int e = tid + kThreads * k;            // 16-byte chunk over both 8K blocks
-            const int qb = e >> 9, i = (e & 511) >> 3;   // block, token row
-            const uint32_t off = (uint32_t)((e & 511) << 4);
-            const uint4 kv = *reinterpret_cast<const uint4 *>(sm + qb * 16384 + off);
-            *reinterpret_cast<uint4 *>(rest + kRestKt + qb * 8192 + off) = scale8(kv, s_w[i]);
-            if (want_bound) k2[k & 1] += sum_sq8(kv);
-        }
-        if (want_bound) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                float x = k2[r];
-                x += __shfl_xor_sync(0xffffffffu, x, 1);
-                x += __shfl_xor_sync(0xffffffffu, x, 2);
-                x += __shfl_xor_sync(0xffffffffu, x, 4);
-                const int i = 32 * r + (tid >> 3);
-                bad = bad || (i < L && !(s_beta[i] >= 0.f && s_beta[i] * x <= kBetaK2Max));
-            }
-        }
-    }
-    __syncthreads();  // every thread is done reading Q before A overwrites it
     ok = ok && mbar_wait(&bar_mma, 0);
     tc_fence_after();
 
     // Epilogue 1: accumulator row r = qd*32 + lane, columns [32 hf, 32 hf + 32).
-    // Rows 0..63 (K K^T) -> A in fp32; rows 64..127 (Q K^T) -> P rows (bf16).
+    // Rows 0..63 (K K^T) -> A in fp32; rows 64..127 (Q K^T) -> P rows (bf16).  A's
+    // diagonal, which the solve never reads, holds beta_i |k_i|^2 for the decay bound.
     if (ok) {
         const int r = qd * 32 + lane;
         const uint32_t taddr = tm + ((uint32_t)(qd * 32) << 16) + 32 * hf;
@@ -241,7 +214,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int t = 4 * q + e, j = 32 * hf + t;
-                const bool keep = i < L && (is_a ? j < i : j <= i);
+                const bool keep = i < L && j <= i;
                 rr[t] = keep ? pre * dd[e] * (t < 16 ? v0[t] : v1[t - 16]) : 0.f;
             }
         }
@@ -260,9 +233,13 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         }
     }
     tc_fence_before();
-    // (and a gate above 0, outside the documented range, leaves the chunk without a bound)
-    const bool any_bad = __syncthreads_or(bad || (tid < L && !(g_in <= 0.f)));
-    if (tid == 0) reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = (!want_bound || any_bad) ? kLamNone : s_b2[L - 1];
+    __syncthreads();
+    // a token outside the decay bound's range: beta_i < 0 or beta_i |k_i|^2 > kBetaK2Max
+    bool bad = false;
+    if (want_bound && ok && (tid & 3) == 0) {
+        const int i = tid >> 2;
+        bad = i < L && !(s_beta[i] >= 0.f && *reinterpret_cast<const float *>(sm + a_offset(i, i)) <= kBetaK2Max);
+    }
 
     // Blocked solve of T = (I + A)^-1 with 16 x 16 blocks.
     uint8_t *Tf = sm + kPrepTf;
@@ -298,8 +275,11 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     }
     fence_async_smem();  // (T's region is taken over by the V tile below)
     tc_fence_before();
-    __syncthreads();
+    const bool any_bad = __syncthreads_or(bad);
     tc_fence_after();
+    // (a gate above 0, outside the documented range, also leaves the chunk without a bound)
+    if (tid == 0)
+        reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = (!want_bound || !monotone || any_bad) ? kLamNone : s_b2[L - 1];
 
     // W^T = K^T T'^T (M = d_k) now; U^T = V^T T''^T (M = d_v) once V is in; K = 64 tokens.
     bool v_issued = false;
@@ -360,16 +340,18 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
 // ===========================================================================
 // Shared memory (1024-aligned), three stages of per-chunk operands, each the
 // chunk-head's workspace block as it is (two bulk copies; with one gate per head
-// the Q tile comes from q itself, by TMA, where the block holds Qs):
+// the Q and K tiles come from q and k themselves, by TMA, where the block holds Qs
+// and K~):
 //   [0, 16K)      W^T rows: the MN-major B operand of S0 W^T (N = 64)
 //   [16K, 32K)    Q or Qs, two 64-channel halves: the K-major B operand of S0 Q^T
-//   [32K, 48K)    K~: the MN-major B operand of U'^T K~ (N = 128)
+//   [32K, 48K)    K (one gate per head) or K~: the MN-major B operand of the state
+//                 increment (N = 128)
 //   [48K, 56K)    P rows: the K-major B operand of U'^T P^T (N = 64)
 //   [56K, 72K)    U^T rows;  [72K, 73K) gate factors
 // The operands the threads produce (S0 and U' in bf16) are written to TMEM and
 // used as A operands straight from there.
-// TMEM columns: [0,128) D1 = [S0 W^T | S0 Q^T], [128,320) D2 = [U'^T K~ | U'^T P^T],
-// [320,384) S0, [384,416) U'.
+// TMEM columns: [0,128) D1 = [S0 W^T | S0 Q^T], [128,320) D2 = [increment | U'^T P^T],
+// [320,384) S0, [384,416) U', [416,448) diag(w) U' (one gate per head).
 // A tcgen05.ld waits for the MMAs in flight, so every accumulator is read once
 // the chunk's MMAs are done (the output with the state increment), and the
 // output leaves from registers while the next chunk's first MMA group runs.
@@ -377,7 +359,7 @@ constexpr uint32_t kStW = kBlkW, kStQ = kBlkQs, kStRest = kBlkRest, kStage = (ui
 static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled operands");
 constexpr int kStages = 3;
 constexpr uint32_t kScanSmem = kStages * kStage + 1024;
-constexpr uint32_t kTmD1 = 0, kTmD2 = 128, kTmAS = 320, kTmAU = 384;
+constexpr uint32_t kTmD1 = 0, kTmD2 = 128, kTmAS = 320, kTmAU = 384, kTmAUw = 416;
 
 struct ScanBars {
     uint64_t full[kStages];
@@ -433,15 +415,17 @@ constexpr int scan_threads() {
     return KDA || SPLIT ? kThreads : kThreads + 32;
 }
 #define GDN_SCAN_PARAMS                                                                                              \
-    const __grid_constant__ CUtensorMap mq, const float *h0, const int32_t *__restrict__ cu,                          \
+    const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk, const float *h0,                \
+        const int32_t *__restrict__ cu,                                                                              \
         const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk,                  \
         int64_t max_chunks, int64_t snap_stride, int64_t n_snap, const uint8_t *__restrict__ blocks,                  \
         __nv_bfloat16 *__restrict__ out, float *final_state, float *__restrict__ snaps, const ScanSplit sp, int *err
 #define GDN_SCAN_ARGS \
-    mq, h0, cu, off, N, T, rows, H, Hk, max_chunks, snap_stride, n_snap, blocks, out, final_state, snaps, sp, err
+    mq, mk, h0, cu, off, N, T, rows, H, Hk, max_chunks, snap_stride, n_snap, blocks, out, final_state, snaps, sp, err
 
 template <bool KDA, bool SPLIT>
-__device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0, const int32_t *__restrict__ cu,
+__device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorMap &mk, const float *h0,
+                                          const int32_t *__restrict__ cu,
                                           const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
                                           int64_t H, int64_t Hk, int64_t max_chunks, int64_t snap_stride,
                                           int64_t n_snap, const uint8_t *__restrict__ blocks,
@@ -570,7 +554,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
 
     constexpr int kLoader = WS ? kThreads : 128;  // lane 0 of the issuing warp, else warp 4 lane 0
     int64_t issued = 0;                           // (loader) chunks whose copies are issued
-    // (one gate per head) the Q tile of chunk c: token rows q_row0 + 64 c, query/key head hq
+    // (one gate per head) the Q and K tiles of chunk c: token rows q_row0 + 64 c, query/key head hq
     int32_t q_row0 = 0, hq = 0;
     if (!KDA && tid == kLoader) {
         q_row0 = (int32_t)(start + cb * C);
@@ -581,22 +565,29 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
         uint8_t *st = sm + stage * kStage;
         const uint8_t *blk = block_of(c);
         uint64_t *bar = &bars.full[stage];
-        if (ident) {  // a transition map reads W^T, K~ and the factors only
+        const int32_t row0 = q_row0 + (int32_t)c * C;
+        if (ident) {  // a transition map reads W^T, K~ (or K) and the factors only
             mbar_arrive_expect_tx(bar, (uint32_t)(16384 + kTcKt + kTcFac));
             bulk_load(st + kStW, blk + kBlkW, 16384u, bar);
-            bulk_load(st + kStRest + kRestKt, blk + kBlkRest + kRestKt, (uint32_t)kTcKt, bar);
+            if (KDA) {
+                bulk_load(st + kStRest + kRestKt, blk + kBlkRest + kRestKt, (uint32_t)kTcKt, bar);
+            } else {
+                tma_load_3d(st + kStRest + kRestKt, &mk, 0, hq, row0, bar);
+                tma_load_3d(st + kStRest + kRestKt + 8192, &mk, 64, hq, row0, bar);
+            }
             bulk_load(st + kStRest + kRestFac, blk + kBlkRest + kRestFac, (uint32_t)kTcFac, bar);
         } else if (KDA) {
             mbar_arrive_expect_tx(bar, kStage);
             bulk_load(st, blk, (uint32_t)kTcWQ, bar);
             bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
-        } else {  // one gate per head: the Q tile itself (the output is scaled later)
+        } else {  // one gate per head: the Q and K tiles themselves (the output and U' are scaled)
             mbar_arrive_expect_tx(bar, kStage);
-            const int32_t row0 = q_row0 + (int32_t)c * C;
             bulk_load(st + kStW, blk + kBlkW, 16384u, bar);
             tma_load_3d(st + kStQ, &mq, 0, hq, row0, bar);
             tma_load_3d(st + kStQ + 8192, &mq, 64, hq, row0, bar);
-            bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
+            tma_load_3d(st + kStRest + kRestKt, &mk, 0, hq, row0, bar);
+            tma_load_3d(st + kStRest + kRestKt + 8192, &mk, 64, hq, row0, bar);
+            bulk_load(st + kStRest + kRestP, blk + kBlkRest + kRestP, (uint32_t)(kTcRest - kTcKt), bar);
         }
         issued = c + 1;
     };
@@ -703,17 +694,19 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
         // every MMA of chunk c-1 has completed (step (e) waited for them), so its
         // stage can take chunk c+2
         if (tid == kLoader && c >= 1 && c + kStages - 1 < nrun) issue_loads(c + kStages - 1);
-        // (d) D2 = [U'^T K~ | U'^T P^T]   (N = 128 + 64, K = 64 tokens): [state increment |
-        //     intra-chunk output] (the increment only, for a chunk without outputs).  The
-        //     increment is committed on its own (the state is updated while U'^T P^T
+        // (d) D2 = [increment | U'^T P^T]   (N = 128 + 64, K = 64 tokens): [state increment |
+        //     intra-chunk output] (the increment only, for a chunk without outputs); the
+        //     increment is U'^T K~ (per-channel gate) or (diag(w) U')^T K (one gate per
+        //     head).  It is committed on its own (the state is updated while U'^T P^T
         //     runs), then every product of the chunk.
         auto issue_d2 = [&] {
             const uint64_t bk = sdesc_sw128(st_u + kStRest + kRestKt, 8192, 1024),
                            bp = sdesc_sw128(st_u + kStRest + kRestP, 16, 1024);
             const uint32_t id_k = idesc_bf16(128, 128, 0, 1), id_p = idesc_bf16(128, 64, 0, 0);
+            const uint32_t a_inc = tm + (KDA ? kTmAU : kTmAUw);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(tm + kTmD2, tm + kTmAU + kk * 8, bk + (uint64_t)((kk * 2048) >> 4), id_k, kk > 0);
+                mma_bf16_ts(tm + kTmD2, a_inc + kk * 8, bk + (uint64_t)((kk * 2048) >> 4), id_k, kk > 0);
             mma_commit_warp(&bars.mma[1]);
             if (emit)
 #pragma unroll
@@ -742,22 +735,35 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const float *h0
             tmem_ld16(tm + lane_off + kTmD1 + 32 * hf, a0);
             tmem_ld16(tm + lane_off + kTmD1 + 32 * hf + 16, a1);
             tmem_wait_ld();
-            uint32_t wu[16];
+            const float4 *w4 = reinterpret_cast<const float4 *>(fac + kFacW + 32 * hf);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int cq = 4 * hf + q;  // 16-byte chunk = tokens 8 cq .. 8 cq + 7
-                uint4 u8 = make_uint4(0u, 0u, 0u, 0u);
-                if (!ident) u8 = *reinterpret_cast<const uint4 *>(rest + kRestU + sw128_offset(v, cq));
-                const uint32_t uw32[4] = {u8.x, u8.y, u8.z, u8.w};
+            for (int hh = 0; hh < 2; ++hh) {  // tokens 32 hf + 16 hh .. + 15: 8 columns of each operand
+                uint32_t wu[8], ww[8];
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
-                    const float acc_lo = (q < 2 ? a0[8 * q + e] : a1[8 * (q - 2) + e]);
-                    const float acc_hi = (q < 2 ? a0[8 * q + e + 1] : a1[8 * (q - 2) + e + 1]);
-                    wu[4 * q + e / 2] = pack_bf16(__low2float(u2) - acc_lo, __high2float(u2) - acc_hi);
+                for (int qq = 0; qq < 2; ++qq) {
+                    const int q = 2 * hh + qq, cq = 4 * hf + q;  // 16-byte chunk = tokens 8 cq .. 8 cq + 7
+                    uint4 u8 = make_uint4(0u, 0u, 0u, 0u);
+                    if (!ident) u8 = *reinterpret_cast<const uint4 *>(rest + kRestU + sw128_offset(v, cq));
+                    const uint32_t uw32[4] = {u8.x, u8.y, u8.z, u8.w};
+                    float wt[8] = {};
+                    if (!KDA) {
+                        const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
+                        wt[0] = wa.x; wt[1] = wa.y; wt[2] = wa.z; wt[3] = wa.w;
+                        wt[4] = wb.x; wt[5] = wb.y; wt[6] = wb.z; wt[7] = wb.w;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
+                        const float acc_lo = (hh == 0 ? a0[8 * qq + e] : a1[8 * qq + e]);
+                        const float acc_hi = (hh == 0 ? a0[8 * qq + e + 1] : a1[8 * qq + e + 1]);
+                        const float lo = __low2float(u2) - acc_lo, hi = __high2float(u2) - acc_hi;
+                        wu[4 * qq + e / 2] = pack_bf16(lo, hi);
+                        if (!KDA) ww[4 * qq + e / 2] = pack_bf16(wt[e] * lo, wt[e + 1] * hi);
+                    }
                 }
+                tmem_st8u(tm + lane_off + kTmAU + 16 * hf + 8 * hh, wu);
+                if (!KDA) tmem_st8u(tm + lane_off + kTmAUw + 16 * hf + 8 * hh, ww);
             }
-            tmem_st16u(tm + lane_off + kTmAU + 16 * hf, wu);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -1064,7 +1070,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         const dim3 grid((unsigned)a.N, (unsigned)p.H);
         log_launch(p.per_channel ? "gdn_scan_kda_tc" : "gdn_scan_tc", grid, dim3(scan_block), kScanSmem);
         LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc" : "gdn_scan_tc", s);
-        kern<<<grid, scan_block, kScanSmem, s>>>(mq, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk,
+        kern<<<grid, scan_block, kScanSmem, s>>>(mq, mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk,
                                                  p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
                                                  (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, a.status);
         return check_launch("gdn_scan_tc");
@@ -1081,7 +1087,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         log_launch("gdn_scan (pass 1)", dim3((unsigned)grid1), dim3(split_block), kScanSmem);
         LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 1)" : "gdn_scan_split_tc (pass 1)", s);
-        kern<<<(unsigned)grid1, split_block, kScanSmem, s>>>(mq, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
+        kern<<<(unsigned)grid1, split_block, kScanSmem, s>>>(mq, mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
                                                              p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap,
                                                              blocks,
                                                              (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp,
@@ -1099,7 +1105,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         log_launch("gdn_scan (pass 2)", dim3((unsigned)grid2), dim3(split_block), kScanSmem);
         LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 2)" : "gdn_scan_split_tc (pass 2)", s);
-        kern<<<(unsigned)grid2, split_block, kScanSmem, s>>>(mq, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
+        kern<<<(unsigned)grid2, split_block, kScanSmem, s>>>(mq, mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
                                                              p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap,
                                                              blocks,
                                                              (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp,

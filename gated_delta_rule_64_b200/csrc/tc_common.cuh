@@ -33,8 +33,10 @@ static_assert(kBlkQs + 16384 == kTcWQ && kRestP == kTcKt && kRestU == kRestP + k
 // the chunk can shrink a state, in log2 units (below).
 constexpr int kFacGL = 0, kFacLam = 128;
 // One gate per head: scale exp(b_i) per token at [kFacQs, kFacQs + 64) (the scan
-// scales its S0 Q^T output columns by them).
-constexpr int kFacQs = 192;
+// scales its S0 Q^T output columns by them) and w_j = exp(b_L - b_j) per token at
+// [kFacW, kFacW + 64) (zero past the chunk's end): the state increment
+// U'^T (K * w) is taken as (diag(w) U')^T K, so the block holds no K~ for this gate.
+constexpr int kFacW = 64, kFacQs = 192;
 
 // Decay bound of a chunk.  One token maps a state S to S D_t (I - beta_t k_t k_t^T)
 // (+ a write that does not depend on S).  When 0 <= beta_t |k_t|^2 <= 2 the
