@@ -111,24 +111,44 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        rows = []
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 10:
-                continue
-            try:
-                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
-                rows.append((ts, float(parts[2]), float(parts[3]), parts[5:10]))
-            except ValueError:
-                continue
+        return self.summarize(parse_smi_rows(out), self.t0, self.t1)
+
+    @staticmethod
+    def summarize(rows, t0, t1):
+        """Median SM clock (and the lowest) over the samples taken inside [t0, t1]."""
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        inside = [r for r in rows if self.t0 is not None and self.t0 - 1 <= r[0] <= (self.t1 or r[0]) + 1]
+        inside = [r for r in rows if t0 is not None and t0 <= r[0] <= (t1 if t1 is not None else r[0])]
+        if not inside and t0 is not None:  # a region shorter than the sampling period
+            inside = [r for r in rows if t0 - 0.2 <= r[0] <= (t1 if t1 is not None else t0) + 0.2]
         use = inside or rows
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in use for i, v in enumerate(r[3][1:]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_min_mhz": min(r[1] for r in use),
+                "sm_max_mhz": max(r[2] for r in use),
+                "power_w_max": max((r[4] for r in use if r[4] == r[4]), default=None),
                 "reasons": reasons, "samples": len(use)}
+
+
+def parse_smi_rows(text):
+    """(time, clocks.sm, clocks.max.sm, reason flags, power.draw) per line of the sampler's output;
+    the timestamp keeps its milliseconds."""
+    rows = []
+    for line in text.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 10:
+            continue
+        try:
+            whole, _, frac = parts[0].partition(".")
+            ts = time.mktime(time.strptime(whole, "%Y/%m/%d %H:%M:%S")) + (float("0." + frac) if frac.isdigit() else 0.0)
+            try:
+                power = float(parts[4])
+            except ValueError:  # "[N/A]"
+                power = float("nan")
+            rows.append((ts, float(parts[2]), float(parts[3]), parts[5:10], power))
+        except ValueError:
+            continue
+    return rows
 
 
 # ---------------------------------------------------------------------------

@@ -89,7 +89,8 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     // (one barrier per commit: a waiter two phases behind could not tell them apart)
     __shared__ uint64_t bar_ld, bar_v, bar_mma, bar_w, bar_u, bar_drain;
     __shared__ uint32_t tmem_base;
-    __shared__ float s_b[C], s_beta[C], s_bg[C], s_sg[C];
+    __shared__ float s_b[C], s_sg[C];
+    __shared__ __align__(16) float s_beta[C], s_bg[C];
     __shared__ __align__(16) float s_b2[C];  // b in log2 units
     __shared__ __align__(16) float s_f[C];   // 2^(m - b2_j), m = b2 at row 31 (the factored decay)
 
@@ -200,22 +201,28 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         const float bi2 = s_b2[i];
         const bool fact = monotone && s_b2[0] - s_b2[C - 1] <= 120.f;  // uniform over the block
         const float ei = fact ? ex2(bi2 - s_b2[31]) : 0.f;
+        // (in pairs: fp32 x2 multiplies)
+        const float2 pe = make_float2(pre * ei, pre * ei);
         float rr[32];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            float dd[4];
+            float2 d01, d23;  // pre exp(b_i - b_j) for the 4 columns j
             if (fact) {
                 const float4 f4 = *reinterpret_cast<const float4 *>(s_f + 32 * hf + 4 * q);
-                dd[0] = ei * f4.x; dd[1] = ei * f4.y; dd[2] = ei * f4.z; dd[3] = ei * f4.w;
+                d01 = __fmul2_rn(pe, make_float2(f4.x, f4.y));
+                d23 = __fmul2_rn(pe, make_float2(f4.z, f4.w));
             } else {
                 const float4 b4 = *reinterpret_cast<const float4 *>(s_b2 + 32 * hf + 4 * q);
-                dd[0] = ex2(bi2 - b4.x); dd[1] = ex2(bi2 - b4.y); dd[2] = ex2(bi2 - b4.z); dd[3] = ex2(bi2 - b4.w);
+                d01 = make_float2(pre * ex2(bi2 - b4.x), pre * ex2(bi2 - b4.y));
+                d23 = make_float2(pre * ex2(bi2 - b4.z), pre * ex2(bi2 - b4.w));
             }
+            const float *vv = q < 4 ? &v0[4 * q] : &v1[4 * (q - 4)];
+            const float2 r01 = __fmul2_rn(d01, make_float2(vv[0], vv[1])), r23 = __fmul2_rn(d23, make_float2(vv[2], vv[3]));
+            const float r4[4] = {r01.x, r01.y, r23.x, r23.y};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int t = 4 * q + e, j = 32 * hf + t;
-                const bool keep = i < L && j <= i;
-                rr[t] = keep ? pre * dd[e] * (t < 16 ? v0[t] : v1[t - 16]) : 0.f;
+                rr[t] = i < L && j <= i ? r4[e] : 0.f;
             }
         }
         if (is_a) {
@@ -259,18 +266,24 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
             tv[4 * q] = f.x; tv[4 * q + 1] = f.y; tv[4 * q + 2] = f.z; tv[4 * q + 3] = f.w;
         }
         const uint32_t tp = smem_u32(sm + 8192), tpp = smem_u32(sm + 24576);
+        const float4 *bg4 = reinterpret_cast<const float4 *>(s_bg + j0), *be4 = reinterpret_cast<const float4 *>(s_beta + j0);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            float a[8], b[8];
+            uint32_t a[4], b[4];  // packed bf16 pairs (fp32 x2 multiplies)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int j = j0 + 8 * q + e;
-                a[e] = tv[8 * q + e] * s_bg[j];
-                b[e] = tv[8 * q + e] * s_beta[j];
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const float4 g4 = bg4[2 * q + h2], e4 = be4[2 * q + h2];
+                const float *t4 = &tv[8 * q + 4 * h2];
+                const float2 a01 = __fmul2_rn(make_float2(t4[0], t4[1]), make_float2(g4.x, g4.y));
+                const float2 a23 = __fmul2_rn(make_float2(t4[2], t4[3]), make_float2(g4.z, g4.w));
+                const float2 b01 = __fmul2_rn(make_float2(t4[0], t4[1]), make_float2(e4.x, e4.y));
+                const float2 b23 = __fmul2_rn(make_float2(t4[2], t4[3]), make_float2(e4.z, e4.w));
+                a[2 * h2] = pack_bf16(a01.x, a01.y); a[2 * h2 + 1] = pack_bf16(a23.x, a23.y);
+                b[2 * h2] = pack_bf16(b01.x, b01.y); b[2 * h2 + 1] = pack_bf16(b23.x, b23.y);
             }
             const uint32_t o = sw128_offset(i, (j0 >> 3) + q);
-            st_shared_v4(tp + o, pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
-            st_shared_v4(tpp + o, pack_bf16(b[0], b[1]), pack_bf16(b[2], b[3]), pack_bf16(b[4], b[5]), pack_bf16(b[6], b[7]));
+            st_shared_v4(tp + o, a[0], a[1], a[2], a[3]);
+            st_shared_v4(tpp + o, b[0], b[1], b[2], b[3]);
         }
     }
     fence_async_smem();  // (T's region is taken over by the V tile below)
@@ -404,16 +417,8 @@ __device__ __forceinline__ int32_t *split_rec(const ScanSplit &sp, int which, in
 }
 
 // SPLIT: launched as a pass of the split scan (1-D grid; the block's work comes from `sp`).
-// Per-head gate, unsplit: kThreads + 32 threads; warps 0-7 hold the state and warp 8
-// issues the MMAs and the copies, so the state warps spend the MMA groups storing the
-// previous chunk's output.  A ninth warp puts three warps on one SM sub-partition,
-// which caps a thread at 168 registers (gdn_scan_tc).  The split and per-channel
-// scans need more, so there warp 0 issues the MMAs and warp 4 the copies
-// (gdn_scan_split_tc, gdn_scan_kda_tc).
-template <bool KDA, bool SPLIT>
-constexpr int scan_threads() {
-    return KDA || SPLIT ? kThreads : kThreads + 32;
-}
+// Eight warps hold the state (two threads per row, 64 columns each); warp 0 also
+// issues the MMAs and warp 4 the copies.
 #define GDN_SCAN_PARAMS                                                                                              \
     const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk, const float *h0,                \
         const int32_t *__restrict__ cu,                                                                              \
@@ -435,7 +440,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
     uint8_t *sm = align1024(smem_raw);
     __shared__ ScanBars bars;
     __shared__ uint32_t tmem_base;
-    __shared__ float s_red[scan_threads<KDA, SPLIT>() / 32];
+    __shared__ float s_red[kThreads / 32];
     // Packed batches: blocks in launch order take the sequences longest first (the
     // order the chunk table wrote after the chunk offsets), all heads of one
     // sequence after another, so the long sequences start in the first wave.
@@ -449,9 +454,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, hf = warp >> 2;
     const int v = qd * 32 + lane;  // state row; this thread holds columns [64 hf, 64 hf + 64)
-    constexpr bool WS = scan_threads<KDA, SPLIT>() > kThreads;  // a warp of its own issues the MMAs and copies
-    constexpr int kIssuer = WS ? kThreads / 32 : 0;
-    const bool holds_rows = !WS || tid < kThreads;  // this thread holds part of the state
+    constexpr int kIssuer = 0, kLoader = 128;  // warp 0 issues the MMAs, warp 4 lane 0 the copies
 
     // This block's work: sequence n, chunks [cb, cb + nchunks) of it (a segment of the
     // split scan), its start state and where its end state goes.
@@ -552,8 +555,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
     const uint32_t tm = tmem_base;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
 
-    constexpr int kLoader = WS ? kThreads : 128;  // lane 0 of the issuing warp, else warp 4 lane 0
-    int64_t issued = 0;                           // (loader) chunks whose copies are issued
+    int64_t issued = 0;  // (loader) chunks whose copies are issued
     // (one gate per head) the Q and K tiles of chunk c: token rows q_row0 + 64 c, query/key head hq
     int32_t q_row0 = 0, hq = 0;
     if (!KDA && tid == kLoader) {
@@ -596,10 +598,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
 
     float S[64];
     const int64_t srow = (int64_t)v * D + 64 * hf;  // this thread's part of a state
-    if (!holds_rows) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) S[c] = 0.f;
-    } else if (start_kind == kStartGiven && s_init) {
+    if (start_kind == kStartGiven && s_init) {
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
             const float4 t = *reinterpret_cast<const float4 *>(s_init + srow + c);
@@ -616,19 +615,19 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
     auto store_output = [&](int64_t c, int half) {
         const int64_t ca = cb + c;
         const int L = (int)(len - ca * C < C ? len - ca * C : C);
-        // 4 x 4 transposes among the quads of lanes (4 adjacent channels): afterwards
-        // lane j of a quad holds those 4 channels of token 4 b + j -> one 8-byte store.
+        // 4 x 4 transposes (bf16) among the quads of lanes (4 adjacent channels):
+        // afterwards lane j of a quad holds those 4 channels of token 4 b + j -> one
+        // 8-byte store.
         const int j4 = lane & 3;
         const int64_t tstride = H * D;
         __nv_bfloat16 *op = out + ((start + ca * C + 32 * hf + j4) * H + h) * D + (v - j4);
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
             const int b = 4 * half + bb;
-            float x0 = o[b >> 2][4 * (b & 3)], x1 = o[b >> 2][4 * (b & 3) + 1], x2 = o[b >> 2][4 * (b & 3) + 2],
-                  x3 = o[b >> 2][4 * (b & 3) + 3];
-            quad_transpose(x0, x1, x2, x3, lane);
-            if (32 * hf + 4 * b + j4 < L)
-                *reinterpret_cast<uint2 *>(op + (int64_t)(4 * b) * tstride) = make_uint2(pack_bf16(x0, x1), pack_bf16(x2, x3));
+            const float *x = &o[b >> 2][4 * (b & 3)];
+            uint32_t p01 = pack_bf16(x[0], x[1]), p23 = pack_bf16(x[2], x[3]);
+            quad_transpose_bf16(p01, p23, lane);
+            if (32 * hf + 4 * b + j4 < L) *reinterpret_cast<uint2 *>(op + (int64_t)(4 * b) * tstride) = make_uint2(p01, p23);
         }
     };
 
@@ -648,7 +647,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
         const float *fac = reinterpret_cast<const float *>(rest + kRestFac);
 
         // (a) S0 -> bf16 pairs -> TMEM A operand (this thread: 32 columns of its row)
-        if (holds_rows) {
+        {
             uint32_t w[16];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -660,14 +659,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
         }
         ok = mbar_wait(&bars.full[stage], (uint32_t)((c / kStages) & 1)) && ok;
         tc_fence_before();
-        if (WS) {
-            if (__syncthreads_or(!ok)) {  // a wait gave up: every thread leaves as failed
-                ok = false;
-                break;
-            }
-        } else {
-            __syncthreads();
-        }
+        __syncthreads();
         tc_fence_after();
         // does this chunk write outputs, and its snapshot?
         const float lam_next = lam + fac[kFacLam];
@@ -714,15 +706,6 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
                     mma_bf16_ts(tm + kTmD2 + 128, tm + kTmAU + kk * 8, bp + (uint64_t)((kk * 32) >> 4), id_p, kk > 0);
             mma_commit_warp(&bars.mma[2]);
         };
-        if (WS && warp == kIssuer) {
-            // (d) once every row's U' is in TMEM (named barrier 1)
-            named_bar_sync(1, kThreads + 32);
-            tc_fence_after();
-            issue_d2();
-            lam = lam_next;
-            emit_prev = emit;
-            continue;
-        }
         // the first half of the previous chunk's output, while these MMAs run
         if (c >= 1 && emit_prev) store_output(c - 1, 0);
 
@@ -754,11 +737,15 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
                         const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
-                        const float acc_lo = (hh == 0 ? a0[8 * qq + e] : a1[8 * qq + e]);
-                        const float acc_hi = (hh == 0 ? a0[8 * qq + e + 1] : a1[8 * qq + e + 1]);
-                        const float lo = __low2float(u2) - acc_lo, hi = __high2float(u2) - acc_hi;
-                        wu[4 * qq + e / 2] = pack_bf16(lo, hi);
-                        if (!KDA) ww[4 * qq + e / 2] = pack_bf16(wt[e] * lo, wt[e + 1] * hi);
+                        const float *acc = hh == 0 ? &a0[8 * qq + e] : &a1[8 * qq + e];
+                        // u - acc (one rounding, as the subtraction), then w (u - acc)
+                        const float2 d = __ffma2_rn(make_float2(acc[0], acc[1]), make_float2(-1.f, -1.f),
+                                                    make_float2(__low2float(u2), __high2float(u2)));
+                        wu[4 * qq + e / 2] = pack_bf16(d.x, d.y);
+                        if (!KDA) {
+                            const float2 dw = __fmul2_rn(make_float2(wt[e], wt[e + 1]), d);
+                            ww[4 * qq + e / 2] = pack_bf16(dw.x, dw.y);
+                        }
                     }
                 }
                 tmem_st8u(tm + lane_off + kTmAU + 16 * hf + 8 * hh, wu);
@@ -767,15 +754,11 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
             tmem_wait_st();
         }
         tc_fence_before();
-        if (WS) {
-            named_bar_arrive(1, kThreads + 32);  // the issuing warp waits for these
-        } else {
-            __syncthreads();
-            tc_fence_after();
-        }
+        __syncthreads();
+        tc_fence_after();
 
         // (d)
-        if (!WS && warp == 0) issue_d2();
+        if (warp == kIssuer) issue_d2();
 
         // the second half of the previous chunk's output, while these MMAs run
         if (c >= 1 && emit_prev) store_output(c - 1, 1);
@@ -796,16 +779,24 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
 #pragma unroll
                 for (int c4 = 0; c4 < 16; ++c4) {
                     const float4 f = gl4[c4];
-                    S[4 * c4] = f.x * S[4 * c4] + a[c4 >> 2][(4 * c4) & 15];
-                    S[4 * c4 + 1] = f.y * S[4 * c4 + 1] + a[c4 >> 2][(4 * c4 + 1) & 15];
-                    S[4 * c4 + 2] = f.z * S[4 * c4 + 2] + a[c4 >> 2][(4 * c4 + 2) & 15];
-                    S[4 * c4 + 3] = f.w * S[4 * c4 + 3] + a[c4 >> 2][(4 * c4 + 3) & 15];
+                    const float *ai = &a[c4 >> 2][(4 * c4) & 15];
+                    const float2 s01 = __ffma2_rn(make_float2(f.x, f.y), make_float2(S[4 * c4], S[4 * c4 + 1]),
+                                                  make_float2(ai[0], ai[1]));
+                    const float2 s23 = __ffma2_rn(make_float2(f.z, f.w), make_float2(S[4 * c4 + 2], S[4 * c4 + 3]),
+                                                  make_float2(ai[2], ai[3]));
+                    S[4 * c4] = s01.x; S[4 * c4 + 1] = s01.y; S[4 * c4 + 2] = s23.x; S[4 * c4 + 3] = s23.y;
                 }
             } else {
+                const float2 gl2 = make_float2(gl, gl);
 #pragma unroll
                 for (int c0 = 0; c0 < 4; ++c0)
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) S[16 * c0 + t] = gl * S[16 * c0 + t] + a[c0][t];
+                    for (int t = 0; t < 16; t += 2) {
+                        const float2 r = __ffma2_rn(gl2, make_float2(S[16 * c0 + t], S[16 * c0 + t + 1]),
+                                                    make_float2(a[c0][t], a[c0][t + 1]));
+                        S[16 * c0 + t] = r.x;
+                        S[16 * c0 + t + 1] = r.y;
+                    }
             }
         }
         ok = mbar_wait(&bars.mma[2], par) && ok;
@@ -824,7 +815,11 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
 #pragma unroll
                 for (int q = 0; q < 2; ++q)
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) o[q][t] += o2[q][t];
+                    for (int t = 0; t < 16; t += 2) {
+                        const float2 r = __fadd2_rn(make_float2(o[q][t], o[q][t + 1]), make_float2(o2[q][t], o2[q][t + 1]));
+                        o[q][t] = r.x;
+                        o[q][t + 1] = r.y;
+                    }
             } else {  // S0 Q^T scaled per token by scale exp(b_i)
                 const float4 *sg4 = reinterpret_cast<const float4 *>(fac + kFacQs + 32 * hf);
 #pragma unroll
@@ -832,10 +827,11 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
 #pragma unroll
                     for (int t4 = 0; t4 < 4; ++t4) {
                         const float4 f = sg4[4 * q + t4];
-                        o[q][4 * t4] = fmaf(o[q][4 * t4], f.x, o2[q][4 * t4]);
-                        o[q][4 * t4 + 1] = fmaf(o[q][4 * t4 + 1], f.y, o2[q][4 * t4 + 1]);
-                        o[q][4 * t4 + 2] = fmaf(o[q][4 * t4 + 2], f.z, o2[q][4 * t4 + 2]);
-                        o[q][4 * t4 + 3] = fmaf(o[q][4 * t4 + 3], f.w, o2[q][4 * t4 + 3]);
+                        float *ot = &o[q][4 * t4];
+                        const float *o2t = &o2[q][4 * t4];
+                        const float2 r01 = __ffma2_rn(make_float2(ot[0], ot[1]), make_float2(f.x, f.y), make_float2(o2t[0], o2t[1]));
+                        const float2 r23 = __ffma2_rn(make_float2(ot[2], ot[3]), make_float2(f.z, f.w), make_float2(o2t[2], o2t[3]));
+                        ot[0] = r01.x; ot[1] = r01.y; ot[2] = r23.x; ot[3] = r23.y;
                     }
             }
         }
@@ -852,13 +848,12 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
         }
         lam = lam_next;
         emit_prev = emit;
-        if (!WS && __syncthreads_or(!ok)) {  // a wait gave up: every thread leaves as failed
+        if (__syncthreads_or(!ok)) {  // a wait gave up: every thread leaves as failed
             ok = false;
             break;
         }
     }
-    if (WS) ok = !__syncthreads_or(!ok);  // the last chunk's waits
-    if (ok && nrun > 0 && emit_prev && holds_rows) {
+    if (ok && nrun > 0 && emit_prev) {
         store_output(nrun - 1, 0);
         store_output(nrun - 1, 1);
     }
@@ -880,7 +875,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
         if (ok && tid == 0) *split_rec(sp, 0, N, n, g, H, h) = (int32_t)(exact_end ? m_first : nchunks);
         if (exact_end && g == sp.G - 1 && final_state) s_end2 = final_state + sh;
     }
-    if (ok && holds_rows) {
+    if (ok) {
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
             float *dst = k ? s_end2 : s_end;
@@ -895,7 +890,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
     if (warp == 0) tmem_dealloc(tm, 512);
 }
 
-__global__ void __maxnreg__(168) gdn_scan_tc(GDN_SCAN_PARAMS) { scan_body<false, false>(GDN_SCAN_ARGS); }
+__global__ void __launch_bounds__(kThreads, 1) gdn_scan_tc(GDN_SCAN_PARAMS) { scan_body<false, false>(GDN_SCAN_ARGS); }
 __global__ void __launch_bounds__(kThreads, 1) gdn_scan_split_tc(GDN_SCAN_PARAMS) { scan_body<false, true>(GDN_SCAN_ARGS); }
 template <bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) gdn_scan_kda_tc(GDN_SCAN_PARAMS) { scan_body<true, SPLIT>(GDN_SCAN_ARGS); }
@@ -1063,7 +1058,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         }
     }
     ScanSplit sp{1, 0, 0, nullptr, nullptr};
-    const int scan_block = p.per_channel ? scan_threads<true, false>() : scan_threads<false, false>();
+    const int scan_block = kThreads;
     if (p.split_G < 2) {
         if (a.N * p.H > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "grid too large");
         auto kern = p.per_channel ? gdn_scan_kda_tc<false> : gdn_scan_tc;
@@ -1077,7 +1072,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     }
     // sequence split: pass 1 (every segment, then the transition maps), the chained
     // start states (G >= 3), pass 2 (the leading chunks of segments 1 .. G-1)
-    const int split_block = p.per_channel ? scan_threads<true, true>() : scan_threads<false, true>();
+    const int split_block = kThreads;
     auto kern = p.per_channel ? gdn_scan_kda_tc<true> : gdn_scan_split_tc;
     float *states = reinterpret_cast<float *>(a.ws + p.off_split);
     sp = ScanSplit{p.split_G, p.split_seg, 1, states,

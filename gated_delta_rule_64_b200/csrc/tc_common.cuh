@@ -114,22 +114,19 @@ __device__ __forceinline__ void warp_store16(uint8_t *base, int r0, int c0, cons
     }
 }
 
-// 4 x 4 transpose among the 4 lanes of a quad: lane j of the quad holds x[0..3]
-// = element (row r_j, columns c .. c+3) before, and (rows r_0 .. r_3, column
-// c + j) after (r_j = the quad's j-th lane's row).
-__device__ __forceinline__ void quad_transpose(float &x0, float &x1, float &x2, float &x3, int lane) {
-    {
-        const bool hi = lane & 1;
-        const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x1, 1);
-        const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x2 : x3, 1);
-        if (hi) { x0 = r0; x2 = r1; } else { x1 = r0; x3 = r1; }
-    }
-    {
-        const bool hi = lane & 2;
-        const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x2, 2);
-        const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x1 : x3, 2);
-        if (hi) { x0 = r0; x1 = r1; } else { x2 = r0; x3 = r1; }
-    }
+// 4 x 4 transpose of bf16 values among the 4 lanes of a quad: lane j holds row j as
+// two packed pairs, p01 = (x_j0, x_j1) and p23 = (x_j2, x_j3) (low half first);
+// afterwards p01 = (x_0j, x_1j), p23 = (x_2j, x_3j).  Two exchanges: 32-bit words
+// across lanes j ^ 2, then 16-bit halves across lanes j ^ 1 (byte permutes).
+__device__ __forceinline__ void quad_transpose_bf16(uint32_t &p01, uint32_t &p23, int lane) {
+    const bool b1 = lane & 2, b0 = lane & 1;
+    // lanes 0, 1 keep their columns 0-1 and take those of row j + 2; lanes 2, 3 the reverse
+    const uint32_t r = __shfl_xor_sync(0xffffffffu, b1 ? p01 : p23, 2);
+    const uint32_t A = b1 ? r : p01, B = b1 ? p23 : r;  // rows {j&1, (j&1) + 2}, columns 2 b1 + {0, 1}
+    // even lanes keep column 2 b1 and send the other; odd lanes the reverse
+    const uint32_t R = __shfl_xor_sync(0xffffffffu, __byte_perm(A, B, b0 ? 0x5410u : 0x7632u), 1);
+    p01 = __byte_perm(A, R, b0 ? 0x3254u : 0x5410u);
+    p23 = __byte_perm(B, R, b0 ? 0x3276u : 0x7610u);
 }
 
 // Eight bf16 values (one 16-byte chunk) times f, rounded back to bf16.

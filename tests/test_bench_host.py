@@ -1,5 +1,6 @@
 """Host logic of bench.py (CPU): the recorded ncu traffic of a kernel is reported
-only while the kernel's source text and the files it depends on are unchanged."""
+only while the kernel's source text and the files it depends on are unchanged; the
+SM clock record covers the timed region only."""
 import hashlib
 import importlib.util
 import json
@@ -96,3 +97,18 @@ def test_algorithmic_work_of_the_headline_workload(bench):
     state = 128 * 128 * 4
     assert nbytes == T * H * (4 * 128 * 2 + 8) + (1 + T // 256) * H * state
     assert flops == T * H * (10 * 64 * 128 + 6 * 128 * 128 + 2 * 64 * 64 / 3)
+
+
+def test_clock_samples_keep_milliseconds_and_stay_inside_the_timed_region(bench):
+    text = "\n".join([
+        "2026/12/02 22:20:00.100, 0, 1965, 1965, 250.0, Not Active, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/02 22:20:00.500, 0, 1800, 1965, 700.0, Active, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 22:20:00.600, 0, 1700, 1965, [N/A], Active, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 22:20:00.900, 0, 1965, 1965, 260.0, Not Active, Not Active, Not Active, Not Active, Not Active",
+    ])
+    rows = bench.parse_smi_rows(text)
+    assert len(rows) == 4 and abs((rows[1][0] - rows[0][0]) - 0.4) < 1e-6
+    t0 = rows[0][0] + 0.3
+    out = bench.ClockSampler.summarize(rows, t0, t0 + 0.4)
+    assert out["samples"] == 2 and out["sm_mhz"] == 1750 and out["sm_min_mhz"] == 1700
+    assert out["reasons"] == ["sw_power_cap"] and out["power_w_max"] == 700.0
