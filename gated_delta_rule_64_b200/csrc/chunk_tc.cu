@@ -636,6 +636,10 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
     float lam = 0.f;
     int64_t m_first = nchunks;
     bool emit_prev = false;  // chunk c - 1 has an output to store
+    // chunks until the next snapshot, and its index (snapshot strides are multiples of C)
+    const int32_t kc = snap_stride > 0 ? (int32_t)(snap_stride / C) : 0;
+    int32_t snap_left = kc > 0 ? kc - (int32_t)(cb % kc) : 0;
+    int64_t snap_idx = kc > 0 ? cb / kc : 0;
     bool ok = true;
     int64_t c = 0;
     for (; c < nrun; ++c) {
@@ -836,15 +840,17 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
             }
         }
 
-        // snapshot after n * stride tokens of the sequence
-        if (emit_state && snaps && snap_stride > 0 && ((cb + c + 1) * C) % snap_stride == 0 && (cb + c + 1) * C <= len) {
-            const int64_t s = (cb + c + 1) * C / snap_stride - 1;
-            if (s < n_snap) {
-                float *dst = snaps + (((n * n_snap + s) * H + h) * D + v) * (int64_t)D + 64 * hf;
+        // snapshot after every snap_stride tokens of the sequence (a multiple of the
+        // chunk): snapshot snap_idx follows chunk (snap_idx + 1) kc - 1 of the sequence
+        if (kc > 0 && --snap_left == 0) {
+            snap_left = kc;
+            if (emit_state && snaps && snap_idx < n_snap) {
+                float *dst = snaps + (((n * n_snap + snap_idx) * H + h) * D + v) * (int64_t)D + 64 * hf;
 #pragma unroll
                 for (int cc = 0; cc < 64; cc += 4)
                     *reinterpret_cast<float4 *>(dst + cc) = make_float4(S[cc], S[cc + 1], S[cc + 2], S[cc + 3]);
             }
+            ++snap_idx;
         }
         lam = lam_next;
         emit_prev = emit;
