@@ -63,15 +63,14 @@ using namespace tc;
 //   [0, 32K)    K and Q tiles stacked as the M = 128 operand of the first MMA:
 //               [c-block 0: K rows | Q rows][c-block 1: K rows | Q rows].
 //               After that MMA the Q rows hold A (fp32; rows 0-31 | 32-63),
-//               then T diag(beta gam) at [8K,16K) and T diag(beta) at [24K,32K)
-//               (bf16 operand images).
-//   [32K, 48K)  T (fp32), then the V tile: V is prefetched into L2 at the start
-//               and loaded here once T has become the bf16 images above
+//               then T diag(beta gam) at [8K,16K) (the bf16 operand image of W)
+//   [32K, 48K)  T (fp32)
 //   [48K, 52K)  per-warp 16 x 16 scratch of the blocked solve
-// The results (W^T rows, K~, P rows, U^T rows, gate factors) are written straight
-// to the workspace block of the chunk-head.  About 54 KB of shared memory and 64
+// The results (W^T rows, P rows, -T'' rows, gate factors) are written straight to
+// the workspace block of the chunk-head; U = T'' V is not formed here (the scan
+// accumulates V^T (-T'')^T onto S0 W^T).  About 54 KB of shared memory and 64
 // registers a thread let four blocks share an SM.
-constexpr uint32_t kPrepTf = 32768, kPrepV = 32768, kPrepY = 49152;
+constexpr uint32_t kPrepTf = 32768, kPrepY = 49152;
 constexpr uint32_t kPrepSmem = kPrepY + 4096 + 1024;
 
 __device__ __forceinline__ uint32_t a_offset(int i, int j) {
@@ -81,13 +80,13 @@ __device__ __forceinline__ uint32_t a_offset(int i, int j) {
 
 __global__ void __launch_bounds__(kThreads, 4)
 gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-            const __grid_constant__ CUtensorMap mv, const float *__restrict__ g, const float *__restrict__ beta,
+            const float *__restrict__ g, const float *__restrict__ beta,
             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
             int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks, int want_bound, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     // (one barrier per commit: a waiter two phases behind could not tell them apart)
-    __shared__ uint64_t bar_ld, bar_v, bar_mma, bar_w, bar_u, bar_drain;
+    __shared__ uint64_t bar_ld, bar_mma, bar_w, bar_drain;
     __shared__ uint32_t tmem_base;
     __shared__ float s_b[C], s_sg[C];
     __shared__ __align__(16) float s_beta[C], s_bg[C];
@@ -114,10 +113,8 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     }
     if (tid == 0) {  // the tile loads first: their latency overlaps the rest of the set-up
         mbar_init(&bar_ld, 1);
-        mbar_init(&bar_v, 1);
         mbar_init(&bar_mma, 1);
         mbar_init(&bar_w, 1);
-        mbar_init(&bar_u, 1);
         mbar_init(&bar_drain, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(&bar_ld, 4 * 8192);
@@ -126,11 +123,9 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         tma_load_3d(sm + 16384, &mk, 64, hq, tok0, &bar_ld);
         tma_load_3d(sm + 8192, &mq, 0, hq, tok0, &bar_ld);
         tma_load_3d(sm + 24576, &mq, 64, hq, tok0, &bar_ld);
-        tma_prefetch_3d(&mv, 0, (int32_t)h, tok0);  // loaded after the solve
-        tma_prefetch_3d(&mv, 64, (int32_t)h, tok0);
     }
     if (warp == 0) {
-        tmem_alloc(&tmem_base, 128);
+        tmem_alloc(&tmem_base, 64);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -253,8 +248,9 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     blocked_solve<kPrepTf, kPrepY>(sm, [](int i, int j) { return a_offset(i, j); },
                                    [](int i) { return (i < 32 ? 8192u : 24576u) + (uint32_t)(i & 31) * 256u; }, ok);
 
-    // T' = T diag(beta gam), T'' = T diag(beta) as bf16 operand images (K-major rows i);
-    // the blocks of T above its block diagonal are zero (the solve leaves them unwritten).
+    // T' = T diag(beta gam) as the bf16 operand image of W (K-major rows i, shared
+    // memory) and -T'' = -T diag(beta) as rows of the block (the scan's operand); the
+    // blocks of T above its block diagonal are zero (the solve leaves them unwritten).
     if (ok) {
         const int i = tid >> 2, j0 = (tid & 3) * 16;
         const bool upper = (tid & 3) > (i >> 4);
@@ -265,7 +261,7 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
             if (!upper) f = *reinterpret_cast<const float4 *>(Tf + f32_offset(i, j0 + 4 * q));
             tv[4 * q] = f.x; tv[4 * q + 1] = f.y; tv[4 * q + 2] = f.z; tv[4 * q + 3] = f.w;
         }
-        const uint32_t tp = smem_u32(sm + 8192), tpp = smem_u32(sm + 24576);
+        const uint32_t tp = smem_u32(sm + 8192);
         const float4 *bg4 = reinterpret_cast<const float4 *>(s_bg + j0), *be4 = reinterpret_cast<const float4 *>(s_beta + j0);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -276,17 +272,17 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
                 const float *t4 = &tv[8 * q + 4 * h2];
                 const float2 a01 = __fmul2_rn(make_float2(t4[0], t4[1]), make_float2(g4.x, g4.y));
                 const float2 a23 = __fmul2_rn(make_float2(t4[2], t4[3]), make_float2(g4.z, g4.w));
-                const float2 b01 = __fmul2_rn(make_float2(t4[0], t4[1]), make_float2(e4.x, e4.y));
-                const float2 b23 = __fmul2_rn(make_float2(t4[2], t4[3]), make_float2(e4.z, e4.w));
+                const float2 b01 = __fmul2_rn(make_float2(t4[0], t4[1]), make_float2(-e4.x, -e4.y));
+                const float2 b23 = __fmul2_rn(make_float2(t4[2], t4[3]), make_float2(-e4.z, -e4.w));
                 a[2 * h2] = pack_bf16(a01.x, a01.y); a[2 * h2 + 1] = pack_bf16(a23.x, a23.y);
                 b[2 * h2] = pack_bf16(b01.x, b01.y); b[2 * h2 + 1] = pack_bf16(b23.x, b23.y);
             }
             const uint32_t o = sw128_offset(i, (j0 >> 3) + q);
             st_shared_v4(tp + o, a[0], a[1], a[2], a[3]);
-            st_shared_v4(tpp + o, b[0], b[1], b[2], b[3]);
+            *reinterpret_cast<uint4 *>(rest + kRestTn + o) = make_uint4(b[0], b[1], b[2], b[3]);
         }
     }
-    fence_async_smem();  // (T's region is taken over by the V tile below)
+    fence_async_smem();  // (T' is read by the tensor core)
     tc_fence_before();
     const bool any_bad = __syncthreads_or(bad);
     tc_fence_after();
@@ -294,42 +290,20 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     if (tid == 0)
         reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = (!want_bound || !monotone || any_bad) ? kLamNone : s_b2[L - 1];
 
-    // W^T = K^T T'^T (M = d_k) now; U^T = V^T T''^T (M = d_v) once V is in; K = 64 tokens.
-    bool v_issued = false;
-    if (tid == 0 && ok) {
-        mbar_arrive_expect_tx(&bar_v, 2 * 8192);
-        tma_load_3d(sm + kPrepV, &mv, 0, (int32_t)h, tok0, &bar_v);
-        tma_load_3d(sm + kPrepV + 8192, &mv, 64, (int32_t)h, tok0, &bar_v);
-        v_issued = true;
-    }
-    const uint32_t id_wu = idesc_bf16(128, 64, 1, 0);
+    // W^T = K^T T'^T (M = d_k, K = 64 tokens)
     if (warp == 0 && __all_sync(0xffffffffu, ok)) {
+        const uint32_t id_w = idesc_bf16(128, 64, 1, 0);
         const uint64_t dk = sdesc_sw128(smem_u32(sm), 16384, 1024), dtp = sdesc_sw128(smem_u32(sm + 8192), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm, dk + ((kk * 2048) >> 4), dtp + ((kk * 32) >> 4), id_wu, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm, dk + ((kk * 2048) >> 4), dtp + ((kk * 32) >> 4), id_w, kk > 0);
         mma_commit_warp(&bar_w);
-        const bool vok = mbar_wait(&bar_v, 0);
-        ok = vok;  // (warp 0 reports a V wait that gave up)
-        if (__all_sync(0xffffffffu, vok)) {
-            tc_fence_after();
-            const uint64_t dv = sdesc_sw128(smem_u32(sm + kPrepV), 8192, 1024),
-                           dtpp = sdesc_sw128(smem_u32(sm + 24576), 16, 1024);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tm + 64, dv + ((kk * 2048) >> 4), dtpp + ((kk * 32) >> 4), id_wu, kk > 0);
-        }
-        mma_commit_warp(&bar_u);  // (after a failed V wait this tracks no new product: U is garbage, ok is false)
     }
 
-    // Epilogue 2: thread row r is channel r of W^T and U^T, tokens [32 hf, 32 hf + 32).
-    // W goes out as a K-major operand image (rows = tokens, two 64-channel
-    // blocks) while U^T is formed, then U^T as 128-byte-swizzled rows (row = channel).
+    // Epilogue 2: thread row r is channel r of W^T, tokens [32 hf, 32 hf + 32), out as
+    // 128-byte swizzled rows (row = channel).
     ok = ok && mbar_wait(&bar_w, 0);
     tc_fence_after();
     if (ok) store_w(tm, blk, qd, hf, lane);
-    ok = ok && mbar_wait(&bar_u, 0);
-    tc_fence_after();
-    if (ok) store_u(tm, blk, qd, hf, lane);
     tc_fence_before();
     if (__syncthreads_or(!ok)) {
         // A wait gave up: record it, then wait (bounded) for the tile copies and for
@@ -337,7 +311,6 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         if (tid == 0) {
             flag_error(err, GDN_DEV_TIMEOUT_PREP);
             mbar_wait(&bar_ld, 0);
-            if (v_issued) mbar_wait(&bar_v, 0);
         }
         if (warp == 0) {
             mma_commit_warp(&bar_drain);
@@ -345,32 +318,35 @@ gdn_prep_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
         }
         __syncthreads();
     }
-    if (warp == 0) tmem_dealloc(tm, 128);
+    if (warp == 0) tmem_dealloc(tm, 64);
 }
 
 // ===========================================================================
 // Scan
 // ===========================================================================
-// Shared memory (1024-aligned), three stages of per-chunk operands, each the
-// chunk-head's workspace block as it is (two bulk copies; with one gate per head
-// the Q and K tiles come from q and k themselves, by TMA, where the block holds Qs
-// and K~):
+// Shared memory (1024-aligned), two stages of per-chunk operands, each the
+// chunk-head's workspace block as it is (bulk copies; with one gate per head the Q
+// and K tiles come from q and k themselves, by TMA, where the block holds Qs and K~)
+// followed by the V tile (TMA):
 //   [0, 16K)      W^T rows: the MN-major B operand of S0 W^T (N = 64)
 //   [16K, 32K)    Q or Qs, two 64-channel halves: the K-major B operand of S0 Q^T
 //   [32K, 48K)    K (one gate per head) or K~: the MN-major B operand of the state
 //                 increment (N = 128)
 //   [48K, 56K)    P rows: the K-major B operand of U'^T P^T (N = 64)
-//   [56K, 72K)    U^T rows;  [72K, 73K) gate factors
+//   [56K, 64K)    -T'' rows: the K-major B operand of V^T (-T'')^T
+//   [64K, 65K)    gate factors
+//   [65K, 81K)    the V tile: the MN-major A operand of V^T (-T'')^T
 // The operands the threads produce (S0 and U' in bf16) are written to TMEM and
 // used as A operands straight from there.
-// TMEM columns: [0,128) D1 = [S0 W^T | S0 Q^T], [128,320) D2 = [increment | U'^T P^T],
-// [320,384) S0, [384,416) U', [416,448) diag(w) U' (one gate per head).
+// TMEM columns: [0,128) D1 = [S0 W^T - U^T | S0 Q^T], [128,320) D2 = [increment |
+// U'^T P^T], [320,384) S0, [384,416) U', [416,448) diag(w) U' (one gate per head).
 // A tcgen05.ld waits for the MMAs in flight, so every accumulator is read once
 // the chunk's MMAs are done (the output with the state increment), and the
 // output leaves from registers while the next chunk's first MMA group runs.
-constexpr uint32_t kStW = kBlkW, kStQ = kBlkQs, kStRest = kBlkRest, kStage = (uint32_t)kTcBlock;
-static_assert(kStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled operands");
-constexpr int kStages = 3;
+constexpr uint32_t kStW = kBlkW, kStQ = kBlkQs, kStRest = kBlkRest, kStV = (uint32_t)kTcBlock;
+constexpr uint32_t kStage = kStV + 16384;
+static_assert(kStV % 1024 == 0 && kStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled operands");
+constexpr int kStages = 2;
 constexpr uint32_t kScanSmem = kStages * kStage + 1024;
 constexpr uint32_t kTmD1 = 0, kTmD2 = 128, kTmAS = 320, kTmAU = 384, kTmAUw = 416;
 
@@ -420,16 +396,18 @@ __device__ __forceinline__ int32_t *split_rec(const ScanSplit &sp, int which, in
 // Eight warps hold the state (two threads per row, 64 columns each); warp 0 also
 // issues the MMAs and warp 4 the copies.
 #define GDN_SCAN_PARAMS                                                                                              \
-    const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk, const float *h0,                \
+    const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,                                  \
+        const __grid_constant__ CUtensorMap mv, const float *h0,                                                     \
         const int32_t *__restrict__ cu,                                                                              \
         const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk,                  \
         int64_t max_chunks, int64_t snap_stride, int64_t n_snap, const uint8_t *__restrict__ blocks,                  \
         __nv_bfloat16 *__restrict__ out, float *final_state, float *__restrict__ snaps, const ScanSplit sp, int *err
 #define GDN_SCAN_ARGS \
-    mq, mk, h0, cu, off, N, T, rows, H, Hk, max_chunks, snap_stride, n_snap, blocks, out, final_state, snaps, sp, err
+    mq, mk, mv, h0, cu, off, N, T, rows, H, Hk, max_chunks, snap_stride, n_snap, blocks, out, final_state, snaps, sp, err
 
 template <bool KDA, bool SPLIT>
-__device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorMap &mk, const float *h0,
+__device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                          const float *h0,
                                           const int32_t *__restrict__ cu,
                                           const int32_t *__restrict__ off, int64_t N, int64_t T, int64_t rows,
                                           int64_t H, int64_t Hk, int64_t max_chunks, int64_t snap_stride,
@@ -556,9 +534,10 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
 
     int64_t issued = 0;  // (loader) chunks whose copies are issued
-    // (one gate per head) the Q and K tiles of chunk c: token rows q_row0 + 64 c, query/key head hq
+    // the V tile (and, one gate per head, the Q and K tiles) of chunk c: token rows
+    // q_row0 + 64 c; query/key head hq
     int32_t q_row0 = 0, hq = 0;
-    if (!KDA && tid == kLoader) {
+    if (tid == kLoader) {
         q_row0 = (int32_t)(start + cb * C);
         hq = (int32_t)(h / (H / Hk));
     }
@@ -582,6 +561,8 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
             mbar_arrive_expect_tx(bar, kStage);
             bulk_load(st, blk, (uint32_t)kTcWQ, bar);
             bulk_load(st + kStRest, blk + kBlkRest, (uint32_t)kTcRest, bar);
+            tma_load_3d(st + kStV, &mv, 0, h, row0, bar);
+            tma_load_3d(st + kStV + 8192, &mv, 64, h, row0, bar);
         } else {  // one gate per head: the Q and K tiles themselves (the output and U' are scaled)
             mbar_arrive_expect_tx(bar, kStage);
             bulk_load(st + kStW, blk + kBlkW, 16384u, bar);
@@ -590,6 +571,8 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
             tma_load_3d(st + kStRest + kRestKt, &mk, 0, hq, row0, bar);
             tma_load_3d(st + kStRest + kRestKt + 8192, &mk, 64, hq, row0, bar);
             bulk_load(st + kStRest + kRestP, blk + kBlkRest + kRestP, (uint32_t)(kTcRest - kTcKt), bar);
+            tma_load_3d(st + kStV, &mv, 0, h, row0, bar);
+            tma_load_3d(st + kStV + 8192, &mv, 64, h, row0, bar);
         }
         issued = c + 1;
     };
@@ -671,15 +654,23 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
         const bool emit_state = spec ? lam_next < kLamDrop : emit_any;
         if (spec && emit && m_first == nchunks) m_first = c;
 
-        // (b) D1 = [S0 W^T | S0 Q^T]   (N = 64 + 64, K = 128): [U correction | inter-chunk
-        //     output] (S0 W^T only, for a chunk without outputs).  S0 W^T is committed
-        //     on its own: U' needs only it, and is formed while S0 Q^T runs.
+        // (b) D1 = [S0 W^T + V^T (-T'')^T | S0 Q^T]   (N = 64 + 64): [-U'^T, with U = T'' V |
+        //     inter-chunk output]; a transition map drops the writes (D1 = S0 W^T, so
+        //     again -U'^T) and has no output.  -U'^T is committed on its own: U' is formed
+        //     from it while S0 Q^T runs.
         if (warp == kIssuer) {
             const uint64_t bw = sdesc_sw128(st_u + kStW, 8192, 1024), bq = sdesc_sw128(st_u + kStQ, 16, 1024);
             const uint32_t id_w = idesc_bf16(128, 64, 0, 1), id_q = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
                 mma_bf16_ts(tm + kTmD1, tm + kTmAS + kk * 8, bw + (uint64_t)((kk * 2048) >> 4), id_w, kk > 0);
+            if (!ident) {
+                const uint64_t av = sdesc_sw128(st_u + kStV, 8192, 1024), bt = sdesc_sw128(st_u + kStRest + kRestTn, 16, 1024);
+                const uint32_t id_v = idesc_bf16(128, 64, 1, 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tm + kTmD1, av + (uint64_t)((kk * 2048) >> 4), bt + (uint64_t)((kk * 32) >> 4), id_v, 1);
+            }
             mma_commit_warp(&bars.mma[0]);
             if (emit)
 #pragma unroll
@@ -713,8 +704,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
         // the first half of the previous chunk's output, while these MMAs run
         if (c >= 1 && emit_prev) store_output(c - 1, 0);
 
-        // (c) U' = U - S0 W^T over tokens [32 hf, 32 hf + 32) -> TMEM A operand
-        //     (a transition map drops the writes: U' = -S0 W^T)
+        // (c) U' = -D1 over tokens [32 hf, 32 hf + 32) -> TMEM A operand (and diag(w) U')
         ok = mbar_wait(&bars.mma[0], par) && ok;
         tc_fence_after();
         {
@@ -728,10 +718,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
                 uint32_t wu[8], ww[8];
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
-                    const int q = 2 * hh + qq, cq = 4 * hf + q;  // 16-byte chunk = tokens 8 cq .. 8 cq + 7
-                    uint4 u8 = make_uint4(0u, 0u, 0u, 0u);
-                    if (!ident) u8 = *reinterpret_cast<const uint4 *>(rest + kRestU + sw128_offset(v, cq));
-                    const uint32_t uw32[4] = {u8.x, u8.y, u8.z, u8.w};
+                    const int q = 2 * hh + qq;  // tokens 32 hf + 8 q .. + 7
                     float wt[8] = {};
                     if (!KDA) {
                         const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
@@ -740,11 +727,8 @@ __device__ __forceinline__ void scan_body(const CUtensorMap &mq, const CUtensorM
                     }
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
-                        const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&uw32[e / 2]);
                         const float *acc = hh == 0 ? &a0[8 * qq + e] : &a1[8 * qq + e];
-                        // u - acc (one rounding, as the subtraction), then w (u - acc)
-                        const float2 d = __ffma2_rn(make_float2(acc[0], acc[1]), make_float2(-1.f, -1.f),
-                                                    make_float2(__low2float(u2), __high2float(u2)));
+                        const float2 d = make_float2(-acc[0], -acc[1]);  // U'
                         wu[4 * qq + e / 2] = pack_bf16(d.x, d.y);
                         if (!KDA) {
                             const float2 dw = __fmul2_rn(make_float2(wt[e], wt[e + 1]), d);
@@ -1052,12 +1036,12 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     if (attr_err != cudaSuccess) return fail(GDN_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(attr_err));
     if (p.max_chunks > 0 && p.rows > 0) {
         if (p.per_channel) {
-            if ((st = tc::launch_prep_kda(mq, mk, mv, mg, p, a, off, blocks, s)) != GDN_OK) return st;
+            if ((st = tc::launch_prep_kda(mq, mk, mg, p, a, off, blocks, s)) != GDN_OK) return st;
         } else {
             const dim3 grid((unsigned)p.max_chunks, (unsigned)p.H);
             log_launch("gdn_prep_tc", grid, dim3(kThreads), kPrepSmem);
             LaunchScope ls("gdn_prep_tc", s);
-            gdn_prep_tc<<<grid, kThreads, kPrepSmem, s>>>(mq, mk, mv, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows,
+            gdn_prep_tc<<<grid, kThreads, kPrepSmem, s>>>(mq, mk, a.g, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows,
                                                           p.H, a.Hk, a.scale, blocks, p.split_G >= 2 ? 1 : 0,
                                                           a.status);
             if ((st = check_launch("gdn_prep_tc")) != GDN_OK) return st;
@@ -1071,7 +1055,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
         const dim3 grid((unsigned)a.N, (unsigned)p.H);
         log_launch(p.per_channel ? "gdn_scan_kda_tc" : "gdn_scan_tc", grid, dim3(scan_block), kScanSmem);
         LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc" : "gdn_scan_tc", s);
-        kern<<<grid, scan_block, kScanSmem, s>>>(mq, mk, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk,
+        kern<<<grid, scan_block, kScanSmem, s>>>(mq, mk, mv, a.h0, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk,
                                                  p.max_chunks, a.snapshot_stride, a.n_snap, blocks,
                                                  (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp, a.status);
         return check_launch("gdn_scan_tc");
@@ -1088,7 +1072,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         log_launch("gdn_scan (pass 1)", dim3((unsigned)grid1), dim3(split_block), kScanSmem);
         LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 1)" : "gdn_scan_split_tc (pass 1)", s);
-        kern<<<(unsigned)grid1, split_block, kScanSmem, s>>>(mq, mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
+        kern<<<(unsigned)grid1, split_block, kScanSmem, s>>>(mq, mk, mv, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
                                                              p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap,
                                                              blocks,
                                                              (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp,
@@ -1106,7 +1090,7 @@ gdn_status launch_chunk_tc(const ChunkPlan &p, const ChunkArgs &a, cudaStream_t 
     {
         log_launch("gdn_scan (pass 2)", dim3((unsigned)grid2), dim3(split_block), kScanSmem);
         LaunchScope ls(p.per_channel ? "gdn_scan_kda_tc (pass 2)" : "gdn_scan_split_tc (pass 2)", s);
-        kern<<<(unsigned)grid2, split_block, kScanSmem, s>>>(mq, mk, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
+        kern<<<(unsigned)grid2, split_block, kScanSmem, s>>>(mq, mk, mv, a.h0, nullptr, nullptr, a.N, a.T, p.rows,
                                                              p.H, a.Hk, p.max_chunks, a.snapshot_stride, a.n_snap,
                                                              blocks,
                                                              (__nv_bfloat16 *)a.out, a.final_state, a.snapshots, sp,

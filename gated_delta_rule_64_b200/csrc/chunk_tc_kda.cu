@@ -10,6 +10,8 @@
 //   A_ij = beta_i sum_c k_ic k_jc exp(b_ic - b_jc)       (j < i)
 //   P_ij = scale  sum_c q_ic k_jc exp(b_ic - b_jc)       (j <= i)
 //   W    = T diag(beta) (K * Gam),   U = T diag(beta) V,   T = (I + A)^-1
+//   (U itself is not formed here: the block holds -T diag(beta) and the scan
+//   accumulates V^T (-T diag(beta))^T onto S0 W^T)
 //   Qs   = scale Q * Gam,            K~ = K * exp(b_L - b)
 //
 // (Gam_i = exp(b_i)); the scan then carries S0 Diag(Gam_L) + U'^T K~.
@@ -49,12 +51,12 @@ namespace {
 //               K * L and Q * L, and then K * L becomes K * Gam (the A operand of W).
 //   [32K, 64K)  gate tile (TMA: four [64 tokens][32 channels] fp32 quarters, 128-byte
 //               swizzle), turned in place into b in log2 units; once the factors are
-//               formed: A (fp32, f32_offset layout) at 32K and the V tile at 48K
+//               formed: A (fp32, f32_offset layout) at 32K
 //   [64K, 80K)  K * R (layout of a K tile, channel halves 8K apart); after the blocks:
 //               T (fp32)
 //   [80K, 96K)  after the blocks: the solve's scratch (4K) and T diag(beta) (8K at 88K)
 //   [96K, 104K) P rows (bf16, row = query token i, 64 key tokens j, 128-byte swizzle)
-constexpr uint32_t kSmKQ = 0, kSmB = 32768, kSmA = 32768, kSmV = 49152, kSmZ = 65536, kSmP = 98304;
+constexpr uint32_t kSmKQ = 0, kSmB = 32768, kSmA = 32768, kSmZ = 65536, kSmP = 98304;
 constexpr uint32_t kSmT = 65536, kSmY = 81920, kSmTp = 90112;
 constexpr uint32_t kSmem = kSmP + 8192 + 1024;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -246,13 +248,13 @@ __device__ __forceinline__ void diag_exact_store(uint8_t *sm, const DiagKeep &ke
 
 __global__ void __launch_bounds__(kThreads, 2)
 gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
+                const __grid_constant__ CUtensorMap mg,
                 const float *__restrict__ beta, const int32_t *__restrict__ cu, const int32_t *__restrict__ off,
                 int64_t N, int64_t T, int64_t rows, int64_t H, int64_t Hk, float scale, uint8_t *__restrict__ blocks,
                 int want_bound, int *err) {
     extern __shared__ unsigned char smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    __shared__ uint64_t bar_g, bar_ld, bar_v, bar_mma, bar_drain;
+    __shared__ uint64_t bar_g, bar_ld, bar_mma, bar_drain;
     __shared__ uint32_t tmem_base;
     __shared__ float s_beta[C], s_tot[D], s_lam[kThreads / 32];
     __shared__ __align__(16) Factors fct;
@@ -272,7 +274,6 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     if (tid == 0) {
         mbar_init(&bar_g, 1);
         mbar_init(&bar_ld, 1);
-        mbar_init(&bar_v, 1);
         mbar_init(&bar_mma, 1);
         mbar_init(&bar_drain, 1);
         fence_mbar_init();
@@ -465,18 +466,12 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             float *fac = reinterpret_cast<float *>(rest + kRestFac);
             if (tid < D) fac[kFacGL + tid] = ex2(*reinterpret_cast<const float *>(sm + kSmB + b_off(Lm1, tid)));
         }
-        fence_async_smem();  // the b region is taken over by the V tile (TMA) below
         const bool any_bad = __syncthreads_or(bad);
         if (tid == 0) {
             float lam = 0.f;
 #pragma unroll
             for (int w = 0; w < kThreads / 32; ++w) lam += s_lam[w];
             reinterpret_cast<float *>(rest + kRestFac)[kFacLam] = (!want_bound || any_bad) ? kLamNone : lam * kLog2e;
-        }
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_v, 2 * 8192);
-            tma_load_3d(sm + kSmV, &mv, 0, (int32_t)h, tok0, &bar_v);
-            tma_load_3d(sm + kSmV + 8192, &mv, 64, (int32_t)h, tok0, &bar_v);
         }
 
         // A and P.  Warp w takes row block p against column blocks [q0, q0 + nq);
@@ -565,8 +560,9 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     blocked_solve<kSmT, kSmY>(sm, [](int i, int j) { return kSmA + f32_offset(i, j); },
                               [](int i) { return kSmA + (uint32_t)i * 256u; }, ok);
 
-    // T'' = T diag(beta) as a bf16 operand image (K-major rows i); the blocks of T above
-    // its block diagonal are zero (the solve leaves them unwritten).
+    // T'' = T diag(beta) as a bf16 operand image (K-major rows i), and -T'' as rows of
+    // the block (the scan's operand); the blocks of T above its block diagonal are zero
+    // (the solve leaves them unwritten).
     if (ok) {
         const int i = tid >> 2, j0 = (tid & 3) * 16;
         const bool upper = (tid & 3) > (i >> 4);
@@ -583,8 +579,10 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             float b[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) b[e] = tv[8 * q + e] * s_beta[j0 + 8 * q + e];
-            st_shared_v4(tp + sw128_offset(i, (j0 >> 3) + q), pack_bf16(b[0], b[1]), pack_bf16(b[2], b[3]),
-                         pack_bf16(b[4], b[5]), pack_bf16(b[6], b[7]));
+            const uint32_t o = sw128_offset(i, (j0 >> 3) + q);
+            st_shared_v4(tp + o, pack_bf16(b[0], b[1]), pack_bf16(b[2], b[3]), pack_bf16(b[4], b[5]), pack_bf16(b[6], b[7]));
+            *reinterpret_cast<uint4 *>(rest + kRestTn + o) = make_uint4(pack_bf16(-b[0], -b[1]), pack_bf16(-b[2], -b[3]),
+                                                                        pack_bf16(-b[4], -b[5]), pack_bf16(-b[6], -b[7]));
         }
     }
     fence_async_smem();
@@ -592,21 +590,17 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
 
-    // W^T = (K * Gam)^T T''^T (M = d_k), U^T = V^T T''^T (M = d_v); K = 64 tokens.
-    ok = mbar_wait(&bar_v, 0) && ok;
+    // W^T = (K * Gam)^T T''^T (M = d_k, K = 64 tokens)
     if (warp == 0 && __all_sync(0xffffffffu, ok)) {
-        const uint64_t dk = sdesc_sw128(smem_u32(sm + kSmKQ), 16384, 1024), dv = sdesc_sw128(smem_u32(sm + kSmV), 8192, 1024),
-                       dt = sdesc_sw128(smem_u32(sm + kSmTp), 16, 1024);
+        const uint64_t dk = sdesc_sw128(smem_u32(sm + kSmKQ), 16384, 1024), dt = sdesc_sw128(smem_u32(sm + kSmTp), 16, 1024);
         const uint32_t id = idesc_bf16(128, 64, 1, 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm, dk + ((kk * 2048) >> 4), dt + ((kk * 32) >> 4), id, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tm + 64, dv + ((kk * 2048) >> 4), dt + ((kk * 32) >> 4), id, kk > 0);
         mma_commit_warp(&bar_mma);
     }
     ok = ok && mbar_wait(&bar_mma, fast ? 1 : 0);
     tc_fence_after();
-    if (ok) store_wu(tm, blk, qd, hf, lane);
+    if (ok) store_w(tm, blk, qd, hf, lane);
     tc_fence_before();
     if (__syncthreads_or(!ok)) {
         // A wait gave up: record it, then wait (bounded) for the tile copies and for
@@ -615,7 +609,6 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             flag_error(err, GDN_DEV_TIMEOUT_PREP);
             mbar_wait(&bar_g, 0);
             mbar_wait(&bar_ld, 0);
-            mbar_wait(&bar_v, 0);
         }
         if (warp == 0) {
             mma_commit_warp(&bar_drain);
@@ -628,9 +621,9 @@ gdn_prep_kda_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
 
 }  // namespace
 
-gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                           const CUtensorMap &mg, const ChunkPlan &p, const ChunkArgs &a, const int32_t *off,
-                           uint8_t *blocks, cudaStream_t s) {
+gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mg,
+                           const ChunkPlan &p, const ChunkArgs &a, const int32_t *off, uint8_t *blocks,
+                           cudaStream_t s) {
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [] {
@@ -640,7 +633,7 @@ gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const C
     log_launch("gdn_prep_kda_tc", dim3((unsigned)p.max_chunks, (unsigned)p.H), dim3(kThreads), kSmem);
     LaunchScope ls("gdn_prep_kda_tc", s);
     gdn_prep_kda_tc<<<dim3((unsigned)p.max_chunks, (unsigned)p.H), kThreads, kSmem, s>>>(
-        mq, mk, mv, mg, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, p.split_G >= 2 ? 1 : 0,
+        mq, mk, mg, a.beta, a.cu_seqlens, off, a.N, a.T, p.rows, p.H, a.Hk, a.scale, blocks, p.split_G >= 2 ? 1 : 0,
         a.status);
     return check_launch("gdn_prep_kda_tc");
 }

@@ -90,17 +90,19 @@ bool tc_eligible(const gdn_desc &d);
 
 // Per chunk-head workspace block of the tensor-core path (bytes), both gate kinds:
 //   [W^T rows 16K][Qs (channels 0-63) 8K][Qs (64-127) 8K]
-//   [K~ 16K][P rows 8K][U^T rows 16K][gate factors 1K]
+//   [K~ 16K][P rows 8K][-T'' rows 8K][gate factors 1K]
 // Every operand is 128-byte swizzled rows of 128 bytes (64 bf16), in 8-row groups
 // 1 KB apart.  W^T (row = key channel, 64 tokens) is the MN-major B operand of
 // S0 W^T; Qs = scale Q * Gam (per-channel gate only; row = token, the layout of a
-// Q tile) the K-major one of S0 Qs^T.  K~ = K * exp(b_L - b) (the layout of a K
-// tile: rows = tokens, two 64-channel halves) is the MN-major B operand of
-// U'^T K~; P (row = query token i, 64 key tokens j) the K-major one of U'^T P^T.
-// The scan copies a block with two bulk copies.
-constexpr size_t kTcWQ = 32768, kTcKt = 64 * 128 * 2, kTcPImg = 64 * 128, kTcUt = 128 * 128, kTcFac = 1024;
-constexpr size_t kTcRest = kTcKt + kTcPImg + kTcUt + kTcFac;  // 41984
-constexpr size_t kTcBlock = kTcWQ + kTcRest;                  // 74752
+// Q tile) the K-major one of S0 Qs^T.  K~ = K * exp(b_L - b) (per-channel gate only;
+// the layout of a K tile: rows = tokens, two 64-channel halves) is the MN-major B
+// operand of U'^T K~; P (row = query token i, 64 key tokens j) the K-major one of
+// U'^T P^T; -T'' = -T diag(beta) (row = token i, 64 tokens j) the K-major one of
+// V^T (-T'')^T, which the scan accumulates onto S0 W^T to get -U'^T.  The scan
+// copies a block with two or three bulk copies.
+constexpr size_t kTcWQ = 32768, kTcKt = 64 * 128 * 2, kTcPImg = 64 * 128, kTcTn = 64 * 128, kTcFac = 1024;
+constexpr size_t kTcRest = kTcKt + kTcPImg + kTcTn + kTcFac;  // 33792
+constexpr size_t kTcBlock = kTcWQ + kTcRest;                  // 66560
 gdn_status launch_decode(const gdn_desc &d, const void *q, const void *k, const void *v,
                          const float *g, const float *beta, float *state, void *out,
                          cudaStream_t s);

@@ -21,12 +21,12 @@ constexpr int D = 128;     // d_k = d_v
 constexpr int kThreads = 256;
 
 // Offsets inside one workspace block: W^T rows at 0, the Qs halves (per-channel
-// gate) at kBlkQs and kBlkQs + 8K, then the rest at kBlkRest: K~, P rows, U^T rows,
+// gate) at kBlkQs and kBlkQs + 8K, then the rest at kBlkRest: K~, P rows, -T'' rows,
 // gate factors.
 constexpr uint32_t kBlkW = 0, kBlkQs = 16384, kBlkRest = (uint32_t)kTcWQ;
-constexpr uint32_t kRestKt = 0, kRestP = 16384, kRestU = 24576, kRestFac = 40960;
-static_assert(kBlkQs + 16384 == kTcWQ && kRestP == kTcKt && kRestU == kRestP + kTcPImg &&
-                  kRestFac == kRestU + kTcUt && kRestFac + kTcFac == kTcRest,
+constexpr uint32_t kRestKt = 0, kRestP = 16384, kRestTn = 24576, kRestFac = 32768;
+static_assert(kBlkQs + 16384 == kTcWQ && kRestP == kTcKt && kRestTn == kRestP + kTcPImg &&
+                  kRestFac == kRestTn + kTcTn && kRestFac + kTcFac == kTcRest,
               "block layout");
 // Gate factors (floats): exp(b_L), at [0] for the per-head gate and per key
 // channel at [0, 128) for the per-channel gate; at [kFacLam] a bound on how much
@@ -273,10 +273,10 @@ __device__ __forceinline__ void blocked_solve(uint8_t *sm, OffA offA, RowA rowA,
     __syncthreads();
 }
 
-// Epilogue of the W / U MMAs: TMEM columns [0, 64) hold W^T and [64, 128) U^T
-// (lane = channel, column = token).  Thread row r = qd*32 + lane writes tokens
-// [32 hf, 32 hf + 32) of its channel row of W^T and of U^T (128-byte swizzled rows).
-// (Kept out of line: inlined, they push the per-head prep kernel past its register budget.)
+// Epilogue of the W MMA: TMEM columns [0, 64) hold W^T (lane = channel, column =
+// token).  Thread row r = qd*32 + lane writes tokens [32 hf, 32 hf + 32) of its
+// channel row of W^T (128-byte swizzled rows).
+// (Kept out of line: inlined, it pushes the per-head prep kernel past its register budget.)
 static __device__ __noinline__ void store_rows(uint32_t taddr, uint8_t *dst, int r, int hf) {
     float u0[16], u1[16];
     tmem_ld16(taddr, u0);
@@ -292,19 +292,12 @@ static __device__ __noinline__ void store_rows(uint32_t taddr, uint8_t *dst, int
 __device__ __forceinline__ void store_w(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
     store_rows(tm + ((uint32_t)(qd * 32) << 16) + 32 * hf, blk + kBlkW, qd * 32 + lane, hf);
 }
-__device__ __forceinline__ void store_u(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
-    store_rows(tm + ((uint32_t)(qd * 32) << 16) + 64 + 32 * hf, blk + kBlkRest + kRestU, qd * 32 + lane, hf);
-}
-__device__ __forceinline__ void store_wu(uint32_t tm, uint8_t *blk, int qd, int hf, int lane) {
-    store_w(tm, blk, qd, hf, lane);
-    store_u(tm, blk, qd, hf, lane);
-}
 
 // Prep kernel of the per-channel gate (its own translation unit).
 // (mg: the per-channel log gate as a (rows, H, 128) fp32 tensor, 32 x 1 x 64 boxes, 128-byte swizzle.)
-gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                           const CUtensorMap &mg, const ChunkPlan &p, const ChunkArgs &a, const int32_t *off,
-                           uint8_t *blocks, cudaStream_t s);
+gdn_status launch_prep_kda(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mg,
+                           const ChunkPlan &p, const ChunkArgs &a, const int32_t *off, uint8_t *blocks,
+                           cudaStream_t s);
 
 }  // namespace tc
 }  // namespace gdn

@@ -65,7 +65,7 @@ def test_workspace_size(lib):
         return n.value
     simt = 4 * 64 * (128 + 128 + 64 + 1)          # fp32 W, U, P and gate per chunk-head
     assert 6 * 3 * simt <= size(dtype=gdn.GDN_F32) < 6 * 3 * simt + 4096
-    tc = 32768 + 64 * 128 * 2 + 64 * 128 + 128 * 128 + 1024  # [W;Qs] images, K~, P^T image, U^T rows, factors
+    tc = 32768 + 64 * 128 * 2 + 64 * 128 + 64 * 128 + 1024  # W^T and Qs rows, K~, P rows, -T'' rows, factors
     assert 6 * 3 * tc <= size() < 6 * 3 * tc + 4096
     # the per-channel gate uses the same block
     assert 6 * 3 * tc <= size(gate=gdn.GDN_GATE_CHANNEL) < 6 * 3 * tc + 4096
@@ -338,7 +338,7 @@ def test_split_scan_workspace(lib):
         d = _desc(**kw)
         assert lib.gdn_chunk_workspace_size(ctypes.byref(d), kw.get("B", 2), ctypes.byref(n)) == gdn.GDN_OK
         return n.value
-    blk = 32768 + 64 * 128 * 2 + 64 * 128 + 128 * 128 + 1024
+    blk = 32768 + 64 * 128 * 2 + 64 * 128 + 64 * 128 + 1024  # the tensor-core block of a chunk-head
     up = lambda x: -(-x // 256) * 256
     state = 128 * 128 * 4
 
