@@ -84,6 +84,58 @@ def test_one_group_form_of_a_chunk():
     assert np.max(np.abs(o - o_ref)) <= 1e-12 * max(1, np.abs(o_ref).max())
 
 
+def _grouped_forward(q, k, v, g, beta, S0, C=64, scale=1.0):
+    """The chunk step regrouped the way the tensor-core kernels form it, chunk by chunk:
+    the block holds W^T = (T diag(beta gam) K)^T (per-channel gate: T diag(beta) (K*Gam)),
+    P and -T'' = -T diag(beta), never U; the scan's first group gives
+    D = S0 W^T + V^T (-T'')^T = -U'^T, so U' = -D^T; the state increment is
+    (diag(w) U')^T K with w_j = exp(b_L - b_j) for one gate per head (U'^T K~ with
+    K~ = K * exp(b_L - b) per channel); the output is scale gam_i (S0 q_i) + P U'."""
+    T, dk = k.shape
+    per_channel = g.ndim == 2
+    S = S0.astype(np.float64).copy()
+    out = np.zeros((T, v.shape[1]))
+    for s0 in range(0, T, C):
+        e = min(T, s0 + C)
+        n = e - s0
+        Q, K, V, be = q[s0:e], k[s0:e], v[s0:e], beta[s0:e]
+        b = np.cumsum(g[s0:e], axis=0)
+        dec = np.exp(b[:, None, :] - b[None, :, :]) if per_channel else np.exp(b[:, None] - b[None, :])
+        gram = np.einsum("ic,jc,ijc->ij", K, K, dec) if per_channel else (K @ K.T) * dec
+        qk = np.einsum("ic,jc,ijc->ij", Q, K, dec) if per_channel else (Q @ K.T) * dec
+        Tm = np.linalg.inv(np.eye(n) + np.tril(be[:, None] * gram, -1))
+        Tb = Tm * be[None, :]                                  # T'' = T diag(beta)
+        Wt = (Tb @ (K * np.exp(b))).T if per_channel else (Tm * (be * np.exp(b))[None, :] @ K).T
+        P = scale * np.tril(qk)
+        D = S @ Wt + V.T @ (-Tb).T                              # -U'^T
+        Up = -D.T
+        if per_channel:
+            inc = Up.T @ (K * np.exp(b[-1] - b))
+            out[s0:e] = (scale * Q * np.exp(b)) @ S.T + P @ Up
+            S = S * np.exp(b[-1])[None, :] + inc
+        else:
+            w = np.exp(b[-1] - b)
+            inc = (w[:, None] * Up).T @ K
+            out[s0:e] = (scale * np.exp(b))[:, None] * (Q @ S.T) + P @ Up
+            S = np.exp(b[-1]) * S + inc
+    return out, S
+
+
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_kernel_grouping_matches_token_loop(per_channel):
+    """The regrouping the kernels use (no U in the block; -U'^T as one accumulation of
+    S0 W^T and V^T (-T'')^T; the increment through diag(w) U' for one gate per head)
+    is the same chunk step: equal to the token loop over several chunks and a ragged
+    tail."""
+    q, k, v, g, beta, S0 = _problem(41, 150, 12, 9, per_channel)
+    o_ref, s_ref, _ = oracle.gated_delta_rule(q[None, :, None], k[None, :, None], v[None, :, None],
+                                              g[None, :, None], beta[None, :, None], S0[None, None],
+                                              per_channel=per_channel, scale=0.7)
+    o, s = _grouped_forward(q, k, v, g, beta, S0, C=64, scale=0.7)
+    assert np.max(np.abs(o - o_ref[0, :, 0])) <= 1e-12 * max(1, np.abs(o_ref).max())
+    assert np.max(np.abs(s - s_ref[0, 0])) <= 1e-12 * max(1, np.abs(s_ref).max())
+
+
 @pytest.mark.parametrize("L", [64, 40, 17])
 def test_per_channel_blocks_as_one_product(L):
     """The per-channel prep forms A and P as one product when the decays are
