@@ -20,25 +20,25 @@
 //
 // Two kernels:
 //   gdn_prep_tc  one CTA per (chunk, head), all chunks in parallel.  TMA loads
-//                K, Q, V; one M = 128 MMA gives [K;Q] K^T (the K rows give the
+//                K and Q; one M = 128 MMA gives [K;Q] K^T (the K rows give the
 //                Gram matrix, the Q rows Q K^T); the unit-lower-triangular
 //                system is solved blockwise (16 x 16 diagonal blocks by forward
 //                substitution in fp32, off-diagonal blocks by tf32 warp MMAs);
-//                two MMAs give W^T and U^T.  The results are written as
-//                ready-made operand images (16-byte stores of 128-byte swizzled
-//                rows) into one contiguous block per chunk-head.
+//                one MMA gives W^T.  W^T, P, -T'' = -T diag(beta) and the gate
+//                factors are written as ready-made operand images (16-byte
+//                stores of 128-byte swizzled rows) into one contiguous block per
+//                chunk-head; U itself is never formed.
 //   gdn_scan_tc  one CTA per (sequence, head).  The fp32 state lives in
 //                registers (two threads per state row, 64 columns each); per
 //                chunk it is rounded to a bf16 A operand in TMEM and two MMA
 //                groups with fp32 accumulators in TMEM produce
-//                [S0 W^T | S0 Q^T] and, from U' = U - W S0^T,
+//                [S0 W^T + V^T (-T'')^T | S0 Q^T] (the first part is -U'^T:
+//                U' = U - W S0^T with U = T diag(beta) V) and then
 //                [(diag(w) U')^T K | U'^T P^T] with w_j = exp(b_L - b_j) (the
-//                state increment and the intra-chunk output).  The next chunks'
-//                blocks are prefetched (bulk copies; Q and K tiles by TMA) into
-//                three stages.
-//                A ninth warp issues the MMAs and copies (per-head gate, no
-//                sequence split), so the eight state warps store the previous
-//                chunk's output while the MMA groups run.
+//                state increment and the intra-chunk output).  The next chunk's
+//                block is prefetched (bulk copies; Q, K and V tiles by TMA) into
+//                the second of two stages, and the previous chunk's output is
+//                stored while the MMA groups run.
 //
 // All tcgen05 MMAs are M = 128 (the 128 rows of the state, or the 64 K rows
 // stacked on the 64 Q rows), so accumulator rows map 1:1 onto TMEM lanes and
@@ -352,7 +352,7 @@ constexpr uint32_t kTmD1 = 0, kTmD2 = 128, kTmAS = 320, kTmAU = 384, kTmAUw = 41
 
 struct ScanBars {
     uint64_t full[kStages];
-    uint64_t mma[3];  // per chunk: S0 W^T done; U'^T K~ done; every product of the chunk done
+    uint64_t mma[3];  // per chunk: -U'^T done; the increment done; every product of the chunk done
     uint64_t drain;   // after a failed wait: every MMA issued has completed
 };
 
